@@ -1,0 +1,454 @@
+// api.cu -- the C ABI of libmoe.so (declared in include/moe.h): argument
+// validation, workspace layout and ownership, TMA descriptor encoding, and the
+// enqueue order of the layer's kernels on the caller's stream.
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+#include "moe_internal.h"
+
+namespace moe {
+
+int grouped_smem_bytes(int K);
+
+static thread_local int g_last_cuda_error = 0;
+
+static int cuda_fail(cudaError_t e)
+{
+    g_last_cuda_error = static_cast<int>(e);
+    return MOE_ERR_CUDA;
+}
+
+int num_sms()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+cudaError_t ensure_max_smem(const void *kernel, int bytes)
+{
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, int> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    int &have = done[std::make_pair(kernel, dev)];
+    if (have >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) have = bytes;
+    return e;
+}
+
+static size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+Layout make_layout(int M, int H, int I, int E, int k)
+{
+    Layout L;
+    const size_t n = static_cast<size_t>(M) * k;
+    L.route_splits = (H + kRouteChunkH - 1) / kRouteChunkH;
+    L.max_tiles = static_cast<int>((n < static_cast<size_t>(E) ? n : static_cast<size_t>(E)) +
+                                   (n + kTileTokens - 1) / kTileTokens);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += round_up(bytes > 0 ? bytes : 1, 256);
+        return o;
+    };
+    L.status = take(256);
+    L.partial = take(static_cast<size_t>(L.route_splits) * M * E * sizeof(float));
+    L.x16 = take(static_cast<size_t>(M) * H * 2);
+    L.topk_ids = take(n * 4);
+    L.topk_w = take(n * 4);
+    L.offsets = take(static_cast<size_t>(E + 1) * 4);
+    L.sorted_ids = take(n * 4);
+    L.inv_pos = take(n * 4);
+    L.tiles = take(static_cast<size_t>(L.max_tiles) * sizeof(ExpertTile));
+    L.n_tiles = take(4);
+    L.h = take(n * I * 2);
+    L.y = take(n * H * sizeof(float));
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------------ validation
+
+static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static int check_dims(int M, int H, int I, int E, int k, bool need_hi)
+{
+    if (M < 0 || E <= 0 || k <= 0 || H <= 0 || (need_hi && I <= 0)) return MOE_ERR_INVALID_ARG;
+    if (E > kMaxE || k > kMaxK || k > E) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (H % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (need_hi && (I % 32 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(M) * k > kMaxAssignments) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (need_hi) {
+        if (static_cast<long long>(E) * 2 * I >= (1LL << 31) || static_cast<long long>(E) * H >= (1LL << 31))
+            return MOE_ERR_UNSUPPORTED_SHAPE;
+        if (grouped_smem_bytes(H) > 227 * 1024 || grouped_smem_bytes(I) > 227 * 1024)
+            return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
+    return MOE_OK;
+}
+
+static bool overlaps(const void *a, size_t an, const void *b, size_t bn)
+{
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + bn && pb < pa + an;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Packed E2M1 matrix viewed as [rows][row_bytes] uint8; boxes of 16 rows x 128 bytes, 128-byte swizzle.
+static int make_weight_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kBoxRows)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------------ library-owned workspaces
+
+static std::mutex g_pool_mu;
+static std::map<std::pair<int, uintptr_t>, std::pair<void *, size_t>> g_pool;
+
+// Workspace of (current device, stream), grown outside stream capture only.  A
+// buffer replaced by a larger one stays allocated: work already queued may use it.
+static int library_workspace(cudaStream_t s, size_t need, char **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    auto &ent = g_pool[std::make_pair(dev, reinterpret_cast<uintptr_t>(s))];
+    if (ent.second >= need) {
+        *out = static_cast<char *>(ent.first);
+        return MOE_OK;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(s, &cs);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (cs != cudaStreamCaptureStatusNone) return MOE_ERR_WORKSPACE;
+    const size_t bytes = need > 2 * ent.second ? need : 2 * ent.second;
+    void *p = nullptr;
+    e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ent = std::make_pair(p, bytes);
+    *out = static_cast<char *>(p);
+    return MOE_OK;
+}
+
+#define MOE_TRY(expr)                                   \
+    do {                                                \
+        cudaError_t _e = (expr);                        \
+        if (_e != cudaSuccess) return cuda_fail(_e);    \
+    } while (0)
+
+// ------------------------------------------------------------------ step bodies (arguments already validated)
+
+static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const int32_t *sorted_ids,
+                       const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int H, int I, int E,
+                       int k, int max_tiles, cudaStream_t s)
+{
+    CUtensorMap map;
+    int rc = make_weight_map(&map, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2);
+    if (rc != MOE_OK) return rc;
+    MOE_TRY(launch_gate_up(map, w13_s, x16, sorted_ids, tiles, n_tiles, h, status, H, I, k, max_tiles, s));
+    return MOE_OK;
+}
+
+static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int H,
+                    int I, int E, int max_tiles, cudaStream_t s)
+{
+    CUtensorMap map;
+    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2);
+    if (rc != MOE_OK) return rc;
+    MOE_TRY(launch_down(map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, H, I, max_tiles, s));
+    return MOE_OK;
+}
+
+// Optional per-launch event marks (profiling entry point only).
+struct Marks {
+    cudaEvent_t ev[MOE_PROFILE_KERNELS + 1];
+    int n = 0;
+    cudaError_t mark(cudaStream_t s) { return cudaEventRecord(ev[n++], s); }
+};
+
+#define MOE_MARK(m, s)                                  \
+    do {                                                \
+        if (m) MOE_TRY((m)->mark(s));                   \
+    } while (0)
+
+static int forward_impl(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
+                        const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H,
+                        int I, int E, int k, int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
+                        char *ws, const Layout &L, cudaStream_t s, Marks *marks = nullptr)
+{
+    int *status = reinterpret_cast<int *>(ws + L.status);
+    float *partial = reinterpret_cast<float *>(ws + L.partial);
+    __half *x16 = reinterpret_cast<__half *>(ws + L.x16);
+    int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(ws + L.topk_ids);
+    float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(ws + L.topk_w);
+    int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
+    int32_t *sorted_ids = reinterpret_cast<int32_t *>(ws + L.sorted_ids);
+    int32_t *inv_pos = reinterpret_cast<int32_t *>(ws + L.inv_pos);
+    ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
+    int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
+    __half *h = reinterpret_cast<__half *>(ws + L.h);
+    float *y = reinterpret_cast<float *>(ws + L.y);
+
+    MOE_MARK(marks, s);
+    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, M, H, E, L.route_splits, s));
+    MOE_MARK(marks, s);
+    MOE_TRY(launch_route_topk(partial, router_bias, ids, tw, M, E, k, L.route_splits, s));
+    MOE_MARK(marks, s);
+    MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, s));
+    MOE_MARK(marks, s);
+    int rc = run_gate_up(w13_q, w13_s, x16, sorted_ids, tiles, n_tiles, h, status, H, I, E, k, L.max_tiles, s);
+    if (rc != MOE_OK) return rc;
+    MOE_MARK(marks, s);
+    rc = run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, status, H, I, E, L.max_tiles, s);
+    if (rc != MOE_OK) return rc;
+    MOE_MARK(marks, s);
+    MOE_TRY(launch_combine(y, out, status, status_out, M, H, k, s));
+    MOE_MARK(marks, s);
+    return MOE_OK;
+}
+
+static int check_forward_args(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
+                              const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M,
+                              int H, int I, int E, int k, const int32_t *topk_ids_out, const float *topk_w_out,
+                              const int32_t *status_out)
+{
+    int rc = check_dims(M, H, I, E, k, true);
+    if (rc != MOE_OK) return rc;
+    if (!x || !router_w || !w13_q || !w13_s || !w2_q || !w2_s || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(w13_q, 16) || !aligned(w13_s, 16) ||
+        !aligned(w2_q, 16) || !aligned(w2_s, 16) || !aligned(out, 16))
+        return MOE_ERR_INVALID_ARG;
+    if ((router_bias && !aligned(router_bias, 4)) || (topk_ids_out && !aligned(topk_ids_out, 4)) ||
+        (topk_w_out && !aligned(topk_w_out, 4)) || (status_out && !aligned(status_out, 4)))
+        return MOE_ERR_INVALID_ARG;
+    const size_t xbytes = static_cast<size_t>(M) * H * 2;
+    if (M > 0 && overlaps(x, xbytes, out, xbytes)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_status_string(int status)
+{
+    switch (status) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    default: return "MOE_ERR_UNKNOWN";
+    }
+}
+
+int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t moe_workspace_bytes(int M, int H, int I, int E, int k)
+{
+    if (check_dims(M, H, I, E, k, true) != MOE_OK) return 0;
+    return make_layout(M, H, I, E, k).total;
+}
+
+int moe_route(const void *x_bf16, const float *router_w, const float *router_bias, int32_t *topk_ids, float *topk_w,
+              int M, int H, int E, int k, cudaStream_t stream)
+{
+    int rc = check_dims(M, H, 32, E, k, false);
+    if (rc != MOE_OK) return rc;
+    if (!x_bf16 || !router_w || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(router_w, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
+        (router_bias && !aligned(router_bias, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, 32, E, k);
+    char *ws = nullptr;
+    rc = library_workspace(stream, L.total, &ws);
+    if (rc != MOE_OK) return rc;
+    float *partial = reinterpret_cast<float *>(ws + L.partial);
+    MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, reinterpret_cast<int *>(ws + L.status), M, H, E,
+                                L.route_splits, stream));
+    MOE_TRY(launch_route_topk(partial, router_bias, topk_ids, topk_w, M, E, k, L.route_splits, stream));
+    return MOE_OK;
+}
+
+int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorted_ids, int32_t *inv_pos, int M, int E,
+                int k, cudaStream_t stream)
+{
+    int rc = check_dims(M, 32, 32, E, k, false);
+    if (rc != MOE_OK) return rc;
+    if (!topk_ids || !expert_offsets || !sorted_ids || !inv_pos) return MOE_ERR_INVALID_ARG;
+    if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (M == 0) return MOE_OK;
+    MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, nullptr, nullptr, M, E, k, stream));
+    return MOE_OK;
+}
+
+int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *w13_s, const int32_t *expert_offsets,
+                       const int32_t *sorted_ids, void *h_f16, int M, int H, int I, int E, int k, cudaStream_t stream)
+{
+    int rc = check_dims(M, H, I, E, k, true);
+    if (rc != MOE_OK) return rc;
+    if (!x_bf16 || !w13_q || !w13_s || !expert_offsets || !sorted_ids || !h_f16) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(w13_q, 16) || !aligned(w13_s, 16) || !aligned(h_f16, 16) ||
+        !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, I, E, k);
+    char *ws = nullptr;
+    rc = library_workspace(stream, L.total, &ws);
+    if (rc != MOE_OK) return rc;
+    int *status = reinterpret_cast<int *>(ws + L.status);
+    __half *x16 = reinterpret_cast<__half *>(ws + L.x16);
+    ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
+    int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
+    MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
+    MOE_TRY(launch_build_tiles(expert_offsets, tiles, n_tiles, nullptr, E, stream));
+    return run_gate_up(w13_q, w13_s, x16, sorted_ids, tiles, n_tiles, static_cast<__half *>(h_f16), status, H, I, E,
+                       k, L.max_tiles, stream);
+}
+
+int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
+                     const int32_t *expert_offsets, const int32_t *sorted_ids, void *out_bf16, int M, int H, int I,
+                     int E, int k, cudaStream_t stream)
+{
+    int rc = check_dims(M, H, I, E, k, true);
+    if (rc != MOE_OK) return rc;
+    if (!h_f16 || !w2_q || !w2_s || !topk_w || !expert_offsets || !sorted_ids || !out_bf16) return MOE_ERR_INVALID_ARG;
+    if (!aligned(h_f16, 16) || !aligned(w2_q, 16) || !aligned(w2_s, 16) || !aligned(out_bf16, 16) ||
+        !aligned(topk_w, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, I, E, k);
+    char *ws = nullptr;
+    rc = library_workspace(stream, L.total, &ws);
+    if (rc != MOE_OK) return rc;
+    int *status = reinterpret_cast<int *>(ws + L.status);
+    ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
+    int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
+    float *y = reinterpret_cast<float *>(ws + L.y);
+    MOE_TRY(launch_build_tiles(expert_offsets, tiles, n_tiles, status, E, stream));
+    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, status, H, I,
+                  E, L.max_tiles, stream);
+    if (rc != MOE_OK) return rc;
+    MOE_TRY(launch_combine(y, out_bf16, status, nullptr, M, H, k, stream));
+    return MOE_OK;
+}
+
+int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
+                         const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H,
+                         int I, int E, int k, int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    int rc = check_forward_args(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, topk_ids_out,
+                                topk_w_out, status_out);
+    if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, I, E, k);
+    if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    return forward_impl(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, topk_ids_out,
+                        topk_w_out, status_out, static_cast<char *>(workspace), L, stream);
+}
+
+int moe_mxfp4_forward_profile(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
+                              const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H,
+                              int I, int E, int k, int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream, float *kernel_ms)
+{
+    int rc = check_forward_args(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, topk_ids_out,
+                                topk_w_out, status_out);
+    if (rc != MOE_OK) return rc;
+    if (!kernel_ms) return MOE_ERR_INVALID_ARG;
+    for (int i = 0; i < MOE_PROFILE_KERNELS; ++i) kernel_ms[i] = 0.f;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, I, E, k);
+    if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    Marks marks;
+    int created = 0;
+    cudaError_t e = cudaSuccess;
+    for (; created <= MOE_PROFILE_KERNELS && e == cudaSuccess; ++created) e = cudaEventCreate(&marks.ev[created]);
+    if (e == cudaSuccess) {
+        rc = forward_impl(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, topk_ids_out,
+                          topk_w_out, status_out, static_cast<char *>(workspace), L, stream, &marks);
+        if (rc == MOE_OK) {
+            e = cudaEventSynchronize(marks.ev[MOE_PROFILE_KERNELS]);
+            for (int i = 0; i < MOE_PROFILE_KERNELS && e == cudaSuccess; ++i)
+                e = cudaEventElapsedTime(&kernel_ms[i], marks.ev[i], marks.ev[i + 1]);
+        }
+    } else {
+        --created;
+    }
+    for (int i = 0; i < created; ++i) cudaEventDestroy(marks.ev[i]);
+    if (rc != MOE_OK) return rc;
+    if (e != cudaSuccess) return cuda_fail(e);
+    return MOE_OK;
+}
+
+int moe_mxfp4_forward(const void *x, const float *router_w, const uint8_t *w13_q, const uint8_t *w13_s,
+                      const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H, int I, int E, int k,
+                      cudaStream_t stream)
+{
+    int rc = check_forward_args(x, router_w, nullptr, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, nullptr, nullptr,
+                                nullptr);
+    if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, I, E, k);
+    char *ws = nullptr;
+    rc = library_workspace(stream, L.total, &ws);
+    if (rc != MOE_OK) return rc;
+    return forward_impl(x, router_w, nullptr, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, nullptr, nullptr, nullptr,
+                        ws, L, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,370 @@
+// grouped_gemm.cu -- grouped MXFP4 expert GEMMs for small per-expert token counts.
+//
+// "Compact routed MXFP4 GEMM" (gate_up and down), "Routed MoE gather" and
+// "Routed clamp-SwiGLU" rows of "Post-Portfolio Device Attribution" ("MTP1
+// Post-Portfolio Eager-Cycle Profile"); the page's "Decision" section plans a
+// fused gate/up producer with a bf16-rounded exchange, and
+// "row/QUANT-CT-MXFP4-C8-DIFF" measures the unfused gate_up (more grouped GEMM
+// launches and CTAs per layer) as the dominant decode cost.  At decode token
+// counts these GEMMs stream each touched expert's weights once and are bound by
+// HBM bandwidth ("The Systematic Optimization Campaign", chunk 8.0).
+//
+// Design (one persistent CTA per SM, warp specialised):
+//  * Work item = (expert tile of <= 8 assignments, block of 32 weight rows).
+//    gate_up rows: 16 gate rows n0.. and the 16 matching up rows I+n0..;
+//    down rows: 32 consecutive rows r0.. of W2.  Items are spread round-robin
+//    over the CTAs; all tiles of one row block are adjacent, so CTAs that share
+//    weights run together and hit L2.
+//  * Producer warp: TMA 2-D tiled copies (16 rows x 128 B boxes, 128-byte
+//    swizzle) of packed E2M1 bytes through an 8-stage ring of 8 KB stages; in
+//    the same stage, one 1-D bulk copy per tile token of its binary16
+//    activation chunk (the routed gather: x rows for gate_up, h rows for down);
+//    and one pair of bulk copies of the item's E8M0 scale rows into a double
+//    buffer.
+//  * 8 consumer warps split each stage's 16 blocks of 32 K: a thread reads the
+//    32-bit word q of its rows' 16-byte block (conflict-free thanks to the
+//    swizzle), decodes it with the hardware E2M1 -> f16x2 conversion straight
+//    into MMA A-fragment registers, and runs two m16n8k16 f16 MMAs per block and
+//    token group.  Inside a block the K order is permuted (thread q's word covers
+//    K 8q..8q+7) identically for A and for the activation fragment, so each MMA
+//    pair spans exactly one scale block and the E8M0 scale is applied once to the
+//    fp32 partial sum.
+//  * gate_up m-tile = 8 gate rows (fragment rows 0-7) + the same 8 up rows
+//    (fragment rows 8-15): each thread holds g and u of one output row, so
+//    clamp-SwiGLU and the bf16 rounding run in registers.
+//  * The K split over warps is reduced through shared memory in warp order.
+// Activations (x or h) are read as binary16; bf16 x converts exactly for
+// 2^-17 <= |x| <= 65504, E2M1 values are exact in binary16, and products
+// accumulate in fp32.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kRedFloats = kConsumerWarps * 2 * 32 * 4;   // [warp][mt][lane][4]
+
+struct SmemPlan {
+    int wst_off, act_off, sbuf_off, sbuf_bytes, red_off, bars_off, total;
+};
+
+__host__ __device__ inline SmemPlan smem_plan(int K)
+{
+    SmemPlan p;
+    p.wst_off = 0;
+    p.act_off = kStages * kStageBytes;
+    p.sbuf_off = p.act_off + kStages * kActStageBytes;
+    p.sbuf_bytes = ((kRowsPerItem * (K / 32)) + 127) / 128 * 128;
+    p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
+    p.bars_off = p.red_off + kRedFloats * 4;
+    p.total = p.bars_off + (2 * kStages + 4) * 8 + 1024;   // + alignment slack
+    return p;
+}
+
+__device__ __forceinline__ float clamp_swiglu(float g, float u)
+{
+    const float a = fminf(g, 7.0f);
+    const float c = fminf(fmaxf(u, -7.0f), 7.0f);
+    return a / (1.0f + expf(-a)) * c;
+}
+
+__device__ __forceinline__ __half round_h(float v)
+{
+    // bf16 round-to-nearest-even, then the exact move into binary16
+    return __float2half_rn(__bfloat162float(__float2bfloat16_rn(v)));
+}
+
+template <bool kGateUp>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ wscale,
+                     const __half *__restrict__ act, const int32_t *__restrict__ sorted_ids,
+                     const float *__restrict__ topk_w, const ExpertTile *__restrict__ tiles,
+                     const int *__restrict__ n_tiles_ptr, __half *__restrict__ hout, float *__restrict__ yout,
+                     int *status, int K, int I, int H, int ktop)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    const SmemPlan plan = smem_plan(K);
+    uint8_t *wst = smem + plan.wst_off;
+    uint8_t *ast = smem + plan.act_off;
+    uint8_t *sbuf = smem + plan.sbuf_off;
+    float *red = reinterpret_cast<float *>(smem + plan.red_off);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bars_off);
+    uint64_t *full = bars, *empty = bars + kStages, *sfull = bars + 2 * kStages, *sempty = sfull + 2;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = *n_tiles_ptr;
+    const int row_blocks = kGateUp ? I / 16 : H / 32;
+    const int n_items = n_tiles * row_blocks;
+    const int kblocks = K / 32;               // scale bytes per row
+    const int n_chunks = (K + kChunkK - 1) / kChunkK;
+    const int kbytes = K / 2;                 // packed bytes per row
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sfull[b], 1);
+            mbar_init(&sempty[b], kConsumerWarps);
+        }
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    bool aborted = false;
+
+    if (warp == kConsumerWarps) {
+        // ---------------------------------------------------------------- producer warp
+        // lane 0: scale rows and weight boxes; lane i < count: token i's activation chunk
+        if (lane == 0) prefetch_tensormap(&wmap);
+        int stage_ctr = 0, item_ctr = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
+            const ExpertTile tl = tiles[item % n_tiles];
+            const int rb = item / n_tiles;
+            const int e = tl.expert;
+            int row_a, row_b;   // first global rows of the two 16-row halves
+            if (kGateUp) {
+                row_a = e * 2 * I + rb * 16;
+                row_b = row_a + I;
+            } else {
+                row_a = e * H + rb * 32;
+                row_b = row_a + 16;
+            }
+            // this lane's activation row (gate_up: the token's x row; down: the h row)
+            const int li = min(lane, tl.count - 1);
+            const __half *arow = kGateUp ? act + static_cast<size_t>(sorted_ids[tl.p0 + li] / ktop) * K
+                                         : act + static_cast<size_t>(tl.p0 + li) * K;
+            const int b = item_ctr & 1;
+            mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
+            aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
+            if (lane == 0 && !aborted) {
+                uint8_t *dst = sbuf + b * plan.sbuf_bytes;
+                const uint32_t half_bytes = 16u * kblocks;
+                mbar_arrive_expect_tx(&sfull[b], 2u * half_bytes);
+                bulk_load(dst, wscale + static_cast<size_t>(row_a) * kblocks, half_bytes, &sfull[b]);
+                bulk_load(dst + half_bytes, wscale + static_cast<size_t>(row_b) * kblocks, half_bytes, &sfull[b]);
+            }
+            for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
+                const int s = stage_ctr % kStages;
+                mbar_wait(&empty[s], ((stage_ctr / kStages) & 1) ^ 1, aborted, status);
+                aborted = __any_sync(0xffffffffu, aborted);
+                const int kb = c * (kChunkK / 2);
+                const int kc = c * kChunkK;
+                const uint32_t act_bytes = 2u * static_cast<uint32_t>(min(kChunkK, K - kc));
+                const int nbox_half = (kb + 128 < kbytes) ? 2 : 1;   // skip a box wholly past K
+                if (lane == 0 && !aborted)
+                    mbar_arrive_expect_tx(&full[s], 2u * nbox_half * kBoxBytes + tl.count * act_bytes);
+                __syncwarp();
+                if (aborted) continue;
+                if (lane == 0) {
+                    uint8_t *st = wst + s * kStageBytes;
+                    // boxes: 0 = half a lo, 1 = half a hi, 2 = half b lo, 3 = half b hi
+                    tma_load_2d(st + 0 * kBoxBytes, &wmap, kb, row_a, &full[s]);
+                    tma_load_2d(st + 2 * kBoxBytes, &wmap, kb, row_b, &full[s]);
+                    if (nbox_half == 2) {
+                        tma_load_2d(st + 1 * kBoxBytes, &wmap, kb + 128, row_a, &full[s]);
+                        tma_load_2d(st + 3 * kBoxBytes, &wmap, kb + 128, row_b, &full[s]);
+                    }
+                }
+                if (lane < tl.count)
+                    bulk_load(ast + s * kActStageBytes + lane * kActPitch, arow + kc, act_bytes, &full[s]);
+            }
+        }
+        // let every copy this CTA issued land before the CTA can exit
+        for (int i = 0; i < kStages && i < stage_ctr; ++i) {
+            const int sc = stage_ctr - 1 - i;
+            mbar_wait(&full[sc % kStages], (sc / kStages) & 1, aborted, status);
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumer warps
+    const int g = lane >> 2, q = lane & 3;
+    const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+    int stage_ctr = 0, item_ctr = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
+        const ExpertTile tl = tiles[item % n_tiles];
+        const int rb = item / n_tiles;
+        const int cnt = tl.count;
+        const int b = item_ctr & 1;
+        const uint8_t *sb = sbuf + b * plan.sbuf_bytes;
+        mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
+
+        float acc[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[mt][r] = 0.f;
+
+        for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
+            const int s = stage_ctr % kStages;
+            const int kc = c * kChunkK;
+            mbar_wait(&full[s], (stage_ctr / kStages) & 1, aborted, status);
+            const uint8_t *st = wst + s * kStageBytes;
+            const uint8_t *xa = ast + s * kActStageBytes + g * kActPitch;   // token g of the tile
+#pragma unroll
+            for (int bi = 0; bi < 2; ++bi) {
+                const int blk = 2 * warp + bi;    // block of 32 K inside the stage
+                const int kg = kc + 32 * blk;
+                if (kg >= K) continue;
+                const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * blk + 8 * q) * 2);
+                const int half = blk >> 3, bb = blk & 7;
+                const int sw = ((bb ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    int top_box, top_row, bot_box, bot_row, top_s, bot_s;
+                    if (kGateUp) {
+                        top_box = half;          top_row = 8 * mt + g;
+                        bot_box = 2 + half;      bot_row = 8 * mt + g;
+                        top_s = 8 * mt + g;      bot_s = 16 + 8 * mt + g;
+                    } else {
+                        top_box = 2 * mt + half; top_row = g;
+                        bot_box = 2 * mt + half; bot_row = 8 + g;
+                        top_s = 16 * mt + g;     bot_s = 16 * mt + 8 + g;
+                    }
+                    const uint32_t wt = *reinterpret_cast<const uint32_t *>(st + top_box * kBoxBytes + top_row * 128 + sw);
+                    const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_box * kBoxBytes + bot_row * 128 + sw);
+                    const float st_scale = e8m0_times2(sb[top_s * kblocks + (kg >> 5)]);
+                    const float sb_scale = e8m0_times2(sb[bot_s * kblocks + (kg >> 5)]);
+                    uint32_t t0, t1, t2, t3, u0, u1, u2, u3;
+                    e2m1x8_to_f16x2(wt, t0, t1, t2, t3);
+                    e2m1x8_to_f16x2(wb, u0, u1, u2, u3);
+                    const uint32_t a0[4] = {t0, u0, t1, u1};
+                    const uint32_t a1[4] = {t2, u2, t3, u3};
+                    float tmp[4];
+                    mma_f16_16816(tmp, a0, xb.x, xb.y, zero4);
+                    mma_f16_16816(tmp, a1, xb.z, xb.w, tmp);
+                    acc[mt][0] = fmaf(tmp[0], st_scale, acc[mt][0]);
+                    acc[mt][1] = fmaf(tmp[1], st_scale, acc[mt][1]);
+                    acc[mt][2] = fmaf(tmp[2], sb_scale, acc[mt][2]);
+                    acc[mt][3] = fmaf(tmp[3], sb_scale, acc[mt][3]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[b]);
+
+        // ---------------------------------------------------------------- cross-warp reduction
+        named_bar_sync(1, kConsumerWarps * 32);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+            *reinterpret_cast<float4 *>(red + ((warp * 2 + mt) * 32 + lane) * 4) =
+                make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]);
+        named_bar_sync(1, kConsumerWarps * 32);
+        if (warp < 2) {
+            const int mt = warp;
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float4 v = *reinterpret_cast<const float4 *>(red + ((w * 2 + mt) * 32 + lane) * 4);
+                sum.x += v.x;
+                sum.y += v.y;
+                sum.z += v.z;
+                sum.w += v.w;
+            }
+            // remove the factor 2 carried by e8m0_times2
+            sum.x *= 0.5f;
+            sum.y *= 0.5f;
+            sum.z *= 0.5f;
+            sum.w *= 0.5f;
+            const int li0 = 2 * q, li1 = li0 + 1;
+            if (kGateUp) {
+                const int n = rb * 16 + 8 * mt + g;
+                if (li0 < cnt) hout[static_cast<size_t>(tl.p0 + li0) * I + n] = round_h(clamp_swiglu(sum.x, sum.z));
+                if (li1 < cnt) hout[static_cast<size_t>(tl.p0 + li1) * I + n] = round_h(clamp_swiglu(sum.y, sum.w));
+            } else {
+                const int ra = rb * 32 + 16 * mt + g, rbw = ra + 8;
+                if (li0 < cnt) {
+                    const int f = sorted_ids[tl.p0 + li0];
+                    const float w = topk_w[f];
+                    yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
+                    yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
+                }
+                if (li1 < cnt) {
+                    const int f = sorted_ids[tl.p0 + li1];
+                    const float w = topk_w[f];
+                    yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
+                    yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
+                }
+            }
+        }
+    }
+}
+
+// out[t] = bf16( sum_j y[t*k + j] ), j ascending; y already carries the routing weight.
+__global__ void combine_kernel(const float *__restrict__ y, __nv_bfloat16 *__restrict__ out, const int *status,
+                               int32_t *status_out, int M, int H, int k)
+{
+    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx == 0 && status_out) *status_out = *status;
+    const int per_row = H / 8;
+    if (idx >= static_cast<size_t>(M) * per_row) return;
+    const int t = static_cast<int>(idx / per_row);
+    const int c = static_cast<int>(idx - static_cast<size_t>(t) * per_row) * 8;
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+        const float4 *p = reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H + c);
+        const float4 u = p[0], v = p[1];
+        a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
+        a[4] += v.x; a[5] += v.y; a[6] += v.z; a[7] += v.w;
+    }
+    __nv_bfloat162 o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint4 *>(o);
+}
+
+template <bool kGateUp>
+static cudaError_t launch_grouped(const CUtensorMap &map, const uint8_t *scales, const __half *act,
+                                  const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
+                                  const int *n_tiles, __half *h, float *y, int *status, int K, int I, int H, int ktop,
+                                  int max_tiles, cudaStream_t s)
+{
+    const SmemPlan plan = smem_plan(K);
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
+    if (e != cudaSuccess) return e;
+    const long long row_blocks = kGateUp ? I / 16 : H / 32;
+    const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
+    const int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
+    grouped_mxfp4_kernel<kGateUp><<<grid > 0 ? grid : 1, kThreads, plan.total, s>>>(
+        map, scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, K, I, H, ktop);
+    return cudaGetLastError();
+}
+
+int grouped_smem_bytes(int K) { return smem_plan(K).total; }
+
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const uint8_t *w13_s, const __half *x16,
+                           const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, __half *h,
+                           int *status, int H, int I, int k, int max_tiles, cudaStream_t s)
+{
+    return launch_grouped<true>(w13_map, w13_s, x16, sorted_ids, nullptr, tiles, n_tiles, h, nullptr, status, H, I,
+                                H, k, max_tiles, s);
+}
+
+cudaError_t launch_down(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+                        const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+                        int H, int I, int max_tiles, cudaStream_t s)
+{
+    return launch_grouped<false>(w2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, status, I, I, H, 1,
+                                 max_tiles, s);
+}
+
+cudaError_t launch_combine(const float *y, void *out, const int *status, int32_t *status_out, int M, int H, int k,
+                           cudaStream_t s)
+{
+    const size_t n = static_cast<size_t>(M) * H / 8;
+    const int threads = 256;
+    const unsigned blocks = static_cast<unsigned>((n + threads - 1) / threads);
+    combine_kernel<<<blocks > 0 ? blocks : 1, threads, 0, s>>>(y, static_cast<__nv_bfloat16 *>(out), status,
+                                                               status_out, M, H, k);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

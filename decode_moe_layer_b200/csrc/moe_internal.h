@@ -1,0 +1,76 @@
+// moe_internal.h -- declarations shared by the library's translation units
+// (constants, workspace layout, kernel launchers).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = -5;
+
+// Grouped GEMM tiling (both projections).
+constexpr int kTileTokens = 8;       // assignments per expert tile (one MMA n-tile)
+constexpr int kRowsPerItem = 32;     // weight rows per work item (2 MMA m-tiles of 16)
+constexpr int kChunkK = 512;         // K elements per pipeline stage
+constexpr int kBoxRows = 16;         // TMA box: 16 rows x 128 bytes (256 K elements)
+constexpr int kBoxBytes = 16 * 128;
+constexpr int kStageBytes = 4 * kBoxBytes;          // packed weights of one stage
+constexpr int kActPitch = kChunkK * 2 + 64;         // one token's binary16 chunk, padded against bank conflicts
+constexpr int kActStageBytes = kTileTokens * kActPitch;
+constexpr int kStages = 8;
+constexpr int kConsumerWarps = 8;
+
+// Router.
+constexpr int kRouteChunkH = 1024;   // H elements per partial-logit chunk
+constexpr int kRouteTokens = 32;     // tokens per router CTA
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 32;
+constexpr int kMaxAssignments = 16384;
+
+struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignments
+    int expert;
+    int p0;           // first position in the expert-grouped order
+    int count;
+    int pad;
+};
+
+// Byte offsets of every buffer inside one call's workspace (256-byte aligned).
+struct Layout {
+    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, total;
+    int route_splits;   // number of H chunks of the router
+    int max_tiles;
+};
+
+Layout make_layout(int M, int H, int I, int E, int k);
+
+// Kernel launchers (return cudaError_t of the launch).
+cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
+                                int M, int H, int E, int splits, cudaStream_t s);
+cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E,
+                              int k, int splits, cudaStream_t s);
+cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos,
+                           ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s);
+cudaError_t launch_build_tiles(const int32_t *offsets, ExpertTile *tiles, int *n_tiles, int *status, int E,
+                               cudaStream_t s);
+cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const uint8_t *w13_s, const __half *x16,
+                           const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, __half *h,
+                           int *status, int H, int I, int k, int max_tiles, cudaStream_t s);
+cudaError_t launch_down(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+                        const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+                        int H, int I, int max_tiles, cudaStream_t s);
+cudaError_t launch_combine(const float *y, void *out, const int *status, int32_t *status_out, int M, int H, int k,
+                           cudaStream_t s);
+
+int num_sms();
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_max_smem(const void *kernel, int bytes);
+
+}  // namespace moe

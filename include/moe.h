@@ -1,0 +1,185 @@
+/*
+ * moe.h -- C ABI of libmoe.so: one routed MXFP4 Mixture-of-Experts layer call
+ * for LLM decode on NVIDIA B200 (sm_100a).
+ *
+ * The layer (the kernel family that "MTP1 Post-Portfolio Eager-Cycle Profile",
+ * table "Post-Portfolio Device Attribution", lists as native router
+ * select/normalize, direct route remap, routed MoE gather, compact routed MXFP4
+ * GEMM and routed clamp-SwiGLU; the grouped MoE GEMM structure that
+ * "row/QUANT-CT-MXFP4-C8-DIFF" (vllm.cpp PR #52) traces at c8 decode):
+ *
+ *   logits = x W_r^T (+ b)              fp32, one per expert            moe_route
+ *   ids    = top-k(softmax(logits))     descending, ties -> lower id    moe_route
+ *   w      = renormalised top-k probs   sum to 1 per token              moe_route
+ *   order  = expert-grouped assignments stable in flat id t*k+j         moe_permute
+ *   h      = bf16(silu(min(g,7)) * clamp(u,-7,7)),
+ *            g,u = gate/up rows of expert ids[t,j] applied to x[t]    moe_gate_up_swiglu
+ *   out[t] = bf16( sum_j w[t,j] * (W2_{ids[t,j]} h[t,j]) )            moe_down_combine
+ *
+ * Data formats (all tensors row-major, contiguous, in caller-owned DEVICE memory):
+ *   x, out            bf16 [M, H]
+ *   router_w          fp32 [E, H];   router_bias fp32 [E] (nullable)
+ *   w13_q             uint8 [E, 2I, H/2]  packed FP4 E2M1 (OCP MX v1.0), low nibble = even K
+ *                                         rows 0..I-1 are gate, rows I..2I-1 are up
+ *   w13_s             uint8 [E, 2I, H/32] E8M0 scale per 32 consecutive K of a row
+ *   w2_q              uint8 [E, H, I/2];  w2_s uint8 [E, H, I/32]
+ *   weight value      E2M1(code) * 2^(scale - 127)
+ *   topk_ids / topk_w int32 / fp32 [M, k], slot j in descending router probability
+ *   expert_offsets    int32 [E+1];  sorted_ids, inv_pos int32 [M*k]
+ *   h                 binary16 [M*k, I] in expert-grouped order (row p holds the
+ *                     assignment sorted_ids[p]); every element is a bf16-rounded
+ *                     value, exact in binary16 for |h| >= 2^-17 (|h| <= 49 always)
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device pointers the caller owns; the library keeps none after
+ *     returning.  Bulk tensors (x, out, router_w, w13_*, w2_*, h) must be 16-byte
+ *     aligned; int32/fp32 index and weight arrays 4-byte aligned.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).  They
+ *     never synchronise the host, and allocate nothing while `stream` is being
+ *     captured into a CUDA graph.
+ *   - Arguments are validated before anything is enqueued; a call that returns an
+ *     error status has enqueued nothing.  M == 0 returns MOE_OK and enqueues nothing.
+ *   - Supported shapes: H % 32 == 0, I % 32 == 0, H,I >= 32, 1 <= k <= min(E, 32),
+ *     E <= 1024, M*k <= 16384.  Others return MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - Out of contract (undefined output, no fault): NaN/Inf or |x| > 65504 in x,
+ *     E8M0 scale bytes 254 and 255.
+ *   - Determinism: for a given device and inputs, every output is bitwise
+ *     reproducible (no floating-point atomics; fixed reduction orders).
+ *
+ * Workspace: the forms without a workspace argument use a library-owned device
+ * buffer per (device, stream).  It grows with cudaMalloc on first use and never
+ * while the stream is capturing; a capture that needs a larger one fails with
+ * MOE_ERR_WORKSPACE (warm up once outside capture).  Two calls on the same stream
+ * share it safely (stream order); calls on different streams get different
+ * buffers.  moe_mxfp4_forward_ex takes the caller's buffer instead.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *cudaStream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = -1,        /* null/misaligned pointer, negative size, aliasing */
+    MOE_ERR_UNSUPPORTED_SHAPE = -2,  /* shape outside the supported set above */
+    MOE_ERR_WORKSPACE = -3,          /* workspace too small (or growth refused during capture) */
+    MOE_ERR_CUDA = -4,               /* a CUDA runtime/driver call or launch failed */
+    MOE_ERR_TIMEOUT = -5             /* a bounded device-side wait gave up (reported via status_out) */
+} moe_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *moe_status_string(int status);
+
+/* Last CUDA error code seen by the library on this host thread (0 if none). */
+int moe_last_cuda_error(void);
+
+/*
+ * Router select/normalize.  Defined by the "Native router select/normalize" row
+ * of "Post-Portfolio Device Attribution" ("MTP1 Post-Portfolio Eager-Cycle
+ * Profile"): per token, fp32 logits x.W_r^T (+ router_bias), softmax over the E
+ * experts, the k largest in descending order (ties -> lower expert id), and their
+ * probabilities renormalised to sum to 1 (equal to a softmax over the k selected
+ * logits).  Writes topk_ids [M,k] int32 and topk_w [M,k] fp32.
+ * Uses the library-owned workspace of `stream` for per-chunk partial logits.
+ */
+int moe_route(const void *x_bf16, const float *router_w, const float *router_bias,
+              int32_t *topk_ids, float *topk_w, int M, int H, int E, int k, cudaStream_t stream);
+
+/*
+ * Route remap: expert-grouped order of the M*k assignments.  Defined by the
+ * "Direct M=2 route remap" row of the same table (route-direct compact routes):
+ * a histogram of topk_ids, its exclusive prefix sum expert_offsets [E+1], and a
+ * stable scatter of the flat ids f = t*k + j into sorted_ids [M*k] (ascending f
+ * within an expert); inv_pos[f] is the position of f in sorted_ids.
+ * topk_ids values must lie in [0, E).  No workspace.
+ */
+int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorted_ids,
+                int32_t *inv_pos, int M, int E, int k, cudaStream_t stream);
+
+/*
+ * Grouped MXFP4 gate_up GEMM with the routed gather and clamp-SwiGLU fused in.
+ * Defined by the "Compact routed MXFP4 GEMM", "Routed MoE gather" and "Routed
+ * clamp-SwiGLU" rows of the same table, with the gate and up producers fused and
+ * the intermediate rounded to bf16 (the "Decision" section of the same page).
+ * For each position p of the expert-grouped order, f = sorted_ids[p], t = f / k,
+ * e = the expert whose offsets range holds p:
+ *   g = W_gate,e x[t], u = W_up,e x[t] (bf16 products, fp32 accumulation),
+ *   h[p] = bf16_rne(silu(min(g,7)) * clamp(u,-7,7)), stored as binary16.
+ * expert_offsets/sorted_ids are moe_permute's outputs.  Uses the library-owned
+ * workspace of `stream`.
+ */
+int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *w13_s,
+                       const int32_t *expert_offsets, const int32_t *sorted_ids, void *h_f16,
+                       int M, int H, int I, int E, int k, cudaStream_t stream);
+
+/*
+ * Down GEMM with the weighted top-k combine fused behind it.  Defined by the
+ * down half of the "Compact routed MXFP4 GEMM" row of the same table:
+ *   y[f] = W2_e h[inv position of f] (fp32 accumulation),
+ *   out[t] = bf16_rne( sum_{j=0..k-1} topk_w[t,j] * y[t*k+j] ), summed in slot
+ *   order j with no atomics.
+ * Uses the library-owned workspace of `stream` for the fp32 per-assignment rows.
+ */
+int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
+                     const int32_t *expert_offsets, const int32_t *sorted_ids, void *out_bf16,
+                     int M, int H, int I, int E, int k, cudaStream_t stream);
+
+/*
+ * Whole layer: moe_route -> moe_permute -> moe_gate_up_swiglu -> moe_down_combine,
+ * enqueued back to back on `stream` with the library-owned workspace and no router
+ * bias.  `out` must not overlap `x`.
+ */
+int moe_mxfp4_forward(const void *x, const float *router_w, const uint8_t *w13_q, const uint8_t *w13_s,
+                      const uint8_t *w2_q, const uint8_t *w2_s, void *out,
+                      int M, int H, int I, int E, int k, cudaStream_t stream);
+
+/* Bytes of device workspace moe_mxfp4_forward_ex needs for this shape (0 if unsupported). */
+size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
+
+/*
+ * Whole layer with a caller-owned workspace (>= moe_workspace_bytes, 256-byte
+ * aligned; its contents need no initialisation and are overwritten), an optional
+ * router bias, optional copies of the routing (topk_ids_out [M,k] int32,
+ * topk_w_out [M,k] fp32) and an optional device int32 `status_out` that receives
+ * MOE_OK or MOE_ERR_TIMEOUT once the enqueued work has run.
+ * A workspace smaller than required returns MOE_ERR_WORKSPACE.
+ */
+int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *router_bias,
+                         const uint8_t *w13_q, const uint8_t *w13_s, const uint8_t *w2_q,
+                         const uint8_t *w2_s, void *out, int M, int H, int I, int E, int k,
+                         int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Number of kernels one layer call launches (the entries of moe_mxfp4_forward_profile's output). */
+#define MOE_PROFILE_KERNELS 6
+
+/*
+ * Per-kernel device-time attribution of one layer call, in the manner of the
+ * per-kernel buckets of "Post-Portfolio Device Attribution" ("MTP1 Post-Portfolio
+ * Eager-Cycle Profile").  Same arguments and results as moe_mxfp4_forward_ex;
+ * additionally records a CUDA event before and after each of the
+ * MOE_PROFILE_KERNELS launches (router logits, router top-k, route remap,
+ * gate_up + clamp-SwiGLU, down, weighted combine), WAITS for the stream to finish
+ * (host synchronisation: not for use under stream capture) and writes each
+ * kernel's event-to-event time in milliseconds into the HOST array kernel_ms.
+ */
+int moe_mxfp4_forward_profile(const void *x, const float *router_w, const float *router_bias,
+                              const uint8_t *w13_q, const uint8_t *w13_s, const uint8_t *w2_q,
+                              const uint8_t *w2_s, void *out, int M, int H, int I, int E, int k,
+                              int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                              float *kernel_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,92 @@
+"""Shared helpers for the GPU parity tests: device upload of the seeded inputs,
+calls into the oracle for the same inputs, and the tolerance checks.
+
+Tolerances (derivations in the design notes):
+  * routing ids, expert offsets, sorted ids, inverse positions: bit-exact;
+  * routing weights: |w - w_oracle| <= 1e-5 (fp32 logits and softmax vs fp64);
+  * h: each element equal to the oracle's bf16 value or one bf16 ulp away
+    (fp32 vs fp64 accumulation may flip a rounding), flips counted;
+  * out: relative L2 error <= 5e-3 and max abs error <= 2e-2 * rms, both against
+    the oracle's fp64 out64.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from moe_inputs import generator as gen
+
+W_TOL = 1e-5
+REL_L2_TOL = 5e-3
+MAX_ABS_RMS_TOL = 2e-2
+
+
+def bits_to_bf16_tensor(bits: np.ndarray, device="cuda") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def bf16_tensor_to_f64(t: torch.Tensor) -> np.ndarray:
+    return gen.bf16_bits_to_f64(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def device_inputs(inp: gen.MoEInputs, device="cuda"):
+    def dev(a):
+        if isinstance(a, torch.Tensor):
+            return a.to(device).contiguous()
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    d = {
+        "x": bits_to_bf16_tensor(inp.x, device),
+        "router_w": torch.from_numpy(inp.router_w).to(device),
+        "router_bias": None if inp.router_bias is None else torch.from_numpy(inp.router_bias).to(device),
+        "w13_q": dev(inp.w13_q), "w13_s": dev(inp.w13_s), "w2_q": dev(inp.w2_q), "w2_s": dev(inp.w2_s),
+    }
+    return d
+
+
+def oracle_forward(inp: gen.MoEInputs, tokens=None):
+    """Oracle layer output for `tokens` (all when None), regenerating only the experts they touch."""
+    k = inp.shape.k
+    if isinstance(inp.w13_q, np.ndarray):
+        return oracle.forward(inp.x, inp.router_w, inp.router_bias, inp.w13_q, inp.w13_s, inp.w2_q, inp.w2_s, k,
+                              tokens=tokens, I=inp.shape.I)
+    ids, _, _ = oracle.route(inp.x, inp.router_w, inp.router_bias, k)
+    toks = range(inp.M) if tokens is None else tokens
+    need = sorted(set(int(e) for t in toks for e in ids[t]))
+    ex = {e: inp.expert_weights(e) for e in need}
+    return oracle.forward(inp.x, inp.router_w, inp.router_bias,
+                          {e: v[0] for e, v in ex.items()}, {e: v[1] for e, v in ex.items()},
+                          {e: v[2] for e, v in ex.items()}, {e: v[3] for e, v in ex.items()},
+                          k, tokens=tokens, I=inp.shape.I)
+
+
+def check_out(gpu_out: np.ndarray, ref64: np.ndarray, what=""):
+    """gpu_out: float64 values of the bf16 output rows; ref64: the oracle's fp64 rows."""
+    err = gpu_out - ref64
+    rms = float(np.sqrt(np.mean(ref64 ** 2)))
+    rel_l2 = float(np.linalg.norm(err) / max(np.linalg.norm(ref64), 1e-300))
+    max_abs = float(np.abs(err).max())
+    assert np.all(np.isfinite(gpu_out)), what + ": non-finite output"
+    assert rel_l2 <= REL_L2_TOL, "%s: rel L2 %.3e > %.1e" % (what, rel_l2, REL_L2_TOL)
+    assert max_abs <= MAX_ABS_RMS_TOL * rms, "%s: max abs %.3e > %.1e * rms %.3e" % (what, max_abs,
+                                                                                    MAX_ABS_RMS_TOL, rms)
+    return rel_l2, max_abs / rms
+
+
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    a = np.maximum(np.abs(v), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def check_h(gpu_h: np.ndarray, ref_bits: np.ndarray, what="", max_flip_frac=0.01):
+    """gpu_h: float64 values (binary16-stored bf16 values); ref_bits: oracle bf16 bit patterns."""
+    ref = gen.bf16_bits_to_f64(ref_bits)
+    diff = np.abs(gpu_h - ref)
+    tol = np.maximum(bf16_ulp(np.maximum(np.abs(gpu_h), np.abs(ref))), 2.0 ** -24)
+    bad = diff > tol
+    assert not bad.any(), "%s: %d elements differ by more than one bf16 ulp (worst %.3e)" % (
+        what, int(bad.sum()), float(diff.max()))
+    flips = int((diff > 0).sum())
+    assert flips <= max_flip_frac * diff.size + 1, "%s: %d of %d elements flipped" % (what, flips, diff.size)
+    return flips

@@ -1,0 +1,201 @@
+"""GPU parity of every step of the layer against the fp64 oracle, through the C ABI.
+
+Small workloads are compared element by element on every output; the full-size
+DeepSeek-class workloads (6 GB of MXFP4 weights) are compared on the complete
+routing and permutation and on sampled tokens' outputs, with the weights
+generated on the device from the same counter streams the oracle regenerates on
+the host.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_inputs import generator as gen
+from tests import _gpu_util as U
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import decode_moe_layer_b200 as m
+    return m
+
+
+def _gpu_route(moe, d, k):
+    ids, w = moe.moe_route(d["x"], d["router_w"], k, router_bias=d["router_bias"])
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- router + permutation
+
+ROUTE_CASES = [(0, 2), (1, 1), (1, 8), (2, 1), (2, 32), (3, 512), (4, 1024), (1, 37)]
+
+
+@pytest.mark.parametrize("ci,M", ROUTE_CASES)
+def test_route_and_permute_bit_exact(moe, ci, M):
+    inp = gen.make_inputs(ci, M, weights="none")
+    k, E = inp.shape.k, inp.shape.E
+    d = {"x": U.bits_to_bf16_tensor(inp.x), "router_w": torch.from_numpy(inp.router_w).cuda(),
+         "router_bias": None if inp.router_bias is None else torch.from_numpy(inp.router_bias).cuda()}
+    ids, w = _gpu_route(moe, d, k)
+    rids, rw, _ = oracle.route(inp.x, inp.router_w, inp.router_bias, k)
+    assert np.array_equal(ids, rids)
+    assert np.abs(w - rw).max() <= U.W_TOL
+    off, srt, inv = moe.moe_permute(torch.from_numpy(ids).cuda(), E)
+    roff, rsrt, rinv = oracle.permute(rids, E)
+    assert np.array_equal(off.cpu().numpy(), roff)
+    assert np.array_equal(srt.cpu().numpy(), rsrt)
+    assert np.array_equal(inv.cpu().numpy(), rinv)
+
+
+def test_route_ties_and_all_experts(moe):
+    # all-zero x: every logit ties -> experts 0..k-1 with weight 1/k
+    x = torch.zeros((5, 256), dtype=torch.bfloat16, device="cuda")
+    wr = torch.randn((16, 256), device="cuda")
+    ids, w = moe.moe_route(x, wr, 4)
+    assert ids.cpu().tolist() == [[0, 1, 2, 3]] * 5
+    assert torch.allclose(w.cpu(), torch.full((5, 4), 0.25), atol=0, rtol=0)
+    # k == E: every expert selected, weights are the plain softmax
+    inp = gen.make_inputs(0, 2, weights="none")
+    E = inp.shape.E
+    ids, w = moe.moe_route(U.bits_to_bf16_tensor(inp.x), torch.from_numpy(inp.router_w).cuda(), E)
+    rids, rw, _ = oracle.route(inp.x, inp.router_w, None, E)
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    assert np.abs(w.cpu().numpy() - rw).max() <= U.W_TOL
+
+
+def test_permute_edge_cases(moe):
+    E = 64
+    rng = np.random.default_rng(0)
+    for M, k in [(1, 1), (1, 8), (3, 5), (2048, 8), (513, 32)]:
+        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(M)]).astype(np.int32)
+        if M == 2048:
+            ids[:] = np.arange(k)        # every assignment on the first k experts
+        off, srt, inv = moe.moe_permute(torch.from_numpy(ids).cuda(), E)
+        roff, rsrt, rinv = oracle.permute(ids, E)
+        assert np.array_equal(off.cpu().numpy(), roff), (M, k)
+        assert np.array_equal(srt.cpu().numpy(), rsrt), (M, k)
+        assert np.array_equal(inv.cpu().numpy(), rinv), (M, k)
+
+
+# ----------------------------------------------------------------------------- gate_up + clamp-SwiGLU
+
+@pytest.mark.parametrize("ci,M", [(0, 2), (1, 8), (1, 37), (2, 1), (2, 16)])
+def test_gate_up_swiglu(moe, ci, M):
+    big = ci >= 2
+    inp = gen.make_inputs(ci, M, weights="torch" if big else "numpy", device="cuda")
+    k, E = inp.shape.k, inp.shape.E
+    d = U.device_inputs(inp)
+    rids, rw, _ = oracle.route(inp.x, inp.router_w, inp.router_bias, k)
+    roff, rsrt, rinv = oracle.permute(rids, E)
+    h = moe.moe_gate_up_swiglu(d["x"], d["w13_q"], d["w13_s"], torch.from_numpy(roff).cuda(),
+                               torch.from_numpy(rsrt).cuda(), k)
+    torch.cuda.synchronize()
+    h_flat = h.float().cpu().numpy().astype(np.float64)[rinv]      # back to flat order t*k+j
+    toks = list(range(M)) if not big else [0, M - 1]
+    for t in toks:
+        for j in range(k):
+            e = int(rids[t, j])
+            q13, s13 = (inp.w13_q[e], inp.w13_s[e]) if not big else inp.expert_weights(e)[:2]
+            _, _, hb = oracle.expert_swiglu(inp.x[t], q13, s13)
+            U.check_h(h_flat[t * k + j], hb, "h[t=%d,j=%d]" % (t, j), max_flip_frac=0.02)
+
+
+# ----------------------------------------------------------------------------- down + combine
+
+@pytest.mark.parametrize("ci,M", [(0, 2), (1, 8), (1, 37)])
+def test_down_combine(moe, ci, M):
+    inp = gen.make_inputs(ci, M)
+    k, E = inp.shape.k, inp.shape.E
+    d = U.device_inputs(inp)
+    r = U.oracle_forward(inp)
+    rids, rw = r["topk_ids"], r["topk_w"]
+    roff, rsrt, rinv = oracle.permute(rids, E)
+    h_bits = r["h"][rsrt]                                         # oracle h in expert-grouped order
+    h16 = torch.from_numpy(gen.bf16_bits_to_f64(h_bits).astype(np.float16)).cuda()
+    out = moe.moe_down_combine(h16, d["w2_q"], d["w2_s"], torch.from_numpy(rw.astype(np.float32)).cuda(),
+                               torch.from_numpy(roff).cuda(), torch.from_numpy(rsrt).cuda(), M, k)
+    torch.cuda.synchronize()
+    U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "down_combine c%d M=%d" % (ci, M))
+
+
+# ----------------------------------------------------------------------------- whole layer
+
+SMALL_FORWARD = [(0, 2), (1, 1), (1, 2), (1, 4), (1, 8), (1, 37)]
+
+
+@pytest.mark.parametrize("ci,M", SMALL_FORWARD)
+def test_forward_small_full_compare(moe, ci, M):
+    inp = gen.make_inputs(ci, M)
+    d = U.device_inputs(inp)
+    k = inp.shape.k
+    ws = torch.empty(moe.moe_workspace_bytes(M, inp.shape.H, inp.shape.I, inp.shape.E, k), dtype=torch.uint8,
+                     device="cuda")
+    ids = torch.empty((M, k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((M, k), dtype=torch.float32, device="cuda")
+    st = torch.full((1,), 123, dtype=torch.int32, device="cuda")
+    out = moe.moe_mxfp4_forward_ex(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], k, ws,
+                                   router_bias=d["router_bias"], topk_ids_out=ids, topk_w_out=tw, status_out=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == moe.MOE_OK
+    r = U.oracle_forward(inp)
+    assert np.array_equal(ids.cpu().numpy(), r["topk_ids"])
+    assert np.abs(tw.cpu().numpy() - r["topk_w"]).max() <= U.W_TOL
+    U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "forward c%d M=%d" % (ci, M))
+    # the 13-argument form (library workspace, no bias) gives the same bytes here
+    out2 = moe.moe_mxfp4_forward(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], k)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+
+
+LARGE_FORWARD = [(2, 1), (2, 2), (2, 8), (2, 16), (2, 32), (3, 256), (3, 512), (4, 1024)]
+
+
+@pytest.fixture(scope="module")
+def large_weights():
+    cache = {}
+
+    def get(ci, M):
+        key = ci
+        shape = gen.CONFIGS[ci]
+        seed = gen.config_seed(ci, M)
+        if key not in cache or cache[key][0] != seed:
+            cache.clear()
+            torch.cuda.empty_cache()
+            inp = gen.make_inputs(ci, M, weights="torch", device="cuda")
+            cache[key] = (seed, inp)
+        return cache[key][1]
+    yield get
+    cache.clear()
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("ci,M", LARGE_FORWARD)
+def test_forward_large_sampled(moe, large_weights, ci, M):
+    inp = large_weights(ci, M)
+    d = U.device_inputs(inp)
+    k = inp.shape.k
+    ids = torch.empty((M, k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((M, k), dtype=torch.float32, device="cuda")
+    ws = torch.empty(moe.moe_workspace_bytes(M, inp.shape.H, inp.shape.I, inp.shape.E, k), dtype=torch.uint8,
+                     device="cuda")
+    out = moe.moe_mxfp4_forward_ex(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], k, ws,
+                                   router_bias=d["router_bias"], topk_ids_out=ids, topk_w_out=tw)
+    torch.cuda.synchronize()
+    rids, rw, _ = oracle.route(inp.x, inp.router_w, inp.router_bias, k)
+    assert np.array_equal(ids.cpu().numpy(), rids)                 # whole routing, bit-exact
+    assert np.abs(tw.cpu().numpy() - rw).max() <= U.W_TOL
+    rng = np.random.default_rng(M)
+    toks = sorted(set([0, M - 1] + list(rng.choice(M, min(M, 2), replace=False))))
+    if ci == 4:
+        # the most-loaded expert's tokens exercise the longest tile runs
+        heavy = np.nonzero((rids == 0).any(axis=1))[0]
+        toks = sorted(set(toks + [int(heavy[0]), int(heavy[-1])]))
+    r = U.oracle_forward(inp, tokens=toks)
+    got = U.bf16_tensor_to_f64(out)
+    U.check_out(got[toks], r["out64"][toks], "forward c%d M=%d tokens %s" % (ci, M, toks))
+    assert np.all(np.isfinite(got))
