@@ -260,6 +260,7 @@ static int check_forward_args(const void *x, const float *router_w, const float 
 {
     int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;   // nothing is read or written
     if (!x || !router_w || !w13_q || !w13_s || !w2_q || !w2_s || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(w13_q, 16) || !aligned(w13_s, 16) ||
         !aligned(w2_q, 16) || !aligned(w2_s, 16) || !aligned(out, 16))
@@ -304,6 +305,7 @@ int moe_route(const void *x_bf16, const float *router_w, const float *router_bia
 {
     int rc = check_dims(M, H, 32, E, k, false);
     if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
     if (!x_bf16 || !router_w || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
     if (!aligned(x_bf16, 16) || !aligned(router_w, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
         (router_bias && !aligned(router_bias, 4)))
@@ -325,6 +327,7 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
 {
     int rc = check_dims(M, 32, 32, E, k, false);
     if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
     if (!topk_ids || !expert_offsets || !sorted_ids || !inv_pos) return MOE_ERR_INVALID_ARG;
     if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
         return MOE_ERR_INVALID_ARG;
@@ -338,6 +341,7 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
 {
     int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
     if (!x_bf16 || !w13_q || !w13_s || !expert_offsets || !sorted_ids || !h_f16) return MOE_ERR_INVALID_ARG;
     if (!aligned(x_bf16, 16) || !aligned(w13_q, 16) || !aligned(w13_s, 16) || !aligned(h_f16, 16) ||
         !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4))
@@ -363,6 +367,7 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
 {
     int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
     if (!h_f16 || !w2_q || !w2_s || !topk_w || !expert_offsets || !sorted_ids || !out_bf16) return MOE_ERR_INVALID_ARG;
     if (!aligned(h_f16, 16) || !aligned(w2_q, 16) || !aligned(w2_s, 16) || !aligned(out_bf16, 16) ||
         !aligned(topk_w, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4))

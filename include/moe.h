@@ -38,7 +38,8 @@
  *     never synchronise the host, and allocate nothing while `stream` is being
  *     captured into a CUDA graph.
  *   - Arguments are validated before anything is enqueued; a call that returns an
- *     error status has enqueued nothing.  M == 0 returns MOE_OK and enqueues nothing.
+ *     error status has enqueued nothing.  M == 0 returns MOE_OK after the shape checks,
+ *     reads no pointer (they may be NULL) and enqueues nothing.
  *   - Supported shapes: H % 32 == 0, I % 32 == 0, H,I >= 32, 1 <= k <= min(E, 32),
  *     E <= 1024, M*k <= 16384.  Others return MOE_ERR_UNSUPPORTED_SHAPE.
  *   - Out of contract (undefined output, no fault): NaN/Inf or |x| > 65504 in x,

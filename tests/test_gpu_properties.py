@@ -56,14 +56,15 @@ def test_graph_replay_matches_eager_and_follows_input(moe):
     g.replay()
     torch.cuda.synchronize()
     assert np.array_equal(_bits(out), _bits(eager))
-    # change x in place, replay: the output must follow and match the oracle
+    # change x and the router in place (a margin-checked pair), replay: the output
+    # must follow and match the oracle
     inp2 = gen.make_inputs(1, 8, seed=777)
     d["x"].copy_(U.bits_to_bf16_tensor(inp2.x))
+    d["router_w"].copy_(torch.from_numpy(inp2.router_w))
     g.replay()
     torch.cuda.synchronize()
     assert not np.array_equal(_bits(out), _bits(eager))
     inp2.w13_q, inp2.w13_s, inp2.w2_q, inp2.w2_s = inp.w13_q, inp.w13_s, inp.w2_q, inp.w2_s
-    inp2.router_w = inp.router_w
     r = U.oracle_forward(inp2)
     U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "graph replay after x change")
 
