@@ -49,7 +49,7 @@ NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
 KERNEL_SRC = os.path.join(ROOT, "decode_moe_layer_b200", "csrc", "grouped_gemm.cu")
-TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gate_up_swiglu_decode_h2048_i768_e128_k8_M8.md")
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "grouped_mxfp4_decode_h2048_i768_e128_k8_M8.md")
 
 
 def parse_args():
