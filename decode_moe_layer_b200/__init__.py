@@ -6,6 +6,7 @@ the library and fails loudly if it has not been built.
 """
 from ._lib import (  # noqa: F401
     EXPORTS,
+    H_STORAGE_SCALE,
     LIB_PATH,
     MOE_ERR_CUDA,
     MOE_ERR_INVALID_ARG,

@@ -24,6 +24,7 @@ EXPORTS = (
     "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_mxfp4_forward_ex",
     "moe_mxfp4_forward_profile",
 )
+H_STORAGE_SCALE = 1024.0   # moe_gate_up_swiglu stores binary16(h * 2^10)
 PROFILE_KERNELS = ("route_logits", "route_topk", "permute", "gate_up_swiglu", "down", "combine")
 
 _lib = None
@@ -128,7 +129,7 @@ def moe_permute(topk_ids, E: int, stream=None):
 
 
 def moe_gate_up_swiglu(x, w13_q, w13_s, expert_offsets, sorted_ids, k: int, stream=None):
-    """-> h binary16 [M*k, I] in expert-grouped order (bf16-rounded values)."""
+    """-> h binary16 [M*k, I] in expert-grouped order, element = bf16_rne(h) * 2^10."""
     _need(x, torch.bfloat16, "x")
     M, H = x.shape
     E, I2, _ = w13_q.shape
@@ -141,7 +142,7 @@ def moe_gate_up_swiglu(x, w13_q, w13_s, expert_offsets, sorted_ids, k: int, stre
 
 
 def moe_down_combine(h, w2_q, w2_s, topk_w, expert_offsets, sorted_ids, M: int, k: int, stream=None):
-    """h binary16 [M*k, I] (expert-grouped) -> out bf16 [M, H]."""
+    """h binary16 [M*k, I] (expert-grouped, element = h * 2^10) -> out bf16 [M, H]."""
     _need(h, torch.float16, "h")
     E, H, _ = w2_q.shape
     I = h.shape[1]

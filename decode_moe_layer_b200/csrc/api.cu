@@ -128,14 +128,14 @@ static EncodeTiledFn encode_fn()
     return fn;
 }
 
-// Packed E2M1 matrix viewed as [rows][row_bytes] uint8; boxes of 16 rows x 128 bytes, 128-byte swizzle.
-static int make_weight_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes)
+// Packed E2M1 matrix viewed as [rows][row_bytes] uint8; boxes of box_rows rows x 128 bytes, 128-byte swizzle.
+static int make_weight_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, int box_rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cuda_fail(cudaErrorNotSupported);
     const cuuint64_t dims[2] = {row_bytes, rows};
     const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kBoxRows)};
+    const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -188,7 +188,9 @@ static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x1
                        int k, int max_tiles, cudaStream_t s)
 {
     CUtensorMap map;
-    int rc = make_weight_map(&map, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2);
+    // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
+    int rc = make_weight_map(&map, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2,
+                             kItemRows / 2);
     if (rc != MOE_OK) return rc;
     MOE_TRY(launch_gate_up(map, w13_s, x16, sorted_ids, tiles, n_tiles, h, status, H, I, k, max_tiles, s));
     return MOE_OK;
@@ -199,7 +201,7 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
                     int I, int E, int max_tiles, cudaStream_t s)
 {
     CUtensorMap map;
-    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2);
+    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
     if (rc != MOE_OK) return rc;
     MOE_TRY(launch_down(map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, H, I, max_tiles, s));
     return MOE_OK;

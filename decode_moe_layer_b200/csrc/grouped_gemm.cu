@@ -10,31 +10,33 @@
 // HBM bandwidth ("The Systematic Optimization Campaign", chunk 8.0).
 //
 // Design (one persistent CTA per SM, warp specialised):
-//  * Work item = (expert tile of <= 8 assignments, block of 32 weight rows).
-//    gate_up rows: 16 gate rows n0.. and the 16 matching up rows I+n0..;
-//    down rows: 32 consecutive rows r0.. of W2.  Items are spread round-robin
-//    over the CTAs; all tiles of one row block are adjacent, so CTAs that share
-//    weights run together and hit L2.
-//  * Producer warp: TMA 2-D tiled copies (16 rows x 128 B boxes, 128-byte
-//    swizzle) of packed E2M1 bytes through an 8-stage ring of 8 KB stages; in
-//    the same stage, one 1-D bulk copy per tile token of its binary16
+//  * Work item = (expert tile of <= 8 assignments, 64 weight rows).  gate_up:
+//    gate rows n0..n0+31 and the matching up rows I+n0..; down: W2 rows
+//    r0..r0+63.  The item is 4 MMA m-tiles of 16 rows; for gate_up an m-tile
+//    holds 8 gate rows (fragment rows 0-7) and the same 8 up rows (fragment rows
+//    8-15), so every thread ends with g and u of one output row and applies
+//    clamp-SwiGLU and the bf16 rounding in registers.  Items are spread
+//    round-robin over the CTAs; all tiles of one row block are adjacent, so
+//    CTAs that share weights run together and hit L2.
+//  * Producer warp: per 512-K stage, TMA 2-D tiled copies of the item's packed
+//    E2M1 bytes (boxes of 32 or 64 rows x 128 bytes, 128-byte swizzle) into a
+//    6-stage ring of 16 KB, and one 1-D bulk copy per tile token of its binary16
 //    activation chunk (the routed gather: x rows for gate_up, h rows for down);
-//    and one pair of bulk copies of the item's E8M0 scale rows into a double
-//    buffer.
-//  * 8 consumer warps split each stage's 16 blocks of 32 K: a thread reads the
-//    32-bit word q of its rows' 16-byte block (conflict-free thanks to the
-//    swizzle), decodes it with the hardware E2M1 -> f16x2 conversion straight
-//    into MMA A-fragment registers, and runs two m16n8k16 f16 MMAs per block and
-//    token group.  Inside a block the K order is permuted (thread q's word covers
-//    K 8q..8q+7) identically for A and for the activation fragment, so each MMA
-//    pair spans exactly one scale block and the E8M0 scale is applied once to the
-//    fp32 partial sum.
-//  * gate_up m-tile = 8 gate rows (fragment rows 0-7) + the same 8 up rows
-//    (fragment rows 8-15): each thread holds g and u of one output row, so
-//    clamp-SwiGLU and the bf16 rounding run in registers.
-//  * The K split over warps is reduced through shared memory in warp order.
+//    per item, the 64 E8M0 scale rows into a double buffer (one copy per row at
+//    a padded pitch when rows are 16-byte multiples, so that the 8 row-distinct
+//    scale reads of a warp fall in distinct banks).
+//  * 16 consumer warps = 2 m-tile pairs x 8 K slots.  Per stage a warp takes 2
+//    of the 16 blocks of 32 K for its 2 m-tiles: a thread reads the 32-bit word
+//    q of its rows' 16-byte block (conflict-free thanks to the swizzle), decodes
+//    it with the hardware E2M1 -> f16x2 conversion straight into MMA A-fragment
+//    registers, and runs two m16n8k16 f16 MMAs per block.  Inside a block the K
+//    order is permuted (thread q's word covers K 8q..8q+7) identically for A and
+//    for the activation fragment, so each MMA pair spans exactly one scale block
+//    and the E8M0 scale is applied once to the fp32 partial sum.
+//  * The 8 K slots of an m-tile are reduced through shared memory in slot order.
 // Activations (x or h) are read as binary16; bf16 x converts exactly for
-// 2^-17 <= |x| <= 65504, E2M1 values are exact in binary16, and products
+// 2^-17 <= |x| <= 65504, h is stored scaled by 2^10 (exact for |h| >= 2^-27,
+// |h| <= 49 so no overflow), E2M1 values are exact in binary16, and products
 // accumulate in fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -44,11 +46,19 @@
 namespace moe {
 
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kRedFloats = kConsumerWarps * 2 * 32 * 4;   // [warp][mt][lane][4]
+constexpr int kRedFloats = kKSlots * kItemMTiles * 32 * 4;   // [kslot][m-tile][lane][4]
 
 struct SmemPlan {
-    int wst_off, act_off, sbuf_off, sbuf_bytes, red_off, bars_off, total;
+    int wst_off, act_off, sbuf_off, spitch, sbuf_bytes, red_off, bars_off, total;
 };
+
+// Scale rows are copied one per row at a padded pitch when they are 16-byte
+// multiples, else as one contiguous block (pitch = row length).
+__host__ __device__ inline int scale_pitch(int K)
+{
+    const int kb = K / 32;
+    return (kb % 16 == 0) ? kb + 16 : kb;
+}
 
 __host__ __device__ inline SmemPlan smem_plan(int K)
 {
@@ -56,7 +66,8 @@ __host__ __device__ inline SmemPlan smem_plan(int K)
     p.wst_off = 0;
     p.act_off = kStages * kStageBytes;
     p.sbuf_off = p.act_off + kStages * kActStageBytes;
-    p.sbuf_bytes = ((kRowsPerItem * (K / 32)) + 127) / 128 * 128;
+    p.spitch = scale_pitch(K);
+    p.sbuf_bytes = (kItemRows * p.spitch + 127) / 128 * 128;
     p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
     p.bars_off = p.red_off + kRedFloats * 4;
     p.total = p.bars_off + (2 * kStages + 4) * 8 + 1024;   // + alignment slack
@@ -70,10 +81,10 @@ __device__ __forceinline__ float clamp_swiglu(float g, float u)
     return a / (1.0f + expf(-a)) * c;
 }
 
-__device__ __forceinline__ __half round_h(float v)
+// bf16 round-to-nearest-even, then the exact move into binary16 with the 2^10 storage scale
+__device__ __forceinline__ __half store_h(float v)
 {
-    // bf16 round-to-nearest-even, then the exact move into binary16
-    return __float2half_rn(__bfloat162float(__float2bfloat16_rn(v)));
+    return __float2half_rn(__bfloat162float(__float2bfloat16_rn(v)) * kHScale);
 }
 
 template <bool kGateUp>
@@ -97,11 +108,14 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = *n_tiles_ptr;
-    const int row_blocks = kGateUp ? I / 16 : H / 32;
+    const int rows_total = kGateUp ? I : H;                 // output rows of this projection
+    const int row_blocks = kGateUp ? I / 32 : (H + kItemRows - 1) / kItemRows;
     const int n_items = n_tiles * row_blocks;
     const int kblocks = K / 32;               // scale bytes per row
+    const int spitch = plan.spitch;
     const int n_chunks = (K + kChunkK - 1) / kChunkK;
     const int kbytes = K / 2;                 // packed bytes per row
+    constexpr int kBoxBytes = (kGateUp ? 32 : 64) * 128;   // one TMA box: rows x 128 bytes
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -120,21 +134,16 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
 
     if (warp == kConsumerWarps) {
         // ---------------------------------------------------------------- producer warp
-        // lane 0: scale rows and weight boxes; lane i < count: token i's activation chunk
         if (lane == 0) prefetch_tensormap(&wmap);
         int stage_ctr = 0, item_ctr = 0;
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
             const ExpertTile tl = tiles[item % n_tiles];
             const int rb = item / n_tiles;
             const int e = tl.expert;
-            int row_a, row_b;   // first global rows of the two 16-row halves
-            if (kGateUp) {
-                row_a = e * 2 * I + rb * 16;
-                row_b = row_a + I;
-            } else {
-                row_a = e * H + rb * 32;
-                row_b = row_a + 16;
-            }
+            // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
+            const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
+            const int row_b = row_a + I;                               // gate_up only
+            const int valid_rows = kGateUp ? kItemRows : min(kItemRows, H - rb * kItemRows);
             // this lane's activation row (gate_up: the token's x row; down: the h row)
             const int li = min(lane, tl.count - 1);
             const __half *arow = kGateUp ? act + static_cast<size_t>(sorted_ids[tl.p0 + li] / ktop) * K
@@ -142,33 +151,48 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
             const int b = item_ctr & 1;
             mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
             aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
-            if (lane == 0 && !aborted) {
+            if (!aborted) {
                 uint8_t *dst = sbuf + b * plan.sbuf_bytes;
-                const uint32_t half_bytes = 16u * kblocks;
-                mbar_arrive_expect_tx(&sfull[b], 2u * half_bytes);
-                bulk_load(dst, wscale + static_cast<size_t>(row_a) * kblocks, half_bytes, &sfull[b]);
-                bulk_load(dst + half_bytes, wscale + static_cast<size_t>(row_b) * kblocks, half_bytes, &sfull[b]);
+                if (lane == 0) mbar_arrive_expect_tx(&sfull[b], static_cast<uint32_t>(valid_rows * kblocks));
+                __syncwarp();
+                if (spitch != kblocks) {
+                    // one copy per row into the padded pitch (kblocks is a multiple of 16)
+                    for (int r = lane; r < valid_rows; r += 32) {
+                        const int grow = kGateUp ? (r < 32 ? row_a + r : row_b + r - 32) : row_a + r;
+                        bulk_load(dst + r * spitch, wscale + static_cast<size_t>(grow) * kblocks, kblocks, &sfull[b]);
+                    }
+                } else if (lane == 0) {
+                    if (kGateUp) {
+                        bulk_load(dst, wscale + static_cast<size_t>(row_a) * kblocks, 32u * kblocks, &sfull[b]);
+                        bulk_load(dst + 32 * kblocks, wscale + static_cast<size_t>(row_b) * kblocks, 32u * kblocks,
+                                  &sfull[b]);
+                    } else {
+                        bulk_load(dst, wscale + static_cast<size_t>(row_a) * kblocks,
+                                  static_cast<uint32_t>(valid_rows * kblocks), &sfull[b]);
+                    }
+                }
             }
             for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
                 const int s = stage_ctr % kStages;
                 mbar_wait(&empty[s], ((stage_ctr / kStages) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);
+                if (aborted) continue;
                 const int kb = c * (kChunkK / 2);
                 const int kc = c * kChunkK;
                 const uint32_t act_bytes = 2u * static_cast<uint32_t>(min(kChunkK, K - kc));
-                const int nbox_half = (kb + 128 < kbytes) ? 2 : 1;   // skip a box wholly past K
-                if (lane == 0 && !aborted)
-                    mbar_arrive_expect_tx(&full[s], 2u * nbox_half * kBoxBytes + tl.count * act_bytes);
+                const int nkh = (kb + 128 < kbytes) ? 2 : 1;   // skip the K-hi box when wholly past K
+                const int nbox = (kGateUp ? 2 : 1) * nkh;
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], nbox * kBoxBytes + tl.count * act_bytes);
                 __syncwarp();
-                if (aborted) continue;
                 if (lane == 0) {
                     uint8_t *st = wst + s * kStageBytes;
-                    // boxes: 0 = half a lo, 1 = half a hi, 2 = half b lo, 3 = half b hi
-                    tma_load_2d(st + 0 * kBoxBytes, &wmap, kb, row_a, &full[s]);
-                    tma_load_2d(st + 2 * kBoxBytes, &wmap, kb, row_b, &full[s]);
-                    if (nbox_half == 2) {
-                        tma_load_2d(st + 1 * kBoxBytes, &wmap, kb + 128, row_a, &full[s]);
-                        tma_load_2d(st + 3 * kBoxBytes, &wmap, kb + 128, row_b, &full[s]);
+                    // gate_up boxes: 0 = gate K-lo, 1 = gate K-hi, 2 = up K-lo, 3 = up K-hi
+                    // down boxes:    0 = K-lo, 1 = K-hi
+                    tma_load_2d(st, &wmap, kb, row_a, &full[s]);
+                    if (nkh == 2) tma_load_2d(st + kBoxBytes, &wmap, kb + 128, row_a, &full[s]);
+                    if (kGateUp) {
+                        tma_load_2d(st + 2 * kBoxBytes, &wmap, kb, row_b, &full[s]);
+                        if (nkh == 2) tma_load_2d(st + 3 * kBoxBytes, &wmap, kb + 128, row_b, &full[s]);
                     }
                 }
                 if (lane < tl.count)
@@ -185,7 +209,31 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
 
     // -------------------------------------------------------------------- consumer warps
     const int g = lane >> 2, q = lane & 3;
+    const int pair = warp & 1;              // m-tiles 2*pair, 2*pair+1
+    const int kslot = warp >> 1;            // blocks 2*kslot, 2*kslot+1 of every stage
+    const int khalf = kslot >> 2;           // both blocks lie in the same 128-byte box column
+    const int bb0 = (2 * kslot) & 7;
     const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+
+    // per m-tile: smem byte offsets (inside a stage) of the top/bottom rows' 16-byte blocks,
+    // and scale-row offsets inside the item's scale buffer
+    int top_off[2], bot_off[2], top_srow[2], bot_srow[2];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+        const int j = 2 * pair + m;
+        if (kGateUp) {
+            top_off[m] = (0 + khalf) * kBoxBytes + (8 * j + g) * 128;
+            bot_off[m] = (2 + khalf) * kBoxBytes + (8 * j + g) * 128;
+            top_srow[m] = (8 * j + g) * spitch;
+            bot_srow[m] = (32 + 8 * j + g) * spitch;
+        } else {
+            top_off[m] = khalf * kBoxBytes + (16 * j + g) * 128;
+            bot_off[m] = khalf * kBoxBytes + (16 * j + 8 + g) * 128;
+            top_srow[m] = (16 * j + g) * spitch;
+            bot_srow[m] = (16 * j + 8 + g) * spitch;
+        }
+    }
+
     int stage_ctr = 0, item_ctr = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
         const ExpertTile tl = tiles[item % n_tiles];
@@ -197,40 +245,28 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
 
         float acc[2][4];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) acc[mt][r] = 0.f;
+            for (int r = 0; r < 4; ++r) acc[m][r] = 0.f;
 
         for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
             const int s = stage_ctr % kStages;
-            const int kc = c * kChunkK;
             mbar_wait(&full[s], (stage_ctr / kStages) & 1, aborted, status);
             const uint8_t *st = wst + s * kStageBytes;
             const uint8_t *xa = ast + s * kActStageBytes + g * kActPitch;   // token g of the tile
+            const int kblk0 = c * (kChunkK / 32) + 2 * kslot;                 // global block index
 #pragma unroll
             for (int bi = 0; bi < 2; ++bi) {
-                const int blk = 2 * warp + bi;    // block of 32 K inside the stage
-                const int kg = kc + 32 * blk;
-                if (kg >= K) continue;
-                const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * blk + 8 * q) * 2);
-                const int half = blk >> 3, bb = blk & 7;
-                const int sw = ((bb ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
+                const int kblk = kblk0 + bi;
+                if (kblk >= kblocks) continue;
+                const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (2 * kslot + bi) + 8 * q) * 2);
+                const int sw = (((bb0 + bi) ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
-                    int top_box, top_row, bot_box, bot_row, top_s, bot_s;
-                    if (kGateUp) {
-                        top_box = half;          top_row = 8 * mt + g;
-                        bot_box = 2 + half;      bot_row = 8 * mt + g;
-                        top_s = 8 * mt + g;      bot_s = 16 + 8 * mt + g;
-                    } else {
-                        top_box = 2 * mt + half; top_row = g;
-                        bot_box = 2 * mt + half; bot_row = 8 + g;
-                        top_s = 16 * mt + g;     bot_s = 16 * mt + 8 + g;
-                    }
-                    const uint32_t wt = *reinterpret_cast<const uint32_t *>(st + top_box * kBoxBytes + top_row * 128 + sw);
-                    const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_box * kBoxBytes + bot_row * 128 + sw);
-                    const float st_scale = e8m0_times2(sb[top_s * kblocks + (kg >> 5)]);
-                    const float sb_scale = e8m0_times2(sb[bot_s * kblocks + (kg >> 5)]);
+                for (int m = 0; m < 2; ++m) {
+                    const uint32_t wt = *reinterpret_cast<const uint32_t *>(st + top_off[m] + sw);
+                    const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_off[m] + sw);
+                    const float st_scale = e8m0_times2(sb[top_srow[m] + kblk]);
+                    const float sb_scale = e8m0_times2(sb[bot_srow[m] + kblk]);
                     uint32_t t0, t1, t2, t3, u0, u1, u2, u3;
                     e2m1x8_to_f16x2(wt, t0, t1, t2, t3);
                     e2m1x8_to_f16x2(wb, u0, u1, u2, u3);
@@ -239,10 +275,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
                     float tmp[4];
                     mma_f16_16816(tmp, a0, xb.x, xb.y, zero4);
                     mma_f16_16816(tmp, a1, xb.z, xb.w, tmp);
-                    acc[mt][0] = fmaf(tmp[0], st_scale, acc[mt][0]);
-                    acc[mt][1] = fmaf(tmp[1], st_scale, acc[mt][1]);
-                    acc[mt][2] = fmaf(tmp[2], sb_scale, acc[mt][2]);
-                    acc[mt][3] = fmaf(tmp[3], sb_scale, acc[mt][3]);
+                    acc[m][0] = fmaf(tmp[0], st_scale, acc[m][0]);
+                    acc[m][1] = fmaf(tmp[1], st_scale, acc[m][1]);
+                    acc[m][2] = fmaf(tmp[2], sb_scale, acc[m][2]);
+                    acc[m][3] = fmaf(tmp[3], sb_scale, acc[m][3]);
                 }
             }
             __syncwarp();
@@ -251,47 +287,49 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
         __syncwarp();
         if (lane == 0) mbar_arrive(&sempty[b]);
 
-        // ---------------------------------------------------------------- cross-warp reduction
+        // ---------------------------------------------------------------- K-slot reduction
         named_bar_sync(1, kConsumerWarps * 32);
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-            *reinterpret_cast<float4 *>(red + ((warp * 2 + mt) * 32 + lane) * 4) =
-                make_float4(acc[mt][0], acc[mt][1], acc[mt][2], acc[mt][3]);
+        for (int m = 0; m < 2; ++m)
+            *reinterpret_cast<float4 *>(red + ((kslot * kItemMTiles + 2 * pair + m) * 32 + lane) * 4) =
+                make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
         named_bar_sync(1, kConsumerWarps * 32);
-        if (warp < 2) {
-            const int mt = warp;
+        if (warp < kItemMTiles) {
+            const int j = warp;
             float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float4 v = *reinterpret_cast<const float4 *>(red + ((w * 2 + mt) * 32 + lane) * 4);
+            for (int ks = 0; ks < kKSlots; ++ks) {
+                const float4 v = *reinterpret_cast<const float4 *>(red + ((ks * kItemMTiles + j) * 32 + lane) * 4);
                 sum.x += v.x;
                 sum.y += v.y;
                 sum.z += v.z;
                 sum.w += v.w;
             }
-            // remove the factor 2 carried by e8m0_times2
-            sum.x *= 0.5f;
-            sum.y *= 0.5f;
-            sum.z *= 0.5f;
-            sum.w *= 0.5f;
             const int li0 = 2 * q, li1 = li0 + 1;
             if (kGateUp) {
-                const int n = rb * 16 + 8 * mt + g;
-                if (li0 < cnt) hout[static_cast<size_t>(tl.p0 + li0) * I + n] = round_h(clamp_swiglu(sum.x, sum.z));
-                if (li1 < cnt) hout[static_cast<size_t>(tl.p0 + li1) * I + n] = round_h(clamp_swiglu(sum.y, sum.w));
+                // remove the factor 2 carried by e8m0_times2
+                sum.x *= 0.5f;
+                sum.y *= 0.5f;
+                sum.z *= 0.5f;
+                sum.w *= 0.5f;
+                const int n = rb * 32 + 8 * j + g;
+                if (li0 < cnt) hout[static_cast<size_t>(tl.p0 + li0) * I + n] = store_h(clamp_swiglu(sum.x, sum.z));
+                if (li1 < cnt) hout[static_cast<size_t>(tl.p0 + li1) * I + n] = store_h(clamp_swiglu(sum.y, sum.w));
             } else {
-                const int ra = rb * 32 + 16 * mt + g, rbw = ra + 8;
+                // remove e8m0_times2's factor 2 and h's 2^10 storage scale
+                const float unscale = 0.5f / kHScale;
+                const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
                 if (li0 < cnt) {
                     const int f = sorted_ids[tl.p0 + li0];
-                    const float w = topk_w[f];
-                    yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
-                    yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
+                    const float w = topk_w[f] * unscale;
+                    if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
+                    if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
                 }
                 if (li1 < cnt) {
                     const int f = sorted_ids[tl.p0 + li1];
-                    const float w = topk_w[f];
-                    yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
-                    yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
+                    const float w = topk_w[f] * unscale;
+                    if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
+                    if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
                 }
             }
         }
@@ -330,7 +368,7 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const uint8_t *scales,
     const SmemPlan plan = smem_plan(K);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
     if (e != cudaSuccess) return e;
-    const long long row_blocks = kGateUp ? I / 16 : H / 32;
+    const long long row_blocks = kGateUp ? I / 32 : (H + kItemRows - 1) / kItemRows;
     const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
     const int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     grouped_mxfp4_kernel<kGateUp><<<grid > 0 ? grid : 1, kThreads, plan.total, s>>>(

@@ -15,15 +15,16 @@ constexpr int kStatusTimeout = -5;
 
 // Grouped GEMM tiling (both projections).
 constexpr int kTileTokens = 8;       // assignments per expert tile (one MMA n-tile)
-constexpr int kRowsPerItem = 32;     // weight rows per work item (2 MMA m-tiles of 16)
-constexpr int kChunkK = 512;         // K elements per pipeline stage
-constexpr int kBoxRows = 16;         // TMA box: 16 rows x 128 bytes (256 K elements)
-constexpr int kBoxBytes = 16 * 128;
-constexpr int kStageBytes = 4 * kBoxBytes;          // packed weights of one stage
+constexpr int kItemMTiles = 4;       // MMA m-tiles (16 weight rows each) per work item
+constexpr int kItemRows = 16 * kItemMTiles;
+constexpr int kChunkK = 512;         // K elements per pipeline stage (256 bytes of E2M1 per row)
+constexpr int kStageBytes = kItemRows * kChunkK / 2;   // packed weights of one stage (16 KB)
 constexpr int kActPitch = kChunkK * 2 + 64;         // one token's binary16 chunk, padded against bank conflicts
 constexpr int kActStageBytes = kTileTokens * kActPitch;
-constexpr int kStages = 8;
-constexpr int kConsumerWarps = 8;
+constexpr int kStages = 6;
+constexpr int kConsumerWarps = 16;   // 2 m-tile pairs x 8 K slots
+constexpr int kKSlots = kConsumerWarps / 2;
+constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact for |h| >= 2^-27
 
 // Router.
 constexpr int kRouteChunkH = 1024;   // H elements per partial-logit chunk

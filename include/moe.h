@@ -27,8 +27,8 @@
  *   topk_ids / topk_w int32 / fp32 [M, k], slot j in descending router probability
  *   expert_offsets    int32 [E+1];  sorted_ids, inv_pos int32 [M*k]
  *   h                 binary16 [M*k, I] in expert-grouped order (row p holds the
- *                     assignment sorted_ids[p]); every element is a bf16-rounded
- *                     value, exact in binary16 for |h| >= 2^-17 (|h| <= 49 always)
+ *                     assignment sorted_ids[p]); element = bf16_rne(h) * 2^10,
+ *                     exact in binary16 for |h| >= 2^-27 (|h| <= 49, so no overflow)
  *
  * Conventions for every entry point:
  *   - Pointers are device pointers the caller owns; the library keeps none after
@@ -113,7 +113,7 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
  * For each position p of the expert-grouped order, f = sorted_ids[p], t = f / k,
  * e = the expert whose offsets range holds p:
  *   g = W_gate,e x[t], u = W_up,e x[t] (bf16 products, fp32 accumulation),
- *   h[p] = bf16_rne(silu(min(g,7)) * clamp(u,-7,7)), stored as binary16.
+ *   h[p] = bf16_rne(silu(min(g,7)) * clamp(u,-7,7)), stored as binary16(h[p] * 2^10).
  * expert_offsets/sorted_ids are moe_permute's outputs.  Uses the library-owned
  * workspace of `stream`.
  */
@@ -123,7 +123,8 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
 
 /*
  * Down GEMM with the weighted top-k combine fused behind it.  Defined by the
- * down half of the "Compact routed MXFP4 GEMM" row of the same table:
+ * down half of the "Compact routed MXFP4 GEMM" row of the same table (h in the
+ * binary16(h * 2^10) format moe_gate_up_swiglu writes):
  *   y[f] = W2_e h[inv position of f] (fp32 accumulation),
  *   out[t] = bf16_rne( sum_{j=0..k-1} topk_w[t,j] * y[t*k+j] ), summed in slot
  *   order j with no atomics.

@@ -95,7 +95,7 @@ def test_gate_up_swiglu(moe, ci, M):
     h = moe.moe_gate_up_swiglu(d["x"], d["w13_q"], d["w13_s"], torch.from_numpy(roff).cuda(),
                                torch.from_numpy(rsrt).cuda(), k)
     torch.cuda.synchronize()
-    h_flat = h.float().cpu().numpy().astype(np.float64)[rinv]      # back to flat order t*k+j
+    h_flat = h.float().cpu().numpy().astype(np.float64)[rinv] / moe.H_STORAGE_SCALE   # flat order t*k+j
     toks = list(range(M)) if not big else [0, M - 1]
     for t in toks:
         for j in range(k):
@@ -119,7 +119,7 @@ def test_down_combine(moe, ci, M):
     rids, rw = r["topk_ids"], r["topk_w"]
     roff, rsrt, rinv = oracle.permute(rids, E)
     h_bits = r["h"][rsrt]                                         # oracle h in expert-grouped order
-    h16 = torch.from_numpy(gen.bf16_bits_to_f64(h_bits).astype(np.float16)).cuda()
+    h16 = torch.from_numpy((gen.bf16_bits_to_f64(h_bits) * moe.H_STORAGE_SCALE).astype(np.float16)).cuda()
     out = moe.moe_down_combine(h16, d["w2_q"], d["w2_s"], torch.from_numpy(rw.astype(np.float32)).cuda(),
                                torch.from_numpy(roff).cuda(), torch.from_numpy(rsrt).cuda(), M, k)
     torch.cuda.synchronize()
