@@ -84,7 +84,7 @@ def algorithmic(shape, M, ids):
     total = w_bytes + E * H * 4 + 2 * M * H * 2 + M * k * 8
     flops = 6 * I * H * M * k + 2 * M * E * H
     gate_up = touched * (2 * I * H * 17 // 32) + M * H * 2 + M * k * I * 2
-    down = touched * (I * H * 17 // 32) + M * k * I * 2 + M * k * H * 4
+    down = touched * (I * H * 17 // 32) + M * k * I * 2 + M * H * 2
     return {"touched": touched, "bytes": total, "flops": flops, "weight_bytes": w_bytes,
             "gate_up_bytes": gate_up, "down_bytes": down}
 
@@ -352,7 +352,7 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     roof_us = max(work["bytes"] / (hbm * 1e3), work["flops"] / (tflops * 1e6))
     roof_nominal_us = max(work["bytes"] / (NOMINAL_HBM_GBS * 1e3), work["flops"] / (NOMINAL_BF16_TFLOPS * 1e6))
     dominant = max(kern_us, key=kern_us.get)
-    dom_bytes = {"gate_up_swiglu": work["gate_up_bytes"], "down": work["down_bytes"]}.get(dominant)
+    dom_bytes = {"gate_up_swiglu": work["gate_up_bytes"], "down_combine": work["down_bytes"]}.get(dominant)
     if dom_bytes is None:
         dom_bytes = work["bytes"]
     achieved = dom_bytes / (kern_us[dominant] * 1e3)          # GB/s
@@ -377,7 +377,7 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
                      "algorithmic_bytes_per_launch": dom_bytes},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": M * H * 2,
                 "path": "pinned host x -> moe_mxfp4_forward_ex (eager C-ABI call) -> pinned host out"},
-        "gpu_launches": len(moe.PROFILE_KERNELS) * args.steps,
+        "gpu_launches": (4 if M <= 256 else 5) * args.steps,
         "clocks": clk,
     }
     if baselines and rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -78,6 +78,7 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.n_tiles = take(4);
     L.h = take(n * I * 2);
     L.y = take(n * H * sizeof(float));
+    L.counters = take(static_cast<size_t>(M) * down_row_blocks(H) * sizeof(int));
     L.total = off;
     return L;
 }
@@ -183,27 +184,29 @@ static int library_workspace(cudaStream_t s, size_t need, char **out)
 
 // ------------------------------------------------------------------ step bodies (arguments already validated)
 
-static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const int32_t *sorted_ids,
-                       const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int H, int I, int E,
-                       int k, int max_tiles, cudaStream_t s)
+static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const ExpertTile *tiles,
+                       const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E,
+                       int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map;
     // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
     int rc = make_weight_map(&map, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2,
                              kItemRows / 2);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_gate_up(map, w13_s, x16, sorted_ids, tiles, n_tiles, h, status, H, I, k, max_tiles, s));
+    MOE_TRY(launch_gate_up(map, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, max_tiles, s, pdl));
     return MOE_OK;
 }
 
 static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
-                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int H,
-                    int I, int E, int max_tiles, cudaStream_t s)
+                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *counters,
+                    void *out, int *status, int32_t *status_out, int H, int I, int E, int k, int max_tiles,
+                    cudaStream_t s, bool pdl)
 {
     CUtensorMap map;
     int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_down(map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, H, I, max_tiles, s));
+    MOE_TRY(launch_down_combine(map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, counters, out, status,
+                                status_out, H, I, k, max_tiles, s, pdl));
     return MOE_OK;
 }
 
@@ -236,21 +239,33 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     __half *h = reinterpret_cast<__half *>(ws + L.h);
     float *y = reinterpret_cast<float *>(ws + L.y);
+    int *counters = reinterpret_cast<int *>(ws + L.counters);
+    // The first kernel is ordered after everything before it on the stream; each later
+    // kernel of the call is launched early (programmatic dependent launch) and waits on
+    // device for its predecessor.  Event marks (profiling) break that overlap, so the
+    // profiling entry point launches without it.
+    const bool pdl = (marks == nullptr);
 
     MOE_MARK(marks, s);
-    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, M, H, E, L.route_splits, s));
+    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, counters, down_row_blocks(H), M, H, E,
+                                L.route_splits, s));
     MOE_MARK(marks, s);
-    MOE_TRY(launch_route_topk(partial, router_bias, ids, tw, M, E, k, L.route_splits, s));
+    if (M <= kFusedSelectMaxM) {
+        MOE_TRY(launch_route_select_permute(partial, router_bias, ids, tw, offsets, sorted_ids, inv_pos, tiles,
+                                            n_tiles, M, E, k, L.route_splits, s, pdl));
+        MOE_MARK(marks, s);
+    } else {
+        MOE_TRY(launch_route_topk(partial, router_bias, ids, tw, M, E, k, L.route_splits, s, pdl));
+        MOE_MARK(marks, s);
+        MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, s, pdl));
+    }
     MOE_MARK(marks, s);
-    MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, s));
-    MOE_MARK(marks, s);
-    int rc = run_gate_up(w13_q, w13_s, x16, sorted_ids, tiles, n_tiles, h, status, H, I, E, k, L.max_tiles, s);
+    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
     MOE_MARK(marks, s);
-    rc = run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, status, H, I, E, L.max_tiles, s);
+    rc = run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, counters, out, status, status_out, H, I, E, k,
+                  L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
-    MOE_MARK(marks, s);
-    MOE_TRY(launch_combine(y, out, status, status_out, M, H, k, s));
     MOE_MARK(marks, s);
     return MOE_OK;
 }
@@ -318,9 +333,9 @@ int moe_route(const void *x_bf16, const float *router_w, const float *router_bia
     rc = library_workspace(stream, L.total, &ws);
     if (rc != MOE_OK) return rc;
     float *partial = reinterpret_cast<float *>(ws + L.partial);
-    MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, reinterpret_cast<int *>(ws + L.status), M, H, E,
-                                L.route_splits, stream));
-    MOE_TRY(launch_route_topk(partial, router_bias, topk_ids, topk_w, M, E, k, L.route_splits, stream));
+    MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, reinterpret_cast<int *>(ws + L.status), nullptr,
+                                nullptr, 0, M, H, E, L.route_splits, stream));
+    MOE_TRY(launch_route_topk(partial, router_bias, topk_ids, topk_w, M, E, k, L.route_splits, stream, false));
     return MOE_OK;
 }
 
@@ -334,7 +349,7 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
     if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
         return MOE_ERR_INVALID_ARG;
     if (M == 0) return MOE_OK;
-    MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, nullptr, nullptr, M, E, k, stream));
+    MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, nullptr, nullptr, M, E, k, stream, false));
     return MOE_OK;
 }
 
@@ -358,9 +373,9 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
-    MOE_TRY(launch_build_tiles(expert_offsets, tiles, n_tiles, nullptr, E, stream));
-    return run_gate_up(w13_q, w13_s, x16, sorted_ids, tiles, n_tiles, static_cast<__half *>(h_f16), status, H, I, E,
-                       k, L.max_tiles, stream);
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, nullptr, nullptr, 0, E, k, stream));
+    return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E,
+                       L.max_tiles, stream, false);
 }
 
 int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
@@ -383,12 +398,11 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
-    MOE_TRY(launch_build_tiles(expert_offsets, tiles, n_tiles, status, E, stream));
-    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, status, H, I,
-                  E, L.max_tiles, stream);
-    if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_combine(y, out_bf16, status, nullptr, M, H, k, stream));
-    return MOE_OK;
+    int *counters = reinterpret_cast<int *>(ws + L.counters);
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, counters, M * down_row_blocks(H),
+                               E, k, stream));
+    return run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, counters,
+                    out_bf16, status, nullptr, H, I, E, k, L.max_tiles, stream, false);
 }
 
 int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,

@@ -21,10 +21,26 @@ namespace moe {
 // ~2 s at 2 GHz: far above any legitimate wait inside one layer call.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
-__device__ __forceinline__ void record_timeout(int *status)
+// Where a call's device status goes: the workspace word, and the caller's optional slot.
+struct StatusPtrs {
+    int *ws;
+    int32_t *out;
+};
+
+__device__ __forceinline__ void record_timeout(const StatusPtrs &st)
 {
-    if (status) atomicExch(status, kStatusTimeout);
+    if (st.ws) atomicExch(st.ws, kStatusTimeout);
+    if (st.out) atomicExch(st.out, kStatusTimeout);
 }
+
+// ------------------------------------------------------------------ programmatic dependent launch
+
+// Block until the grids this one depends on have completed and their writes are visible
+// (returns at once when the kernel was launched without a programmatic dependency).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel in the stream to begin launching; it still waits in pdl_wait().
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ------------------------------------------------------------------ shared-memory addressing
 
@@ -72,7 +88,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 // Bounded wait for the phase with the given parity to complete.  Once a wait
 // has timed out (`aborted` set) later waits return at once, so every thread
 // still reaches every CTA barrier and the kernel ends.
-__device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &aborted, int *status)
+__device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &aborted, const StatusPtrs &st)
 {
     if (aborted) return;
     if (mbar_try_wait(bar, parity)) return;
@@ -80,7 +96,7 @@ __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > kWaitLimitCycles) {
             aborted = true;
-            record_timeout(status);
+            record_timeout(st);
             return;
         }
     }

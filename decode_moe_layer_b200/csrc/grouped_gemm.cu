@@ -93,7 +93,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
                      const __half *__restrict__ act, const int32_t *__restrict__ sorted_ids,
                      const float *__restrict__ topk_w, const ExpertTile *__restrict__ tiles,
                      const int *__restrict__ n_tiles_ptr, __half *__restrict__ hout, float *__restrict__ yout,
-                     int *status, int K, int I, int H, int ktop)
+                     int *__restrict__ counters, __nv_bfloat16 *__restrict__ out, int *status_ws,
+                     int32_t *status_out, int K, int I, int H, int ktop)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -107,10 +108,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
     uint64_t *full = bars, *empty = bars + kStages, *sfull = bars + 2 * kStages, *sempty = sfull + 2;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_tiles = *n_tiles_ptr;
+    const StatusPtrs status{status_ws, status_out};
+    __shared__ int s_last[kTileTokens];      // down: tokens whose row block this CTA completes
     const int rows_total = kGateUp ? I : H;                 // output rows of this projection
-    const int row_blocks = kGateUp ? I / 32 : (H + kItemRows - 1) / kItemRows;
-    const int n_items = n_tiles * row_blocks;
+    const int row_blocks = kGateUp ? I / 32 : down_row_blocks(H);
     const int kblocks = K / 32;               // scale bytes per row
     const int spitch = plan.spitch;
     const int n_chunks = (K + kChunkK - 1) / kChunkK;
@@ -129,6 +130,11 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
         fence_barrier_init();
     }
     __syncthreads();
+    // everything below reads what the previous kernels of this call wrote
+    pdl_wait();
+    pdl_trigger();
+    const int n_tiles = *n_tiles_ptr;
+    const int n_items = n_tiles * row_blocks;
 
     bool aborted = false;
 
@@ -136,18 +142,29 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
         // ---------------------------------------------------------------- producer warp
         if (lane == 0) prefetch_tensormap(&wmap);
         int stage_ctr = 0, item_ctr = 0;
+        // the next item's descriptor, loaded one item ahead so that no copy waits on it
+        int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
+        auto fetch = [&](int it) {
+            if (it < n_items) {
+                const ExpertTile *tp = tiles + it % n_tiles;
+                nx_e = tp->expert;
+                nx_p0 = tp->p0;
+                nx_cnt = tp->count;
+                nx_tok = tp->tok[lane & (kTileTokens - 1)];
+            }
+        };
+        fetch(blockIdx.x);
         for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
-            const ExpertTile tl = tiles[item % n_tiles];
+            const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, tok = nx_tok;
+            fetch(item + gridDim.x);
             const int rb = item / n_tiles;
-            const int e = tl.expert;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
             const int row_b = row_a + I;                               // gate_up only
             const int valid_rows = kGateUp ? kItemRows : min(kItemRows, H - rb * kItemRows);
             // this lane's activation row (gate_up: the token's x row; down: the h row)
-            const int li = min(lane, tl.count - 1);
-            const __half *arow = kGateUp ? act + static_cast<size_t>(sorted_ids[tl.p0 + li] / ktop) * K
-                                         : act + static_cast<size_t>(tl.p0 + li) * K;
+            const __half *arow = kGateUp ? act + static_cast<size_t>(tok) * K
+                                         : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
             const int b = item_ctr & 1;
             mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
             aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
@@ -182,7 +199,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
                 const uint32_t act_bytes = 2u * static_cast<uint32_t>(min(kChunkK, K - kc));
                 const int nkh = (kb + 128 < kbytes) ? 2 : 1;   // skip the K-hi box when wholly past K
                 const int nbox = (kGateUp ? 2 : 1) * nkh;
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], nbox * kBoxBytes + tl.count * act_bytes);
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], nbox * kBoxBytes + cnt * act_bytes);
                 __syncwarp();
                 if (lane == 0) {
                     uint8_t *st = wst + s * kStageBytes;
@@ -195,7 +212,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
                         if (nkh == 2) tma_load_2d(st + 3 * kBoxBytes, &wmap, kb + 128, row_b, &full[s]);
                     }
                 }
-                if (lane < tl.count)
+                if (lane < cnt)
                     bulk_load(ast + s * kActStageBytes + lane * kActPitch, arow + kc, act_bytes, &full[s]);
             }
         }
@@ -331,78 +348,69 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
                     if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
                     if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
                 }
+                // ---------------------------------------------------- weighted top-k combine
+                // The CTA that writes the last of a token's k weighted rows for this row block
+                // sums the k rows in slot order and writes out[t] (integer arrival counters
+                // decide who is last; the floating-point sum itself has a fixed order).
+                __threadfence();                               // my y stores before the arrival below
+                named_bar_sync(2, kItemMTiles * 32);
+                if (warp == 0 && lane < cnt) {
+                    const int t = sorted_ids[tl.p0 + lane] / ktop;
+                    const int old = atomicAdd(&counters[t * row_blocks + rb], 1);
+                    __threadfence();                           // order the reads below after the count
+                    s_last[lane] = (old == ktop - 1) ? t : -1;
+                }
+                named_bar_sync(2, kItemMTiles * 32);
+                const int r = rb * kItemRows + threadIdx.x;
+                for (int i = 0; i < cnt; ++i) {
+                    const int t = s_last[i];
+                    if (t < 0 || threadIdx.x >= kItemRows || r >= rows_total) continue;
+                    float a = 0.f;
+                    for (int jj = 0; jj < ktop; ++jj)
+                        a += __ldcg(yout + (static_cast<size_t>(t) * ktop + jj) * H + r);
+                    out[static_cast<size_t>(t) * H + r] = __float2bfloat16_rn(a);
+                }
             }
         }
     }
 }
 
-// out[t] = bf16( sum_j y[t*k + j] ), j ascending; y already carries the routing weight.
-__global__ void combine_kernel(const float *__restrict__ y, __nv_bfloat16 *__restrict__ out, const int *status,
-                               int32_t *status_out, int M, int H, int k)
-{
-    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx == 0 && status_out) *status_out = *status;
-    const int per_row = H / 8;
-    if (idx >= static_cast<size_t>(M) * per_row) return;
-    const int t = static_cast<int>(idx / per_row);
-    const int c = static_cast<int>(idx - static_cast<size_t>(t) * per_row) * 8;
-    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-        const float4 *p = reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H + c);
-        const float4 u = p[0], v = p[1];
-        a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
-        a[4] += v.x; a[5] += v.y; a[6] += v.z; a[7] += v.w;
-    }
-    __nv_bfloat162 o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
-    *reinterpret_cast<uint4 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint4 *>(o);
-}
-
 template <bool kGateUp>
 static cudaError_t launch_grouped(const CUtensorMap &map, const uint8_t *scales, const __half *act,
                                   const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
-                                  const int *n_tiles, __half *h, float *y, int *status, int K, int I, int H, int ktop,
-                                  int max_tiles, cudaStream_t s)
+                                  const int *n_tiles, __half *h, float *y, int *counters, void *out, int *status,
+                                  int32_t *status_out, int K, int I, int H, int ktop, int max_tiles, cudaStream_t s,
+                                  bool pdl)
 {
     const SmemPlan plan = smem_plan(K);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
     if (e != cudaSuccess) return e;
-    const long long row_blocks = kGateUp ? I / 32 : (H + kItemRows - 1) / kItemRows;
+    const long long row_blocks = kGateUp ? I / 32 : down_row_blocks(H);
     const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
-    const int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
-    grouped_mxfp4_kernel<kGateUp><<<grid > 0 ? grid : 1, kThreads, plan.total, s>>>(
-        map, scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, K, I, H, ktop);
-    return cudaGetLastError();
+    int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
+    if (grid < 1) grid = 1;
+    return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, scales, act,
+                     sorted_ids, topk_w, tiles, n_tiles, h, y, counters, static_cast<__nv_bfloat16 *>(out), status,
+                     status_out, K, I, H, ktop);
 }
 
 int grouped_smem_bytes(int K) { return smem_plan(K).total; }
 
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const uint8_t *w13_s, const __half *x16,
-                           const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, __half *h,
-                           int *status, int H, int I, int k, int max_tiles, cudaStream_t s)
+                           const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int32_t *status_out,
+                           int H, int I, int max_tiles, cudaStream_t s, bool pdl)
 {
-    return launch_grouped<true>(w13_map, w13_s, x16, sorted_ids, nullptr, tiles, n_tiles, h, nullptr, status, H, I,
-                                H, k, max_tiles, s);
+    return launch_grouped<true>(w13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, nullptr, nullptr,
+                                status, status_out, H, I, H, 1, max_tiles, s, pdl);
 }
 
-cudaError_t launch_down(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
-                        const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
-                        int H, int I, int max_tiles, cudaStream_t s)
+cudaError_t launch_down_combine(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h,
+                                const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
+                                const int *n_tiles, float *y, int *counters, void *out, int *status,
+                                int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl)
 {
-    return launch_grouped<false>(w2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, status, I, I, H, 1,
-                                 max_tiles, s);
-}
-
-cudaError_t launch_combine(const float *y, void *out, const int *status, int32_t *status_out, int M, int H, int k,
-                           cudaStream_t s)
-{
-    const size_t n = static_cast<size_t>(M) * H / 8;
-    const int threads = 256;
-    const unsigned blocks = static_cast<unsigned>((n + threads - 1) / threads);
-    combine_kernel<<<blocks > 0 ? blocks : 1, threads, 0, s>>>(y, static_cast<__nv_bfloat16 *>(out), status,
-                                                               status_out, M, H, k);
-    return cudaGetLastError();
+    return launch_grouped<false>(w2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, counters, out,
+                                 status, status_out, I, I, H, k, max_tiles, s, pdl);
 }
 
 }  // namespace moe

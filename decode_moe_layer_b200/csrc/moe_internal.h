@@ -27,7 +27,7 @@ constexpr int kKSlots = kConsumerWarps / 2;
 constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact for |h| >= 2^-27
 
 // Router.
-constexpr int kRouteChunkH = 1024;   // H elements per partial-logit chunk
+constexpr int kRouteChunkH = 512;    // H elements per partial-logit chunk
 constexpr int kRouteTokens = 32;     // tokens per router CTA
 
 constexpr int kMaxE = 1024;
@@ -39,35 +39,65 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
     int p0;           // first position in the expert-grouped order
     int count;
     int pad;
+    int tok[kTileTokens];   // token of each assignment (sorted_ids[p0+i] / k); entries >= count repeat the last
 };
 
 // Byte offsets of every buffer inside one call's workspace (256-byte aligned).
 struct Layout {
-    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, total;
+    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, counters,
+        total;
     int route_splits;   // number of H chunks of the router
     int max_tiles;
 };
 
 Layout make_layout(int M, int H, int I, int E, int k);
 
+// Launch with an optional programmatic dependency on the previous kernel in the stream
+// (the kernel must call pdl_wait() before touching what that kernel writes).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                      Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Largest M for which router top-k and the permutation run as one single-CTA kernel.
+constexpr int kFusedSelectMaxM = 256;
+
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
-                                int M, int H, int E, int splits, cudaStream_t s);
-cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E,
-                              int k, int splits, cudaStream_t s);
+                                int32_t *status_out, int *counters, int n_counters_per_token, int M, int H, int E,
+                                int splits, cudaStream_t s);
+cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
+                              int splits, cudaStream_t s, bool pdl);
+cudaError_t launch_route_select_permute(const float *partial, const float *bias, int32_t *ids, float *w,
+                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
+                                        int *n_tiles, int M, int E, int k, int splits, cudaStream_t s, bool pdl);
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos,
-                           ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s);
-cudaError_t launch_build_tiles(const int32_t *offsets, ExpertTile *tiles, int *n_tiles, int *status, int E,
-                               cudaStream_t s);
+                           ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl);
+cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
+                               int *status, int *counters, int n_counters, int E, int k, cudaStream_t s);
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const uint8_t *w13_s, const __half *x16,
-                           const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, __half *h,
-                           int *status, int H, int I, int k, int max_tiles, cudaStream_t s);
-cudaError_t launch_down(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
-                        const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
-                        int H, int I, int max_tiles, cudaStream_t s);
-cudaError_t launch_combine(const float *y, void *out, const int *status, int32_t *status_out, int M, int H, int k,
-                           cudaStream_t s);
+                           const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int32_t *status_out,
+                           int H, int I, int max_tiles, cudaStream_t s, bool pdl);
+cudaError_t launch_down_combine(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h,
+                                const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
+                                const int *n_tiles, float *y, int *counters, void *out, int *status,
+                                int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl);
+
+// Row blocks of the down projection per token (one arrival counter each).
+__host__ __device__ inline int down_row_blocks(int H) { return (H + kItemRows - 1) / kItemRows; }
 
 int num_sms();
 

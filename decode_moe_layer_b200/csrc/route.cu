@@ -1,23 +1,25 @@
 // route.cu -- router select/normalize ("Native router select/normalize" row of
 // "Post-Portfolio Device Attribution", "MTP1 Post-Portfolio Eager-Cycle Profile").
 //
-// Two kernels:
 //  1. route_logits: fp32 partial logits x.W_r^T over H chunks of kRouteChunkH.
 //     Grid (E/8, H chunks, M/32).  A CTA stages its 32 tokens' x chunk in shared
 //     memory once; each warp owns one expert, keeps that expert's W_r chunk in
-//     registers (read from HBM exactly once per token tile) and reduces with a
-//     fixed xor-butterfly.  The CTAs of expert group 0 also write the binary16 copy
-//     of x that the grouped GEMM consumes.
-//  2. route_topk: one warp per token.  Sums the chunk partials in chunk order,
-//     adds the bias, selects the top k by k rounds of a warp argmax over
-//     (value desc, expert id asc), and renormalises with a softmax over the k
+//     registers (read from HBM once per token tile) and reduces with a fixed
+//     xor-butterfly.  The CTAs of expert group 0 also write the binary16 copy of
+//     x that the grouped GEMM consumes, reset the call's status words and zero the
+//     down kernel's arrival counters (no separate zeroing kernel).
+//  2. top-k per token, one warp per token: sum the chunk partials in chunk order,
+//     add the bias, select the top k by k rounds of a warp argmax over
+//     (value desc, expert id asc), and renormalise with a softmax over the k
 //     selected logits (equal to softmax-over-E followed by renormalisation).
+//     Either its own kernel (route_topk), or, for M <= kFusedSelectMaxM, fused
+//     with the route remap into one single-CTA kernel (route_select_permute).
 // Every reduction has a fixed order, so ids and weights are bitwise reproducible.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math_constants.h>
 
-#include "common.cuh"
+#include "permute_impl.cuh"
 
 namespace moe {
 
@@ -32,15 +34,25 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
 
 __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__restrict__ x,
                                                            const float *__restrict__ wr, float *__restrict__ partial,
-                                                           __half *__restrict__ x16, int *status, int M, int H, int E)
+                                                           __half *__restrict__ x16, int *status, int32_t *status_out,
+                                                           int *counters, int counters_per_token, int M, int H, int E)
 {
     extern __shared__ __align__(16) uint16_t xs[];   // [kRouteTokens][kRouteChunkH] bf16 bits
+    pdl_trigger();
     const int split = blockIdx.y;
     const int h0 = split * kRouteChunkH;
     const int len = min(H - h0, kRouteChunkH);        // multiple of 32
     const int t0 = blockIdx.z * kRouteTokens;
     const int nt = min(kRouteTokens, M - t0);
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0 && status) *status = kStatusOk;
+    if (blockIdx.x == 0 && blockIdx.y == 0) {
+        if (blockIdx.z == 0 && threadIdx.x == 0) {
+            if (status) *status = kStatusOk;
+            if (status_out) *status_out = kStatusOk;
+        }
+        if (counters)
+            for (int i = threadIdx.x; i < nt * counters_per_token; i += blockDim.x)
+                counters[t0 * counters_per_token + i] = 0;
+    }
 
     const int vec_per_row = len / 8;
     const bool write_x16 = (blockIdx.x == 0) && (x16 != nullptr);
@@ -80,7 +92,6 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
 #pragma unroll
         for (int i = 0; i < kVec; ++i) {
             const int c = 128 * i + 4 * lane;
-            if (128 * i >= len) break;
             if (c < len) {
 #pragma unroll
                 for (int tt = 0; tt < 8; ++tt) {
@@ -110,14 +121,12 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
     }
 }
 
+// One warp selects token t's top k.  Lane j < k ends with (sel_e, sel_w) of slot j.
 template <int kPerLane>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ partial,
-                                                         const float *__restrict__ bias, int32_t *__restrict__ ids,
-                                                         float *__restrict__ wout, int M, int E, int k, int splits)
+__device__ __forceinline__ void select_topk(const float *__restrict__ partial, const float *__restrict__ bias, int t,
+                                            int M, int E, int k, int splits, int &sel_e, float &sel_w)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= M) return;
+    const int lane = threadIdx.x & 31;
     float v[kPerLane];
 #pragma unroll
     for (int j = 0; j < kPerLane; ++j) {
@@ -132,7 +141,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     }
     uint32_t taken = 0;
     float sel_v = 0.f, vmax = 0.f;
-    int sel_e = 0;
+    sel_e = 0;
     for (int r = 0; r < k; ++r) {
         float bv = -CUDART_INF_F;
         int be = 0x7fffffff;
@@ -160,14 +169,62 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
         }
         if (r == 0) vmax = bv;
     }
-    float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
+    const float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
     float sum = ex;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    sel_w = ex / sum;
+}
+
+template <int kPerLane>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ partial,
+                                                         const float *__restrict__ bias, int32_t *__restrict__ ids,
+                                                         float *__restrict__ wout, int M, int E, int k, int splits)
+{
+    pdl_wait();
+    pdl_trigger();
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= M) return;
+    int sel_e;
+    float sel_w;
+    select_topk<kPerLane>(partial, bias, t, M, E, k, splits, sel_e, sel_w);
     if (lane < k) {
         ids[static_cast<size_t>(t) * k + lane] = sel_e;
-        wout[static_cast<size_t>(t) * k + lane] = ex / sum;
+        wout[static_cast<size_t>(t) * k + lane] = sel_w;
     }
+}
+
+// Top-k of every token (32 warps loop over the tokens) and the route remap, in one CTA.
+template <int kPerLane>
+__global__ void __launch_bounds__(1024, 1)
+route_select_permute_kernel(const float *__restrict__ partial, const float *__restrict__ bias,
+                            int32_t *__restrict__ ids, float *__restrict__ wout, int32_t *__restrict__ offsets,
+                            int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
+                            ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k, int splits,
+                            int n2)
+{
+    extern __shared__ uint32_t keys[];
+    __shared__ int s_off[kMaxE + 1];
+    __shared__ int scan_buf[33];
+    pdl_wait();
+    pdl_trigger();
+    const int n = M * k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = n + threadIdx.x; i < n2; i += blockDim.x) keys[i] = 0xFFFFFFFFu;
+    for (int t = warp; t < M; t += 32) {
+        int sel_e;
+        float sel_w;
+        select_topk<kPerLane>(partial, bias, t, M, E, k, splits, sel_e, sel_w);
+        if (lane < k) {
+            const int f = t * k + lane;
+            ids[f] = sel_e;
+            wout[f] = sel_w;
+            keys[f] = (static_cast<uint32_t>(sel_e) << 16) | static_cast<uint32_t>(f);
+        }
+    }
+    __syncthreads();
+    sort_and_emit(keys, n, n2, E, k, offsets, sorted_ids, inv_pos, tiles, n_tiles, s_off, scan_buf);
 }
 
 __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
@@ -185,28 +242,65 @@ __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restr
 }
 
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
-                                int M, int H, int E, int splits, cudaStream_t s)
+                                int32_t *status_out, int *counters, int counters_per_token, int M, int H, int E,
+                                int splits, cudaStream_t s)
 {
     const size_t smem = static_cast<size_t>(kRouteTokens) * kRouteChunkH * sizeof(uint16_t);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_logits_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     dim3 grid((E + 7) / 8, splits, (M + kRouteTokens - 1) / kRouteTokens);
-    route_logits_kernel<<<grid, 256, smem, s>>>(static_cast<const uint16_t *>(x), router_w, partial, x16, status, M,
-                                                H, E);
+    // first kernel of a call: fully ordered after whatever precedes it in the stream
+    route_logits_kernel<<<grid, 256, smem, s>>>(static_cast<const uint16_t *>(x), router_w, partial, x16, status,
+                                                status_out, counters, counters_per_token, M, H, E);
     return cudaGetLastError();
 }
 
-cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
-                              int splits, cudaStream_t s)
+template <int P>
+static cudaError_t topk_p(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
+                          int splits, cudaStream_t s, bool pdl)
 {
-    dim3 grid((M + 7) / 8);
-    if (E <= 32) route_topk_kernel<1><<<grid, 256, 0, s>>>(partial, bias, ids, w, M, E, k, splits);
-    else if (E <= 64) route_topk_kernel<2><<<grid, 256, 0, s>>>(partial, bias, ids, w, M, E, k, splits);
-    else if (E <= 128) route_topk_kernel<4><<<grid, 256, 0, s>>>(partial, bias, ids, w, M, E, k, splits);
-    else if (E <= 256) route_topk_kernel<8><<<grid, 256, 0, s>>>(partial, bias, ids, w, M, E, k, splits);
-    else if (E <= 512) route_topk_kernel<16><<<grid, 256, 0, s>>>(partial, bias, ids, w, M, E, k, splits);
-    else route_topk_kernel<32><<<grid, 256, 0, s>>>(partial, bias, ids, w, M, E, k, splits);
-    return cudaGetLastError();
+    return launch_ex(route_topk_kernel<P>, dim3((M + 7) / 8), dim3(256), 0, s, pdl, partial, bias, ids, w, M, E, k,
+                     splits);
+}
+
+cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
+                              int splits, cudaStream_t s, bool pdl)
+{
+    if (E <= 32) return topk_p<1>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+    if (E <= 64) return topk_p<2>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+    if (E <= 128) return topk_p<4>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+    if (E <= 256) return topk_p<8>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+    if (E <= 512) return topk_p<16>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+    return topk_p<32>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+}
+
+template <int P>
+static cudaError_t select_permute_p(const float *partial, const float *bias, int32_t *ids, float *w, int32_t *offsets,
+                                    int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles, int *n_tiles, int M,
+                                    int E, int k, int splits, cudaStream_t s, bool pdl)
+{
+    const int n2 = pow2_at_least(M * k);
+    const size_t smem = static_cast<size_t>(n2) * sizeof(uint32_t);
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>),
+                                    static_cast<int>(kMaxAssignments * sizeof(uint32_t)));
+    if (e != cudaSuccess) return e;
+    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(1024), smem, s, pdl, partial, bias, ids, w,
+                     offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, splits, n2);
+}
+
+cudaError_t launch_route_select_permute(const float *partial, const float *bias, int32_t *ids, float *w,
+                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
+                                        int *n_tiles, int M, int E, int k, int splits, cudaStream_t s, bool pdl)
+{
+#define MOE_SEL(P) select_permute_p<P>(partial, bias, ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, \
+                                       splits, s, pdl)
+    if (E <= 32) return MOE_SEL(1);
+    if (E <= 64) return MOE_SEL(2);
+    if (E <= 128) return MOE_SEL(4);
+    if (E <= 256) return MOE_SEL(8);
+    if (E <= 512) return MOE_SEL(16);
+    return MOE_SEL(32);
+#undef MOE_SEL
 }
 
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s)

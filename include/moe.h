@@ -160,18 +160,21 @@ int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *rout
                          int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
-/* Number of kernels one layer call launches (the entries of moe_mxfp4_forward_profile's output). */
-#define MOE_PROFILE_KERNELS 6
+/* Entries of moe_mxfp4_forward_profile's output. */
+#define MOE_PROFILE_KERNELS 5
 
 /*
  * Per-kernel device-time attribution of one layer call, in the manner of the
  * per-kernel buckets of "Post-Portfolio Device Attribution" ("MTP1 Post-Portfolio
  * Eager-Cycle Profile").  Same arguments and results as moe_mxfp4_forward_ex;
- * additionally records a CUDA event before and after each of the
- * MOE_PROFILE_KERNELS launches (router logits, router top-k, route remap,
- * gate_up + clamp-SwiGLU, down, weighted combine), WAITS for the stream to finish
- * (host synchronisation: not for use under stream capture) and writes each
- * kernel's event-to-event time in milliseconds into the HOST array kernel_ms.
+ * additionally records a CUDA event between consecutive launches, WAITS for the
+ * stream to finish (host synchronisation: not for use under stream capture) and
+ * writes into the HOST array kernel_ms the event-to-event milliseconds of:
+ *   [0] router logits, [1] router top-k (fused with the route remap when
+ *   M <= 256), [2] route remap (0 when fused), [3] gate_up + clamp-SwiGLU,
+ *   [4] down + weighted combine.
+ * Kernels run back to back here instead of overlapping their launches as in
+ * moe_mxfp4_forward_ex, so the sum exceeds a normal call's time.
  */
 int moe_mxfp4_forward_profile(const void *x, const float *router_w, const float *router_bias,
                               const uint8_t *w13_q, const uint8_t *w13_s, const uint8_t *w2_q,

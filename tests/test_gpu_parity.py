@@ -101,8 +101,8 @@ def test_gate_up_swiglu(moe, ci, M):
         for j in range(k):
             e = int(rids[t, j])
             q13, s13 = (inp.w13_q[e], inp.w13_s[e]) if not big else inp.expert_weights(e)[:2]
-            _, _, hb = oracle.expert_swiglu(inp.x[t], q13, s13)
-            U.check_h(h_flat[t * k + j], hb, "c%d M=%d h[t=%d,j=%d]" % (ci, M, t, j))
+            g, u, hb = oracle.expert_swiglu(inp.x[t], q13, s13)
+            U.check_h_bound(h_flat[t * k + j], hb, g, u, inp.x[t], q13, s13, "c%d M=%d h[t=%d,j=%d]" % (ci, M, t, j))
     flips = sum(f for w, f, n in U.FLIP_LOG if w.startswith("c%d M=%d " % (ci, M)))
     total = sum(n for w, f, n in U.FLIP_LOG if w.startswith("c%d M=%d " % (ci, M)))
     print("h rounding flips vs the fp64 oracle: %d of %d (%.2f%%)" % (flips, total, 100.0 * flips / total))
