@@ -315,6 +315,9 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     with torch.cuda.stream(stream):
         for i in range(max(10, min(args.steps, 50))):
             flush.fill_(i & 0xFF)
+            # a short device-side sleep queued first lets the host enqueue every kernel and
+            # event of the call before the GPU reaches them: event gaps then hold device time only
+            torch.cuda._sleep(2_000_000)
             _, ms = moe.moe_mxfp4_forward_profile(xb, wr, w13q, w13s, w2q, w2s, k, ws, router_bias=bias, out=out)
             for n, v in ms.items():
                 prof[n].append(v)

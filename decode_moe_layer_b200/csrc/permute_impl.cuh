@@ -45,7 +45,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &t
 
 // sorted_flat(p) returns the flat assignment id at position p of the expert-grouped order.
 template <typename SortedFlat>
-__device__ void emit_tiles(const int *off, int E, int k, ExpertTile *tiles, int *n_tiles, int *scan_buf,
+__device__ inline void emit_tiles(const int *off, int E, int k, ExpertTile *tiles, int *n_tiles, int *scan_buf,
                            SortedFlat sorted_flat)
 {
     const int e = threadIdx.x;
@@ -70,7 +70,7 @@ __device__ void emit_tiles(const int *off, int E, int k, ExpertTile *tiles, int 
 // keys[0..n2) hold the n assignment keys followed by 0xFFFFFFFF padding (n2 a power of two).
 // Sorts them, then writes expert_offsets [E+1], sorted_ids [n], inv_pos [n] and (when
 // tiles != nullptr) the expert tiles.  s_off must hold E+1 ints, scan_buf 33.
-__device__ void sort_and_emit(uint32_t *keys, int n, int n2, int E, int k, int32_t *__restrict__ offsets,
+__device__ inline void sort_and_emit(uint32_t *keys, int n, int n2, int E, int k, int32_t *__restrict__ offsets,
                               int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
                               ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int *s_off, int *scan_buf)
 {
