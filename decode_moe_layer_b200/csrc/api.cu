@@ -1,6 +1,7 @@
 // api.cu -- the C ABI of libmoe.so (declared in include/moe.h): argument
 // validation, workspace layout and ownership, TMA descriptor encoding, and the
 // enqueue order of the layer's kernels on the caller's stream.
+#include <cstring>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -8,7 +9,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "moe_internal.h"
 
 namespace moe {
@@ -145,6 +146,23 @@ static int make_weight_map(CUtensorMap *map, const void *base, uint64_t rows, ui
     return MOE_OK;
 }
 
+// E8M0 scale matrix viewed as [rows][row_bytes] uint8; boxes of box_rows rows x (kChunkK / 32) bytes,
+// unswizzled.  Only used when row_bytes is a multiple of 16 (per_stage_scales).
+static int make_scale_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, int box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK / 32), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return MOE_OK;
+}
+
 // ------------------------------------------------------------------ library-owned workspaces
 
 static std::mutex g_pool_mu;
@@ -188,12 +206,18 @@ static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x1
                        const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E,
                        int max_tiles, cudaStream_t s, bool pdl)
 {
-    CUtensorMap map;
+    CUtensorMap map, smap;
     // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
     int rc = make_weight_map(&map, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2,
                              kItemRows / 2);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_gate_up(map, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, max_tiles, s, pdl));
+    memset(&smap, 0, sizeof(smap));
+    if (per_stage_scales(H)) {
+        rc = make_scale_map(&smap, w13_s, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 32,
+                            kItemRows / 2);
+        if (rc != MOE_OK) return rc;
+    }
+    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, max_tiles, s, pdl));
     return MOE_OK;
 }
 
@@ -202,10 +226,15 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
                     void *out, int *status, int32_t *status_out, int H, int I, int E, int k, int max_tiles,
                     cudaStream_t s, bool pdl)
 {
-    CUtensorMap map;
+    CUtensorMap map, smap;
     int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_down_combine(map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, counters, out, status,
+    memset(&smap, 0, sizeof(smap));
+    if (per_stage_scales(I)) {
+        rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
+        if (rc != MOE_OK) return rc;
+    }
+    MOE_TRY(launch_down_combine(map, smap, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, counters, out, status,
                                 status_out, H, I, k, max_tiles, s, pdl));
     return MOE_OK;
 }

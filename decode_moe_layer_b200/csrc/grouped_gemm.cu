@@ -18,22 +18,26 @@
 //    clamp-SwiGLU and the bf16 rounding in registers.  Items are spread
 //    round-robin over the CTAs; all tiles of one row block are adjacent, so
 //    CTAs that share weights run together and hit L2.
-//  * Producer warp: per 512-K stage, TMA 2-D tiled copies of the item's packed
-//    E2M1 bytes (boxes of 32 or 64 rows x 128 bytes, 128-byte swizzle) into a
-//    6-stage ring of 16 KB, and one 1-D bulk copy per tile token of its binary16
-//    activation chunk (the routed gather: x rows for gate_up, h rows for down);
-//    per item, the 64 E8M0 scale rows into a double buffer (one copy per row at
-//    a padded pitch when rows are 16-byte multiples, so that the 8 row-distinct
-//    scale reads of a warp fall in distinct banks).
-//  * 16 consumer warps = 2 m-tile pairs x 8 K slots.  Per stage a warp takes 2
-//    of the 16 blocks of 32 K for its 2 m-tiles: a thread reads the 32-bit word
-//    q of its rows' 16-byte block (conflict-free thanks to the swizzle), decodes
-//    it with the hardware E2M1 -> f16x2 conversion straight into MMA A-fragment
-//    registers, and runs two m16n8k16 f16 MMAs per block.  Inside a block the K
-//    order is permuted (thread q's word covers K 8q..8q+7) identically for A and
-//    for the activation fragment, so each MMA pair spans exactly one scale block
-//    and the E8M0 scale is applied once to the fp32 partial sum.
-//  * The 8 K slots of an m-tile are reduced through shared memory in slot order.
+//  * Producer warp: per 1024-K stage, TMA 2-D tiled copies of the item's packed
+//    E2M1 bytes -- 4 column boxes of 32 or 64 rows x 128 bytes per row block,
+//    issued together so that each row's 512 contiguous bytes are read at once --
+//    with a 128-byte swizzle into a 3-stage ring of 32 KB; in the same stage a TMA
+//    box of the matching E8M0 scales (when scale rows are 16-byte multiples, else
+//    the item's scale rows once per item), and one 1-D bulk copy per tile token of
+//    its binary16 activation chunk (the routed gather: x rows for gate_up, h rows
+//    for down).
+//  * 16 compute warps = 2 m-tile pairs x 8 K slots.  Per stage a warp takes 4 of
+//    the 32 blocks of 32 K for its 2 m-tiles: a thread reads the 32-bit word q of
+//    its rows' 16-byte block (conflict-free thanks to the swizzle), decodes it with
+//    the hardware E2M1 -> f16x2 conversion straight into MMA A-fragment registers,
+//    and runs two m16n8k16 f16 MMAs per block.  Inside a block the K order is
+//    permuted (thread q's word covers K 8q..8q+7) identically for A and for the
+//    activation fragment, so each MMA pair spans exactly one scale block and the
+//    E8M0 scale is applied once to the fp32 partial sum.  At the end of an item a
+//    warp parks its partial sums in a double-buffered reduction area and moves on.
+//  * 2 epilogue warps sum the 8 K slots in slot order, then gate_up applies
+//    clamp-SwiGLU and stores h; down applies the routing weight, stores the fp32
+//    row and performs the weighted top-k combine (below) -- off the compute path.
 // Activations (x or h) are read as binary16; bf16 x converts exactly for
 // 2^-17 <= |x| <= 65504, h is stored scaled by 2^10 (exact for |h| >= 2^-27,
 // |h| <= 49 so no overflow), E2M1 values are exact in binary16, and products
@@ -45,32 +49,30 @@
 
 namespace moe {
 
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kRedFloats = kKSlots * kItemMTiles * 32 * 4;   // [kslot][m-tile][lane][4]
+constexpr int kThreads = (kComputeWarps + 1 + kEpilogueWarps) * 32;
+constexpr int kProducerWarp = kComputeWarps;
+constexpr int kFirstEpilogueWarp = kComputeWarps + 1;
+constexpr int kRedFloats = kKSlots * kItemMTiles * 32 * 4;   // one buffer: [kslot][m-tile][lane][4]
+constexpr int kBlocksPerStage = kChunkK / 32;
+constexpr int kBlocksPerWarp = kBlocksPerStage / kKSlots;
+static_assert(kBlocksPerWarp * kKSlots == kBlocksPerStage, "stage blocks split evenly over K slots");
+static_assert(8 % kBlocksPerWarp == 0, "a warp's blocks stay inside one 128-byte box column");
 
 struct SmemPlan {
-    int wst_off, act_off, sbuf_off, spitch, sbuf_bytes, red_off, bars_off, total;
+    int wst_off, act_off, sst_off, sbuf_off, sbuf_bytes, red_off, bars_off, total;
 };
-
-// Scale rows are copied one per row at a padded pitch when they are 16-byte
-// multiples, else as one contiguous block (pitch = row length).
-__host__ __device__ inline int scale_pitch(int K)
-{
-    const int kb = K / 32;
-    return (kb % 16 == 0) ? kb + 16 : kb;
-}
 
 __host__ __device__ inline SmemPlan smem_plan(int K)
 {
     SmemPlan p;
     p.wst_off = 0;
     p.act_off = kStages * kStageBytes;
-    p.sbuf_off = p.act_off + kStages * kActStageBytes;
-    p.spitch = scale_pitch(K);
-    p.sbuf_bytes = (kItemRows * p.spitch + 127) / 128 * 128;
+    p.sst_off = p.act_off + kStages * kActStageBytes;
+    p.sbuf_off = p.sst_off + kStages * kStageScaleBytes;
+    p.sbuf_bytes = per_stage_scales(K) ? 0 : (kItemRows * (K / 32) + 127) / 128 * 128;
     p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
-    p.bars_off = p.red_off + kRedFloats * 4;
-    p.total = p.bars_off + (2 * kStages + 4) * 8 + 1024;   // + alignment slack
+    p.bars_off = p.red_off + 2 * kRedFloats * 4;
+    p.total = p.bars_off + (2 * kStages + 8) * 8 + 1024;   // + alignment slack
     return p;
 }
 
@@ -89,12 +91,13 @@ __device__ __forceinline__ __half store_h(float v)
 
 template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ wscale,
-                     const __half *__restrict__ act, const int32_t *__restrict__ sorted_ids,
-                     const float *__restrict__ topk_w, const ExpertTile *__restrict__ tiles,
-                     const int *__restrict__ n_tiles_ptr, __half *__restrict__ hout, float *__restrict__ yout,
-                     int *__restrict__ counters, __nv_bfloat16 *__restrict__ out, int *status_ws,
-                     int32_t *status_out, int K, int I, int H, int ktop)
+grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
+                     const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
+                     const int32_t *__restrict__ sorted_ids, const float *__restrict__ topk_w,
+                     const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
+                     __half *__restrict__ hout, float *__restrict__ yout, int *__restrict__ counters,
+                     __nv_bfloat16 *__restrict__ out, int *status_ws, int32_t *status_out, int K, int I, int H,
+                     int ktop)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -102,30 +105,36 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
     const SmemPlan plan = smem_plan(K);
     uint8_t *wst = smem + plan.wst_off;
     uint8_t *ast = smem + plan.act_off;
+    uint8_t *sst = smem + plan.sst_off;
     uint8_t *sbuf = smem + plan.sbuf_off;
     float *red = reinterpret_cast<float *>(smem + plan.red_off);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bars_off);
-    uint64_t *full = bars, *empty = bars + kStages, *sfull = bars + 2 * kStages, *sempty = sfull + 2;
+    uint64_t *full = bars, *empty = bars + kStages;
+    uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
+    __shared__ int s_last[kTileTokens];      // down: tokens whose row block this CTA completes
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
-    __shared__ int s_last[kTileTokens];      // down: tokens whose row block this CTA completes
     const int rows_total = kGateUp ? I : H;                 // output rows of this projection
     const int row_blocks = kGateUp ? I / 32 : down_row_blocks(H);
-    const int kblocks = K / 32;               // scale bytes per row
-    const int spitch = plan.spitch;
+    const int kblocks = K / 32;                             // scale bytes per row
+    const bool stage_scales = per_stage_scales(K);
     const int n_chunks = (K + kChunkK - 1) / kChunkK;
-    const int kbytes = K / 2;                 // packed bytes per row
-    constexpr int kBoxBytes = (kGateUp ? 32 : 64) * 128;   // one TMA box: rows x 128 bytes
+    const int kbytes = K / 2;                               // packed bytes per row
+    constexpr int kBoxRows = kGateUp ? 32 : 64;
+    constexpr int kBoxBytes = kBoxRows * 128;               // one weight box: rows x 128 bytes
+    constexpr int kScaleBoxBytes = kBoxRows * (kChunkK / 32);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
+            mbar_init(&empty[s], kComputeWarps);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sfull[b], 1);
-            mbar_init(&sempty[b], kConsumerWarps);
+            mbar_init(&sempty[b], kComputeWarps);
+            mbar_init(&rfull[b], kComputeWarps);
+            mbar_init(&rempty[b], kEpilogueWarps);
         }
         fence_barrier_init();
     }
@@ -138,9 +147,12 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
 
     bool aborted = false;
 
-    if (warp == kConsumerWarps) {
+    if (warp == kProducerWarp) {
         // ---------------------------------------------------------------- producer warp
-        if (lane == 0) prefetch_tensormap(&wmap);
+        if (lane == 0) {
+            prefetch_tensormap(&wmap);
+            if (stage_scales) prefetch_tensormap(&smap);
+        }
         int stage_ctr = 0, item_ctr = 0;
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
         int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
@@ -165,20 +177,13 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
             // this lane's activation row (gate_up: the token's x row; down: the h row)
             const __half *arow = kGateUp ? act + static_cast<size_t>(tok) * K
                                          : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
-            const int b = item_ctr & 1;
-            mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
-            aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
-            if (!aborted) {
-                uint8_t *dst = sbuf + b * plan.sbuf_bytes;
-                if (lane == 0) mbar_arrive_expect_tx(&sfull[b], static_cast<uint32_t>(valid_rows * kblocks));
-                __syncwarp();
-                if (spitch != kblocks) {
-                    // one copy per row into the padded pitch (kblocks is a multiple of 16)
-                    for (int r = lane; r < valid_rows; r += 32) {
-                        const int grow = kGateUp ? (r < 32 ? row_a + r : row_b + r - 32) : row_a + r;
-                        bulk_load(dst + r * spitch, wscale + static_cast<size_t>(grow) * kblocks, kblocks, &sfull[b]);
-                    }
-                } else if (lane == 0) {
+            if (!stage_scales) {
+                const int b = item_ctr & 1;
+                mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
+                aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
+                if (!aborted && lane == 0) {
+                    uint8_t *dst = sbuf + b * plan.sbuf_bytes;
+                    mbar_arrive_expect_tx(&sfull[b], static_cast<uint32_t>(valid_rows * kblocks));
                     if (kGateUp) {
                         bulk_load(dst, wscale + static_cast<size_t>(row_a) * kblocks, 32u * kblocks, &sfull[b]);
                         bulk_load(dst + 32 * kblocks, wscale + static_cast<size_t>(row_b) * kblocks, 32u * kblocks,
@@ -197,23 +202,27 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
                 const int kb = c * (kChunkK / 2);
                 const int kc = c * kChunkK;
                 const uint32_t act_bytes = 2u * static_cast<uint32_t>(min(kChunkK, K - kc));
-                const int nkh = (kb + 128 < kbytes) ? 2 : 1;   // skip the K-hi box when wholly past K
-                const int nbox = (kGateUp ? 2 : 1) * nkh;
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], nbox * kBoxBytes + cnt * act_bytes);
+                const int ncols = min(kBoxCols, (kbytes - kb + 127) / 128);   // skip columns wholly past K
+                const int halves = kGateUp ? 2 : 1;
+                const uint32_t bytes = halves * (ncols * kBoxBytes + (stage_scales ? kScaleBoxBytes : 0)) +
+                                       cnt * act_bytes;
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
                 __syncwarp();
-                if (lane == 0) {
-                    uint8_t *st = wst + s * kStageBytes;
-                    // gate_up boxes: 0 = gate K-lo, 1 = gate K-hi, 2 = up K-lo, 3 = up K-hi
-                    // down boxes:    0 = K-lo, 1 = K-hi
-                    tma_load_2d(st, &wmap, kb, row_a, &full[s]);
-                    if (nkh == 2) tma_load_2d(st + kBoxBytes, &wmap, kb + 128, row_a, &full[s]);
-                    if (kGateUp) {
-                        tma_load_2d(st + 2 * kBoxBytes, &wmap, kb, row_b, &full[s]);
-                        if (nkh == 2) tma_load_2d(st + 3 * kBoxBytes, &wmap, kb + 128, row_b, &full[s]);
-                    }
+                uint8_t *st = wst + s * kStageBytes;
+                // gate_up boxes: columns of the gate rows, then columns of the up rows; down: columns
+                if (lane < ncols) {
+                    tma_load_2d(st + lane * kBoxBytes, &wmap, kb + 128 * lane, row_a, &full[s]);
+                    if (kGateUp) tma_load_2d(st + (kBoxCols + lane) * kBoxBytes, &wmap, kb + 128 * lane, row_b, &full[s]);
                 }
-                if (lane < cnt)
-                    bulk_load(ast + s * kActStageBytes + lane * kActPitch, arow + kc, act_bytes, &full[s]);
+                if (stage_scales && lane == 8) {
+                    uint8_t *ss = sst + s * kStageScaleBytes;
+                    tma_load_2d(ss, &smap, kc / 32, row_a, &full[s]);
+                    if (kGateUp) tma_load_2d(ss + kScaleBoxBytes, &smap, kc / 32, row_b, &full[s]);
+                }
+                if (lane >= 16 && lane - 16 < cnt)
+                    bulk_load(ast + s * kActStageBytes + (lane - 16) * kActPitch,
+                              (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc, act_bytes,
+                              &full[s]);
             }
         }
         // let every copy this CTA issued land before the CTA can exit
@@ -224,41 +233,129 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
         return;
     }
 
-    // -------------------------------------------------------------------- consumer warps
+    if (warp >= kFirstEpilogueWarp) {
+        // ---------------------------------------------------------------- epilogue warps
+        const int et = threadIdx.x - kFirstEpilogueWarp * 32;   // 0..63
+        const int ep = warp - kFirstEpilogueWarp;
+        const int g = lane >> 2, q = lane & 3;
+        int item_ctr = 0;
+        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
+            const ExpertTile *tp = tiles + item % n_tiles;
+            const int rb = item / n_tiles;
+            const int cnt = tp->count, p0 = tp->p0;
+            const int b = item_ctr & 1;
+            const float *rbuf = red + b * kRedFloats;
+            mbar_wait(&rfull[b], (item_ctr >> 1) & 1, aborted, status);
+            float4 sums[2];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int j = ep + 2 * m;
+                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int ks = 0; ks < kKSlots; ++ks) {
+                    const float4 v = *reinterpret_cast<const float4 *>(rbuf + ((ks * kItemMTiles + j) * 32 + lane) * 4);
+                    sum.x += v.x;
+                    sum.y += v.y;
+                    sum.z += v.z;
+                    sum.w += v.w;
+                }
+                sums[m] = sum;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&rempty[b]);
+            const int li0 = 2 * q, li1 = li0 + 1;
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int j = ep + 2 * m;
+                float4 sum = sums[m];
+                if (kGateUp) {
+                    // remove the factor 2 carried by e8m0_times2
+                    const int n = rb * 32 + 8 * j + g;
+                    if (li0 < cnt)
+                        hout[static_cast<size_t>(p0 + li0) * I + n] = store_h(clamp_swiglu(0.5f * sum.x, 0.5f * sum.z));
+                    if (li1 < cnt)
+                        hout[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
+                } else {
+                    // remove e8m0_times2's factor 2 and h's 2^10 storage scale
+                    const float unscale = 0.5f / kHScale;
+                    const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
+                    if (li0 < cnt) {
+                        const int f = sorted_ids[p0 + li0];
+                        const float w = topk_w[f] * unscale;
+                        if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
+                        if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
+                    }
+                    if (li1 < cnt) {
+                        const int f = sorted_ids[p0 + li1];
+                        const float w = topk_w[f] * unscale;
+                        if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
+                        if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
+                    }
+                }
+            }
+            if (!kGateUp) {
+                // ---------------------------------------------------- weighted top-k combine
+                // The CTA that writes the last of a token's k weighted rows for this row block
+                // sums the k rows in slot order and writes out[t] (integer arrival counters
+                // decide who is last; the floating-point sum itself has a fixed order).
+                __threadfence();                               // my y stores before the arrival below
+                named_bar_sync(2, kEpilogueWarps * 32);
+                if (et < cnt) {
+                    const int t = tiles[item % n_tiles].tok[et];
+                    const int old = atomicAdd(&counters[t * row_blocks + rb], 1);
+                    __threadfence();                           // order the reads below after the count
+                    s_last[et] = (old == ktop - 1) ? t : -1;
+                }
+                named_bar_sync(2, kEpilogueWarps * 32);
+                const int r = rb * kItemRows + et;
+                for (int i = 0; i < cnt; ++i) {
+                    const int t = s_last[i];
+                    if (t < 0 || r >= rows_total) continue;
+                    float a = 0.f;
+                    for (int jj = 0; jj < ktop; ++jj)
+                        a += __ldcg(yout + (static_cast<size_t>(t) * ktop + jj) * H + r);
+                    out[static_cast<size_t>(t) * H + r] = __float2bfloat16_rn(a);
+                }
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------------- compute warps
     const int g = lane >> 2, q = lane & 3;
     const int pair = warp & 1;              // m-tiles 2*pair, 2*pair+1
-    const int kslot = warp >> 1;            // blocks 2*kslot, 2*kslot+1 of every stage
-    const int khalf = kslot >> 2;           // both blocks lie in the same 128-byte box column
-    const int bb0 = (2 * kslot) & 7;
+    const int kslot = warp >> 1;            // blocks kslot*kBlocksPerWarp .. of every stage
+    const int col = (kslot * kBlocksPerWarp) >> 3;
+    const int bb0 = (kslot * kBlocksPerWarp) & 7;
     const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
     // per m-tile: smem byte offsets (inside a stage) of the top/bottom rows' 16-byte blocks,
-    // and scale-row offsets inside the item's scale buffer
-    int top_off[2], bot_off[2], top_srow[2], bot_srow[2];
+    // and scale-row indices (rows of the item's 64 weight rows)
+    int top_off[2], bot_off[2], top_sr[2], bot_sr[2];
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
         const int j = 2 * pair + m;
         if (kGateUp) {
-            top_off[m] = (0 + khalf) * kBoxBytes + (8 * j + g) * 128;
-            bot_off[m] = (2 + khalf) * kBoxBytes + (8 * j + g) * 128;
-            top_srow[m] = (8 * j + g) * spitch;
-            bot_srow[m] = (32 + 8 * j + g) * spitch;
+            top_off[m] = col * kBoxBytes + (8 * j + g) * 128;
+            bot_off[m] = (kBoxCols + col) * kBoxBytes + (8 * j + g) * 128;
+            top_sr[m] = 8 * j + g;
+            bot_sr[m] = 32 + 8 * j + g;
         } else {
-            top_off[m] = khalf * kBoxBytes + (16 * j + g) * 128;
-            bot_off[m] = khalf * kBoxBytes + (16 * j + 8 + g) * 128;
-            top_srow[m] = (16 * j + g) * spitch;
-            bot_srow[m] = (16 * j + 8 + g) * spitch;
+            top_off[m] = col * kBoxBytes + (16 * j + g) * 128;
+            bot_off[m] = col * kBoxBytes + (16 * j + 8 + g) * 128;
+            top_sr[m] = 16 * j + g;
+            bot_sr[m] = 16 * j + 8 + g;
         }
     }
+    // scale addressing: per stage, row pitch kChunkK/32 bytes and block index within the stage;
+    // per item, row pitch kblocks and the global block index
+    const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
 
     int stage_ctr = 0, item_ctr = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
-        const ExpertTile tl = tiles[item % n_tiles];
-        const int rb = item / n_tiles;
-        const int cnt = tl.count;
         const int b = item_ctr & 1;
-        const uint8_t *sb = sbuf + b * plan.sbuf_bytes;
-        mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
+        const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
+        if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
 
         float acc[2][4];
 #pragma unroll
@@ -271,19 +368,20 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
             mbar_wait(&full[s], (stage_ctr / kStages) & 1, aborted, status);
             const uint8_t *st = wst + s * kStageBytes;
             const uint8_t *xa = ast + s * kActStageBytes + g * kActPitch;   // token g of the tile
-            const int kblk0 = c * (kChunkK / 32) + 2 * kslot;                 // global block index
+            const uint8_t *sc_base = stage_scales ? sst + s * kStageScaleBytes : sbi;
+            const int blk_base = kslot * kBlocksPerWarp;                      // block index within the stage
+            const int sc_col0 = stage_scales ? blk_base : c * kBlocksPerStage + blk_base;
 #pragma unroll
-            for (int bi = 0; bi < 2; ++bi) {
-                const int kblk = kblk0 + bi;
-                if (kblk >= kblocks) continue;
-                const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (2 * kslot + bi) + 8 * q) * 2);
+            for (int bi = 0; bi < kBlocksPerWarp; ++bi) {
+                if (c * kBlocksPerStage + blk_base + bi >= kblocks) continue;
+                const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (blk_base + bi) + 8 * q) * 2);
                 const int sw = (((bb0 + bi) ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
                     const uint32_t wt = *reinterpret_cast<const uint32_t *>(st + top_off[m] + sw);
                     const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_off[m] + sw);
-                    const float st_scale = e8m0_times2(sb[top_srow[m] + kblk]);
-                    const float sb_scale = e8m0_times2(sb[bot_srow[m] + kblk]);
+                    const float st_scale = e8m0_times2(sc_base[top_sr[m] * s_pitch + sc_col0 + bi]);
+                    const float sb_scale = e8m0_times2(sc_base[bot_sr[m] * s_pitch + sc_col0 + bi]);
                     uint32_t t0, t1, t2, t3, u0, u1, u2, u3;
                     e2m1x8_to_f16x2(wt, t0, t1, t2, t3);
                     e2m1x8_to_f16x2(wb, u0, u1, u2, u3);
@@ -302,85 +400,26 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__
             if (lane == 0) mbar_arrive(&empty[s]);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sempty[b]);
+        if (!stage_scales && lane == 0) mbar_arrive(&sempty[b]);
 
-        // ---------------------------------------------------------------- K-slot reduction
-        named_bar_sync(1, kConsumerWarps * 32);
+        // park the K-slot partial sums for the epilogue warps
+        mbar_wait(&rempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
+        float *rbuf = red + b * kRedFloats;
 #pragma unroll
         for (int m = 0; m < 2; ++m)
-            *reinterpret_cast<float4 *>(red + ((kslot * kItemMTiles + 2 * pair + m) * 32 + lane) * 4) =
+            *reinterpret_cast<float4 *>(rbuf + ((kslot * kItemMTiles + 2 * pair + m) * 32 + lane) * 4) =
                 make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-        named_bar_sync(1, kConsumerWarps * 32);
-        if (warp < kItemMTiles) {
-            const int j = warp;
-            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int ks = 0; ks < kKSlots; ++ks) {
-                const float4 v = *reinterpret_cast<const float4 *>(red + ((ks * kItemMTiles + j) * 32 + lane) * 4);
-                sum.x += v.x;
-                sum.y += v.y;
-                sum.z += v.z;
-                sum.w += v.w;
-            }
-            const int li0 = 2 * q, li1 = li0 + 1;
-            if (kGateUp) {
-                // remove the factor 2 carried by e8m0_times2
-                sum.x *= 0.5f;
-                sum.y *= 0.5f;
-                sum.z *= 0.5f;
-                sum.w *= 0.5f;
-                const int n = rb * 32 + 8 * j + g;
-                if (li0 < cnt) hout[static_cast<size_t>(tl.p0 + li0) * I + n] = store_h(clamp_swiglu(sum.x, sum.z));
-                if (li1 < cnt) hout[static_cast<size_t>(tl.p0 + li1) * I + n] = store_h(clamp_swiglu(sum.y, sum.w));
-            } else {
-                // remove e8m0_times2's factor 2 and h's 2^10 storage scale
-                const float unscale = 0.5f / kHScale;
-                const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
-                if (li0 < cnt) {
-                    const int f = sorted_ids[tl.p0 + li0];
-                    const float w = topk_w[f] * unscale;
-                    if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
-                    if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
-                }
-                if (li1 < cnt) {
-                    const int f = sorted_ids[tl.p0 + li1];
-                    const float w = topk_w[f] * unscale;
-                    if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
-                    if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
-                }
-                // ---------------------------------------------------- weighted top-k combine
-                // The CTA that writes the last of a token's k weighted rows for this row block
-                // sums the k rows in slot order and writes out[t] (integer arrival counters
-                // decide who is last; the floating-point sum itself has a fixed order).
-                __threadfence();                               // my y stores before the arrival below
-                named_bar_sync(2, kItemMTiles * 32);
-                if (warp == 0 && lane < cnt) {
-                    const int t = sorted_ids[tl.p0 + lane] / ktop;
-                    const int old = atomicAdd(&counters[t * row_blocks + rb], 1);
-                    __threadfence();                           // order the reads below after the count
-                    s_last[lane] = (old == ktop - 1) ? t : -1;
-                }
-                named_bar_sync(2, kItemMTiles * 32);
-                const int r = rb * kItemRows + threadIdx.x;
-                for (int i = 0; i < cnt; ++i) {
-                    const int t = s_last[i];
-                    if (t < 0 || threadIdx.x >= kItemRows || r >= rows_total) continue;
-                    float a = 0.f;
-                    for (int jj = 0; jj < ktop; ++jj)
-                        a += __ldcg(yout + (static_cast<size_t>(t) * ktop + jj) * H + r);
-                    out[static_cast<size_t>(t) * H + r] = __float2bfloat16_rn(a);
-                }
-            }
-        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfull[b]);
     }
 }
 
 template <bool kGateUp>
-static cudaError_t launch_grouped(const CUtensorMap &map, const uint8_t *scales, const __half *act,
-                                  const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
-                                  const int *n_tiles, __half *h, float *y, int *counters, void *out, int *status,
-                                  int32_t *status_out, int K, int I, int H, int ktop, int max_tiles, cudaStream_t s,
-                                  bool pdl)
+static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
+                                  const __half *act, const int32_t *sorted_ids, const float *topk_w,
+                                  const ExpertTile *tiles, const int *n_tiles, __half *h, float *y, int *counters,
+                                  void *out, int *status, int32_t *status_out, int K, int I, int H, int ktop,
+                                  int max_tiles, cudaStream_t s, bool pdl)
 {
     const SmemPlan plan = smem_plan(K);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
@@ -389,28 +428,29 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const uint8_t *scales,
     const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
     int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     if (grid < 1) grid = 1;
-    return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, scales, act,
-                     sorted_ids, topk_w, tiles, n_tiles, h, y, counters, static_cast<__nv_bfloat16 *>(out), status,
-                     status_out, K, I, H, ktop);
+    return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, smap,
+                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, counters,
+                     static_cast<__nv_bfloat16 *>(out), status, status_out, K, I, H, ktop);
 }
 
 int grouped_smem_bytes(int K) { return smem_plan(K).total; }
 
-cudaError_t launch_gate_up(const CUtensorMap &w13_map, const uint8_t *w13_s, const __half *x16,
-                           const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int32_t *status_out,
-                           int H, int I, int max_tiles, cudaStream_t s, bool pdl)
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
+                           const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
+                           int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl)
 {
-    return launch_grouped<true>(w13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, nullptr, nullptr,
-                                status, status_out, H, I, H, 1, max_tiles, s, pdl);
+    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, nullptr,
+                                nullptr, status, status_out, H, I, H, 1, max_tiles, s, pdl);
 }
 
-cudaError_t launch_down_combine(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h,
-                                const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
-                                const int *n_tiles, float *y, int *counters, void *out, int *status,
-                                int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl)
+cudaError_t launch_down_combine(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s,
+                                const __half *h, const int32_t *sorted_ids, const float *topk_w,
+                                const ExpertTile *tiles, const int *n_tiles, float *y, int *counters, void *out,
+                                int *status, int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s,
+                                bool pdl)
 {
-    return launch_grouped<false>(w2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, counters, out,
-                                 status, status_out, I, I, H, k, max_tiles, s, pdl);
+    return launch_grouped<false>(w2_map, s2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, counters,
+                                 out, status, status_out, I, I, H, k, max_tiles, s, pdl);
 }
 
 }  // namespace moe

@@ -17,14 +17,21 @@ constexpr int kStatusTimeout = -5;
 constexpr int kTileTokens = 8;       // assignments per expert tile (one MMA n-tile)
 constexpr int kItemMTiles = 4;       // MMA m-tiles (16 weight rows each) per work item
 constexpr int kItemRows = 16 * kItemMTiles;
-constexpr int kChunkK = 512;         // K elements per pipeline stage (256 bytes of E2M1 per row)
-constexpr int kStageBytes = kItemRows * kChunkK / 2;   // packed weights of one stage (16 KB)
+constexpr int kChunkK = 1024;        // K elements per pipeline stage (512 bytes of E2M1 per row)
+constexpr int kBoxCols = kChunkK / 256;              // 128-byte TMA box columns per stage
+constexpr int kStageBytes = kItemRows * kChunkK / 2; // packed weights of one stage (32 KB)
+constexpr int kStageScaleBytes = kItemRows * kChunkK / 32;   // E8M0 bytes of one stage (per-stage mode)
 constexpr int kActPitch = kChunkK * 2 + 64;         // one token's binary16 chunk, padded against bank conflicts
 constexpr int kActStageBytes = kTileTokens * kActPitch;
-constexpr int kStages = 6;
-constexpr int kConsumerWarps = 16;   // 2 m-tile pairs x 8 K slots
-constexpr int kKSlots = kConsumerWarps / 2;
+constexpr int kStages = 3;
+constexpr int kComputeWarps = 16;    // 2 m-tile pairs x 8 K slots
+constexpr int kKSlots = kComputeWarps / 2;
+constexpr int kEpilogueWarps = 2;
 constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact for |h| >= 2^-27
+
+// E8M0 scales travel with each stage (a TMA box of the scale matrix) when a scale row is a
+// multiple of 16 bytes; otherwise the item's scale rows are copied once per item.
+__host__ __device__ inline bool per_stage_scales(int K) { return (K / 32) % 16 == 0; }
 
 // Router.
 constexpr int kRouteChunkH = 512;    // H elements per partial-logit chunk
@@ -88,10 +95,10 @@ cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
                                int *status, int *counters, int n_counters, int E, int k, cudaStream_t s);
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
-cudaError_t launch_gate_up(const CUtensorMap &w13_map, const uint8_t *w13_s, const __half *x16,
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s, const __half *x16,
                            const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int32_t *status_out,
                            int H, int I, int max_tiles, cudaStream_t s, bool pdl);
-cudaError_t launch_down_combine(const CUtensorMap &w2_map, const uint8_t *w2_s, const __half *h,
+cudaError_t launch_down_combine(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
                                 const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
                                 const int *n_tiles, float *y, int *counters, void *out, int *status,
                                 int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl);
