@@ -380,7 +380,7 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
                      "algorithmic_bytes_per_launch": dom_bytes},
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": M * H * 2,
                 "path": "pinned host x -> moe_mxfp4_forward_ex (eager C-ABI call) -> pinned host out"},
-        "gpu_launches": (4 if M <= 256 else 5) * args.steps,
+        "gpu_launches": (5 if M <= 64 else 6) * args.steps,
         "clocks": clk,
     }
     if baselines and rank == 0 and world == 1 and not args.no_cpu_baseline:

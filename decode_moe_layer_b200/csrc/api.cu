@@ -79,7 +79,6 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.n_tiles = take(4);
     L.h = take(n * I * 2);
     L.y = take(n * H * sizeof(float));
-    L.counters = take(static_cast<size_t>(M) * down_row_blocks(H) * sizeof(int));
     L.total = off;
     return L;
 }
@@ -221,24 +220,6 @@ static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x1
     return MOE_OK;
 }
 
-static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
-                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *counters,
-                    void *out, int *status, int32_t *status_out, int H, int I, int E, int k, int max_tiles,
-                    cudaStream_t s, bool pdl)
-{
-    CUtensorMap map, smap;
-    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
-    if (rc != MOE_OK) return rc;
-    memset(&smap, 0, sizeof(smap));
-    if (per_stage_scales(I)) {
-        rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
-        if (rc != MOE_OK) return rc;
-    }
-    MOE_TRY(launch_down_combine(map, smap, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, counters, out, status,
-                                status_out, H, I, k, max_tiles, s, pdl));
-    return MOE_OK;
-}
-
 // Optional per-launch event marks (profiling entry point only).
 struct Marks {
     cudaEvent_t ev[MOE_PROFILE_KERNELS + 1];
@@ -250,6 +231,26 @@ struct Marks {
     do {                                                \
         if (m) MOE_TRY((m)->mark(s));                   \
     } while (0)
+
+static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, void *out, int *status,
+                    int32_t *status_out, int M, int H, int I, int E, int k, int max_tiles, cudaStream_t s, bool pdl,
+                    Marks *marks)
+{
+    CUtensorMap map, smap;
+    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
+    if (rc != MOE_OK) return rc;
+    memset(&smap, 0, sizeof(smap));
+    if (per_stage_scales(I)) {
+        rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
+        if (rc != MOE_OK) return rc;
+    }
+    MOE_TRY(launch_down(map, smap, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, status_out, H, I, max_tiles,
+                        s, pdl));
+    MOE_TRY(launch_combine(y, out, M, H, k, s, pdl));
+    MOE_MARK(marks, s);
+    return MOE_OK;
+}
 
 static int forward_impl(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
                         const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H,
@@ -268,7 +269,6 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     __half *h = reinterpret_cast<__half *>(ws + L.h);
     float *y = reinterpret_cast<float *>(ws + L.y);
-    int *counters = reinterpret_cast<int *>(ws + L.counters);
     // The first kernel is ordered after everything before it on the stream; each later
     // kernel of the call is launched early (programmatic dependent launch) and waits on
     // device for its predecessor.  Event marks (profiling) break that overlap, so the
@@ -276,8 +276,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     const bool pdl = (marks == nullptr);
 
     MOE_MARK(marks, s);
-    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, counters, down_row_blocks(H), M, H, E,
-                                L.route_splits, s));
+    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, M, H, E, L.route_splits, s));
     MOE_MARK(marks, s);
     if (M <= kFusedSelectMaxM) {
         MOE_TRY(launch_route_select_permute(partial, router_bias, ids, tw, offsets, sorted_ids, inv_pos, tiles,
@@ -292,11 +291,8 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
     MOE_MARK(marks, s);
-    rc = run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, counters, out, status, status_out, H, I, E, k,
-                  L.max_tiles, s, pdl);
-    if (rc != MOE_OK) return rc;
-    MOE_MARK(marks, s);
-    return MOE_OK;
+    return run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, out, status, status_out, M, H, I, E, k,
+                    L.max_tiles, s, pdl, marks);
 }
 
 static int check_forward_args(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
@@ -363,7 +359,7 @@ int moe_route(const void *x_bf16, const float *router_w, const float *router_bia
     if (rc != MOE_OK) return rc;
     float *partial = reinterpret_cast<float *>(ws + L.partial);
     MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, reinterpret_cast<int *>(ws + L.status), nullptr,
-                                nullptr, 0, M, H, E, L.route_splits, stream));
+                                M, H, E, L.route_splits, stream));
     MOE_TRY(launch_route_topk(partial, router_bias, topk_ids, topk_w, M, E, k, L.route_splits, stream, false));
     return MOE_OK;
 }
@@ -402,7 +398,7 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, nullptr, nullptr, 0, E, k, stream));
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, nullptr, E, k, stream));
     return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E,
                        L.max_tiles, stream, false);
 }
@@ -427,11 +423,9 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
-    int *counters = reinterpret_cast<int *>(ws + L.counters);
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, counters, M * down_row_blocks(H),
-                               E, k, stream));
-    return run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, counters,
-                    out_bf16, status, nullptr, H, I, E, k, L.max_tiles, stream, false);
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
+    return run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, out_bf16,
+                    status, nullptr, M, H, I, E, k, L.max_tiles, stream, false, nullptr);
 }
 
 int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,

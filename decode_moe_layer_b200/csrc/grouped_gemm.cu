@@ -36,8 +36,9 @@
 //    E8M0 scale is applied once to the fp32 partial sum.  At the end of an item a
 //    warp parks its partial sums in a double-buffered reduction area and moves on.
 //  * 2 epilogue warps sum the 8 K slots in slot order, then gate_up applies
-//    clamp-SwiGLU and stores h; down applies the routing weight, stores the fp32
-//    row and performs the weighted top-k combine (below) -- off the compute path.
+//    clamp-SwiGLU and stores h; down applies the routing weight and stores the
+//    fp32 row of the assignment -- off the compute path.  The weighted top-k
+//    combine that follows is its own small kernel (combine_kernel).
 // Activations (x or h) are read as binary16; bf16 x converts exactly for
 // 2^-17 <= |x| <= 65504, h is stored scaled by 2^10 (exact for |h| >= 2^-27,
 // |h| <= 49 so no overflow), E2M1 values are exact in binary16, and products
@@ -95,9 +96,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                      const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
                      const int32_t *__restrict__ sorted_ids, const float *__restrict__ topk_w,
                      const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
-                     __half *__restrict__ hout, float *__restrict__ yout, int *__restrict__ counters,
-                     __nv_bfloat16 *__restrict__ out, int *status_ws, int32_t *status_out, int K, int I, int H,
-                     int ktop)
+                     __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out, int K,
+                     int I, int H)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -111,7 +111,6 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bars_off);
     uint64_t *full = bars, *empty = bars + kStages;
     uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
-    __shared__ int s_last[kTileTokens];      // down: tokens whose row block this CTA completes
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
@@ -293,30 +292,6 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     }
                 }
             }
-            if (!kGateUp) {
-                // ---------------------------------------------------- weighted top-k combine
-                // The CTA that writes the last of a token's k weighted rows for this row block
-                // sums the k rows in slot order and writes out[t] (integer arrival counters
-                // decide who is last; the floating-point sum itself has a fixed order).
-                __threadfence();                               // my y stores before the arrival below
-                named_bar_sync(2, kEpilogueWarps * 32);
-                if (et < cnt) {
-                    const int t = tiles[item % n_tiles].tok[et];
-                    const int old = atomicAdd(&counters[t * row_blocks + rb], 1);
-                    __threadfence();                           // order the reads below after the count
-                    s_last[et] = (old == ktop - 1) ? t : -1;
-                }
-                named_bar_sync(2, kEpilogueWarps * 32);
-                const int r = rb * kItemRows + et;
-                for (int i = 0; i < cnt; ++i) {
-                    const int t = s_last[i];
-                    if (t < 0 || r >= rows_total) continue;
-                    float a = 0.f;
-                    for (int jj = 0; jj < ktop; ++jj)
-                        a += __ldcg(yout + (static_cast<size_t>(t) * ktop + jj) * H + r);
-                    out[static_cast<size_t>(t) * H + r] = __float2bfloat16_rn(a);
-                }
-            }
         }
         return;
     }
@@ -414,12 +389,34 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     }
 }
 
+// out[t] = bf16( sum_j y[t*k + j] ), slots j ascending (a fixed order, no atomics); y already
+// carries the routing weight.  Four outputs per thread.
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, __nv_bfloat16 *__restrict__ out,
+                                                      int M, int H, int k)
+{
+    pdl_wait();
+    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int per_row = H / 4;
+    if (idx >= static_cast<size_t>(M) * per_row) return;
+    const int t = static_cast<int>(idx / per_row);
+    const int c = static_cast<int>(idx - static_cast<size_t>(t) * per_row) * 4;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+        const float4 v = *reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H + c);
+        a.x += v.x;
+        a.y += v.y;
+        a.z += v.z;
+        a.w += v.w;
+    }
+    __nv_bfloat162 o[2] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w)};
+    *reinterpret_cast<uint2 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint2 *>(o);
+}
+
 template <bool kGateUp>
 static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
                                   const __half *act, const int32_t *sorted_ids, const float *topk_w,
-                                  const ExpertTile *tiles, const int *n_tiles, __half *h, float *y, int *counters,
-                                  void *out, int *status, int32_t *status_out, int K, int I, int H, int ktop,
-                                  int max_tiles, cudaStream_t s, bool pdl)
+                                  const ExpertTile *tiles, const int *n_tiles, __half *h, float *y, int *status,
+                                  int32_t *status_out, int K, int I, int H, int max_tiles, cudaStream_t s, bool pdl)
 {
     const SmemPlan plan = smem_plan(K);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
@@ -429,8 +426,7 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &sma
     int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     if (grid < 1) grid = 1;
     return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, smap,
-                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, counters,
-                     static_cast<__nv_bfloat16 *>(out), status, status_out, K, I, H, ktop);
+                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, status_out, K, I, H);
 }
 
 int grouped_smem_bytes(int K) { return smem_plan(K).total; }
@@ -439,18 +435,25 @@ cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_ma
                            const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
                            int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl)
 {
-    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, nullptr,
-                                nullptr, status, status_out, H, I, H, 1, max_tiles, s, pdl);
+    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, status,
+                                status_out, H, I, H, max_tiles, s, pdl);
 }
 
-cudaError_t launch_down_combine(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s,
-                                const __half *h, const int32_t *sorted_ids, const float *topk_w,
-                                const ExpertTile *tiles, const int *n_tiles, float *y, int *counters, void *out,
-                                int *status, int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s,
-                                bool pdl)
+cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
+                        const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles, const int *n_tiles,
+                        float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
+                        bool pdl)
 {
-    return launch_grouped<false>(w2_map, s2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, counters,
-                                 out, status, status_out, I, I, H, k, max_tiles, s, pdl);
+    return launch_grouped<false>(w2_map, s2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, status,
+                                 status_out, I, I, H, max_tiles, s, pdl);
+}
+
+cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl)
+{
+    const size_t n = static_cast<size_t>(M) * H / 4;
+    const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+    return launch_ex(combine_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, y,
+                     static_cast<__nv_bfloat16 *>(out), M, H, k);
 }
 
 }  // namespace moe

@@ -51,8 +51,7 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
 
 // Byte offsets of every buffer inside one call's workspace (256-byte aligned).
 struct Layout {
-    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, counters,
-        total;
+    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, total;
     int route_splits;   // number of H chunks of the router
     int max_tiles;
 };
@@ -79,12 +78,12 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 }
 
 // Largest M for which router top-k and the permutation run as one single-CTA kernel.
-constexpr int kFusedSelectMaxM = 256;
+constexpr int kFusedSelectMaxM = 64;
+constexpr int kFusedSelectThreads = 512;
 
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
-                                int32_t *status_out, int *counters, int n_counters_per_token, int M, int H, int E,
-                                int splits, cudaStream_t s);
+                                int32_t *status_out, int M, int H, int E, int splits, cudaStream_t s);
 cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
                               int splits, cudaStream_t s, bool pdl);
 cudaError_t launch_route_select_permute(const float *partial, const float *bias, int32_t *ids, float *w,
@@ -93,15 +92,16 @@ cudaError_t launch_route_select_permute(const float *partial, const float *bias,
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos,
                            ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
-                               int *status, int *counters, int n_counters, int E, int k, cudaStream_t s);
+                               int *status, int E, int k, cudaStream_t s);
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
-cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s, const __half *x16,
-                           const ExpertTile *tiles, const int *n_tiles, __half *h, int *status, int32_t *status_out,
-                           int H, int I, int max_tiles, cudaStream_t s, bool pdl);
-cudaError_t launch_down_combine(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                                const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles,
-                                const int *n_tiles, float *y, int *counters, void *out, int *status,
-                                int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl);
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
+                           const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
+                           int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl);
+cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
+                        const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles, const int *n_tiles,
+                        float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
+                        bool pdl);
+cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl);
 
 // Row blocks of the down projection per token (one arrival counter each).
 __host__ __device__ inline int down_row_blocks(int H) { return (H + kItemRows - 1) / kItemRows; }

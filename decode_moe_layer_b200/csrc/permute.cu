@@ -27,17 +27,15 @@ __global__ void __launch_bounds__(1024, 1) permute_kernel(const int32_t *__restr
     sort_and_emit(keys, n, n2, E, k, offsets, sorted_ids, inv_pos, tiles, n_tiles, s_off, scan_buf);
 }
 
-// Expert tiles from given offsets / sorted ids; also resets the call's status word and
-// the down kernel's per-(token, row block) arrival counters.
+// Expert tiles from given offsets / sorted ids; also resets the call's status word.
 __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__restrict__ offsets,
                                                               const int32_t *__restrict__ sorted_ids,
                                                               ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles,
-                                                              int *status, int *counters, int n_counters, int E, int k)
+                                                              int *status, int E, int k)
 {
     __shared__ int s_off[kMaxE + 1];
     __shared__ int scan_buf[33];
     if (threadIdx.x == 0 && status) *status = kStatusOk;
-    for (int i = threadIdx.x; i < n_counters; i += blockDim.x) counters[i] = 0;
     for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
     emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
@@ -57,9 +55,9 @@ cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted
 }
 
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
-                               int *status, int *counters, int n_counters, int E, int k, cudaStream_t s)
+                               int *status, int E, int k, cudaStream_t s)
 {
-    build_tiles_kernel<<<1, 1024, 0, s>>>(offsets, sorted_ids, tiles, n_tiles, status, counters, n_counters, E, k);
+    build_tiles_kernel<<<1, 1024, 0, s>>>(offsets, sorted_ids, tiles, n_tiles, status, E, k);
     return cudaGetLastError();
 }
 

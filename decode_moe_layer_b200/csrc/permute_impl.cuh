@@ -8,17 +8,17 @@
 // yields the same bytes).  Expert offsets are lower bounds found by binary
 // search in the sorted keys, and the expert tiles that drive the grouped GEMMs
 // come from a block-wide exclusive scan of ceil(count_e / kTileTokens).  No
-// atomics.  All functions are called by every thread of a 1024-thread CTA.
+// atomics.  All functions are called by every thread of the CTA (a multiple of 32 threads).
 #pragma once
 
 #include "common.cuh"
 
 namespace moe {
 
-// Exclusive scan of one value per thread over a 1024-thread block.
+// Exclusive scan of one value per thread over the block (blockDim.x a multiple of 32, <= 1024).
 __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &total)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     int incl = v;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -28,14 +28,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &t
     if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        int w = warp_tot[lane];
+        int w = lane < nwarps ? warp_tot[lane] : 0;
         int wi = w;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int o = __shfl_up_sync(0xffffffffu, wi, off);
             if (lane >= off) wi += o;
         }
-        warp_tot[lane] = wi - w;        // exclusive prefix of the warp totals
+        if (lane < nwarps) warp_tot[lane] = wi - w;      // exclusive prefix of the warp totals
         if (lane == 31) warp_tot[32] = wi;
     }
     __syncthreads();
@@ -44,25 +44,29 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &t
 }
 
 // sorted_flat(p) returns the flat assignment id at position p of the expert-grouped order.
+// Each thread owns a contiguous run of ceil(E / blockDim) experts.
 template <typename SortedFlat>
 __device__ inline void emit_tiles(const int *off, int E, int k, ExpertTile *tiles, int *n_tiles, int *scan_buf,
-                           SortedFlat sorted_flat)
+                                  SortedFlat sorted_flat)
 {
-    const int e = threadIdx.x;
-    int cnt = 0;
-    if (e < E) cnt = off[e + 1] - off[e];
-    const int nt = (cnt + kTileTokens - 1) / kTileTokens;
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
+    int mine = 0;
+    for (int e = e0; e < e1; ++e) mine += (off[e + 1] - off[e] + kTileTokens - 1) / kTileTokens;
     int total = 0;
-    const int base = block_exclusive_scan(nt, scan_buf, total);
-    for (int i = 0; i < nt; ++i) {
-        ExpertTile tl;
-        tl.expert = e;
-        tl.p0 = off[e] + i * kTileTokens;
-        tl.count = min(kTileTokens, cnt - i * kTileTokens);
-        tl.pad = 0;
+    int base = block_exclusive_scan(mine, scan_buf, total);
+    for (int e = e0; e < e1; ++e) {
+        const int cnt = off[e + 1] - off[e];
+        for (int i = 0; i * kTileTokens < cnt; ++i) {
+            ExpertTile tl;
+            tl.expert = e;
+            tl.p0 = off[e] + i * kTileTokens;
+            tl.count = min(kTileTokens, cnt - i * kTileTokens);
+            tl.pad = 0;
 #pragma unroll
-        for (int j = 0; j < kTileTokens; ++j) tl.tok[j] = sorted_flat(tl.p0 + min(j, tl.count - 1)) / k;
-        tiles[base + i] = tl;
+            for (int j = 0; j < kTileTokens; ++j) tl.tok[j] = sorted_flat(tl.p0 + min(j, tl.count - 1)) / k;
+            tiles[base++] = tl;
+        }
     }
     if (threadIdx.x == 0) *n_tiles = total;
 }

@@ -6,8 +6,7 @@
 //     memory once; each warp owns one expert, keeps that expert's W_r chunk in
 //     registers (read from HBM once per token tile) and reduces with a fixed
 //     xor-butterfly.  The CTAs of expert group 0 also write the binary16 copy of
-//     x that the grouped GEMM consumes, reset the call's status words and zero the
-//     down kernel's arrival counters (no separate zeroing kernel).
+//     x that the grouped GEMM consumes and reset the call's status words.
 //  2. top-k per token, one warp per token: sum the chunk partials in chunk order,
 //     add the bias, select the top k by k rounds of a warp argmax over
 //     (value desc, expert id asc), and renormalise with a softmax over the k
@@ -35,7 +34,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
 __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__restrict__ x,
                                                            const float *__restrict__ wr, float *__restrict__ partial,
                                                            __half *__restrict__ x16, int *status, int32_t *status_out,
-                                                           int *counters, int counters_per_token, int M, int H, int E)
+                                                           int M, int H, int E)
 {
     extern __shared__ __align__(16) uint16_t xs[];   // [kRouteTokens][kRouteChunkH] bf16 bits
     pdl_trigger();
@@ -44,14 +43,21 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
     const int len = min(H - h0, kRouteChunkH);        // multiple of 32
     const int t0 = blockIdx.z * kRouteTokens;
     const int nt = min(kRouteTokens, M - t0);
-    if (blockIdx.x == 0 && blockIdx.y == 0) {
-        if (blockIdx.z == 0 && threadIdx.x == 0) {
-            if (status) *status = kStatusOk;
-            if (status_out) *status_out = kStatusOk;
-        }
-        if (counters)
-            for (int i = threadIdx.x; i < nt * counters_per_token; i += blockDim.x)
-                counters[t0 * counters_per_token + i] = 0;
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
+        if (status) *status = kStatusOk;
+        if (status_out) *status_out = kStatusOk;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 8 + warp;
+
+    // this warp's expert chunk of W_r, requested before the x staging so both loads overlap
+    constexpr int kVec = kRouteChunkH / 128;   // float4 per lane
+    float4 w[kVec];
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) {
+        const int c = 128 * i + 4 * lane;
+        w[i] = (e < E && c < len) ? *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(e) * H + h0 + c)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
     const int vec_per_row = len / 8;
@@ -72,18 +78,7 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
     }
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 8 + warp;
     if (e >= E) return;
-
-    constexpr int kVec = kRouteChunkH / 128;   // float4 per lane
-    float4 w[kVec];
-#pragma unroll
-    for (int i = 0; i < kVec; ++i) {
-        const int c = 128 * i + 4 * lane;
-        w[i] = (c < len) ? *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(e) * H + h0 + c)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
 
     for (int tg = 0; tg < nt; tg += 8) {
         float acc[8];
@@ -197,7 +192,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
 
 // Top-k of every token (32 warps loop over the tokens) and the route remap, in one CTA.
 template <int kPerLane>
-__global__ void __launch_bounds__(1024, 1)
+__global__ void __launch_bounds__(kFusedSelectThreads, 1)
 route_select_permute_kernel(const float *__restrict__ partial, const float *__restrict__ bias,
                             int32_t *__restrict__ ids, float *__restrict__ wout, int32_t *__restrict__ offsets,
                             int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
@@ -212,7 +207,7 @@ route_select_permute_kernel(const float *__restrict__ partial, const float *__re
     const int n = M * k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int i = n + threadIdx.x; i < n2; i += blockDim.x) keys[i] = 0xFFFFFFFFu;
-    for (int t = warp; t < M; t += 32) {
+    for (int t = warp; t < M; t += kFusedSelectThreads / 32) {
         int sel_e;
         float sel_w;
         select_topk<kPerLane>(partial, bias, t, M, E, k, splits, sel_e, sel_w);
@@ -242,8 +237,7 @@ __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restr
 }
 
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
-                                int32_t *status_out, int *counters, int counters_per_token, int M, int H, int E,
-                                int splits, cudaStream_t s)
+                                int32_t *status_out, int M, int H, int E, int splits, cudaStream_t s)
 {
     const size_t smem = static_cast<size_t>(kRouteTokens) * kRouteChunkH * sizeof(uint16_t);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_logits_kernel), static_cast<int>(smem));
@@ -251,7 +245,7 @@ cudaError_t launch_route_logits(const void *x, const float *router_w, float *par
     dim3 grid((E + 7) / 8, splits, (M + kRouteTokens - 1) / kRouteTokens);
     // first kernel of a call: fully ordered after whatever precedes it in the stream
     route_logits_kernel<<<grid, 256, smem, s>>>(static_cast<const uint16_t *>(x), router_w, partial, x16, status,
-                                                status_out, counters, counters_per_token, M, H, E);
+                                                status_out, M, H, E);
     return cudaGetLastError();
 }
 
@@ -284,7 +278,7 @@ static cudaError_t select_permute_p(const float *partial, const float *bias, int
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>),
                                     static_cast<int>(kMaxAssignments * sizeof(uint32_t)));
     if (e != cudaSuccess) return e;
-    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(1024), smem, s, pdl, partial, bias, ids, w,
+    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kFusedSelectThreads), smem, s, pdl, partial, bias, ids, w,
                      offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, splits, n2);
 }
 
