@@ -15,9 +15,9 @@
 //    r0..r0+63.  The item is 4 MMA m-tiles of 16 rows; for gate_up an m-tile
 //    holds 8 gate rows (fragment rows 0-7) and the same 8 up rows (fragment rows
 //    8-15), so every thread ends with g and u of one output row and applies
-//    clamp-SwiGLU and the bf16 rounding in registers.  Items are spread
-//    round-robin over the CTAs; all tiles of one row block are adjacent, so
-//    CTAs that share weights run together and hit L2.
+//    clamp-SwiGLU and the bf16 rounding in registers.  Each CTA takes a
+//    contiguous run of items in (tile, row block) order, so it streams adjacent
+//    32 KB weight regions of one expert back to back (DRAM page locality).
 //  * Producer warp: per 1024-K stage, TMA 2-D tiled copies of the item's packed
 //    E2M1 bytes -- 4 column boxes of 32 or 64 rows x 128 bytes per row block,
 //    issued together so that each row's 512 contiguous bytes are read at once --
@@ -143,6 +143,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     pdl_trigger();
     const int n_tiles = *n_tiles_ptr;
     const int n_items = n_tiles * row_blocks;
+    // a contiguous run of items per CTA, tile-major: consecutive items are adjacent row
+    // blocks of one expert, so each CTA streams contiguous weight memory
+    const int item_begin = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
+    const int item_end = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
 
     bool aborted = false;
 
@@ -156,19 +160,19 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
         int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
         auto fetch = [&](int it) {
-            if (it < n_items) {
-                const ExpertTile *tp = tiles + it % n_tiles;
+            if (it < item_end) {
+                const ExpertTile *tp = tiles + it / row_blocks;
                 nx_e = tp->expert;
                 nx_p0 = tp->p0;
                 nx_cnt = tp->count;
                 nx_tok = tp->tok[lane & (kTileTokens - 1)];
             }
         };
-        fetch(blockIdx.x);
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
+        fetch(item_begin);
+        for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
             const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, tok = nx_tok;
-            fetch(item + gridDim.x);
-            const int rb = item / n_tiles;
+            fetch(item + 1);
+            const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
             const int row_b = row_a + I;                               // gate_up only
@@ -238,9 +242,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         const int ep = warp - kFirstEpilogueWarp;
         const int g = lane >> 2, q = lane & 3;
         int item_ctr = 0;
-        for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
-            const ExpertTile *tp = tiles + item % n_tiles;
-            const int rb = item / n_tiles;
+        for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
+            const ExpertTile *tp = tiles + item / row_blocks;
+            const int rb = item % row_blocks;
             const int cnt = tp->count, p0 = tp->p0;
             const int b = item_ctr & 1;
             const float *rbuf = red + b * kRedFloats;
@@ -327,7 +331,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
 
     int stage_ctr = 0, item_ctr = 0;
-    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++item_ctr) {
+    for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
         const int b = item_ctr & 1;
         const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
         if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
