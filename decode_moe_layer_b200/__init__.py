@@ -24,6 +24,7 @@ from ._lib import (  # noqa: F401
     PROFILE_KERNELS,
     moe_permute,
     moe_route,
+    moe_route_noalloc,
     moe_status_string,
     moe_workspace_bytes,
 )

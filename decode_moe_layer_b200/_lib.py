@@ -22,7 +22,7 @@ MOE_ERR_TIMEOUT = -5
 EXPORTS = (
     "moe_status_string", "moe_last_cuda_error", "moe_route", "moe_permute", "moe_gate_up_swiglu",
     "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_mxfp4_forward_ex",
-    "moe_mxfp4_forward_profile",
+    "moe_mxfp4_forward_profile", "moe_route_noalloc",
 )
 H_STORAGE_SCALE = 1024.0   # moe_gate_up_swiglu stores binary16(h * 2^10)
 PROFILE_KERNELS = ("route_logits", "route_select", "permute", "gate_up_swiglu", "down_combine")
@@ -55,6 +55,8 @@ def load():
     lib.moe_last_cuda_error.argtypes = []
     lib.moe_route.restype = I
     lib.moe_route.argtypes = [P, P, P, P, P, I, I, I, I, P]
+    lib.moe_route_noalloc.restype = I
+    lib.moe_route_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, P]
     lib.moe_permute.restype = I
     lib.moe_permute.argtypes = [P, P, P, P, I, I, I, P]
     lib.moe_gate_up_swiglu.restype = I
@@ -112,6 +114,20 @@ def moe_route(x, router_w, k: int, router_bias=None, stream=None):
     w = torch.empty((M, k), dtype=torch.float32, device=x.device)
     rc = load().moe_route(_ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(ids), _ptr(w), M, H, E, k, _stream(stream))
     _check(rc, "moe_route")
+    return ids, w
+
+
+def moe_route_noalloc(x, router_w, k: int, router_bias=None, stream=None):
+    """moe_route with its scratch in the library's static device array (no device allocation)."""
+    _need(x, torch.bfloat16, "x")
+    _need(router_w, torch.float32, "router_w")
+    M, H = x.shape
+    E = router_w.shape[0]
+    ids = torch.empty((M, k), dtype=torch.int32, device=x.device)
+    w = torch.empty((M, k), dtype=torch.float32, device=x.device)
+    rc = load().moe_route_noalloc(_ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(ids), _ptr(w), M, H, E, k,
+                                  _stream(stream))
+    _check(rc, "moe_route_noalloc")
     return ids, w
 
 

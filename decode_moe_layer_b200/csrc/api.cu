@@ -18,7 +18,7 @@ int grouped_smem_bytes(int K);
 
 static thread_local int g_last_cuda_error = 0;
 
-static int cuda_fail(cudaError_t e)
+int cuda_fail(cudaError_t e)
 {
     g_last_cuda_error = static_cast<int>(e);
     return MOE_ERR_CUDA;
@@ -87,7 +87,7 @@ Layout make_layout(int M, int H, int I, int E, int k)
 
 static bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-static int check_dims(int M, int H, int I, int E, int k, bool need_hi)
+int check_dims(int M, int H, int I, int E, int k, bool need_hi)
 {
     if (M < 0 || E <= 0 || k <= 0 || H <= 0 || (need_hi && I <= 0)) return MOE_ERR_INVALID_ARG;
     if (E > kMaxE || k > kMaxK || k > E) return MOE_ERR_UNSUPPORTED_SHAPE;

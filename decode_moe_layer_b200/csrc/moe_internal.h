@@ -58,6 +58,11 @@ struct Layout {
 
 Layout make_layout(int M, int H, int I, int E, int k);
 
+// Shared argument checks of the C entry points (api.cu): the MOE_* status of a shape, and
+// recording a failed CUDA call (returns MOE_ERR_CUDA).
+int check_dims(int M, int H, int I, int E, int k, bool need_hi);
+int cuda_fail(cudaError_t e);
+
 // Launch with an optional programmatic dependency on the previous kernel in the stream
 // (the kernel must call pdl_wait() before touching what that kernel writes).
 template <typename... KArgs, typename... Args>

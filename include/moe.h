@@ -143,6 +143,25 @@ int moe_mxfp4_forward(const void *x, const float *router_w, const uint8_t *w13_q
                       const uint8_t *w2_q, const uint8_t *w2_s, void *out,
                       int M, int H, int I, int E, int k, cudaStream_t stream);
 
+/*
+ * moe_route without any device allocation, for callers that cannot allocate at the
+ * point where they route (an allocator that owns all device memory, a decode loop
+ * that must not allocate between steps).  The pages have no counterpart: this is
+ * an interface choice of this library.  Same arguments, results and checks as
+ * moe_route; the scratch (partial logits and a status word) lives in a 4 MiB
+ * device array compiled into the library instead of the library-owned workspace.
+ *   - Limit: 256 + ceil(H/512) * M * E * 4 bytes must fit in 4 MiB (for example
+ *     M <= 2048 at H=2048, E=128); larger shapes return MOE_ERR_WORKSPACE and
+ *     enqueue nothing.
+ *   - The first call on a device looks the array's device address up (once per
+ *     device); make that first call before any stream capture.
+ *   - Calls no cudaMalloc/cudaFree.  Every call shares the one array, which keeps
+ *     the last call's contents (nothing in it needs to start at zero): calls that
+ *     overlap on the GPU (other streams, other host threads) race on it.
+ */
+int moe_route_noalloc(const void *x_bf16, const float *router_w, const float *router_bias,
+                      int32_t *topk_ids, float *topk_w, int M, int H, int E, int k, cudaStream_t stream);
+
 /* Bytes of device workspace moe_mxfp4_forward_ex needs for this shape (0 if unsupported). */
 size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
 
