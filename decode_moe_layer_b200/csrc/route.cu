@@ -8,9 +8,10 @@
 //     xor-butterfly.  The CTAs of expert group 0 also write the binary16 copy of
 //     x that the grouped GEMM consumes and reset the call's status words.
 //  2. top-k per token, one warp per token: sum the chunk partials in chunk order,
-//     add the bias, select the top k by k rounds of a warp argmax over
-//     (value desc, expert id asc), and renormalise with a softmax over the k
-//     selected logits (equal to softmax-over-E followed by renormalisation).
+//     add the bias, select the top k by k rounds of a warp arg-max (warp max of
+//     order-preserving logit keys, then warp min of the ids holding it: value
+//     desc, expert id asc), and renormalise with a softmax over the k selected
+//     logits (equal to softmax-over-E followed by renormalisation).
 //     Either its own kernel (route_topk), or, for M <= kFusedSelectMaxM, fused
 //     with the route remap into one single-CTA kernel (route_select_permute).
 // Every reduction has a fixed order, so ids and weights are bitwise reproducible.
@@ -102,21 +103,45 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
                 }
             }
         }
+        // transpose-reduce: 3 halving exchanges leave each lane one token's sum over 8 lanes
+        // (token index = lane bits 4,3,2), 2 more levels finish the 32-lane sum; 9 shuffles
+        const bool b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
+        float r1[4], r2[2];
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt) {
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc[tt] += __shfl_xor_sync(0xffffffffu, acc[tt], off);
+        for (int i = 0; i < 4; ++i) {
+            const float keep = b4 ? acc[i + 4] : acc[i], send = b4 ? acc[i] : acc[i + 4];
+            r1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
         }
-        float mine = 0.f;
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt)
-            if (tt == lane) mine = acc[tt];
-        if (lane < 8 && tg + lane < nt)
-            partial[(static_cast<size_t>(split) * M + t0 + tg + lane) * E + e] = mine;
+        for (int i = 0; i < 2; ++i) {
+            const float keep = b3 ? r1[i + 2] : r1[i], send = b3 ? r1[i] : r1[i + 2];
+            r2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+        float mine = (b2 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? r2[0] : r2[1], 4);
+        mine += __shfl_xor_sync(0xffffffffu, mine, 2);
+        mine += __shfl_xor_sync(0xffffffffu, mine, 1);
+        const int tt = 4 * b4 + 2 * b3 + b2;
+        if ((lane & 3) == 0 && tg + tt < nt)
+            partial[(static_cast<size_t>(split) * M + t0 + tg + tt) * E + e] = mine;
     }
 }
 
+// Order-preserving map of fp32 to uint32 (larger float -> larger integer; -inf -> 0x007FFFFF).
+__device__ __forceinline__ uint32_t ordered_key(float v)
+{
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float from_ordered_key(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // One warp selects token t's top k.  Lane j < k ends with (sel_e, sel_w) of slot j.
+// Each round: every lane offers its best untaken (logit, id); a warp max over the
+// ordered logit keys and a warp min over the ids of the lanes holding that max pick
+// the winner (value desc, ties -> lower id).
 template <int kPerLane>
 __device__ __forceinline__ void select_topk(const float *__restrict__ partial, const float *__restrict__ bias, int t,
                                             int M, int E, int k, int splits, int &sel_e, float &sel_w)
@@ -140,29 +165,27 @@ __device__ __forceinline__ void select_topk(const float *__restrict__ partial, c
     for (int r = 0; r < k; ++r) {
         float bv = -CUDART_INF_F;
         int be = 0x7fffffff;
+        bool any = false;
 #pragma unroll
         for (int j = 0; j < kPerLane; ++j) {
             const int e = lane + 32 * j;
-            if (!((taken >> j) & 1u) && e < E && (v[j] > bv || (v[j] == bv && e < be))) {
+            if (!((taken >> j) & 1u) && e < E && (!any || v[j] > bv)) {
                 bv = v[j];
                 be = e;
+                any = true;
             }
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (ov > bv || (ov == bv && oe < be)) {
-                bv = ov;
-                be = oe;
-            }
-        }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
+        const uint32_t key = any ? ordered_key(bv) : 0u;
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, (any && key == kmax) ? static_cast<uint32_t>(be)
+                                                                                              : 0xffffffffu));
+        if ((win & 31) == lane) taken |= 1u << (win >> 5);
+        const float wv = from_ordered_key(kmax);
         if (lane == r) {
-            sel_v = bv;
-            sel_e = be;
+            sel_v = wv;
+            sel_e = win;
         }
-        if (r == 0) vmax = bv;
+        if (r == 0) vmax = wv;
     }
     const float ex = (lane < k) ? expf(sel_v - vmax) : 0.f;
     float sum = ex;
@@ -190,23 +213,26 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     }
 }
 
-// Top-k of every token (32 warps loop over the tokens) and the route remap, in one CTA.
+// Top-k of every token (warps loop over the tokens) and the route remap, in one CTA.
+// With n = M*k <= kFusedSelectMaxM*k unique keys (expert << 16 | f), the position of a key
+// in the expert-grouped order is the number of smaller keys, and expert e's offset is
+// the number of keys of experts below e: both are counted over broadcast shared-memory
+// reads, so the remap needs no sort and only three block barriers.
 template <int kPerLane>
 __global__ void __launch_bounds__(kFusedSelectThreads, 1)
 route_select_permute_kernel(const float *__restrict__ partial, const float *__restrict__ bias,
                             int32_t *__restrict__ ids, float *__restrict__ wout, int32_t *__restrict__ offsets,
                             int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
-                            ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k, int splits,
-                            int n2)
+                            ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k, int splits)
 {
-    extern __shared__ uint32_t keys[];
+    __shared__ uint32_t keys[kFusedSelectMaxM * kMaxK];
+    __shared__ int sorted_s[kFusedSelectMaxM * kMaxK];
     __shared__ int s_off[kMaxE + 1];
     __shared__ int scan_buf[33];
     pdl_wait();
     pdl_trigger();
     const int n = M * k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = n + threadIdx.x; i < n2; i += blockDim.x) keys[i] = 0xFFFFFFFFu;
     for (int t = warp; t < M; t += kFusedSelectThreads / 32) {
         int sel_e;
         float sel_w;
@@ -219,7 +245,23 @@ route_select_permute_kernel(const float *__restrict__ partial, const float *__re
         }
     }
     __syncthreads();
-    sort_and_emit(keys, n, n2, E, k, offsets, sorted_ids, inv_pos, tiles, n_tiles, s_off, scan_buf);
+    for (int f = threadIdx.x; f < n; f += blockDim.x) {
+        const uint32_t key = keys[f];
+        int pos = 0;
+        for (int i = 0; i < n; ++i) pos += keys[i] < key;
+        sorted_ids[pos] = f;
+        sorted_s[pos] = f;
+        inv_pos[f] = pos;
+    }
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+        const uint32_t target = static_cast<uint32_t>(e) << 16;
+        int off = 0;
+        for (int i = 0; i < n; ++i) off += keys[i] < target;
+        s_off[e] = off;
+        offsets[e] = off;
+    }
+    __syncthreads();
+    emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return sorted_s[p]; });
 }
 
 __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
@@ -273,13 +315,8 @@ static cudaError_t select_permute_p(const float *partial, const float *bias, int
                                     int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles, int *n_tiles, int M,
                                     int E, int k, int splits, cudaStream_t s, bool pdl)
 {
-    const int n2 = pow2_at_least(M * k);
-    const size_t smem = static_cast<size_t>(n2) * sizeof(uint32_t);
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>),
-                                    static_cast<int>(kMaxAssignments * sizeof(uint32_t)));
-    if (e != cudaSuccess) return e;
-    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kFusedSelectThreads), smem, s, pdl, partial, bias, ids, w,
-                     offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, splits, n2);
+    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kFusedSelectThreads), 0, s, pdl, partial, bias,
+                     ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, splits);
 }
 
 cudaError_t launch_route_select_permute(const float *partial, const float *bias, int32_t *ids, float *w,
