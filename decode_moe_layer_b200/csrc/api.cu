@@ -58,7 +58,7 @@ Layout make_layout(int M, int H, int I, int E, int k)
 {
     Layout L;
     const size_t n = static_cast<size_t>(M) * k;
-    L.route_splits = (H + kRouteChunkH - 1) / kRouteChunkH;
+    L.route_splits = route_splits(H);
     L.max_tiles = static_cast<int>((n < static_cast<size_t>(E) ? n : static_cast<size_t>(E)) +
                                    (n + kTileTokens - 1) / kTileTokens);
     size_t off = 0;
@@ -94,6 +94,7 @@ int check_dims(int M, int H, int I, int E, int k, bool need_hi)
     if (H % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (need_hi && (I % 32 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (static_cast<long long>(M) * k > kMaxAssignments) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (route_splits(H) > kMaxRouteSplits) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (need_hi) {
         if (static_cast<long long>(E) * 2 * I >= (1LL << 31) || static_cast<long long>(E) * H >= (1LL << 31))
             return MOE_ERR_UNSUPPORTED_SHAPE;

@@ -34,7 +34,11 @@ constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact
 __host__ __device__ inline bool per_stage_scales(int K) { return (K / 32) % 16 == 0; }
 
 // Router.
-constexpr int kRouteChunkH = 512;    // H elements per partial-logit chunk
+constexpr int kRouteChunkH = 512;    // H elements per partial-logit chunk (H < 4096)
+constexpr int kMaxRouteSplits = 16;  // partial-logit chunks at most (H <= 16384)
+// Router chunk: 512 elements for H < 4096 (more CTAs), 1024 above (fewer partial sums).
+__host__ __device__ inline int route_chunk(int H) { return H >= 4096 ? 1024 : 512; }
+__host__ __device__ inline int route_splits(int H) { return (H + route_chunk(H) - 1) / route_chunk(H); }
 constexpr int kRouteTokens = 32;     // tokens per router CTA
 
 constexpr int kMaxE = 1024;

@@ -1,7 +1,8 @@
 // route.cu -- router select/normalize ("Native router select/normalize" row of
 // "Post-Portfolio Device Attribution", "MTP1 Post-Portfolio Eager-Cycle Profile").
 //
-//  1. route_logits: fp32 partial logits x.W_r^T over H chunks of kRouteChunkH.
+//  1. route_logits: fp32 partial logits x.W_r^T over H chunks of 512 (H < 4096) or
+//     1024 elements.
 //     Grid (E/8, H chunks, M/32).  A CTA stages its 32 tokens' x chunk in shared
 //     memory once; each warp owns one expert, keeps that expert's W_r chunk in
 //     registers (read from HBM once per token tile) and reduces with a fixed
@@ -32,16 +33,17 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+template <int kChunk>
 __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__restrict__ x,
                                                            const float *__restrict__ wr, float *__restrict__ partial,
                                                            __half *__restrict__ x16, int *status, int32_t *status_out,
                                                            int M, int H, int E)
 {
-    extern __shared__ __align__(16) uint16_t xs[];   // [kRouteTokens][kRouteChunkH] bf16 bits
+    extern __shared__ __align__(16) uint16_t xs[];   // [kRouteTokens][kChunk] bf16 bits
     pdl_trigger();
     const int split = blockIdx.y;
-    const int h0 = split * kRouteChunkH;
-    const int len = min(H - h0, kRouteChunkH);        // multiple of 32
+    const int h0 = split * kChunk;
+    const int len = min(H - h0, kChunk);              // multiple of 32
     const int t0 = blockIdx.z * kRouteTokens;
     const int nt = min(kRouteTokens, M - t0);
     if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
@@ -52,7 +54,7 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
     const int e = blockIdx.x * 8 + warp;
 
     // this warp's expert chunk of W_r, requested before the x staging so both loads overlap
-    constexpr int kVec = kRouteChunkH / 128;   // float4 per lane
+    constexpr int kVec = kChunk / 128;   // float4 per lane
     float4 w[kVec];
 #pragma unroll
     for (int i = 0; i < kVec; ++i) {
@@ -67,7 +69,7 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
         const int r = i / vec_per_row, c = i - r * vec_per_row;
         const size_t g = static_cast<size_t>(t0 + r) * H + h0 + 8 * c;
         uint4 v = *reinterpret_cast<const uint4 *>(x + g);
-        *reinterpret_cast<uint4 *>(xs + r * kRouteChunkH + 8 * c) = v;
+        *reinterpret_cast<uint4 *>(xs + r * kChunk + 8 * c) = v;
         if (write_x16) {
             uint4 o;
             o.x = bf16x2_to_f16x2(v.x);
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
 #pragma unroll
                 for (int tt = 0; tt < 8; ++tt) {
                     if (tg + tt < nt) {
-                        const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (tg + tt) * kRouteChunkH + c);
+                        const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (tg + tt) * kChunk + c);
                         float a = acc[tt];
                         a = fmaf(bf16_lo(xv.x), w[i].x, a);
                         a = fmaf(bf16_hi(xv.x), w[i].y, a);
@@ -153,8 +155,14 @@ __device__ __forceinline__ void select_topk(const float *__restrict__ partial, c
         const int e = lane + 32 * j;
         float s = -CUDART_INF_F;
         if (e < E) {
+            // the splits' loads are independent: issue them together, then add in split order
+            float part[kMaxRouteSplits];
+#pragma unroll
+            for (int sp = 0; sp < kMaxRouteSplits; ++sp)
+                part[sp] = sp < splits ? partial[(static_cast<size_t>(sp) * M + t) * E + e] : 0.f;
             s = 0.f;
-            for (int sp = 0; sp < splits; ++sp) s += partial[(static_cast<size_t>(sp) * M + t) * E + e];
+#pragma unroll
+            for (int sp = 0; sp < kMaxRouteSplits; ++sp) s += part[sp];
             if (bias) s += bias[e];
         }
         v[j] = s;
@@ -281,13 +289,14 @@ __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restr
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
                                 int32_t *status_out, int M, int H, int E, int splits, cudaStream_t s)
 {
-    const size_t smem = static_cast<size_t>(kRouteTokens) * kRouteChunkH * sizeof(uint16_t);
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_logits_kernel), static_cast<int>(smem));
+    const int chunk = route_chunk(H);
+    const size_t smem = static_cast<size_t>(kRouteTokens) * chunk * sizeof(uint16_t);
+    auto kern = chunk == 1024 ? route_logits_kernel<1024> : route_logits_kernel<512>;
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     dim3 grid((E + 7) / 8, splits, (M + kRouteTokens - 1) / kRouteTokens);
     // first kernel of a call: fully ordered after whatever precedes it in the stream
-    route_logits_kernel<<<grid, 256, smem, s>>>(static_cast<const uint16_t *>(x), router_w, partial, x16, status,
-                                                status_out, M, H, E);
+    kern<<<grid, 256, smem, s>>>(static_cast<const uint16_t *>(x), router_w, partial, x16, status, status_out, M, H, E);
     return cudaGetLastError();
 }
 

@@ -17,7 +17,7 @@
 namespace moe {
 
 // Scratch of moe_route_noalloc: 256 bytes of status, then the partial logits
-// [ceil(H/512)][M][E] fp32.  Every GPU that loads the library holds these 4 MiB
+// [route_splits(H)][M][E] fp32.  Every GPU that loads the library holds these 4 MiB
 // until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 constexpr size_t kNoAllocStatusBytes = 256;
@@ -60,7 +60,7 @@ extern "C" int moe_route_noalloc(const void *x_bf16, const float *router_w, cons
     if ((ax % 16) || (aw % 16) || (reinterpret_cast<uintptr_t>(topk_ids) % 4) ||
         (reinterpret_cast<uintptr_t>(topk_w) % 4) || (router_bias && reinterpret_cast<uintptr_t>(router_bias) % 4))
         return MOE_ERR_INVALID_ARG;
-    const int splits = (H + kRouteChunkH - 1) / kRouteChunkH;
+    const int splits = route_splits(H);
     const size_t need = kNoAllocStatusBytes + static_cast<size_t>(splits) * M * E * sizeof(float);
     if (need > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
     void *base = nullptr;

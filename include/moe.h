@@ -40,8 +40,9 @@
  *   - Arguments are validated before anything is enqueued; a call that returns an
  *     error status has enqueued nothing.  M == 0 returns MOE_OK after the shape checks,
  *     reads no pointer (they may be NULL) and enqueues nothing.
- *   - Supported shapes: H % 32 == 0, I % 32 == 0, H,I >= 32, 1 <= k <= min(E, 32),
- *     E <= 1024, M*k <= 16384.  Others return MOE_ERR_UNSUPPORTED_SHAPE.
+ *   - Supported shapes: H % 32 == 0, I % 32 == 0, H,I >= 32, H <= 16384,
+ *     1 <= k <= min(E, 32), E <= 1024, M*k <= 16384.  Others return
+ *     MOE_ERR_UNSUPPORTED_SHAPE.
  *   - Out of contract (undefined output, no fault): NaN/Inf or |x| > 65504 in x,
  *     E8M0 scale bytes 254 and 255.
  *   - Determinism: for a given device and inputs, every output is bitwise
@@ -150,9 +151,9 @@ int moe_mxfp4_forward(const void *x, const float *router_w, const uint8_t *w13_q
  * an interface choice of this library.  Same arguments, results and checks as
  * moe_route; the scratch (partial logits and a status word) lives in a 4 MiB
  * device array compiled into the library instead of the library-owned workspace.
- *   - Limit: 256 + ceil(H/512) * M * E * 4 bytes must fit in 4 MiB (for example
- *     M <= 2048 at H=2048, E=128); larger shapes return MOE_ERR_WORKSPACE and
- *     enqueue nothing.
+ *   - Limit: 256 + S * M * E * 4 bytes must fit in 4 MiB, S = ceil(H/512) for
+ *     H < 4096 and ceil(H/1024) above (for example M <= 2048 at H=2048, E=128);
+ *     larger shapes return MOE_ERR_WORKSPACE and enqueue nothing.
  *   - The first call on a device looks the array's device address up (once per
  *     device); make that first call before any stream capture.
  *   - Calls no cudaMalloc/cudaFree.  Every call shares the one array, which keeps
