@@ -214,7 +214,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
                 if (per_stage_scales(I)) prefetch_tensormap(&s2_map);
             }
         }
-        int stage_ctr = 0, item_ctr = 0;
+        int stage_ctr = 0, scale_ctr = 0;    // scale_ctr: items that use the per-item scale buffer
         int ready_tile = -1;                 // tile whose h is known to be complete
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
         int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
@@ -228,7 +228,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
             }
         };
         fetch(item_begin);
-        for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
+        for (int item = item_begin; item < item_end; ++item) {
             const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, tok = nx_tok;
             fetch(item + 1);
             const ItemInfo it = item_info(item, n_gu, rb_gu, rb_dn);
@@ -251,8 +251,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
             const __half *arow = gu ? a.x16 + static_cast<size_t>(tok) * K
                                     : a.h + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
             if (!stage_scales) {
-                const int b = item_ctr & 1;
-                mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
+                const int b = scale_ctr & 1;
+                mbar_wait(&sempty[b], ((scale_ctr >> 1) & 1) ^ 1, aborted, status);
+                ++scale_ctr;
                 aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
                 if (!aborted && lane == 0) {
                     uint8_t *dst = sbuf + b * plan.sbuf_bytes;
@@ -408,7 +409,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
     const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
 
-    int stage_ctr = 0, item_ctr = 0;
+    int stage_ctr = 0, item_ctr = 0, scale_ctr = 0;
     for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
         const ItemInfo it = item_info(item, n_gu, rb_gu, rb_dn);
         const int K = it.gu ? H : I;
@@ -436,9 +437,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
         // scale addressing: per stage, row pitch kChunkK/32 bytes and block index within the stage;
         // per item, row pitch kblocks and the global block index
         const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
-        const int b = item_ctr & 1;
-        const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
-        if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
+        const int b = item_ctr & 1;                         // reduction buffer of this item
+        const int sb = scale_ctr & 1;                       // per-item scale buffer (when used)
+        const uint8_t *sbi = sbuf + sb * plan.sbuf_bytes;
+        if (!stage_scales) mbar_wait(&sfull[sb], (scale_ctr >> 1) & 1, aborted, status);
 
         float acc[2][4];
 #pragma unroll
@@ -483,7 +485,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
             if (lane == 0) mbar_arrive(&empty[s]);
         }
         __syncwarp();
-        if (!stage_scales && lane == 0) mbar_arrive(&sempty[b]);
+        if (!stage_scales) {
+            if (lane == 0) mbar_arrive(&sempty[sb]);
+            ++scale_ctr;
+        }
 
         // park the K-slot partial sums for the epilogue warps
         mbar_wait(&rempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
