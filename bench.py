@@ -83,10 +83,10 @@ def algorithmic(shape, M, ids):
     w_bytes = touched * (51 * I * H // 32)
     total = w_bytes + E * H * 4 + 2 * M * H * 2 + M * k * 8
     flops = 6 * I * H * M * k + 2 * M * E * H
-    # the expert-GEMM kernel must read the touched experts' weights and scales and the tokens' x;
-    # its h and y round trips are intermediates, not algorithmic bytes
-    gemms = w_bytes + M * H * 2
-    return {"touched": touched, "bytes": total, "flops": flops, "weight_bytes": w_bytes, "gemm_bytes": gemms}
+    gate_up = touched * (2 * I * H * 17 // 32) + M * H * 2 + M * k * I * 2
+    down = touched * (I * H * 17 // 32) + M * k * I * 2 + M * H * 2
+    return {"touched": touched, "bytes": total, "flops": flops, "weight_bytes": w_bytes,
+            "gate_up_bytes": gate_up, "down_bytes": down}
 
 
 def kernel_source_hash():
@@ -355,11 +355,11 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     roof_us = max(work["bytes"] / (hbm * 1e3), work["flops"] / (tflops * 1e6))
     roof_nominal_us = max(work["bytes"] / (NOMINAL_HBM_GBS * 1e3), work["flops"] / (NOMINAL_BF16_TFLOPS * 1e6))
     dominant = max(kern_us, key=kern_us.get)
-    dom_bytes = {"expert_gemms": work["gemm_bytes"]}.get(dominant)
+    dom_bytes = {"gate_up_swiglu": work["gate_up_bytes"], "down_combine": work["down_bytes"]}.get(dominant)
     if dom_bytes is None:
         dom_bytes = work["bytes"]
     achieved = dom_bytes / (kern_us[dominant] * 1e3)          # GB/s
-    traffic = profiled_traffic() if (ci, M) == (1, 8) and dominant == "expert_gemms" else None
+    traffic = profiled_traffic() if (ci, M) == (1, 8) and dominant == "gate_up_swiglu" else None
     sorted_ms = sorted(step_ms)
     rec = {
         "metric": METRIC, "value": mean_us, "unit": UNIT, "n_gpus": world, "steps": args.steps,

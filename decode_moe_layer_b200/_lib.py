@@ -25,7 +25,7 @@ EXPORTS = (
     "moe_mxfp4_forward_profile", "moe_route_noalloc",
 )
 H_STORAGE_SCALE = 1024.0   # moe_gate_up_swiglu stores binary16(h * 2^10)
-PROFILE_KERNELS = ("route_logits", "route_select", "permute", "expert_gemms", "combine")
+PROFILE_KERNELS = ("route_logits", "route_select", "permute", "gate_up_swiglu", "down_combine")
 
 _lib = None
 

@@ -14,6 +14,7 @@
 
 namespace moe {
 
+int grouped_smem_bytes(int K);
 
 static thread_local int g_last_cuda_error = 0;
 
@@ -97,7 +98,8 @@ int check_dims(int M, int H, int I, int E, int k, bool need_hi)
     if (need_hi) {
         if (static_cast<long long>(E) * 2 * I >= (1LL << 31) || static_cast<long long>(E) * H >= (1LL << 31))
             return MOE_ERR_UNSUPPORTED_SHAPE;
-        if (grouped_smem_bytes(H, I) > 227 * 1024) return MOE_ERR_UNSUPPORTED_SHAPE;
+        if (grouped_smem_bytes(H) > 227 * 1024 || grouped_smem_bytes(I) > 227 * 1024)
+            return MOE_ERR_UNSUPPORTED_SHAPE;
     }
     return MOE_OK;
 }
@@ -200,35 +202,22 @@ static int library_workspace(cudaStream_t s, size_t need, char **out)
 
 // ------------------------------------------------------------------ step bodies (arguments already validated)
 
-// Encode the tensor maps a grouped launch needs and launch it (phases: 1 gate_up, 2 down, 3 both).
-static int run_grouped(int phases, const void *w13_q, const uint8_t *w13_s, const void *w2_q, const uint8_t *w2_s,
-                       GroupedLaunch g, int E, cudaStream_t s, bool pdl)
+static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const ExpertTile *tiles,
+                       const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E,
+                       int max_tiles, cudaStream_t s, bool pdl)
 {
-    CUtensorMap m13, s13, m2, s2;
-    memset(&m13, 0, sizeof(m13));
-    memset(&s13, 0, sizeof(s13));
-    memset(&m2, 0, sizeof(m2));
-    memset(&s2, 0, sizeof(s2));
-    const int H = g.H, I = g.I;
-    int rc = MOE_OK;
-    if (phases & 1) {
-        // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
-        rc = make_weight_map(&m13, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2,
+    CUtensorMap map, smap;
+    // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
+    int rc = make_weight_map(&map, w13_q, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 2,
                              kItemRows / 2);
-        if (rc == MOE_OK && per_stage_scales(H))
-            rc = make_scale_map(&s13, w13_s, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 32,
-                                kItemRows / 2);
-    }
-    if (rc == MOE_OK && (phases & 2)) {
-        rc = make_weight_map(&m2, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
-        if (rc == MOE_OK && per_stage_scales(I))
-            rc = make_scale_map(&s2, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
-    }
     if (rc != MOE_OK) return rc;
-    g.w13_s = w13_s;
-    g.w2_s = w2_s;
-    g.phases = phases;
-    MOE_TRY(launch_grouped(m13, s13, m2, s2, g, s, pdl));
+    memset(&smap, 0, sizeof(smap));
+    if (per_stage_scales(H)) {
+        rc = make_scale_map(&smap, w13_s, static_cast<uint64_t>(E) * 2 * I, static_cast<uint64_t>(H) / 32,
+                            kItemRows / 2);
+        if (rc != MOE_OK) return rc;
+    }
+    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, max_tiles, s, pdl));
     return MOE_OK;
 }
 
@@ -243,6 +232,26 @@ struct Marks {
     do {                                                \
         if (m) MOE_TRY((m)->mark(s));                   \
     } while (0)
+
+static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, void *out, int *status,
+                    int32_t *status_out, int M, int H, int I, int E, int k, int max_tiles, cudaStream_t s, bool pdl,
+                    Marks *marks)
+{
+    CUtensorMap map, smap;
+    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
+    if (rc != MOE_OK) return rc;
+    memset(&smap, 0, sizeof(smap));
+    if (per_stage_scales(I)) {
+        rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
+        if (rc != MOE_OK) return rc;
+    }
+    MOE_TRY(launch_down(map, smap, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, status_out, H, I, max_tiles,
+                        s, pdl));
+    MOE_TRY(launch_combine(y, out, M, H, k, s, pdl));
+    MOE_MARK(marks, s);
+    return MOE_OK;
+}
 
 static int forward_impl(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
                         const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H,
@@ -280,25 +289,11 @@ static int forward_impl(const void *x, const float *router_w, const float *route
         MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, s, pdl));
     }
     MOE_MARK(marks, s);
-    GroupedLaunch g = {};
-    g.x16 = x16;
-    g.h = h;
-    g.y = y;
-    g.sorted_ids = sorted_ids;
-    g.topk_w = tw;
-    g.tiles = tiles;
-    g.n_tiles = n_tiles;
-    g.status = status;
-    g.status_out = status_out;
-    g.H = H;
-    g.I = I;
-    g.max_tiles = L.max_tiles;
-    int rc = run_grouped(3, w13_q, w13_s, w2_q, w2_s, g, E, s, pdl);
+    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
     MOE_MARK(marks, s);
-    MOE_TRY(launch_combine(y, out, M, H, k, s, pdl));
-    MOE_MARK(marks, s);
-    return MOE_OK;
+    return run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, out, status, status_out, M, H, I, E, k,
+                    L.max_tiles, s, pdl, marks);
 }
 
 static int check_forward_args(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
@@ -405,16 +400,8 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, nullptr, E, k, stream));
-    GroupedLaunch g = {};
-    g.x16 = x16;
-    g.h = static_cast<__half *>(h_f16);
-    g.tiles = tiles;
-    g.n_tiles = n_tiles;
-    g.status = status;
-    g.H = H;
-    g.I = I;
-    g.max_tiles = L.max_tiles;
-    return run_grouped(1, w13_q, w13_s, nullptr, nullptr, g, E, stream, false);
+    return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E,
+                       L.max_tiles, stream, false);
 }
 
 int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
@@ -438,21 +425,8 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
-    GroupedLaunch g = {};
-    g.h = const_cast<__half *>(static_cast<const __half *>(h_f16));
-    g.y = y;
-    g.sorted_ids = sorted_ids;
-    g.topk_w = topk_w;
-    g.tiles = tiles;
-    g.n_tiles = n_tiles;
-    g.status = status;
-    g.H = H;
-    g.I = I;
-    g.max_tiles = L.max_tiles;
-    rc = run_grouped(2, nullptr, nullptr, w2_q, w2_s, g, E, stream, false);
-    if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_combine(y, out_bf16, M, H, k, stream, false));
-    return MOE_OK;
+    return run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, out_bf16,
+                    status, nullptr, M, H, I, E, k, L.max_tiles, stream, false, nullptr);
 }
 
 int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,

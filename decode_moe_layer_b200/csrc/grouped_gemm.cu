@@ -9,17 +9,15 @@
 // counts these GEMMs stream each touched expert's weights once and are bound by
 // HBM bandwidth ("The Systematic Optimization Campaign", chunk 8.0).
 //
-// Design (one persistent CTA per SM, warp specialised; one kernel runs both
-// projections, gate_up items first, then down items):
+// Design (one persistent CTA per SM, warp specialised):
 //  * Work item = (expert tile of <= 8 assignments, 64 weight rows).  gate_up:
 //    gate rows n0..n0+31 and the matching up rows I+n0..; down: W2 rows
 //    r0..r0+63.  The item is 4 MMA m-tiles of 16 rows; for gate_up an m-tile
 //    holds 8 gate rows (fragment rows 0-7) and the same 8 up rows (fragment rows
 //    8-15), so every thread ends with g and u of one output row and applies
 //    clamp-SwiGLU and the bf16 rounding in registers.  Each CTA takes a
-//    contiguous run of items of equal weight-byte cost, in (phase, tile, row
-//    block) order, so it streams adjacent 32 KB weight regions of one expert back
-//    to back (DRAM page locality).
+//    contiguous run of items in (tile, row block) order, so it streams adjacent
+//    32 KB weight regions of one expert back to back (DRAM page locality).
 //  * Producer warp: per 1024-K stage, TMA 2-D tiled copies of the item's packed
 //    E2M1 bytes -- 4 column boxes of 32 or 64 rows x 128 bytes per row block,
 //    issued together so that each row's 512 contiguous bytes are read at once --
@@ -28,12 +26,6 @@
 //    the item's scale rows once per item), and one 1-D bulk copy per tile token of
 //    its binary16 activation chunk (the routed gather: x rows for gate_up, h rows
 //    for down).
-//  * gate_up -> down hand-off inside the kernel: after storing an item's h rows
-//    the epilogue counts the item in its tile's ready counter (fence, then
-//    atomic add); before a down item's first stage the producer issues the W2
-//    and scale boxes at once and waits (bounded) only before the h copies, until
-//    every gate_up row block of that tile is counted.  The launch is cooperative,
-//    so every CTA is resident and the wait always ends.
 //  * 16 compute warps = 2 m-tile pairs x 8 K slots.  Per stage a warp takes 4 of
 //    the 32 blocks of 32 K for its 2 m-tiles: a thread reads the 32-bit word q of
 //    its rows' 16-byte block (conflict-free thanks to the swizzle), decodes it with
@@ -66,43 +58,19 @@ constexpr int kBlocksPerStage = kChunkK / 32;
 constexpr int kBlocksPerWarp = kBlocksPerStage / kKSlots;
 static_assert(kBlocksPerWarp * kKSlots == kBlocksPerStage, "stage blocks split evenly over K slots");
 static_assert(8 % kBlocksPerWarp == 0, "a warp's blocks stay inside one 128-byte box column");
-constexpr int kGuBoxRows = kItemRows / 2, kDnBoxRows = kItemRows;   // weight box heights
-// ~2 s at 2 GHz for a down item's wait on its tile's h.
-constexpr long long kReadyWaitCycles = 4000000000LL;
-
-struct GemmArgs {
-    const uint8_t *w13_s, *w2_s;        // E8M0 scale matrices (per-item copies read them directly)
-    const __half *x16;                  // gate_up activations [M][H]
-    __half *h;                          // gate_up output / down activations [M*k][I], expert-grouped
-    float *y;                           // down output [M*k][H] (weighted), flat order
-    const int32_t *sorted_ids;
-    const float *topk_w;
-    ExpertTile *tiles;                  // .ready counts finished gate_up row blocks per tile
-    const int *n_tiles;
-    int *status_ws;
-    int32_t *status_out;
-    int H, I;
-    int phases;                         // bit 0: gate_up items, bit 1: down items
-    int wait_ready;                     // down items wait for their tile's gate_up items
-};
-
-__host__ __device__ inline int item_scale_bytes(int K) { return per_stage_scales(K) ? 0 : kItemRows * (K / 32); }
 
 struct SmemPlan {
     int wst_off, act_off, sst_off, sbuf_off, sbuf_bytes, red_off, bars_off, total;
 };
 
-__host__ __device__ inline SmemPlan smem_plan(int H, int I, int phases)
+__host__ __device__ inline SmemPlan smem_plan(int K)
 {
     SmemPlan p;
     p.wst_off = 0;
     p.act_off = kStages * kStageBytes;
     p.sst_off = p.act_off + kStages * kActStageBytes;
     p.sbuf_off = p.sst_off + kStages * kStageScaleBytes;
-    int sb = 0;
-    if (phases & 1) sb = item_scale_bytes(H);
-    if ((phases & 2) && item_scale_bytes(I) > sb) sb = item_scale_bytes(I);
-    p.sbuf_bytes = (sb + 127) / 128 * 128;
+    p.sbuf_bytes = per_stage_scales(K) ? 0 : (kItemRows * (K / 32) + 127) / 128 * 128;
     p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
     p.bars_off = p.red_off + 2 * kRedFloats * 4;
     p.total = p.bars_off + (2 * kStages + 8) * 8 + 1024;   // + alignment slack
@@ -122,40 +90,19 @@ __device__ __forceinline__ __half store_h(float v)
     return __float2half_rn(__bfloat162float(__float2bfloat16_rn(v)) * kHScale);
 }
 
-__device__ __forceinline__ int load_acquire(const int *p)
-{
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Item i of the work list: phase (gate_up first), tile and row block.
-struct ItemInfo {
-    bool gu;
-    int tile, rb;
-};
-
-__device__ __forceinline__ ItemInfo item_info(int i, int n_gu, int rb_gu, int rb_dn)
-{
-    ItemInfo it;
-    it.gu = i < n_gu;
-    const int j = it.gu ? i : i - n_gu;
-    const int rbs = it.gu ? rb_gu : rb_dn;
-    it.tile = j / rbs;
-    it.rb = j - it.tile * rbs;
-    return it;
-}
-
+template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
-grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_constant__ CUtensorMap s13_map,
-                     const __grid_constant__ CUtensorMap w2_map, const __grid_constant__ CUtensorMap s2_map,
-                     const __grid_constant__ GemmArgs a)
+grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
+                     const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
+                     const int32_t *__restrict__ sorted_ids, const float *__restrict__ topk_w,
+                     const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
+                     __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out, int K,
+                     int I, int H)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    const int H = a.H, I = a.I;
-    const SmemPlan plan = smem_plan(H, I, a.phases);
+    const SmemPlan plan = smem_plan(K);
     uint8_t *wst = smem + plan.wst_off;
     uint8_t *ast = smem + plan.act_off;
     uint8_t *sst = smem + plan.sst_off;
@@ -166,9 +113,16 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
     uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const StatusPtrs status{a.status_ws, a.status_out};
-    const int rb_gu = I / 32, rb_dn = down_row_blocks(H);
-    const int chunks_gu = (H + kChunkK - 1) / kChunkK, chunks_dn = (I + kChunkK - 1) / kChunkK;
+    const StatusPtrs status{status_ws, status_out};
+    const int rows_total = kGateUp ? I : H;                 // output rows of this projection
+    const int row_blocks = kGateUp ? I / 32 : down_row_blocks(H);
+    const int kblocks = K / 32;                             // scale bytes per row
+    const bool stage_scales = per_stage_scales(K);
+    const int n_chunks = (K + kChunkK - 1) / kChunkK;
+    const int kbytes = K / 2;                               // packed bytes per row
+    constexpr int kBoxRows = kGateUp ? 32 : 64;
+    constexpr int kBoxBytes = kBoxRows * 128;               // one weight box: rows x 128 bytes
+    constexpr int kScaleBoxBytes = kBoxRows * (kChunkK / 32);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -187,40 +141,27 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
     // everything below reads what the previous kernels of this call wrote
     pdl_wait();
     pdl_trigger();
-    const int n_tiles = *a.n_tiles;
-    const int n_gu = (a.phases & 1) ? n_tiles * rb_gu : 0;
-    const int n_dn = (a.phases & 2) ? n_tiles * rb_dn : 0;
-    // contiguous item runs of equal stage count per CTA
-    const long long cost_gu = static_cast<long long>(n_gu) * chunks_gu;
-    const long long cost_all = cost_gu + static_cast<long long>(n_dn) * chunks_dn;
-    auto first_item_at = [&](long long c) -> int {   // first item whose cost offset is >= c
-        if (c <= cost_gu) return static_cast<int>((c + chunks_gu - 1) / chunks_gu);
-        return n_gu + static_cast<int>((c - cost_gu + chunks_dn - 1) / chunks_dn);
-    };
-    const int item_begin = first_item_at((cost_all * blockIdx.x + gridDim.x - 1) / gridDim.x);
-    const int item_end = first_item_at((cost_all * (blockIdx.x + 1) + gridDim.x - 1) / gridDim.x);
+    const int n_tiles = *n_tiles_ptr;
+    const int n_items = n_tiles * row_blocks;
+    // a contiguous run of items per CTA, tile-major: consecutive items are adjacent row
+    // blocks of one expert, so each CTA streams contiguous weight memory
+    const int item_begin = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
+    const int item_end = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
 
     bool aborted = false;
 
     if (warp == kProducerWarp) {
         // ---------------------------------------------------------------- producer warp
         if (lane == 0) {
-            if (a.phases & 1) {
-                prefetch_tensormap(&w13_map);
-                if (per_stage_scales(H)) prefetch_tensormap(&s13_map);
-            }
-            if (a.phases & 2) {
-                prefetch_tensormap(&w2_map);
-                if (per_stage_scales(I)) prefetch_tensormap(&s2_map);
-            }
+            prefetch_tensormap(&wmap);
+            if (stage_scales) prefetch_tensormap(&smap);
         }
-        int stage_ctr = 0, scale_ctr = 0;    // scale_ctr: items that use the per-item scale buffer
-        int ready_tile = -1;                 // tile whose h is known to be complete
+        int stage_ctr = 0, item_ctr = 0;
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
         int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
-        auto fetch = [&](int i) {
-            if (i < item_end) {
-                const ExpertTile *tp = a.tiles + item_info(i, n_gu, rb_gu, rb_dn).tile;
+        auto fetch = [&](int it) {
+            if (it < item_end) {
+                const ExpertTile *tp = tiles + it / row_blocks;
                 nx_e = tp->expert;
                 nx_p0 = tp->p0;
                 nx_cnt = tp->count;
@@ -228,37 +169,25 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
             }
         };
         fetch(item_begin);
-        for (int item = item_begin; item < item_end; ++item) {
+        for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
             const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, tok = nx_tok;
             fetch(item + 1);
-            const ItemInfo it = item_info(item, n_gu, rb_gu, rb_dn);
-            const bool gu = it.gu;
-            const int K = gu ? H : I;
-            const int kblocks = K / 32, kbytes = K / 2;
-            const bool stage_scales = per_stage_scales(K);
-            const int n_chunks = gu ? chunks_gu : chunks_dn;
-            const CUtensorMap *wmap = gu ? &w13_map : &w2_map;
-            const CUtensorMap *smap = gu ? &s13_map : &s2_map;
-            const uint8_t *wscale = gu ? a.w13_s : a.w2_s;
-            const int box_bytes = (gu ? kGuBoxRows : kDnBoxRows) * 128;
-            const int sbox_bytes = (gu ? kGuBoxRows : kDnBoxRows) * (kChunkK / 32);
+            const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
-            const int row_a = gu ? e * 2 * I + it.rb * 32 : e * H + it.rb * kItemRows;
+            const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
             const int row_b = row_a + I;                               // gate_up only
-            const int valid_rows = gu ? kItemRows : min(kItemRows, H - it.rb * kItemRows);
-            const bool need_ready = !gu && a.wait_ready && it.tile != ready_tile;
+            const int valid_rows = kGateUp ? kItemRows : min(kItemRows, H - rb * kItemRows);
             // this lane's activation row (gate_up: the token's x row; down: the h row)
-            const __half *arow = gu ? a.x16 + static_cast<size_t>(tok) * K
-                                    : a.h + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
+            const __half *arow = kGateUp ? act + static_cast<size_t>(tok) * K
+                                         : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
             if (!stage_scales) {
-                const int b = scale_ctr & 1;
-                mbar_wait(&sempty[b], ((scale_ctr >> 1) & 1) ^ 1, aborted, status);
-                ++scale_ctr;
+                const int b = item_ctr & 1;
+                mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
                 if (!aborted && lane == 0) {
                     uint8_t *dst = sbuf + b * plan.sbuf_bytes;
                     mbar_arrive_expect_tx(&sfull[b], static_cast<uint32_t>(valid_rows * kblocks));
-                    if (gu) {
+                    if (kGateUp) {
                         bulk_load(dst, wscale + static_cast<size_t>(row_a) * kblocks, 32u * kblocks, &sfull[b]);
                         bulk_load(dst + 32 * kblocks, wscale + static_cast<size_t>(row_b) * kblocks, 32u * kblocks,
                                   &sfull[b]);
@@ -277,48 +206,26 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
                 const int kc = c * kChunkK;
                 const uint32_t act_bytes = 2u * static_cast<uint32_t>(min(kChunkK, K - kc));
                 const int ncols = min(kBoxCols, (kbytes - kb + 127) / 128);   // skip columns wholly past K
-                const int halves = gu ? 2 : 1;
-                const uint32_t bytes = halves * (ncols * box_bytes + (stage_scales ? sbox_bytes : 0)) +
+                const int halves = kGateUp ? 2 : 1;
+                const uint32_t bytes = halves * (ncols * kBoxBytes + (stage_scales ? kScaleBoxBytes : 0)) +
                                        cnt * act_bytes;
                 if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
                 __syncwarp();
                 uint8_t *st = wst + s * kStageBytes;
                 // gate_up boxes: columns of the gate rows, then columns of the up rows; down: columns
                 if (lane < ncols) {
-                    tma_load_2d(st + lane * box_bytes, wmap, kb + 128 * lane, row_a, &full[s]);
-                    if (gu) tma_load_2d(st + (kBoxCols + lane) * box_bytes, wmap, kb + 128 * lane, row_b, &full[s]);
+                    tma_load_2d(st + lane * kBoxBytes, &wmap, kb + 128 * lane, row_a, &full[s]);
+                    if (kGateUp) tma_load_2d(st + (kBoxCols + lane) * kBoxBytes, &wmap, kb + 128 * lane, row_b, &full[s]);
                 }
                 if (stage_scales && lane == 8) {
                     uint8_t *ss = sst + s * kStageScaleBytes;
-                    tma_load_2d(ss, smap, kc / 32, row_a, &full[s]);
-                    if (gu) tma_load_2d(ss + sbox_bytes, smap, kc / 32, row_b, &full[s]);
-                }
-                if (c == 0 && need_ready) {
-                    // the W2 and scale boxes above are already in flight; the h rows of this tile
-                    // must be complete before they are copied
-                    const int *ctr = &a.tiles[it.tile].pad;
-                    if (lane == 0 && load_acquire(ctr) < rb_gu) {
-                        const long long t0 = clock64();
-                        while (load_acquire(ctr) < rb_gu) {
-                            if (clock64() - t0 > kReadyWaitCycles) {
-                                aborted = true;
-                                record_timeout(status);
-                                break;
-                            }
-                            __nanosleep(64);
-                        }
-                    }
-                    __syncwarp();
-                    aborted = __shfl_sync(0xffffffffu, aborted, 0);
-                    // every lane that copies h acquires the count itself, then orders the TMA engine's
-                    // reads (async proxy) after that acquire
-                    (void)load_acquire(ctr);
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                    ready_tile = it.tile;
+                    tma_load_2d(ss, &smap, kc / 32, row_a, &full[s]);
+                    if (kGateUp) tma_load_2d(ss + kScaleBoxBytes, &smap, kc / 32, row_b, &full[s]);
                 }
                 if (lane >= 16 && lane - 16 < cnt)
                     bulk_load(ast + s * kActStageBytes + (lane - 16) * kActPitch,
-                              (gu ? arow : a.h + static_cast<size_t>(p0 + lane - 16) * K) + kc, act_bytes, &full[s]);
+                              (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc, act_bytes,
+                              &full[s]);
             }
         }
         // let every copy this CTA issued land before the CTA can exit
@@ -331,12 +238,13 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
 
     if (warp >= kFirstEpilogueWarp) {
         // ---------------------------------------------------------------- epilogue warps
+        const int et = threadIdx.x - kFirstEpilogueWarp * 32;   // 0..63
         const int ep = warp - kFirstEpilogueWarp;
         const int g = lane >> 2, q = lane & 3;
         int item_ctr = 0;
         for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
-            const ItemInfo it = item_info(item, n_gu, rb_gu, rb_dn);
-            const ExpertTile *tp = a.tiles + it.tile;
+            const ExpertTile *tp = tiles + item / row_blocks;
+            const int rb = item % row_blocks;
             const int cnt = tp->count, p0 = tp->p0;
             const int b = item_ctr & 1;
             const float *rbuf = red + b * kRedFloats;
@@ -362,38 +270,30 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 const int j = ep + 2 * m;
-                const float4 sum = sums[m];
-                if (it.gu) {
+                float4 sum = sums[m];
+                if (kGateUp) {
                     // remove the factor 2 carried by e8m0_times2
-                    const int n = it.rb * 32 + 8 * j + g;
+                    const int n = rb * 32 + 8 * j + g;
                     if (li0 < cnt)
-                        a.h[static_cast<size_t>(p0 + li0) * I + n] = store_h(clamp_swiglu(0.5f * sum.x, 0.5f * sum.z));
+                        hout[static_cast<size_t>(p0 + li0) * I + n] = store_h(clamp_swiglu(0.5f * sum.x, 0.5f * sum.z));
                     if (li1 < cnt)
-                        a.h[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
+                        hout[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
                 } else {
                     // remove e8m0_times2's factor 2 and h's 2^10 storage scale
                     const float unscale = 0.5f / kHScale;
-                    const int ra = it.rb * kItemRows + 16 * j + g, rbw = ra + 8;
+                    const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
                     if (li0 < cnt) {
-                        const int f = a.sorted_ids[p0 + li0];
-                        const float w = a.topk_w[f] * unscale;
-                        if (ra < H) a.y[static_cast<size_t>(f) * H + ra] = w * sum.x;
-                        if (rbw < H) a.y[static_cast<size_t>(f) * H + rbw] = w * sum.z;
+                        const int f = sorted_ids[p0 + li0];
+                        const float w = topk_w[f] * unscale;
+                        if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
+                        if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
                     }
                     if (li1 < cnt) {
-                        const int f = a.sorted_ids[p0 + li1];
-                        const float w = a.topk_w[f] * unscale;
-                        if (ra < H) a.y[static_cast<size_t>(f) * H + ra] = w * sum.y;
-                        if (rbw < H) a.y[static_cast<size_t>(f) * H + rbw] = w * sum.w;
+                        const int f = sorted_ids[p0 + li1];
+                        const float w = topk_w[f] * unscale;
+                        if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
+                        if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
                     }
-                }
-            }
-            if (it.gu && a.wait_ready) {
-                // publish this row block of the tile's h to the down items of other CTAs
-                named_bar_sync(2, kEpilogueWarps * 32);
-                if (ep == 0 && lane == 0) {
-                    __threadfence();
-                    atomicAdd(&a.tiles[it.tile].pad, 1);
                 }
             }
         }
@@ -408,39 +308,33 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
     const int bb0 = (kslot * kBlocksPerWarp) & 7;
     const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
-
-    int stage_ctr = 0, item_ctr = 0, scale_ctr = 0;
-    for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
-        const ItemInfo it = item_info(item, n_gu, rb_gu, rb_dn);
-        const int K = it.gu ? H : I;
-        // per m-tile: smem byte offsets (inside a stage) of the top/bottom rows' 16-byte blocks and
-        // scale-row indices; gate_up: 8 gate rows over the same 8 up rows, down: 16 consecutive rows
-        int top_off[2], bot_off[2], top_sr[2], bot_sr[2];
+    // per m-tile: smem byte offsets (inside a stage) of the top/bottom rows' 16-byte blocks,
+    // and scale-row indices (rows of the item's 64 weight rows)
+    int top_off[2], bot_off[2], top_sr[2], bot_sr[2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            const int j = 2 * pair + m;
-            if (it.gu) {
-                top_off[m] = col * kGuBoxRows * 128 + (8 * j + g) * 128;
-                bot_off[m] = (kBoxCols + col) * kGuBoxRows * 128 + (8 * j + g) * 128;
-                top_sr[m] = 8 * j + g;
-                bot_sr[m] = 32 + 8 * j + g;
-            } else {
-                top_off[m] = col * kDnBoxRows * 128 + (16 * j + g) * 128;
-                bot_off[m] = col * kDnBoxRows * 128 + (16 * j + 8 + g) * 128;
-                top_sr[m] = 16 * j + g;
-                bot_sr[m] = 16 * j + 8 + g;
-            }
+    for (int m = 0; m < 2; ++m) {
+        const int j = 2 * pair + m;
+        if (kGateUp) {
+            top_off[m] = col * kBoxBytes + (8 * j + g) * 128;
+            bot_off[m] = (kBoxCols + col) * kBoxBytes + (8 * j + g) * 128;
+            top_sr[m] = 8 * j + g;
+            bot_sr[m] = 32 + 8 * j + g;
+        } else {
+            top_off[m] = col * kBoxBytes + (16 * j + g) * 128;
+            bot_off[m] = col * kBoxBytes + (16 * j + 8 + g) * 128;
+            top_sr[m] = 16 * j + g;
+            bot_sr[m] = 16 * j + 8 + g;
         }
-        const int kblocks = K / 32;
-        const bool stage_scales = per_stage_scales(K);
-        const int n_chunks = it.gu ? chunks_gu : chunks_dn;
-        // scale addressing: per stage, row pitch kChunkK/32 bytes and block index within the stage;
-        // per item, row pitch kblocks and the global block index
-        const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
-        const int b = item_ctr & 1;                         // reduction buffer of this item
-        const int sb = scale_ctr & 1;                       // per-item scale buffer (when used)
-        const uint8_t *sbi = sbuf + sb * plan.sbuf_bytes;
-        if (!stage_scales) mbar_wait(&sfull[sb], (scale_ctr >> 1) & 1, aborted, status);
+    }
+    // scale addressing: per stage, row pitch kChunkK/32 bytes and block index within the stage;
+    // per item, row pitch kblocks and the global block index
+    const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
+
+    int stage_ctr = 0, item_ctr = 0;
+    for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
+        const int b = item_ctr & 1;
+        const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
+        if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
 
         float acc[2][4];
 #pragma unroll
@@ -485,10 +379,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap w13_map, const __grid_c
             if (lane == 0) mbar_arrive(&empty[s]);
         }
         __syncwarp();
-        if (!stage_scales) {
-            if (lane == 0) mbar_arrive(&sempty[sb]);
-            ++scale_ctr;
-        }
+        if (!stage_scales && lane == 0) mbar_arrive(&sempty[b]);
 
         // park the K-slot partial sums for the epilogue warps
         mbar_wait(&rempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
@@ -525,56 +416,40 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     *reinterpret_cast<uint2 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint2 *>(o);
 }
 
-int grouped_smem_bytes(int H, int I) { return smem_plan(H, I, 3).total; }
-
-cudaError_t launch_grouped(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const CUtensorMap &w2_map,
-                           const CUtensorMap &s2_map, const GroupedLaunch &g, cudaStream_t s, bool pdl)
+template <bool kGateUp>
+static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
+                                  const __half *act, const int32_t *sorted_ids, const float *topk_w,
+                                  const ExpertTile *tiles, const int *n_tiles, __half *h, float *y, int *status,
+                                  int32_t *status_out, int K, int I, int H, int max_tiles, cudaStream_t s, bool pdl)
 {
-    GemmArgs a;
-    a.w13_s = g.w13_s;
-    a.w2_s = g.w2_s;
-    a.x16 = g.x16;
-    a.h = g.h;
-    a.y = g.y;
-    a.sorted_ids = g.sorted_ids;
-    a.topk_w = g.topk_w;
-    a.tiles = g.tiles;
-    a.n_tiles = g.n_tiles;
-    a.status_ws = g.status;
-    a.status_out = g.status_out;
-    a.H = g.H;
-    a.I = g.I;
-    a.phases = g.phases;
-    a.wait_ready = g.phases == 3 ? 1 : 0;
-    const SmemPlan plan = smem_plan(g.H, g.I, g.phases);
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel), plan.total);
+    const SmemPlan plan = smem_plan(K);
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
     if (e != cudaSuccess) return e;
-    long long max_items = 0;
-    if (g.phases & 1) max_items += static_cast<long long>(g.max_tiles) * (g.I / 32);
-    if (g.phases & 2) max_items += static_cast<long long>(g.max_tiles) * down_row_blocks(g.H);
+    const long long row_blocks = kGateUp ? I / 32 : down_row_blocks(H);
+    const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
     int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     if (grid < 1) grid = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = plan.total;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[2];
-    int n = 0;
-    if (a.wait_ready) {
-        // down items wait on other CTAs' gate_up items: every CTA must be resident
-        attr[n].id = cudaLaunchAttributeCooperative;
-        attr[n].val.cooperative = 1;
-        ++n;
-    }
-    if (pdl && !a.wait_ready) {
-        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[n].val.programmaticStreamSerializationAllowed = 1;
-        ++n;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = n;
-    return cudaLaunchKernelEx(&cfg, grouped_mxfp4_kernel, w13_map, s13_map, w2_map, s2_map, a);
+    return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, smap,
+                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, status_out, K, I, H);
+}
+
+int grouped_smem_bytes(int K) { return smem_plan(K).total; }
+
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
+                           const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
+                           int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl)
+{
+    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, status,
+                                status_out, H, I, H, max_tiles, s, pdl);
+}
+
+cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
+                        const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles, const int *n_tiles,
+                        float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
+                        bool pdl)
+{
+    return launch_grouped<false>(w2_map, s2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, status,
+                                 status_out, I, I, H, max_tiles, s, pdl);
 }
 
 cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl)

@@ -49,7 +49,7 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
     int expert;
     int p0;           // first position in the expert-grouped order
     int count;
-    int pad;          // written 0; counts finished gate_up row blocks when both projections share a launch
+    int pad;
     int tok[kTileTokens];   // token of each assignment (sorted_ids[p0+i] / k); entries >= count repeat the last
 };
 
@@ -103,24 +103,13 @@ cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
                                int *status, int E, int k, cudaStream_t s);
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
-// One launch of the grouped MXFP4 GEMM kernel: gate_up items (phases bit 0), down items
-// (bit 1), or both in one persistent cooperative launch (phases == 3).
-struct GroupedLaunch {
-    const uint8_t *w13_s, *w2_s;
-    const __half *x16;
-    __half *h;
-    float *y;
-    const int32_t *sorted_ids;
-    const float *topk_w;
-    ExpertTile *tiles;
-    const int *n_tiles;
-    int *status;
-    int32_t *status_out;
-    int H, I, max_tiles, phases;
-};
-cudaError_t launch_grouped(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const CUtensorMap &w2_map,
-                           const CUtensorMap &s2_map, const GroupedLaunch &g, cudaStream_t s, bool pdl);
-int grouped_smem_bytes(int H, int I);
+cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
+                           const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
+                           int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl);
+cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
+                        const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles, const int *n_tiles,
+                        float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
+                        bool pdl);
 cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl);
 
 // Row blocks of the down projection per token (one arrival counter each).

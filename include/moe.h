@@ -191,8 +191,8 @@ int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *rout
  * stream to finish (host synchronisation: not for use under stream capture) and
  * writes into the HOST array kernel_ms the event-to-event milliseconds of:
  *   [0] router logits, [1] router top-k (fused with the route remap when
- *   M <= 64), [2] route remap (0 when fused), [3] the expert GEMMs (gate_up +
- *   clamp-SwiGLU and down, one kernel), [4] the weighted combine.
+ *   M <= 64), [2] route remap (0 when fused), [3] gate_up + clamp-SwiGLU,
+ *   [4] down and the weighted combine (two kernels).
  * Kernels run back to back here instead of overlapping their launches as in
  * moe_mxfp4_forward_ex, so the sum exceeds a normal call's time.
  */
