@@ -279,7 +279,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     MOE_MARK(marks, s);
     MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, M, H, E, L.route_splits, s));
     MOE_MARK(marks, s);
-    if (M <= kFusedSelectMaxM) {
+    if (fused_select(M, E, k)) {
         MOE_TRY(launch_route_select_permute(partial, router_bias, ids, tw, offsets, sorted_ids, inv_pos, tiles,
                                             n_tiles, M, E, k, L.route_splits, s, pdl));
         MOE_MARK(marks, s);

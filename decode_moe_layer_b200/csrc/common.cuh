@@ -102,6 +102,14 @@ __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &
     }
 }
 
+// Bounded wait for copies already issued to land before a CTA exits.  It runs even after an
+// earlier wait gave up: shared memory must not be released with copies still in flight.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, const StatusPtrs &st)
+{
+    bool gave_up = false;
+    mbar_wait(bar, parity, gave_up, st);
+}
+
 // ------------------------------------------------------------------ bulk copies (TMA engine)
 
 // 2-D tiled tensor copy global -> shared, completion counted on `bar` in bytes.

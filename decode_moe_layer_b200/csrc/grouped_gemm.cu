@@ -138,10 +138,15 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         fence_barrier_init();
     }
     __syncthreads();
-    // everything below reads what the previous kernels of this call wrote
-    pdl_wait();
+    // gate_up reads the tile list its predecessor (the permutation) writes, so it waits here.
+    // The down kernel's predecessor is gate_up, which lets dependents launch only after its own
+    // wait, so the tile list, sorted ids and routing weights (written before gate_up) are complete
+    // when any down CTA runs.  Only h comes from gate_up: the down producer waits before its first
+    // h copy, and the W2 weights and scales of its first stages stream in during gate_up's tail.
+    // The producer's early reads of the tile list bypass L1 (ld.global.cg).
+    if (kGateUp) pdl_wait();
     pdl_trigger();
-    const int n_tiles = *n_tiles_ptr;
+    const int n_tiles = __ldcg(n_tiles_ptr);
     const int n_items = n_tiles * row_blocks;
     // a contiguous run of items per CTA, tile-major: consecutive items are adjacent row
     // blocks of one expert, so each CTA streams contiguous weight memory
@@ -157,16 +162,31 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             if (stage_scales) prefetch_tensormap(&smap);
         }
         int stage_ctr = 0, item_ctr = 0;
+        int stages_issued = 0, scales_issued = 0;   // copies in flight must land before exit
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
         int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
         auto fetch = [&](int it) {
             if (it < item_end) {
                 const ExpertTile *tp = tiles + it / row_blocks;
-                nx_e = tp->expert;
-                nx_p0 = tp->p0;
-                nx_cnt = tp->count;
-                nx_tok = tp->tok[lane & (kTileTokens - 1)];
+                nx_e = __ldcg(&tp->expert);
+                nx_p0 = __ldcg(&tp->p0);
+                nx_cnt = __ldcg(&tp->count);
+                nx_tok = __ldcg(&tp->tok[lane & (kTileTokens - 1)]);
             }
+        };
+        // down: h copies of the first stages, held back until gate_up has completed
+        bool h_ready = kGateUp;
+        const __half *pend_src[kStages];
+        uint32_t pend_bytes[kStages];
+#pragma unroll
+        for (int i = 0; i < kStages; ++i) pend_bytes[i] = 0;
+        auto release_h = [&]() {
+            pdl_wait();
+#pragma unroll
+            for (int i = 0; i < kStages; ++i)
+                if (pend_bytes[i] != 0)
+                    bulk_load(ast + i * kActStageBytes + (lane - 16) * kActPitch, pend_src[i], pend_bytes[i], &full[i]);
+            h_ready = true;
         };
         fetch(item_begin);
         for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
@@ -182,6 +202,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                                          : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
             if (!stage_scales) {
                 const int b = item_ctr & 1;
+                // the scale buffer frees only when compute has finished item_ctr - 2, which may
+                // need the held-back h copies
+                if (!h_ready && item_ctr >= 2) release_h();
                 mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
                 if (!aborted && lane == 0) {
@@ -196,9 +219,11 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                                   static_cast<uint32_t>(valid_rows * kblocks), &sfull[b]);
                     }
                 }
+                if (!aborted) ++scales_issued;
             }
             for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
                 const int s = stage_ctr % kStages;
+                if (!h_ready && stage_ctr >= kStages) release_h();
                 mbar_wait(&empty[s], ((stage_ctr / kStages) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);
                 if (aborted) continue;
@@ -222,25 +247,43 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     tma_load_2d(ss, &smap, kc / 32, row_a, &full[s]);
                     if (kGateUp) tma_load_2d(ss + kScaleBoxBytes, &smap, kc / 32, row_b, &full[s]);
                 }
-                if (lane >= 16 && lane - 16 < cnt)
-                    bulk_load(ast + s * kActStageBytes + (lane - 16) * kActPitch,
-                              (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc, act_bytes,
-                              &full[s]);
+                if (lane >= 16 && lane - 16 < cnt) {
+                    const __half *src = (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc;
+                    if (h_ready) {
+                        bulk_load(ast + s * kActStageBytes + (lane - 16) * kActPitch, src, act_bytes, &full[s]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < kStages; ++i)   // stage_ctr < kStages here, so s == stage_ctr
+                            if (i == s) {
+                                pend_src[i] = src;
+                                pend_bytes[i] = act_bytes;
+                            }
+                    }
+                }
+                ++stages_issued;
             }
         }
-        // let every copy this CTA issued land before the CTA can exit
-        for (int i = 0; i < kStages && i < stage_ctr; ++i) {
-            const int sc = stage_ctr - 1 - i;
-            mbar_wait(&full[sc % kStages], (sc / kStages) & 1, aborted, status);
+        if (!h_ready) release_h();
+        // let every copy this CTA issued land before the CTA can exit (stages and per-item scale
+        // rows are issued in order until a wait gives up, so the issued ones are a prefix)
+        for (int i = 0; i < kStages && i < stages_issued; ++i) {
+            const int sc = stages_issued - 1 - i;
+            mbar_wait_drain(&full[sc % kStages], (sc / kStages) & 1, status);
+        }
+        for (int i = 0; i < 2 && i < scales_issued; ++i) {
+            const int j = scales_issued - 1 - i;
+            mbar_wait_drain(&sfull[j & 1], (j >> 1) & 1, status);
         }
         return;
     }
 
     if (warp >= kFirstEpilogueWarp) {
         // ---------------------------------------------------------------- epilogue warps
-        const int et = threadIdx.x - kFirstEpilogueWarp * 32;   // 0..63
         const int ep = warp - kFirstEpilogueWarp;
         const int g = lane >> 2, q = lane & 3;
+        // nothing for the epilogue before the first item's partial sums; the down kernel's
+        // epilogue waits for gate_up here so that its plain loads see the current call's data
+        if (!kGateUp) pdl_wait();
         int item_ctr = 0;
         for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
             const ExpertTile *tp = tiles + item / row_blocks;

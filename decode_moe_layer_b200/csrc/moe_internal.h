@@ -86,9 +86,15 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// Largest M for which router top-k and the permutation run as one single-CTA kernel.
-constexpr int kFusedSelectMaxM = 64;
-constexpr int kFusedSelectThreads = 512;
+// Router top-k and the permutation run as one single-CTA kernel when M*k <= kFusedSelectMaxN
+// and E <= kFusedSelectMaxE; otherwise as route_topk followed by the permutation kernel.
+constexpr int kFusedSelectThreads = 1024;
+constexpr int kFusedSelectMaxN = 1024;
+constexpr int kFusedSelectMaxE = 512;
+__host__ __device__ inline bool fused_select(int M, int E, int k)
+{
+    return static_cast<long long>(M) * k <= kFusedSelectMaxN && E <= kFusedSelectMaxE;
+}
 
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,

@@ -13,8 +13,9 @@
 //     order-preserving logit keys, then warp min of the ids holding it: value
 //     desc, expert id asc), and renormalise with a softmax over the k selected
 //     logits (equal to softmax-over-E followed by renormalisation).
-//     Either its own kernel (route_topk), or, for M <= kFusedSelectMaxM, fused
-//     with the route remap into one single-CTA kernel (route_select_permute).
+//     Either its own kernel (route_topk), or, for M*k <= kFusedSelectMaxN and
+//     E <= kFusedSelectMaxE, fused with the route remap into one single-CTA kernel
+//     (route_select_permute).
 // Every reduction has a fixed order, so ids and weights are bitwise reproducible.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -64,19 +65,35 @@ __global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__res
     }
 
     const int vec_per_row = len / 8;
+    const int n_vec = nt * vec_per_row;
     const bool write_x16 = (blockIdx.x == 0) && (x16 != nullptr);
-    for (int i = threadIdx.x; i < nt * vec_per_row; i += blockDim.x) {
-        const int r = i / vec_per_row, c = i - r * vec_per_row;
-        const size_t g = static_cast<size_t>(t0 + r) * H + h0 + 8 * c;
-        uint4 v = *reinterpret_cast<const uint4 *>(x + g);
-        *reinterpret_cast<uint4 *>(xs + r * kChunk + 8 * c) = v;
-        if (write_x16) {
-            uint4 o;
-            o.x = bf16x2_to_f16x2(v.x);
-            o.y = bf16x2_to_f16x2(v.y);
-            o.z = bf16x2_to_f16x2(v.z);
-            o.w = bf16x2_to_f16x2(v.w);
-            *reinterpret_cast<uint4 *>(x16 + g) = o;
+    // a thread's x loads are issued in batches before any is stored, so they overlap
+    constexpr int kBatch = 8;
+    for (int i0 = threadIdx.x; i0 < n_vec; i0 += kBatch * blockDim.x) {
+        uint4 v[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int i = i0 + b * blockDim.x;
+            if (i < n_vec) {
+                const int r = i / vec_per_row, c = i - r * vec_per_row;
+                v[b] = *reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t0 + r) * H + h0 + 8 * c);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int i = i0 + b * blockDim.x;
+            if (i < n_vec) {
+                const int r = i / vec_per_row, c = i - r * vec_per_row;
+                *reinterpret_cast<uint4 *>(xs + r * kChunk + 8 * c) = v[b];
+                if (write_x16) {
+                    uint4 o;
+                    o.x = bf16x2_to_f16x2(v[b].x);
+                    o.y = bf16x2_to_f16x2(v[b].y);
+                    o.z = bf16x2_to_f16x2(v[b].z);
+                    o.w = bf16x2_to_f16x2(v[b].w);
+                    *reinterpret_cast<uint4 *>(x16 + static_cast<size_t>(t0 + r) * H + h0 + 8 * c) = o;
+                }
+            }
         }
     }
     __syncthreads();
@@ -221,11 +238,14 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict
     }
 }
 
-// Top-k of every token (warps loop over the tokens) and the route remap, in one CTA.
-// With n = M*k <= kFusedSelectMaxM*k unique keys (expert << 16 | f), the position of a key
-// in the expert-grouped order is the number of smaller keys, and expert e's offset is
-// the number of keys of experts below e: both are counted over broadcast shared-memory
-// reads, so the remap needs no sort and only three block barriers.
+// Top-k of every token (warps loop over the tokens) and the route remap, in one CTA of
+// kFusedSelectThreads threads, for n = M*k <= kFusedSelectMaxN assignments and E <= kFusedSelectMaxE.
+// Thread f owns assignment f.  Its stable rank inside its expert (the number of earlier
+// assignments routed to the same expert) is its rank among the matching lanes of its warp
+// (__match_any_sync) plus the counts of that expert in the earlier warps, kept in a
+// [warp][expert] table that one pass per expert turns into prefix counts.  One block scan
+// of (tiles, count) per expert gives every expert offset and tile base; thread f then writes
+// its sorted position, inverse position and tile slot directly.  Four block barriers, no sort.
 template <int kPerLane>
 __global__ void __launch_bounds__(kFusedSelectThreads, 1)
 route_select_permute_kernel(const float *__restrict__ partial, const float *__restrict__ bias,
@@ -233,15 +253,19 @@ route_select_permute_kernel(const float *__restrict__ partial, const float *__re
                             int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
                             ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k, int splits)
 {
-    __shared__ uint32_t keys[kFusedSelectMaxM * kMaxK];
-    __shared__ int sorted_s[kFusedSelectMaxM * kMaxK];
-    __shared__ int s_off[kMaxE + 1];
+    constexpr int kWarps = kFusedSelectThreads / 32;
+    static_assert(kFusedSelectMaxN <= kFusedSelectThreads, "one thread per assignment");
+    __shared__ int s_e[kFusedSelectMaxN];                        // expert of assignment f
+    __shared__ uint16_t s_wc[kWarps][kFusedSelectMaxE];          // per-warp counts, then prefix counts
+    __shared__ int s_off[kFusedSelectMaxE], s_cnt[kFusedSelectMaxE], s_tb[kFusedSelectMaxE];
     __shared__ int scan_buf[33];
-    pdl_wait();
-    pdl_trigger();
     const int n = M * k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int t = warp; t < M; t += kFusedSelectThreads / 32) {
+    // the count table is cleared while the previous kernel may still run
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) s_wc[i / E][i % E] = 0;
+    pdl_wait();
+    pdl_trigger();
+    for (int t = warp; t < M; t += kWarps) {
         int sel_e;
         float sel_w;
         select_topk<kPerLane>(partial, bias, t, M, E, k, splits, sel_e, sel_w);
@@ -249,27 +273,60 @@ route_select_permute_kernel(const float *__restrict__ partial, const float *__re
             const int f = t * k + lane;
             ids[f] = sel_e;
             wout[f] = sel_w;
-            keys[f] = (static_cast<uint32_t>(sel_e) << 16) | static_cast<uint32_t>(f);
+            s_e[f] = sel_e;
         }
     }
     __syncthreads();
-    for (int f = threadIdx.x; f < n; f += blockDim.x) {
-        const uint32_t key = keys[f];
-        int pos = 0;
-        for (int i = 0; i < n; ++i) pos += keys[i] < key;
-        sorted_ids[pos] = f;
-        sorted_s[pos] = f;
-        inv_pos[f] = pos;
+    // rank among the lanes of this warp routed to the same expert (lanes past n carry -1)
+    const int f = threadIdx.x;
+    const int e = f < n ? s_e[f] : -1;
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(same & ((1u << lane) - 1u));
+    if (e >= 0 && rank_w == 0) s_wc[warp][e] = static_cast<uint16_t>(__popc(same));
+    __syncthreads();
+    // per expert: prefix counts over the warps, the expert's total and its tile count
+    int packed = 0;                       // (tiles << 16) | count
+    if (threadIdx.x < E) {
+        int run = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = s_wc[w][threadIdx.x];
+            s_wc[w][threadIdx.x] = static_cast<uint16_t>(run);
+            run += c;
+        }
+        packed = (((run + kTileTokens - 1) / kTileTokens) << 16) | run;
+        s_cnt[threadIdx.x] = run;
     }
-    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
-        const uint32_t target = static_cast<uint32_t>(e) << 16;
-        int off = 0;
-        for (int i = 0; i < n; ++i) off += keys[i] < target;
-        s_off[e] = off;
-        offsets[e] = off;
+    int total = 0;
+    const int base = block_exclusive_scan(packed, scan_buf, total);   // ends with a block barrier
+    if (threadIdx.x < E) {
+        s_off[threadIdx.x] = base & 0xFFFF;
+        s_tb[threadIdx.x] = base >> 16;
+        offsets[threadIdx.x] = base & 0xFFFF;
+    }
+    if (threadIdx.x == 0) {
+        offsets[E] = n;
+        *n_tiles = total >> 16;
     }
     __syncthreads();
-    emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return sorted_s[p]; });
+    if (e >= 0) {
+        const int rank = s_wc[warp][e] + rank_w;
+        const int pos = s_off[e] + rank;
+        sorted_ids[pos] = f;
+        inv_pos[f] = pos;
+        const int cnt = s_cnt[e];
+        const int slot = rank % kTileTokens, tile_first = rank - slot;
+        ExpertTile *tp = tiles + s_tb[e] + rank / kTileTokens;
+        const int t = f / k;
+        tp->tok[slot] = t;
+        if (slot == 0) {
+            tp->expert = e;
+            tp->p0 = s_off[e] + tile_first;
+            tp->count = min(kTileTokens, cnt - tile_first);
+            tp->pad = 0;
+        }
+        if (rank == cnt - 1)   // the tile's last assignment repeats its token into the unused slots
+            for (int j = slot + 1; j < kTileTokens; ++j) tp->tok[j] = t;
+    }
 }
 
 __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
