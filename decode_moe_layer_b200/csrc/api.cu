@@ -58,7 +58,6 @@ Layout make_layout(int M, int H, int I, int E, int k)
 {
     Layout L;
     const size_t n = static_cast<size_t>(M) * k;
-    L.route_splits = route_splits(H);
     L.max_tiles = static_cast<int>((n < static_cast<size_t>(E) ? n : static_cast<size_t>(E)) +
                                    (n + kTileTokens - 1) / kTileTokens);
     size_t off = 0;
@@ -68,7 +67,8 @@ Layout make_layout(int M, int H, int I, int E, int k)
         return o;
     };
     L.status = take(256);
-    L.partial = take(static_cast<size_t>(L.route_splits) * M * E * sizeof(float));
+    L.splits = route_plan(M, H, E).splits;
+    L.partial = take(static_cast<size_t>(L.splits) * M * E * sizeof(float));
     L.x16 = take(static_cast<size_t>(M) * H * 2);
     L.topk_ids = take(n * 4);
     L.topk_w = take(n * 4);
@@ -94,7 +94,6 @@ int check_dims(int M, int H, int I, int E, int k, bool need_hi)
     if (H % 32 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (need_hi && (I % 32 != 0)) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (static_cast<long long>(M) * k > kMaxAssignments) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (route_splits(H) > kMaxRouteSplits) return MOE_ERR_UNSUPPORTED_SHAPE;
     if (need_hi) {
         if (static_cast<long long>(E) * 2 * I >= (1LL << 31) || static_cast<long long>(E) * H >= (1LL << 31))
             return MOE_ERR_UNSUPPORTED_SHAPE;
@@ -277,14 +276,14 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     const bool pdl = (marks == nullptr);
 
     MOE_MARK(marks, s);
-    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, M, H, E, L.route_splits, s));
+    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, M, H, E, s));
     MOE_MARK(marks, s);
     if (fused_select(M, E, k)) {
-        MOE_TRY(launch_route_select_permute(partial, router_bias, ids, tw, offsets, sorted_ids, inv_pos, tiles,
-                                            n_tiles, M, E, k, L.route_splits, s, pdl));
+        MOE_TRY(launch_route_select_permute(partial, L.splits, router_bias, ids, tw, offsets, sorted_ids, inv_pos,
+                                            tiles, n_tiles, M, E, k, s, pdl));
         MOE_MARK(marks, s);
     } else {
-        MOE_TRY(launch_route_topk(partial, router_bias, ids, tw, M, E, k, L.route_splits, s, pdl));
+        MOE_TRY(launch_route_topk(partial, L.splits, router_bias, ids, tw, M, E, k, s, pdl));
         MOE_MARK(marks, s);
         MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, s, pdl));
     }
@@ -360,8 +359,8 @@ int moe_route(const void *x_bf16, const float *router_w, const float *router_bia
     if (rc != MOE_OK) return rc;
     float *partial = reinterpret_cast<float *>(ws + L.partial);
     MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, reinterpret_cast<int *>(ws + L.status), nullptr,
-                                M, H, E, L.route_splits, stream));
-    MOE_TRY(launch_route_topk(partial, router_bias, topk_ids, topk_w, M, E, k, L.route_splits, stream, false));
+                                M, H, E, stream));
+    MOE_TRY(launch_route_topk(partial, L.splits, router_bias, topk_ids, topk_w, M, E, k, stream, false));
     return MOE_OK;
 }
 
@@ -399,7 +398,7 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, nullptr, E, k, stream));
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
     return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E,
                        L.max_tiles, stream, false);
 }

@@ -56,6 +56,8 @@ constexpr int kFirstEpilogueWarp = kComputeWarps + 1;
 constexpr int kRedFloats = kKSlots * kItemMTiles * 32 * 4;   // one buffer: [kslot][m-tile][lane][4]
 constexpr int kBlocksPerStage = kChunkK / 32;
 constexpr int kBlocksPerWarp = kBlocksPerStage / kKSlots;
+constexpr int kItemQ = 8;   // item ids in flight between the producer and the compute warps (> kStages)
+constexpr int kRedBufs = 2; // K-slot partial-sum buffers between the compute and epilogue warps
 static_assert(kBlocksPerWarp * kKSlots == kBlocksPerStage, "stage blocks split evenly over K slots");
 static_assert(8 % kBlocksPerWarp == 0, "a warp's blocks stay inside one 128-byte box column");
 
@@ -72,8 +74,8 @@ __host__ __device__ inline SmemPlan smem_plan(int K)
     p.sbuf_off = p.sst_off + kStages * kStageScaleBytes;
     p.sbuf_bytes = per_stage_scales(K) ? 0 : (kItemRows * (K / 32) + 127) / 128 * 128;
     p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
-    p.bars_off = p.red_off + 2 * kRedFloats * 4;
-    p.total = p.bars_off + (2 * kStages + 8) * 8 + 1024;   // + alignment slack
+    p.bars_off = p.red_off + kRedBufs * kRedFloats * 4;
+    p.total = p.bars_off + (2 * kStages + 8) * 8 + (kItemQ + 2) * 4 + 1024;   // + alignment slack
     return p;
 }
 
@@ -96,8 +98,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                      const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
                      const int32_t *__restrict__ sorted_ids, const float *__restrict__ topk_w,
                      const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
-                     __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out, int K,
-                     int I, int H)
+                     __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out,
+                     int *queue, int K, int I, int H)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -111,6 +113,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bars_off);
     uint64_t *full = bars, *empty = bars + kStages;
     uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
+    volatile int *item_q = reinterpret_cast<volatile int *>(bars + 2 * kStages + 8);   // [kItemQ] producer -> compute
+    volatile int *red_item = item_q + kItemQ;                                         // [2] compute -> epilogue
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
@@ -132,6 +136,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sfull[b], 1);
             mbar_init(&sempty[b], kComputeWarps);
+        }
+        for (int b = 0; b < kRedBufs; ++b) {
             mbar_init(&rfull[b], kComputeWarps);
             mbar_init(&rempty[b], kEpilogueWarps);
         }
@@ -148,10 +154,6 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     pdl_trigger();
     const int n_tiles = __ldcg(n_tiles_ptr);
     const int n_items = n_tiles * row_blocks;
-    // a contiguous run of items per CTA, tile-major: consecutive items are adjacent row
-    // blocks of one expert, so each CTA streams contiguous weight memory
-    const int item_begin = static_cast<int>((static_cast<long long>(n_items) * blockIdx.x) / gridDim.x);
-    const int item_end = static_cast<int>((static_cast<long long>(n_items) * (blockIdx.x + 1)) / gridDim.x);
 
     bool aborted = false;
 
@@ -166,7 +168,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
         int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
         auto fetch = [&](int it) {
-            if (it < item_end) {
+            if (it < n_items) {
                 const ExpertTile *tp = tiles + it / row_blocks;
                 nx_e = __ldcg(&tp->expert);
                 nx_p0 = __ldcg(&tp->p0);
@@ -188,10 +190,39 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     bulk_load(ast + i * kActStageBytes + (lane - 16) * kActPitch, pend_src[i], pend_bytes[i], &full[i]);
             h_ready = true;
         };
-        fetch(item_begin);
-        for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
+        // Items come from the call's work queue (an atomic counter, zeroed by the first kernel of
+        // the call) in tile-major order, so faster SMs take more of them and all SMs sweep the
+        // weight matrices together.  With few items per CTA (coarse items, decode sizes) a CTA
+        // first takes a contiguous run of 3/4 of its even share and then single items; with many,
+        // it takes 2 or 4 consecutive items per grab (fewer atomics on the counter).  Two grabs
+        // are always in flight, issued long before their ids are needed; the descriptor of the
+        // next item loads one item ahead.
+        const int per_cta = n_items / static_cast<int>(gridDim.x);
+        const int grab_items = per_cta < 16 ? 1 : (per_cta < 48 ? 2 : 4);
+        const int share = per_cta < 16 ? static_cast<int>((3LL * n_items) / (4LL * gridDim.x)) : 0;
+        const int static_total = share * static_cast<int>(gridDim.x);
+        int run = static_cast<int>(blockIdx.x) * share;
+        int run_end = run + share;
+        auto grab = [&]() { return lane == 0 ? atomicAdd(queue, 1) : 0; };
+        int g0 = grab(), g1 = grab();
+        auto take = [&]() -> int {
+            if (run >= run_end) {
+                run = static_total + grab_items * __shfl_sync(0xffffffffu, g0, 0);
+                run_end = run + grab_items;
+                g0 = g1;
+                g1 = grab();
+            }
+            return run++;
+        };
+        int next_id = take();
+        fetch(next_id);
+        for (;; ++item_ctr) {
+            const int item = next_id;
+            if (item >= n_items) break;
             const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, tok = nx_tok;
-            fetch(item + 1);
+            next_id = take();
+            fetch(next_id);
+            if (lane == 0) item_q[item_ctr % kItemQ] = item;   // published by the first stage's arrival
             const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
@@ -265,7 +296,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         }
         if (!h_ready) release_h();
         // let every copy this CTA issued land before the CTA can exit (stages and per-item scale
-        // rows are issued in order until a wait gives up, so the issued ones are a prefix)
+        // rows are issued in order until a wait gives up, so the issued ones are a prefix).  This
+        // comes before the end marker, whose arrival reuses the ring slot of stage
+        // stages_issued - kStages and would make that stage's phase look pending again.
         for (int i = 0; i < kStages && i < stages_issued; ++i) {
             const int sc = stages_issued - 1 - i;
             mbar_wait_drain(&full[sc % kStages], (sc / kStages) & 1, status);
@@ -273,6 +306,16 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         for (int i = 0; i < 2 && i < scales_issued; ++i) {
             const int j = scales_issued - 1 - i;
             mbar_wait_drain(&sfull[j & 1], (j >> 1) & 1, status);
+        }
+        {
+            // end marker: one more ring slot whose arrival carries item -1 and no copies
+            const int s = stage_ctr % kStages;
+            mbar_wait(&empty[s], ((stage_ctr / kStages) & 1) ^ 1, aborted, status);
+            aborted = __any_sync(0xffffffffu, aborted);
+            if (!aborted && lane == 0) {
+                item_q[item_ctr % kItemQ] = -1;
+                mbar_arrive(&full[s]);
+            }
         }
         return;
     }
@@ -284,14 +327,16 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         // nothing for the epilogue before the first item's partial sums; the down kernel's
         // epilogue waits for gate_up here so that its plain loads see the current call's data
         if (!kGateUp) pdl_wait();
-        int item_ctr = 0;
-        for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
+        for (int item_ctr = 0;; ++item_ctr) {
+            const int b = item_ctr % kRedBufs;
+            const float *rbuf = red + b * kRedFloats;
+            mbar_wait(&rfull[b], (item_ctr / kRedBufs) & 1, aborted, status);
+            if (aborted) break;
+            const int item = red_item[b];   // -1: no further item
+            if (item < 0) break;
             const ExpertTile *tp = tiles + item / row_blocks;
             const int rb = item % row_blocks;
             const int cnt = tp->count, p0 = tp->p0;
-            const int b = item_ctr & 1;
-            const float *rbuf = red + b * kRedFloats;
-            mbar_wait(&rfull[b], (item_ctr >> 1) & 1, aborted, status);
             float4 sums[2];
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
@@ -345,18 +390,19 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 
     // -------------------------------------------------------------------- compute warps
     const int g = lane >> 2, q = lane & 3;
-    const int pair = warp & 1;              // m-tiles 2*pair, 2*pair+1
-    const int kslot = warp >> 1;            // blocks kslot*kBlocksPerWarp .. of every stage
+    constexpr int kGroups = kItemMTiles / kWarpMTiles;
+    const int mgrp = warp % kGroups;        // m-tiles mgrp*kWarpMTiles ..
+    const int kslot = warp / kGroups;       // blocks kslot*kBlocksPerWarp .. of every stage
     const int col = (kslot * kBlocksPerWarp) >> 3;
     const int bb0 = (kslot * kBlocksPerWarp) & 7;
     const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
 
     // per m-tile: smem byte offsets (inside a stage) of the top/bottom rows' 16-byte blocks,
     // and scale-row indices (rows of the item's 64 weight rows)
-    int top_off[2], bot_off[2], top_sr[2], bot_sr[2];
+    int top_off[kWarpMTiles], bot_off[kWarpMTiles], top_sr[kWarpMTiles], bot_sr[kWarpMTiles];
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-        const int j = 2 * pair + m;
+    for (int m = 0; m < kWarpMTiles; ++m) {
+        const int j = mgrp * kWarpMTiles + m;
         if (kGateUp) {
             top_off[m] = col * kBoxBytes + (8 * j + g) * 128;
             bot_off[m] = (kBoxCols + col) * kBoxBytes + (8 * j + g) * 128;
@@ -374,20 +420,24 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
 
     int stage_ctr = 0, item_ctr = 0;
-    for (int item = item_begin; item < item_end; ++item, ++item_ctr) {
+    for (;; ++item_ctr) {
         const int b = item_ctr & 1;
+        // the item's first stage (or the end marker) names the item
+        mbar_wait(&full[stage_ctr % kStages], (stage_ctr / kStages) & 1, aborted, status);
+        if (aborted) break;
+        if (item_q[item_ctr % kItemQ] < 0) break;
         const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
         if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
 
-        float acc[2][4];
+        float acc[kWarpMTiles][4];
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
+        for (int m = 0; m < kWarpMTiles; ++m)
 #pragma unroll
             for (int r = 0; r < 4; ++r) acc[m][r] = 0.f;
 
         for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
             const int s = stage_ctr % kStages;
-            mbar_wait(&full[s], (stage_ctr / kStages) & 1, aborted, status);
+            if (c > 0) mbar_wait(&full[s], (stage_ctr / kStages) & 1, aborted, status);
             const uint8_t *st = wst + s * kStageBytes;
             const uint8_t *xa = ast + s * kActStageBytes + g * kActPitch;   // token g of the tile
             const uint8_t *sc_base = stage_scales ? sst + s * kStageScaleBytes : sbi;
@@ -399,7 +449,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (blk_base + bi) + 8 * q) * 2);
                 const int sw = (((bb0 + bi) ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
+                for (int m = 0; m < kWarpMTiles; ++m) {
                     const uint32_t wt = *reinterpret_cast<const uint32_t *>(st + top_off[m] + sw);
                     const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_off[m] + sw);
                     const float st_scale = e8m0_times2(sc_base[top_sr[m] * s_pitch + sc_col0 + bi]);
@@ -424,15 +474,25 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         __syncwarp();
         if (!stage_scales && lane == 0) mbar_arrive(&sempty[b]);
 
-        // park the K-slot partial sums for the epilogue warps
-        mbar_wait(&rempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
-        float *rbuf = red + b * kRedFloats;
+        // park the K-slot partial sums (and the item id) for the epilogue warps
+        const int rb = item_ctr % kRedBufs;
+        mbar_wait(&rempty[rb], ((item_ctr / kRedBufs) & 1) ^ 1, aborted, status);
+        float *rbuf = red + rb * kRedFloats;
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
-            *reinterpret_cast<float4 *>(rbuf + ((kslot * kItemMTiles + 2 * pair + m) * 32 + lane) * 4) =
+        for (int m = 0; m < kWarpMTiles; ++m)
+            *reinterpret_cast<float4 *>(rbuf + ((kslot * kItemMTiles + mgrp * kWarpMTiles + m) * 32 + lane) * 4) =
                 make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+        if (warp == 0 && lane == 0) red_item[rb] = item_q[item_ctr % kItemQ];
         __syncwarp();
-        if (lane == 0) mbar_arrive(&rfull[b]);
+        if (lane == 0) mbar_arrive(&rfull[rb]);
+    }
+    // end marker for the epilogue warps
+    const int rb = item_ctr % kRedBufs;
+    mbar_wait(&rempty[rb], ((item_ctr / kRedBufs) & 1) ^ 1, aborted, status);
+    if (!aborted) {
+        if (warp == 0 && lane == 0) red_item[rb] = -1;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rfull[rb]);
     }
 }
 
@@ -472,8 +532,9 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &sma
     const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
     int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     if (grid < 1) grid = 1;
+    int *queue = status + (kGateUp ? kQueueGateUp : kQueueDown);
     return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, smap,
-                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, status_out, K, I, H);
+                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, status_out, queue, K, I, H);
 }
 
 int grouped_smem_bytes(int K) { return smem_plan(K).total; }

@@ -12,6 +12,10 @@ namespace moe {
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = -5;
+// The call's 256-byte status block: word 0 is the status; words kQueueGateUp and kQueueDown
+// are the grouped kernels' work-queue counters, zeroed by the first kernel of the call.
+constexpr int kQueueGateUp = 8;
+constexpr int kQueueDown = 16;
 
 // Grouped GEMM tiling (both projections).
 constexpr int kTileTokens = 8;       // assignments per expert tile (one MMA n-tile)
@@ -25,7 +29,8 @@ constexpr int kActPitch = kChunkK * 2 + 64;         // one token's binary16 chun
 constexpr int kActStageBytes = kTileTokens * kActPitch;
 constexpr int kStages = 3;
 constexpr int kComputeWarps = 16;    // 2 m-tile pairs x 8 K slots
-constexpr int kKSlots = kComputeWarps / 2;
+constexpr int kWarpMTiles = 2;       // m-tiles per compute warp (the activation fragment serves both)
+constexpr int kKSlots = kComputeWarps * kWarpMTiles / kItemMTiles;
 constexpr int kEpilogueWarps = 2;
 constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact for |h| >= 2^-27
 
@@ -33,13 +38,42 @@ constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact
 // multiple of 16 bytes; otherwise the item's scale rows are copied once per item.
 __host__ __device__ inline bool per_stage_scales(int K) { return (K / 32) % 16 == 0; }
 
-// Router.
-constexpr int kRouteChunkH = 512;    // H elements per partial-logit chunk (H < 4096)
-constexpr int kMaxRouteSplits = 16;  // partial-logit chunks at most (H <= 16384)
-// Router chunk: 512 elements for H < 4096 (more CTAs), 1024 above (fewer partial sums).
-__host__ __device__ inline int route_chunk(int H) { return H >= 4096 ? 1024 : 512; }
-__host__ __device__ inline int route_splits(int H) { return (H + route_chunk(H) - 1) / route_chunk(H); }
-constexpr int kRouteTokens = 32;     // tokens per router CTA
+// Router logits on the tensor cores (route_plan picks the launch).  A CTA covers 16 experts,
+// one token block (8 tokens per MMA n-tile, `tiles` n-tiles) and `passes` K ranges of
+// 8 warps x 16 * steps elements; the `splits` CTAs of one expert group and token block cover H
+// between them and each writes its partial logits [split][M][E], summed in split order by
+// the top-k.  Small M: one n-tile and short K ranges, so hundreds of light CTAs share the
+// W_r read; large M: full-H CTAs (splits = 1) looping over their K ranges.  The plan uses a
+// fixed SM count so that workspace sizes do not depend on the device.
+constexpr int kRouteExperts = 16;
+constexpr int kRouteWarps = 8;
+constexpr int kPlanSMs = 148;
+struct RoutePlan {
+    int tiles;    // MMA n-tiles (8 tokens) per token block: 1 or 4
+    int steps;    // 16-K MMA steps per pass: 2 or 8
+    int splits;   // CTAs per (expert group, token block), each a partial-logit slice
+    int passes;   // K ranges per warp
+    int blocks_t; // token blocks
+};
+__host__ __device__ inline RoutePlan route_plan(int M, int H, int E)
+{
+    RoutePlan p;
+    p.tiles = M <= 8 ? 1 : 4;
+    p.steps = M <= 8 ? 2 : 8;
+    p.blocks_t = (M + 8 * p.tiles - 1) / (8 * p.tiles);
+    const int gx = (E + kRouteExperts - 1) / kRouteExperts;
+    const int units = (H + kRouteWarps * 16 * p.steps - 1) / (kRouteWarps * 16 * p.steps);
+    const long long base = static_cast<long long>(gx) * p.blocks_t;
+    const int cap = (p.tiles == 1 ? 4 : 1) * kPlanSMs;   // light CTAs share SMs, heavy ones do not
+    if (base * units <= cap) {
+        p.splits = units;
+    } else {
+        const long long sp = cap / base;
+        p.splits = sp < 1 ? 1 : static_cast<int>(sp);
+    }
+    p.passes = (units + p.splits - 1) / p.splits;
+    return p;
+}
 
 constexpr int kMaxE = 1024;
 constexpr int kMaxK = 32;
@@ -56,7 +90,7 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
 // Byte offsets of every buffer inside one call's workspace (256-byte aligned).
 struct Layout {
     size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, total;
-    int route_splits;   // number of H chunks of the router
+    int splits;   // router partial-logit slices (route_plan)
     int max_tiles;
 };
 
@@ -86,24 +120,33 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-// Router top-k and the permutation run as one single-CTA kernel when M*k <= kFusedSelectMaxN
-// and E <= kFusedSelectMaxE; otherwise as route_topk followed by the permutation kernel.
-constexpr int kFusedSelectThreads = 1024;
-constexpr int kFusedSelectMaxN = 1024;
-constexpr int kFusedSelectMaxE = 512;
+// Router top-k and the permutation run as one single-CTA kernel when M <= kFusedSelectMaxM,
+// M*k <= kPermuteThreads (one ranking round) and the M*E logits fit in shared memory; otherwise as route_topk (one warp per token
+// across the grid) followed by the permutation kernel (one ranking round per kPermuteThreads
+// assignments).  Both use kPermuteThreads threads.
+constexpr int kPermuteThreads = 1024;
+constexpr int kFusedSelectMaxM = 64;
+constexpr int kFusedSelectMaxLogits = 16384;   // M * E logits staged in shared memory (64 KB)
 __host__ __device__ inline bool fused_select(int M, int E, int k)
 {
-    return static_cast<long long>(M) * k <= kFusedSelectMaxN && E <= kFusedSelectMaxE;
+    return M <= kFusedSelectMaxM && static_cast<long long>(M) * k <= kPermuteThreads &&
+           static_cast<long long>(M) * E <= kFusedSelectMaxLogits;
+}
+// Dynamic shared memory of the ranking (rank_smem): two [warp][expert] u16 tables (counts and
+// prefix counts), four int arrays over E and a 33-int scan buffer.
+__host__ __device__ inline int permute_smem_bytes(int E)
+{
+    return 2 * (kPermuteThreads / 32) * E * 2 + 4 * E * 4 + 64 * 4;
 }
 
 // Kernel launchers (return cudaError_t of the launch).
 cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
-                                int32_t *status_out, int M, int H, int E, int splits, cudaStream_t s);
-cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
-                              int splits, cudaStream_t s, bool pdl);
-cudaError_t launch_route_select_permute(const float *partial, const float *bias, int32_t *ids, float *w,
+                                int32_t *status_out, int M, int H, int E, cudaStream_t s);
+cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
+                              int E, int k, cudaStream_t s, bool pdl);
+cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
                                         int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
-                                        int *n_tiles, int M, int E, int k, int splits, cudaStream_t s, bool pdl);
+                                        int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos,
                            ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,

@@ -1,30 +1,36 @@
-// permute.cu -- stand-alone route remap kernel and the expert-tile builder used
-// by the step-level entry points (see permute_impl.cuh for the algorithm).
+// permute.cu -- stand-alone route remap kernel (rank_and_scatter of permute_impl.cuh
+// over given topk_ids) and the expert-tile builder used by the step-level entry points.
 #include "permute_impl.cuh"
 
 namespace moe {
 
-__global__ void __launch_bounds__(1024, 1) permute_kernel(const int32_t *__restrict__ ids, int32_t *__restrict__ offsets,
-                                                          int32_t *__restrict__ sorted_ids,
-                                                          int32_t *__restrict__ inv_pos, ExpertTile *__restrict__ tiles,
-                                                          int *__restrict__ n_tiles, int n, int E, int k, int n2)
+// Route remap of given topk_ids (rank_and_scatter in rounds of kPermuteThreads assignments).
+__global__ void __launch_bounds__(kPermuteThreads, 1)
+permute_kernel(const int32_t *__restrict__ topk_ids, int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_ids,
+               int32_t *__restrict__ inv_pos, ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int n, int E,
+               int k)
 {
-    extern __shared__ uint32_t keys[];   // n2 (power of two >= n) entries
-    __shared__ int s_off[kMaxE + 1];
-    __shared__ int scan_buf[33];
+    extern __shared__ __align__(16) uint8_t smem[];
+    int *s_e = reinterpret_cast<int *>(smem + permute_smem_bytes(E));   // [n]
     pdl_wait();                          // topk_ids come from the previous kernel
     pdl_trigger();
-    for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-        uint32_t key = 0xFFFFFFFFu;
-        if (i < n) {
-            int e = ids[i];
-            if (e < 0 || e >= E) e = E;          // out-of-range ids sort after every expert
-            key = (static_cast<uint32_t>(e) << 16) | static_cast<uint32_t>(i);
+    // stage the ids with each thread's loads issued in batches before any is stored
+    constexpr int kBatch = 8;
+    for (int i0 = threadIdx.x; i0 < n; i0 += kBatch * kPermuteThreads) {
+        int v[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int i = i0 + b * kPermuteThreads;
+            v[b] = i < n ? topk_ids[i] : -1;
         }
-        keys[i] = key;
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int i = i0 + b * kPermuteThreads;
+            if (i < n) s_e[i] = v[b];
+        }
     }
     __syncthreads();
-    sort_and_emit(keys, n, n2, E, k, offsets, sorted_ids, inv_pos, tiles, n_tiles, s_off, scan_buf);
+    rank_and_scatter(s_e, n, E, k, rank_smem(smem, E), offsets, sorted_ids, inv_pos, tiles, n_tiles);
 }
 
 // Expert tiles from given offsets / sorted ids; also resets the call's status word.
@@ -35,7 +41,11 @@ __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__r
 {
     __shared__ int s_off[kMaxE + 1];
     __shared__ int scan_buf[33];
-    if (threadIdx.x == 0 && status) *status = kStatusOk;
+    if (threadIdx.x == 0 && status) {
+        status[0] = kStatusOk;
+        status[kQueueGateUp] = 0;
+        status[kQueueDown] = 0;
+    }
     for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
     emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
@@ -45,13 +55,11 @@ cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted
                            ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl)
 {
     const int n = M * k;
-    const int n2 = pow2_at_least(n);
-    const size_t smem = static_cast<size_t>(n2) * sizeof(uint32_t);
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(permute_kernel),
-                                    static_cast<int>(kMaxAssignments * sizeof(uint32_t)));
+    const int smem = permute_smem_bytes(E) + n * static_cast<int>(sizeof(int));
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(permute_kernel), smem);
     if (e != cudaSuccess) return e;
-    return launch_ex(permute_kernel, dim3(1), dim3(1024), smem, s, pdl, ids, offsets, sorted_ids, inv_pos, tiles,
-                     n_tiles, n, E, k, n2);
+    return launch_ex(permute_kernel, dim3(1), dim3(kPermuteThreads), smem, s, pdl, ids, offsets, sorted_ids, inv_pos,
+                     tiles, n_tiles, n, E, k);
 }
 
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,

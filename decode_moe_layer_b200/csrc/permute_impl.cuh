@@ -2,13 +2,19 @@
 // permutation kernel and the fused router-select + permutation kernel.
 //
 // "Direct M=2 route remap" row of "Post-Portfolio Device Attribution" ("MTP1
-// Post-Portfolio Eager-Cycle Profile").  Each assignment f = t*k + j is the
-// unique key (expert << 16) | f; a shared-memory bitonic sort of the keys gives
-// the stable expert-grouped order directly (keys are unique, so every sort
-// yields the same bytes).  Expert offsets are lower bounds found by binary
-// search in the sorted keys, and the expert tiles that drive the grouped GEMMs
-// come from a block-wide exclusive scan of ceil(count_e / kTileTokens).  No
-// atomics.  All functions are called by every thread of the CTA (a multiple of 32 threads).
+// Post-Portfolio Eager-Cycle Profile").  The expert-grouped order is the stable
+// counting sort of the assignments f = t*k + j by expert: position(f) =
+// offset[e_f] + rank(f), rank(f) = the number of earlier assignments on the same
+// expert.  One thread per assignment, in rounds of blockDim assignments:
+//  * a warp's lanes that share an expert find each other with __match_any_sync
+//    (rank inside the warp = matching lanes below it);
+//  * the lowest of them records the warp's count of that expert in a
+//    [warp][expert] table, one pass per expert turns the table into prefix counts
+//    (plus the counts of earlier rounds) and the thread reads its rank back.
+// Counts per expert come first (shared-memory atomics: order-free), then one block
+// scan of (tiles << 16 | count) gives every expert offset and tile base at once.
+// Two block barriers per round, no sort; every result is unique, so the bytes do
+// not depend on scheduling.
 #pragma once
 
 #include "common.cuh"
@@ -43,6 +49,191 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &t
     return warp_tot[warp] + incl - v;
 }
 
+// Shared memory of the ranking, carved from one dynamic buffer of permute_smem_bytes(E) bytes:
+// wc at 0, pref at 64 E, the int arrays at 128 E, the scan buffer at 144 E (+132 bytes).
+struct RankSmem {
+    uint16_t *wc;     // [32][E] counts of the current round's warps
+    uint16_t *pref;   // [32][E] their prefix counts (with earlier rounds)
+    int *cnt, *off, *tb, *base;   // [E] count, offset, first tile, assignments ranked so far
+    int *scan;        // 33
+};
+
+__device__ __forceinline__ RankSmem rank_smem(uint8_t *raw, int E)
+{
+    constexpr int kW = kPermuteThreads / 32;
+    RankSmem r;
+    r.wc = reinterpret_cast<uint16_t *>(raw);
+    r.pref = r.wc + kW * E;
+    int *ints = reinterpret_cast<int *>(raw + 2 * kW * E * 2);
+    r.cnt = ints;
+    r.off = ints + E;
+    r.tb = ints + 2 * E;
+    r.base = ints + 3 * E;
+    r.scan = ints + 4 * E;
+    return r;
+}
+
+// Stable expert-grouped order of n assignments whose experts are s_e[0..n) (shared memory).
+// Writes expert_offsets [E+1], sorted_ids [n], inv_pos [n] and, when tiles != nullptr, the
+// expert tiles and their count.  Assignments with an expert outside [0, E) are out of
+// contract: they are left out (inv_pos = -1, offsets[E] counts only the others) and never
+// index past an array.  Called by every thread of a kPermuteThreads-thread CTA.
+__device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, RankSmem sm,
+                                        int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_ids,
+                                        int32_t *__restrict__ inv_pos, ExpertTile *__restrict__ tiles,
+                                        int *__restrict__ n_tiles)
+{
+    constexpr int kW = kPermuteThreads / 32;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // only the warps that hold assignments in some round use table rows
+    const int rows = min(kW, (n + 31) / 32);
+    for (int i = tid; i < rows * E; i += kPermuteThreads) sm.wc[i] = 0;
+    for (int e = tid; e < E; e += kPermuteThreads) {
+        sm.cnt[e] = 0;
+        sm.base[e] = 0;
+    }
+    __syncthreads();
+    for (int f = tid; f < n; f += kPermuteThreads) {
+        const int e = s_e[f];
+        if (e >= 0 && e < E) atomicAdd(&sm.cnt[e], 1);
+    }
+    __syncthreads();
+    // offsets and tile bases: (tiles << 16) | count per expert, one scan (counts <= 16384)
+    const int mine = tid < E ? (((sm.cnt[tid] + kTileTokens - 1) / kTileTokens) << 16) | sm.cnt[tid] : 0;
+    int total = 0;
+    const int base = block_exclusive_scan(mine, sm.scan, total);   // ends with a block barrier
+    if (tid < E) {
+        sm.off[tid] = base & 0xFFFF;
+        sm.tb[tid] = base >> 16;
+        offsets[tid] = base & 0xFFFF;
+    }
+    if (tid == 0) {
+        offsets[E] = total & 0xFFFF;
+        if (tiles) *n_tiles = total >> 16;
+    }
+    for (int r0 = 0; r0 < n; r0 += kPermuteThreads) {
+        const int f = r0 + tid;
+        int e = f < n ? s_e[f] : -1;
+        if (e >= E) e = -1;
+        if (f < n && e < 0) inv_pos[f] = -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank_w = __popc(same & ((1u << lane) - 1u));
+        if (e >= 0 && rank_w == 0) sm.wc[warp * E + e] = static_cast<uint16_t>(__popc(same));
+        __syncthreads();
+        if (tid < E) {
+            const int active = min(kW, (n - r0 + 31) / 32);   // warps holding assignments this round
+            int c[kW];
+#pragma unroll
+            for (int w = 0; w < kW; ++w) c[w] = w < active ? sm.wc[w * E + tid] : 0;   // all loads first
+            int run = sm.base[tid];
+#pragma unroll
+            for (int w = 0; w < kW; ++w) {
+                if (w < active) {
+                    sm.wc[w * E + tid] = 0;
+                    sm.pref[w * E + tid] = static_cast<uint16_t>(run);
+                }
+                run += c[w];
+            }
+            sm.base[tid] = run;
+        }
+        __syncthreads();
+        if (e >= 0) {
+            const int rank = sm.pref[warp * E + e] + rank_w;
+            const int pos = sm.off[e] + rank;
+            sorted_ids[pos] = f;
+            inv_pos[f] = pos;
+            if (tiles) {
+                const int cnt = sm.cnt[e];
+                const int slot = rank % kTileTokens, tile_first = rank - slot;
+                ExpertTile *tp = tiles + sm.tb[e] + rank / kTileTokens;
+                const int t = f / k;
+                tp->tok[slot] = t;
+                if (slot == 0) {
+                    tp->expert = e;
+                    tp->p0 = sm.off[e] + tile_first;
+                    tp->count = min(kTileTokens, cnt - tile_first);
+                    tp->pad = 0;
+                }
+                if (rank == cnt - 1)   // the tile's last assignment repeats its token into the unused slots
+                    for (int j = slot + 1; j < kTileTokens; ++j) tp->tok[j] = t;
+            }
+        }
+    }
+}
+
+// The same stable order, offsets, sorted ids, inverse positions and tiles, computed by ONE
+// warp (the calling warp) for n assignments whose experts are s_e[0..n) (shared memory; the
+// experts of a fused top-k, all in [0, E)).  Shared scratch: cnt, off, tb [E] and rank [n].
+// Rounds of 32 assignments: each round's matching lanes get their rank from the running
+// per-expert count, whose leader then advances it; one warp scan of (tiles << 16 | count)
+// over the experts gives offsets and tile bases.  Only __syncwarp, no block barrier.
+__device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k, int *cnt, int *off, int *tb,
+                                             int *rank, int32_t *__restrict__ offsets,
+                                             int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
+                                             ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles)
+{
+    const int lane = threadIdx.x & 31;
+    for (int e = lane; e < E; e += 32) cnt[e] = 0;
+    __syncwarp();
+    for (int r0 = 0; r0 < n; r0 += 32) {
+        const int f = r0 + lane;
+        const int e = f < n ? s_e[f] : -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        const int rank_w = __popc(same & ((1u << lane) - 1u));
+        const int before = e >= 0 ? cnt[e] : 0;
+        __syncwarp();
+        if (e >= 0) {
+            rank[f] = before + rank_w;
+            if (rank_w == 0) cnt[e] = before + __popc(same);
+        }
+        __syncwarp();
+    }
+    // lane l scans the contiguous experts [l * per, (l + 1) * per)
+    const int per = (E + 31) / 32;
+    const int ea = min(E, lane * per), eb = min(E, ea + per);
+    int local = 0;
+    for (int e = ea; e < eb; ++e) local += (((cnt[e] + kTileTokens - 1) / kTileTokens) << 16) | cnt[e];
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, d);
+        if (lane >= d) incl += o;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int run = incl - local;
+    for (int e = ea; e < eb; ++e) {
+        off[e] = run & 0xFFFF;
+        tb[e] = run >> 16;
+        offsets[e] = run & 0xFFFF;
+        run += (((cnt[e] + kTileTokens - 1) / kTileTokens) << 16) | cnt[e];
+    }
+    if (lane == 0) {
+        offsets[E] = total & 0xFFFF;
+        *n_tiles = total >> 16;
+    }
+    __syncwarp();
+    for (int f = lane; f < n; f += 32) {
+        const int e = s_e[f];
+        const int r = rank[f];
+        const int pos = off[e] + r;
+        sorted_ids[pos] = f;
+        inv_pos[f] = pos;
+        const int c = cnt[e];
+        const int slot = r % kTileTokens, tile_first = r - slot;
+        ExpertTile *tp = tiles + tb[e] + r / kTileTokens;
+        const int t = f / k;
+        tp->tok[slot] = t;
+        if (slot == 0) {
+            tp->expert = e;
+            tp->p0 = off[e] + tile_first;
+            tp->count = min(kTileTokens, c - tile_first);
+            tp->pad = 0;
+        }
+        if (r == c - 1)   // the tile's last assignment repeats its token into the unused slots
+            for (int j = slot + 1; j < kTileTokens; ++j) tp->tok[j] = t;
+    }
+}
+
 // sorted_flat(p) returns the flat assignment id at position p of the expert-grouped order.
 // Each thread owns a contiguous run of ceil(E / blockDim) experts.
 template <typename SortedFlat>
@@ -69,57 +260,6 @@ __device__ inline void emit_tiles(const int *off, int E, int k, ExpertTile *tile
         }
     }
     if (threadIdx.x == 0) *n_tiles = total;
-}
-
-// keys[0..n2) hold the n assignment keys followed by 0xFFFFFFFF padding (n2 a power of two).
-// Sorts them, then writes expert_offsets [E+1], sorted_ids [n], inv_pos [n] and (when
-// tiles != nullptr) the expert tiles.  s_off must hold E+1 ints, scan_buf 33.
-__device__ inline void sort_and_emit(uint32_t *keys, int n, int n2, int E, int k, int32_t *__restrict__ offsets,
-                              int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
-                              ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int *s_off, int *scan_buf)
-{
-    const int tid = threadIdx.x;
-    for (int size = 2; size <= n2; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = tid; i < (n2 >> 1); i += blockDim.x) {
-                const int lo = 2 * i - (i & (stride - 1));
-                const int hi = lo + stride;
-                const bool up = (lo & size) == 0;
-                const uint32_t a = keys[lo], b = keys[hi];
-                if ((a > b) == up) {
-                    keys[lo] = b;
-                    keys[hi] = a;
-                }
-            }
-            __syncthreads();
-        }
-    }
-    for (int e = tid; e <= E; e += blockDim.x) {
-        const uint32_t target = static_cast<uint32_t>(e) << 16;
-        int lo = 0, hi = n;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (keys[mid] < target) lo = mid + 1;
-            else hi = mid;
-        }
-        s_off[e] = lo;
-        offsets[e] = lo;
-    }
-    for (int p = tid; p < n; p += blockDim.x) {
-        const int f = static_cast<int>(keys[p] & 0xFFFFu);
-        sorted_ids[p] = f;
-        inv_pos[f] = p;
-    }
-    if (tiles == nullptr) return;
-    __syncthreads();
-    emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(keys[p] & 0xFFFFu); });
-}
-
-__host__ __device__ inline int pow2_at_least(int n)
-{
-    int n2 = 2;
-    while (n2 < n) n2 <<= 1;
-    return n2;
 }
 
 }  // namespace moe

@@ -1,21 +1,26 @@
 // route.cu -- router select/normalize ("Native router select/normalize" row of
 // "Post-Portfolio Device Attribution", "MTP1 Post-Portfolio Eager-Cycle Profile").
 //
-//  1. route_logits: fp32 partial logits x.W_r^T over H chunks of 512 (H < 4096) or
-//     1024 elements.
-//     Grid (E/8, H chunks, M/32).  A CTA stages its 32 tokens' x chunk in shared
-//     memory once; each warp owns one expert, keeps that expert's W_r chunk in
-//     registers (read from HBM once per token tile) and reduces with a fixed
-//     xor-butterfly.  The CTAs of expert group 0 also write the binary16 copy of
-//     x that the grouped GEMM consumes and reset the call's status words.
-//  2. top-k per token, one warp per token: sum the chunk partials in chunk order,
-//     add the bias, select the top k by k rounds of a warp arg-max (warp max of
-//     order-preserving logit keys, then warp min of the ids holding it: value
-//     desc, expert id asc), and renormalise with a softmax over the k selected
-//     logits (equal to softmax-over-E followed by renormalisation).
-//     Either its own kernel (route_topk), or, for M*k <= kFusedSelectMaxN and
-//     E <= kFusedSelectMaxE, fused with the route remap into one single-CTA kernel
-//     (route_select_permute).
+//  1. route_logits: fp32 logits x.W_r^T on the tensor cores.  x is bf16 (exact in
+//     a bf16 MMA); each fp32 W_r value is split exactly into three bf16 terms
+//     hi + mid + lo (each residual of an fp32 value after rounding to 8 significant
+//     bits is exact in fp32, and the last one has at most 8 significant bits), so
+//     three bf16 m16n8k16 MMAs with fp32 accumulation form the fp32 dot product up
+//     to accumulation rounding.  A CTA = 16 experts x one token block x the K ranges
+//     of its 8 warps (route_plan); each warp splits its W_r slice once per pass and
+//     runs it against every token tile.  The 8 warp partials are summed in warp
+//     order in shared memory and the CTA writes its slice of partial logits
+//     [split][M][E]; the top-k adds the slices in split order.  The CTAs of expert
+//     group 0 also write the binary16 copy of x that the grouped GEMM consumes; the
+//     first CTA resets the call's status words.
+//  2. top-k per token, one warp per token: sum the slices, add the bias, select the
+//     top k by k rounds of a warp arg-max (warp max of order-preserving logit keys,
+//     then warp min of the ids holding it: value desc, expert id asc), and
+//     renormalise with a softmax over the k selected logits (equal to
+//     softmax-over-E followed by renormalisation).  Either its own kernel
+//     (route_topk), or, for small M (fused_select), fused with the route remap into
+//     one single-CTA kernel (route_select_permute) that first sums the slices into
+//     shared memory with all its threads.
 // Every reduction has a fixed order, so ids and weights are bitwise reproducible.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -34,114 +39,129 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-template <int kChunk>
-__global__ void __launch_bounds__(256) route_logits_kernel(const uint16_t *__restrict__ x,
-                                                           const float *__restrict__ wr, float *__restrict__ partial,
-                                                           __half *__restrict__ x16, int *status, int32_t *status_out,
-                                                           int M, int H, int E)
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
-    extern __shared__ __align__(16) uint16_t xs[];   // [kRouteTokens][kChunk] bf16 bits
-    pdl_trigger();
+    __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);   // .x (low half) = lo
+    return *reinterpret_cast<uint32_t *>(&b);
+}
+
+// (a, b) -> three bf16x2 registers with hi + mid + lo == (a, b) exactly.
+__device__ __forceinline__ void split3_bf16x2(float a, float b, uint32_t &hi, uint32_t &mid, uint32_t &lo)
+{
+    hi = pack_bf16x2(a, b);
+    const float ra = a - bf16_lo(hi), rb = b - bf16_hi(hi);
+    mid = pack_bf16x2(ra, rb);
+    lo = pack_bf16x2(ra - bf16_lo(mid), rb - bf16_hi(mid));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Fragment K order: inside each 16-K step, thread q (= lane & 3) holds the 4 consecutive K
+// elements 4q..4q+3 as MMA k-slots (2q, 2q+1, 2q+8, 2q+9) of both operands, so W_r rows load
+// as float4 and x rows as 8-byte words; the MMA sums over the same K either way.
+template <int kSteps, int kTiles>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr, float *__restrict__ partial,
+                    __half *__restrict__ x16, int *status, int32_t *status_out, int M, int H, int E, int passes)
+{
+    constexpr int kPassK = 16 * kSteps;
+    constexpr int kTokens = 8 * kTiles;
+    constexpr int kPitch = kTokens + 8;                 // padded row of the warp partials
+    __shared__ __align__(16) float red[kRouteWarps][kRouteExperts][kPitch];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, q = lane & 3;
+    const int e0 = blockIdx.x * kRouteExperts;
     const int split = blockIdx.y;
-    const int h0 = split * kChunk;
-    const int len = min(H - h0, kChunk);              // multiple of 32
-    const int t0 = blockIdx.z * kRouteTokens;
-    const int nt = min(kRouteTokens, M - t0);
+    const int t0 = blockIdx.z * kTokens;
+    const bool write_x16 = (blockIdx.x == 0) && (x16 != nullptr);
+    pdl_trigger();
     if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
-        if (status) *status = kStatusOk;
+        if (status) {
+            status[0] = kStatusOk;
+            status[kQueueGateUp] = 0;
+            status[kQueueDown] = 0;
+        }
         if (status_out) *status_out = kStatusOk;
     }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 8 + warp;
-
-    // this warp's expert chunk of W_r, requested before the x staging so both loads overlap
-    constexpr int kVec = kChunk / 128;   // float4 per lane
-    float4 w[kVec];
+    const int wg = split * kRouteWarps + warp;              // this warp's index along H
+    const int ea = e0 + g, eb = e0 + g + 8;                 // its two W_r rows
+    float acc[kTiles][4];
 #pragma unroll
-    for (int i = 0; i < kVec; ++i) {
-        const int c = 128 * i + 4 * lane;
-        w[i] = (e < E && c < len) ? *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(e) * H + h0 + c)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-
-    const int vec_per_row = len / 8;
-    const int n_vec = nt * vec_per_row;
-    const bool write_x16 = (blockIdx.x == 0) && (x16 != nullptr);
-    // a thread's x loads are issued in batches before any is stored, so they overlap
-    constexpr int kBatch = 8;
-    for (int i0 = threadIdx.x; i0 < n_vec; i0 += kBatch * blockDim.x) {
-        uint4 v[kBatch];
+    for (int j = 0; j < kTiles; ++j)
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int i = i0 + b * blockDim.x;
-            if (i < n_vec) {
-                const int r = i / vec_per_row, c = i - r * vec_per_row;
-                v[b] = *reinterpret_cast<const uint4 *>(x + static_cast<size_t>(t0 + r) * H + h0 + 8 * c);
+        for (int r = 0; r < 4; ++r) acc[j][r] = 0.f;
+    for (int pass = 0; pass < passes; ++pass) {
+        const int kw = (wg * passes + pass) * kPassK;       // first K of this pass
+        // issue every load of the pass before any use: W_r rows and the token tiles' x words
+        float4 wa[kSteps], wb[kSteps];
+        uint2 xv[kTiles][kSteps];
+#pragma unroll
+        for (int s = 0; s < kSteps; ++s) {
+            const int kk = kw + 16 * s + 4 * q;
+            const bool kin = kk < H;   // H % 32 == 0: a 4-element group is wholly in or out
+            wa[s] = (kin && ea < E) ? *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(ea) * H + kk)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            wb[s] = (kin && eb < E) ? *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(eb) * H + kk)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < kTiles; ++j) {
+                const int t = t0 + 8 * j + g;
+                xv[j][s] = (kin && t < M) ? *reinterpret_cast<const uint2 *>(x + static_cast<size_t>(t) * H + kk)
+                                          : make_uint2(0u, 0u);
             }
         }
 #pragma unroll
-        for (int b = 0; b < kBatch; ++b) {
-            const int i = i0 + b * blockDim.x;
-            if (i < n_vec) {
-                const int r = i / vec_per_row, c = i - r * vec_per_row;
-                *reinterpret_cast<uint4 *>(xs + r * kChunk + 8 * c) = v[b];
-                if (write_x16) {
-                    uint4 o;
-                    o.x = bf16x2_to_f16x2(v[b].x);
-                    o.y = bf16x2_to_f16x2(v[b].y);
-                    o.z = bf16x2_to_f16x2(v[b].z);
-                    o.w = bf16x2_to_f16x2(v[b].w);
-                    *reinterpret_cast<uint4 *>(x16 + static_cast<size_t>(t0 + r) * H + h0 + 8 * c) = o;
+        for (int s = 0; s < kSteps; ++s) {
+            uint32_t hi[4], mid[4], lo[4];
+            split3_bf16x2(wa[s].x, wa[s].y, hi[0], mid[0], lo[0]);   // row g,   K 4q, 4q+1
+            split3_bf16x2(wb[s].x, wb[s].y, hi[1], mid[1], lo[1]);   // row g+8, K 4q, 4q+1
+            split3_bf16x2(wa[s].z, wa[s].w, hi[2], mid[2], lo[2]);   // row g,   K 4q+2, 4q+3
+            split3_bf16x2(wb[s].z, wb[s].w, hi[3], mid[3], lo[3]);   // row g+8, K 4q+2, 4q+3
+#pragma unroll
+            for (int j = 0; j < kTiles; ++j) {
+                if (t0 + 8 * j >= M) continue;   // warp-uniform
+                mma_bf16_16816(acc[j], hi, xv[j][s].x, xv[j][s].y);
+                mma_bf16_16816(acc[j], mid, xv[j][s].x, xv[j][s].y);
+                mma_bf16_16816(acc[j], lo, xv[j][s].x, xv[j][s].y);
+            }
+        }
+        if (write_x16) {
+#pragma unroll
+            for (int s = 0; s < kSteps; ++s) {
+                const int kk = kw + 16 * s + 4 * q;
+#pragma unroll
+                for (int j = 0; j < kTiles; ++j) {
+                    const int t = t0 + 8 * j + g;
+                    if (kk < H && t < M)
+                        *reinterpret_cast<uint2 *>(x16 + static_cast<size_t>(t) * H + kk) =
+                            make_uint2(bf16x2_to_f16x2(xv[j][s].x), bf16x2_to_f16x2(xv[j][s].y));
                 }
             }
         }
+    }
+    // warp partials: accumulator rows g, g+8 (experts), columns 2q, 2q+1 of tile j (tokens)
+#pragma unroll
+    for (int j = 0; j < kTiles; ++j) {
+        *reinterpret_cast<float2 *>(&red[warp][g][8 * j + 2 * q]) = make_float2(acc[j][0], acc[j][1]);
+        *reinterpret_cast<float2 *>(&red[warp][g + 8][8 * j + 2 * q]) = make_float2(acc[j][2], acc[j][3]);
     }
     __syncthreads();
-
-    if (e >= E) return;
-
-    for (int tg = 0; tg < nt; tg += 8) {
-        float acc[8];
+    for (int i = threadIdx.x; i < kRouteExperts * kTokens; i += blockDim.x) {
+        const int tl = i / kRouteExperts, el = i % kRouteExperts;   // consecutive threads: consecutive experts
+        const int e = e0 + el, t = t0 + tl;
+        if (e < E && t < M) {
+            float v = 0.f;
 #pragma unroll
-        for (int tt = 0; tt < 8; ++tt) acc[tt] = 0.f;
-#pragma unroll
-        for (int i = 0; i < kVec; ++i) {
-            const int c = 128 * i + 4 * lane;
-            if (c < len) {
-#pragma unroll
-                for (int tt = 0; tt < 8; ++tt) {
-                    if (tg + tt < nt) {
-                        const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (tg + tt) * kChunk + c);
-                        float a = acc[tt];
-                        a = fmaf(bf16_lo(xv.x), w[i].x, a);
-                        a = fmaf(bf16_hi(xv.x), w[i].y, a);
-                        a = fmaf(bf16_lo(xv.y), w[i].z, a);
-                        a = fmaf(bf16_hi(xv.y), w[i].w, a);
-                        acc[tt] = a;
-                    }
-                }
-            }
+            for (int w = 0; w < kRouteWarps; ++w) v += red[w][el][tl];
+            partial[(static_cast<size_t>(split) * M + t) * E + e] = v;
         }
-        // transpose-reduce: 3 halving exchanges leave each lane one token's sum over 8 lanes
-        // (token index = lane bits 4,3,2), 2 more levels finish the 32-lane sum; 9 shuffles
-        const bool b4 = (lane >> 4) & 1, b3 = (lane >> 3) & 1, b2 = (lane >> 2) & 1;
-        float r1[4], r2[2];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float keep = b4 ? acc[i + 4] : acc[i], send = b4 ? acc[i] : acc[i + 4];
-            r1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const float keep = b3 ? r1[i + 2] : r1[i], send = b3 ? r1[i] : r1[i + 2];
-            r2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-        float mine = (b2 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? r2[0] : r2[1], 4);
-        mine += __shfl_xor_sync(0xffffffffu, mine, 2);
-        mine += __shfl_xor_sync(0xffffffffu, mine, 1);
-        const int tt = 4 * b4 + 2 * b3 + b2;
-        if ((lane & 3) == 0 && tg + tt < nt)
-            partial[(static_cast<size_t>(split) * M + t0 + tg + tt) * E + e] = mine;
     }
 }
 
@@ -157,33 +177,15 @@ __device__ __forceinline__ float from_ordered_key(uint32_t k)
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// One warp selects token t's top k.  Lane j < k ends with (sel_e, sel_w) of slot j.
-// Each round: every lane offers its best untaken (logit, id); a warp max over the
-// ordered logit keys and a warp min over the ids of the lanes holding that max pick
-// the winner (value desc, ties -> lower id).
+// One warp selects a token's top k from its E logits, lane-strided in v (v[j] = expert
+// lane + 32 j, -inf past E).  Lane j < k ends with (sel_e, sel_w) of slot j.  Each round:
+// every lane offers its best untaken (logit, id); a warp max over the ordered logit keys and a
+// warp min over the ids of the lanes holding that max pick the winner (value desc, ties ->
+// lower id).
 template <int kPerLane>
-__device__ __forceinline__ void select_topk(const float *__restrict__ partial, const float *__restrict__ bias, int t,
-                                            int M, int E, int k, int splits, int &sel_e, float &sel_w)
+__device__ __forceinline__ void topk_from_values(const float (&v)[kPerLane], int E, int k, int &sel_e, float &sel_w)
 {
     const int lane = threadIdx.x & 31;
-    float v[kPerLane];
-#pragma unroll
-    for (int j = 0; j < kPerLane; ++j) {
-        const int e = lane + 32 * j;
-        float s = -CUDART_INF_F;
-        if (e < E) {
-            // the splits' loads are independent: issue them together, then add in split order
-            float part[kMaxRouteSplits];
-#pragma unroll
-            for (int sp = 0; sp < kMaxRouteSplits; ++sp)
-                part[sp] = sp < splits ? partial[(static_cast<size_t>(sp) * M + t) * E + e] : 0.f;
-            s = 0.f;
-#pragma unroll
-            for (int sp = 0; sp < kMaxRouteSplits; ++sp) s += part[sp];
-            if (bias) s += bias[e];
-        }
-        v[j] = s;
-    }
     uint32_t taken = 0;
     float sel_v = 0.f, vmax = 0.f;
     sel_e = 0;
@@ -220,55 +222,106 @@ __device__ __forceinline__ void select_topk(const float *__restrict__ partial, c
 }
 
 template <int kPerLane>
-__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ partial,
+__global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ partial, int splits,
                                                          const float *__restrict__ bias, int32_t *__restrict__ ids,
-                                                         float *__restrict__ wout, int M, int E, int k, int splits)
+                                                         float *__restrict__ wout, int M, int E, int k)
 {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= M) return;
+    float v[kPerLane];
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) v[j] = 0.f;
+    for (int sp = 0; sp < splits; ++sp) {   // slices in split order; each round's loads are independent
+#pragma unroll
+        for (int j = 0; j < kPerLane; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E) v[j] += partial[(static_cast<size_t>(sp) * M + t) * E + e];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) {
+        const int e = lane + 32 * j;
+        v[j] = e < E ? (bias ? v[j] + bias[e] : v[j]) : -CUDART_INF_F;
+    }
     int sel_e;
     float sel_w;
-    select_topk<kPerLane>(partial, bias, t, M, E, k, splits, sel_e, sel_w);
+    topk_from_values<kPerLane>(v, E, k, sel_e, sel_w);
     if (lane < k) {
         ids[static_cast<size_t>(t) * k + lane] = sel_e;
         wout[static_cast<size_t>(t) * k + lane] = sel_w;
     }
 }
 
-// Top-k of every token (warps loop over the tokens) and the route remap, in one CTA of
-// kFusedSelectThreads threads, for n = M*k <= kFusedSelectMaxN assignments and E <= kFusedSelectMaxE.
-// Thread f owns assignment f.  Its stable rank inside its expert (the number of earlier
-// assignments routed to the same expert) is its rank among the matching lanes of its warp
-// (__match_any_sync) plus the counts of that expert in the earlier warps, kept in a
-// [warp][expert] table that one pass per expert turns into prefix counts.  One block scan
-// of (tiles, count) per expert gives every expert offset and tile base; thread f then writes
-// its sorted position, inverse position and tile slot directly.  Four block barriers, no sort.
+// Sums of the partial-logit slices in split order (+ bias) into dst[0..n_log), by all threads.
+// A thread keeps kBatch logits x kChunk slices of loads in flight before adding them.
+template <int kBatch, int kChunk>
+__device__ __forceinline__ void stage_logits(const float *__restrict__ partial, int splits, const float *__restrict__ bias,
+                                             int n_log, int E, float *dst)
+{
+    for (int i0 = threadIdx.x; i0 < n_log; i0 += kBatch * blockDim.x) {
+        float acc[kBatch];
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) acc[b] = 0.f;
+        for (int sp0 = 0; sp0 < splits; sp0 += kChunk) {
+            float v[kBatch][kChunk];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+                for (int u = 0; u < kChunk; ++u) {
+                    const int i = i0 + b * blockDim.x;
+                    v[b][u] = (i < n_log && sp0 + u < splits) ? partial[static_cast<size_t>(sp0 + u) * n_log + i] : 0.f;
+                }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+                for (int u = 0; u < kChunk; ++u) acc[b] += v[b][u];
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; ++b) {
+            const int i = i0 + b * blockDim.x;
+            if (i < n_log) dst[i] = bias ? acc[b] + bias[i % E] : acc[b];
+        }
+    }
+}
+
+// Top-k of every token and the route remap, in one CTA of kPermuteThreads threads, when
+// fused_select(M, E, k): all threads sum the partial-logit slices into shared memory, warps
+// take the tokens' top-k, then warp 0 alone ranks and scatters the M*k assignments
+// (warp_rank_and_scatter) while the other warps exit.
 template <int kPerLane>
-__global__ void __launch_bounds__(kFusedSelectThreads, 1)
-route_select_permute_kernel(const float *__restrict__ partial, const float *__restrict__ bias,
+__global__ void __launch_bounds__(kPermuteThreads, 1)
+route_select_permute_kernel(const float *__restrict__ partial, int splits, const float *__restrict__ bias,
                             int32_t *__restrict__ ids, float *__restrict__ wout, int32_t *__restrict__ offsets,
                             int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
-                            ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k, int splits)
+                            ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k)
 {
-    constexpr int kWarps = kFusedSelectThreads / 32;
-    static_assert(kFusedSelectMaxN <= kFusedSelectThreads, "one thread per assignment");
-    __shared__ int s_e[kFusedSelectMaxN];                        // expert of assignment f
-    __shared__ uint16_t s_wc[kWarps][kFusedSelectMaxE];          // per-warp counts, then prefix counts
-    __shared__ int s_off[kFusedSelectMaxE], s_cnt[kFusedSelectMaxE], s_tb[kFusedSelectMaxE];
-    __shared__ int scan_buf[33];
-    const int n = M * k;
+    extern __shared__ __align__(16) uint8_t smem[];
+    __shared__ int s_e[kPermuteThreads];      // expert of assignment f
+    __shared__ int s_rank[kPermuteThreads];   // its rank inside the expert
+    float *s_log = reinterpret_cast<float *>(smem);                      // [M][E]
+    int *s_cnt = reinterpret_cast<int *>(smem) + M * E;                   // [E] x 3
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // the count table is cleared while the previous kernel may still run
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) s_wc[i / E][i % E] = 0;
     pdl_wait();
     pdl_trigger();
-    for (int t = warp; t < M; t += kWarps) {
+    const int n_log = M * E;
+    if (n_log <= kPermuteThreads)
+        stage_logits<1, 32>(partial, splits, bias, n_log, E, s_log);
+    else
+        stage_logits<4, 8>(partial, splits, bias, n_log, E, s_log);
+    __syncthreads();
+    for (int t = warp; t < M; t += kPermuteThreads / 32) {
+        float v[kPerLane];
+#pragma unroll
+        for (int j = 0; j < kPerLane; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = e < E ? s_log[t * E + e] : -CUDART_INF_F;
+        }
         int sel_e;
         float sel_w;
-        select_topk<kPerLane>(partial, bias, t, M, E, k, splits, sel_e, sel_w);
+        topk_from_values<kPerLane>(v, E, k, sel_e, sel_w);
         if (lane < k) {
             const int f = t * k + lane;
             ids[f] = sel_e;
@@ -277,56 +330,9 @@ route_select_permute_kernel(const float *__restrict__ partial, const float *__re
         }
     }
     __syncthreads();
-    // rank among the lanes of this warp routed to the same expert (lanes past n carry -1)
-    const int f = threadIdx.x;
-    const int e = f < n ? s_e[f] : -1;
-    const unsigned same = __match_any_sync(0xffffffffu, e);
-    const int rank_w = __popc(same & ((1u << lane) - 1u));
-    if (e >= 0 && rank_w == 0) s_wc[warp][e] = static_cast<uint16_t>(__popc(same));
-    __syncthreads();
-    // per expert: prefix counts over the warps, the expert's total and its tile count
-    int packed = 0;                       // (tiles << 16) | count
-    if (threadIdx.x < E) {
-        int run = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int c = s_wc[w][threadIdx.x];
-            s_wc[w][threadIdx.x] = static_cast<uint16_t>(run);
-            run += c;
-        }
-        packed = (((run + kTileTokens - 1) / kTileTokens) << 16) | run;
-        s_cnt[threadIdx.x] = run;
-    }
-    int total = 0;
-    const int base = block_exclusive_scan(packed, scan_buf, total);   // ends with a block barrier
-    if (threadIdx.x < E) {
-        s_off[threadIdx.x] = base & 0xFFFF;
-        s_tb[threadIdx.x] = base >> 16;
-        offsets[threadIdx.x] = base & 0xFFFF;
-    }
-    if (threadIdx.x == 0) {
-        offsets[E] = n;
-        *n_tiles = total >> 16;
-    }
-    __syncthreads();
-    if (e >= 0) {
-        const int rank = s_wc[warp][e] + rank_w;
-        const int pos = s_off[e] + rank;
-        sorted_ids[pos] = f;
-        inv_pos[f] = pos;
-        const int cnt = s_cnt[e];
-        const int slot = rank % kTileTokens, tile_first = rank - slot;
-        ExpertTile *tp = tiles + s_tb[e] + rank / kTileTokens;
-        const int t = f / k;
-        tp->tok[slot] = t;
-        if (slot == 0) {
-            tp->expert = e;
-            tp->p0 = s_off[e] + tile_first;
-            tp->count = min(kTileTokens, cnt - tile_first);
-            tp->pad = 0;
-        }
-        if (rank == cnt - 1)   // the tile's last assignment repeats its token into the unused slots
-            for (int j = slot + 1; j < kTileTokens; ++j) tp->tok[j] = t;
-    }
+    if (warp != 0) return;
+    warp_rank_and_scatter(s_e, M * k, E, k, s_cnt, s_cnt + E, s_cnt + 2 * E, s_rank, offsets, sorted_ids, inv_pos,
+                          tiles, n_tiles);
 }
 
 __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
@@ -343,54 +349,65 @@ __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restr
     reinterpret_cast<uint4 *>(x16)[i] = o;
 }
 
-cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
-                                int32_t *status_out, int M, int H, int E, int splits, cudaStream_t s)
+template <int kSteps, int kTiles>
+static cudaError_t logits_launch(const void *x, const float *router_w, float *partial, __half *x16, int *status,
+                                 int32_t *status_out, int M, int H, int E, const RoutePlan &plan, cudaStream_t s)
 {
-    const int chunk = route_chunk(H);
-    const size_t smem = static_cast<size_t>(kRouteTokens) * chunk * sizeof(uint16_t);
-    auto kern = chunk == 1024 ? route_logits_kernel<1024> : route_logits_kernel<512>;
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    dim3 grid((E + 7) / 8, splits, (M + kRouteTokens - 1) / kRouteTokens);
+    const dim3 grid((E + kRouteExperts - 1) / kRouteExperts, plan.splits, plan.blocks_t);
     // first kernel of a call: fully ordered after whatever precedes it in the stream
-    kern<<<grid, 256, smem, s>>>(static_cast<const uint16_t *>(x), router_w, partial, x16, status, status_out, M, H, E);
+    route_logits_kernel<kSteps, kTiles><<<grid, kRouteWarps * 32, 0, s>>>(
+        static_cast<const uint16_t *>(x), router_w, partial, x16, status, status_out, M, H, E, plan.passes);
     return cudaGetLastError();
 }
 
-template <int P>
-static cudaError_t topk_p(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
-                          int splits, cudaStream_t s, bool pdl)
+cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
+                                int32_t *status_out, int M, int H, int E, cudaStream_t s)
 {
-    return launch_ex(route_topk_kernel<P>, dim3((M + 7) / 8), dim3(256), 0, s, pdl, partial, bias, ids, w, M, E, k,
-                     splits);
-}
-
-cudaError_t launch_route_topk(const float *partial, const float *bias, int32_t *ids, float *w, int M, int E, int k,
-                              int splits, cudaStream_t s, bool pdl)
-{
-    if (E <= 32) return topk_p<1>(partial, bias, ids, w, M, E, k, splits, s, pdl);
-    if (E <= 64) return topk_p<2>(partial, bias, ids, w, M, E, k, splits, s, pdl);
-    if (E <= 128) return topk_p<4>(partial, bias, ids, w, M, E, k, splits, s, pdl);
-    if (E <= 256) return topk_p<8>(partial, bias, ids, w, M, E, k, splits, s, pdl);
-    if (E <= 512) return topk_p<16>(partial, bias, ids, w, M, E, k, splits, s, pdl);
-    return topk_p<32>(partial, bias, ids, w, M, E, k, splits, s, pdl);
+    const RoutePlan plan = route_plan(M, H, E);
+    if (plan.tiles == 1 && plan.steps == 2)
+        return logits_launch<2, 1>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
+    if (plan.tiles == 4 && plan.steps == 8)
+        return logits_launch<8, 4>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
+    return cudaErrorInvalidConfiguration;   // route_plan yields only the two shapes above
 }
 
 template <int P>
-static cudaError_t select_permute_p(const float *partial, const float *bias, int32_t *ids, float *w, int32_t *offsets,
-                                    int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles, int *n_tiles, int M,
-                                    int E, int k, int splits, cudaStream_t s, bool pdl)
+static cudaError_t topk_p(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M, int E,
+                          int k, cudaStream_t s, bool pdl)
 {
-    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kFusedSelectThreads), 0, s, pdl, partial, bias,
-                     ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, splits);
+    return launch_ex(route_topk_kernel<P>, dim3((M + 7) / 8), dim3(256), 0, s, pdl, partial, splits, bias, ids, w, M,
+                     E, k);
 }
 
-cudaError_t launch_route_select_permute(const float *partial, const float *bias, int32_t *ids, float *w,
+cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
+                              int E, int k, cudaStream_t s, bool pdl)
+{
+    if (E <= 32) return topk_p<1>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+    if (E <= 64) return topk_p<2>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+    if (E <= 128) return topk_p<4>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+    if (E <= 256) return topk_p<8>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+    if (E <= 512) return topk_p<16>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+    return topk_p<32>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+}
+
+template <int P>
+static cudaError_t select_permute_p(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
+                                    int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
+                                    int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl)
+{
+    const int smem = (M * E + 3 * E) * static_cast<int>(sizeof(float));
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>), smem);
+    if (e != cudaSuccess) return e;
+    return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kPermuteThreads), smem, s, pdl, partial, splits,
+                     bias, ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k);
+}
+
+cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
                                         int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
-                                        int *n_tiles, int M, int E, int k, int splits, cudaStream_t s, bool pdl)
+                                        int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl)
 {
-#define MOE_SEL(P) select_permute_p<P>(partial, bias, ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, \
-                                       splits, s, pdl)
+#define MOE_SEL(P) select_permute_p<P>(partial, splits, bias, ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, \
+                                       E, k, s, pdl)
     if (E <= 32) return MOE_SEL(1);
     if (E <= 64) return MOE_SEL(2);
     if (E <= 128) return MOE_SEL(4);

@@ -7,8 +7,8 @@
 // steps to keep its latency predictable, or code running where the CUDA
 // allocation calls are not allowed.  moe_route uses a library-owned workspace
 // that is grown with cudaMalloc on first use; moe_route_noalloc runs the same
-// two router kernels but keeps their scratch -- the per-chunk partial logits and
-// the call's status word -- in a fixed device array compiled into the library.
+// two router kernels but keeps their scratch -- the router's partial-logit slices
+// and the call's status word -- in a fixed device array compiled into the library.
 #include <mutex>
 
 #include "moe.h"
@@ -17,8 +17,8 @@
 namespace moe {
 
 // Scratch of moe_route_noalloc: 256 bytes of status, then the partial logits
-// [route_splits(H)][M][E] fp32.  Every GPU that loads the library holds these 4 MiB
-// until the process exits.
+// [splits][M][E] fp32 (splits from route_plan).  Every GPU that loads the library holds
+// these 4 MiB until the process exits.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 constexpr size_t kNoAllocStatusBytes = 256;
 static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
@@ -60,7 +60,7 @@ extern "C" int moe_route_noalloc(const void *x_bf16, const float *router_w, cons
     if ((ax % 16) || (aw % 16) || (reinterpret_cast<uintptr_t>(topk_ids) % 4) ||
         (reinterpret_cast<uintptr_t>(topk_w) % 4) || (router_bias && reinterpret_cast<uintptr_t>(router_bias) % 4))
         return MOE_ERR_INVALID_ARG;
-    const int splits = route_splits(H);
+    const int splits = route_plan(M, H, E).splits;
     const size_t need = kNoAllocStatusBytes + static_cast<size_t>(splits) * M * E * sizeof(float);
     if (need > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
     void *base = nullptr;
@@ -68,11 +68,11 @@ extern "C" int moe_route_noalloc(const void *x_bf16, const float *router_w, cons
     if (rc != MOE_OK) return rc;
     int *status = static_cast<int *>(base);
     float *partial = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + kNoAllocStatusBytes);
-    // every partial logit the top-k kernel reads is written first by the logits kernel,
-    // so nothing in the array has to start at zero
-    cudaError_t e = launch_route_logits(x_bf16, router_w, partial, nullptr, status, nullptr, M, H, E, splits, stream);
+    // every partial logit the top-k kernel reads is written first by the logits kernel, so
+    // nothing in the array has to start at zero
+    cudaError_t e = launch_route_logits(x_bf16, router_w, partial, nullptr, status, nullptr, M, H, E, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = launch_route_topk(partial, router_bias, topk_ids, topk_w, M, E, k, splits, stream, false);
+    e = launch_route_topk(partial, splits, router_bias, topk_ids, topk_w, M, E, k, stream, false);
     if (e != cudaSuccess) return cuda_fail(e);
     return MOE_OK;
 }

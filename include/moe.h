@@ -149,11 +149,14 @@ int moe_mxfp4_forward(const void *x, const float *router_w, const uint8_t *w13_q
  * point where they route (an allocator that owns all device memory, a decode loop
  * that must not allocate between steps).  The pages have no counterpart: this is
  * an interface choice of this library.  Same arguments, results and checks as
- * moe_route; the scratch (partial logits and a status word) lives in a 4 MiB
- * device array compiled into the library instead of the library-owned workspace.
- *   - Limit: 256 + S * M * E * 4 bytes must fit in 4 MiB, S = ceil(H/512) for
- *     H < 4096 and ceil(H/1024) above (for example M <= 2048 at H=2048, E=128);
- *     larger shapes return MOE_ERR_WORKSPACE and enqueue nothing.
+ * moe_route; the scratch (the router's fp32 partial logits and a status word)
+ * lives in a 4 MiB device array compiled into the library instead of the
+ * library-owned workspace.
+ *   - Limit: 256 + S * M * E * 4 bytes must fit in 4 MiB, where S is the number of
+ *     H slices the router splits each expert group into: ceil(H / 256) for M <= 8,
+ *     ceil(H / 1024) for larger M, reduced toward 1 as M * E grows (for example
+ *     33 KB at M = 8, H = 2048, E = 128; 1 MB at M = 1024, H = 7168, E = 256).
+ *     Larger shapes return MOE_ERR_WORKSPACE and enqueue nothing.
  *   - The first call on a device looks the array's device address up (once per
  *     device); make that first call before any stream capture.
  *   - Calls no cudaMalloc/cudaFree.  Every call shares the one array, which keeps

@@ -38,6 +38,6 @@ def test_noalloc_route_rejects_sizes_beyond_its_scratch():
     import decode_moe_layer_b200 as moe
     lib = moe.load()
     a = ctypes.c_void_p(0x1000)
-    # 256 + 14 * 2048 * 256 * 4 bytes of partial logits exceed the 4 MiB array
-    rc = lib.moe_route_noalloc(a, a, None, a, a, 2048, 7168, 256, 8, None)
+    # 256 + 4096 * 512 * 4 bytes of logits exceed the 4 MiB array (M * k stays within limits)
+    rc = lib.moe_route_noalloc(a, a, None, a, a, 4096, 7168, 512, 2, None)
     assert rc == moe.MOE_ERR_WORKSPACE
