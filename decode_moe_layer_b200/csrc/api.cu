@@ -79,6 +79,14 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.n_tiles = take(4);
     L.h = take(n * I * 2);
     L.y = take(n * H * sizeof(float));
+    L.wide = wide_enabled(M, H, I);
+    L.max_wide = L.wide ? static_cast<int>((n / (kTileTokens + 1) < static_cast<size_t>(E) ? n / (kTileTokens + 1)
+                                                                                             : static_cast<size_t>(E)) +
+                                           n / kWideTokens + 1)
+                        : 0;
+    L.wide_tiles = take(static_cast<size_t>(L.max_wide) * sizeof(WideTile));
+    L.n_wide = take(4);
+    L.x_perm = take(L.wide ? n * H * 2 : 0);
     L.total = off;
     return L;
 }
@@ -147,16 +155,34 @@ static int make_weight_map(CUtensorMap *map, const void *base, uint64_t rows, ui
 
 // E8M0 scale matrix viewed as [rows][row_bytes] uint8; boxes of box_rows rows x (kChunkK / 32) bytes,
 // unswizzled.  Only used when row_bytes is a multiple of 16 (per_stage_scales).
-static int make_scale_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, int box_rows)
+static int make_scale_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t row_bytes, int box_rows,
+                          int box_bytes = kChunkK / 32)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cuda_fail(cudaErrorNotSupported);
     const cuuint64_t dims[2] = {row_bytes, rows};
     const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kChunkK / 32), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes), static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    return MOE_OK;
+}
+
+// binary16 activation rows [rows][K] (expert-grouped x or h) for the wide kernel: boxes of 16 rows
+// x 64 elements (128 bytes), 128-byte swizzle, the K-major operand layout of tcgen05.mma.
+static int make_act_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t K)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cuda_fail(cudaErrorNotSupported);
+    const cuuint64_t dims[2] = {K, rows};
+    const cuuint64_t strides[1] = {K * 2};
+    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     return MOE_OK;
@@ -233,9 +259,8 @@ struct Marks {
     } while (0)
 
 static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
-                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, void *out, int *status,
-                    int32_t *status_out, int M, int H, int I, int E, int k, int max_tiles, cudaStream_t s, bool pdl,
-                    Marks *marks)
+                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+                    int32_t *status_out, int H, int I, int E, int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
     int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
@@ -247,8 +272,25 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
     }
     MOE_TRY(launch_down(map, smap, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, status_out, H, I, max_tiles,
                         s, pdl));
-    MOE_TRY(launch_combine(y, out, M, H, k, s, pdl));
-    MOE_MARK(marks, s);
+    return MOE_OK;
+}
+
+// The tensor-core path for the wide tiles of one projection (gate_up: x rows gathered into
+// expert-grouped order -> h; down: h -> y).  Weight boxes of 64 rows x 128 bytes, scale boxes
+// of 64 rows x 16 bytes (one 512-element stage), activation boxes of 16 rows x 64 elements.
+static int run_wide(bool gate_up, const void *wq, const uint8_t *ws_, const __half *act, const WideTile *wtiles,
+                    const int *n_wide, int max_wide, const int32_t *sorted_ids, const float *topk_w, __half *h, float *y,
+                    int *status, int32_t *status_out, int M, int H, int I, int E, int k, cudaStream_t s, bool pdl)
+{
+    CUtensorMap wmap, smap, bmap;
+    const uint64_t rows = gate_up ? static_cast<uint64_t>(E) * 2 * I : static_cast<uint64_t>(E) * H;
+    const uint64_t K = gate_up ? H : I;
+    int rc = make_weight_map(&wmap, wq, rows, K / 2, 64);
+    if (rc == MOE_OK) rc = make_scale_map(&smap, ws_, rows, K / 32, 64, kWideStageK / 32);
+    if (rc == MOE_OK) rc = make_act_map(&bmap, act, static_cast<uint64_t>(M) * k, K);
+    if (rc != MOE_OK) return rc;
+    MOE_TRY(launch_wide(gate_up, wmap, smap, bmap, wtiles, n_wide, max_wide, sorted_ids, topk_w, h, y, status,
+                        status_out, H, I, s, pdl));
     return MOE_OK;
 }
 
@@ -269,6 +311,10 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     __half *h = reinterpret_cast<__half *>(ws + L.h);
     float *y = reinterpret_cast<float *>(ws + L.y);
+    WideTile *wtiles = reinterpret_cast<WideTile *>(ws + L.wide_tiles);
+    int *n_wide = reinterpret_cast<int *>(ws + L.n_wide);
+    __half *x_perm = reinterpret_cast<__half *>(ws + L.x_perm);
+    const TileOut to{tiles, n_tiles, L.wide ? wtiles : nullptr, n_wide};
     // The first kernel is ordered after everything before it on the stream; each later
     // kernel of the call is launched early (programmatic dependent launch) and waits on
     // device for its predecessor.  Event marks (profiling) break that overlap, so the
@@ -279,20 +325,36 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, M, H, E, s));
     MOE_MARK(marks, s);
     if (fused_select(M, E, k)) {
-        MOE_TRY(launch_route_select_permute(partial, L.splits, router_bias, ids, tw, offsets, sorted_ids, inv_pos,
-                                            tiles, n_tiles, M, E, k, s, pdl));
+        MOE_TRY(launch_route_select_permute(partial, L.splits, router_bias, ids, tw, offsets, sorted_ids, inv_pos, to, M,
+                                            E, k, s, pdl));
         MOE_MARK(marks, s);
     } else {
         MOE_TRY(launch_route_topk(partial, L.splits, router_bias, ids, tw, M, E, k, s, pdl));
         MOE_MARK(marks, s);
-        MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k, s, pdl));
+        MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, to, M, E, k, s, pdl));
     }
     MOE_MARK(marks, s);
+    // gate_up: the 8-assignment tiles on mma.sync, then (large M) the wide tiles on tcgen05
     int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
+    if (L.wide) {
+        MOE_TRY(launch_gather_rows(x16, sorted_ids, x_perm, M * k, H, k, s, pdl));
+        rc = run_wide(true, w13_q, w13_s, x_perm, wtiles, n_wide, L.max_wide, sorted_ids, tw, h, y, status, status_out,
+                      M, H, I, E, k, s, pdl);
+        if (rc != MOE_OK) return rc;
+    }
     MOE_MARK(marks, s);
-    return run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, out, status, status_out, M, H, I, E, k,
-                    L.max_tiles, s, pdl, marks);
+    // down likewise, then the weighted top-k combine
+    rc = run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, status, status_out, H, I, E, L.max_tiles, s, pdl);
+    if (rc != MOE_OK) return rc;
+    if (L.wide) {
+        rc = run_wide(false, w2_q, w2_s, h, wtiles, n_wide, L.max_wide, sorted_ids, tw, h, y, status, status_out, M, H, I,
+                      E, k, s, pdl);
+        if (rc != MOE_OK) return rc;
+    }
+    MOE_TRY(launch_combine(y, out, M, H, k, s, pdl));
+    MOE_MARK(marks, s);
+    return MOE_OK;
 }
 
 static int check_forward_args(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
@@ -374,7 +436,8 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
     if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
         return MOE_ERR_INVALID_ARG;
     if (M == 0) return MOE_OK;
-    MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, nullptr, nullptr, M, E, k, stream, false));
+    const TileOut none{nullptr, nullptr, nullptr, nullptr};
+    MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, none, M, E, k, stream, false));
     return MOE_OK;
 }
 
@@ -424,8 +487,11 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
-    return run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, out_bf16,
-                    status, nullptr, M, H, I, E, k, L.max_tiles, stream, false, nullptr);
+    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, status,
+                  nullptr, H, I, E, L.max_tiles, stream, false);
+    if (rc != MOE_OK) return rc;
+    MOE_TRY(launch_combine(y, out_bf16, M, H, k, stream, false));
+    return MOE_OK;
 }
 
 int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,

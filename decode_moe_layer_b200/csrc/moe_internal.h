@@ -12,10 +12,13 @@ namespace moe {
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = -5;
+constexpr int kStatusUnsupported = -2;   // MOE_ERR_UNSUPPORTED_SHAPE: an input outside a kernel's exact range
 // The call's 256-byte status block: word 0 is the status; words kQueueGateUp and kQueueDown
 // are the grouped kernels' work-queue counters, zeroed by the first kernel of the call.
 constexpr int kQueueGateUp = 8;
 constexpr int kQueueDown = 16;
+constexpr int kQueueGateUpWide = 24;
+constexpr int kQueueDownWide = 32;
 
 // Grouped GEMM tiling (both projections).
 constexpr int kTileTokens = 8;       // assignments per expert tile (one MMA n-tile)
@@ -87,11 +90,31 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
     int tok[kTileTokens];   // token of each assignment (sorted_ids[p0+i] / k); entries >= count repeat the last
 };
 
+// Experts with at least kWideMinTokens assignments go to the tensor-core path (grouped_wide.cu)
+// as wide tiles of up to kWideTokens consecutive assignments; it needs H and I to be multiples
+// of its 512-element packed stage.  No expert can exceed M assignments, so M < kWideMinTokens
+// never uses it.
+constexpr int kWideTokens = 128;
+constexpr int kWideStageK = 512;
+constexpr int kWideMinTokens = 32;   // fewer assignments stream faster as 8-assignment tiles
+struct WideTile {
+    int expert;
+    int p0;      // first position in the expert-grouped order
+    int count;   // assignments, 1 .. kWideTokens
+    int pad;
+};
+__host__ __device__ inline bool wide_enabled(int M, int H, int I)
+{
+    return M >= kWideMinTokens && H % kWideStageK == 0 && I % kWideStageK == 0;
+}
+
 // Byte offsets of every buffer inside one call's workspace (256-byte aligned).
 struct Layout {
-    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y, total;
+    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y;
+    size_t wide_tiles, n_wide, x_perm, total;
     int splits;   // router partial-logit slices (route_plan)
-    int max_tiles;
+    int max_tiles, max_wide;
+    bool wide;    // wide_enabled for this shape
 };
 
 Layout make_layout(int M, int H, int I, int E, int k);
@@ -133,10 +156,10 @@ __host__ __device__ inline bool fused_select(int M, int E, int k)
            static_cast<long long>(M) * E <= kFusedSelectMaxLogits;
 }
 // Dynamic shared memory of the ranking (rank_smem): two [warp][expert] u16 tables (counts and
-// prefix counts), four int arrays over E and a 33-int scan buffer.
+// prefix counts), five int arrays over E and a 33-int scan buffer.
 __host__ __device__ inline int permute_smem_bytes(int E)
 {
-    return 2 * (kPermuteThreads / 32) * E * 2 + 4 * E * 4 + 64 * 4;
+    return 2 * (kPermuteThreads / 32) * E * 2 + 5 * E * 4 + 64 * 4;
 }
 
 // Kernel launchers (return cudaError_t of the launch).
@@ -144,11 +167,20 @@ cudaError_t launch_route_logits(const void *x, const float *router_w, float *par
                                 int32_t *status_out, int M, int H, int E, cudaStream_t s);
 cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
                               int E, int k, cudaStream_t s, bool pdl);
+// Tile outputs of the route remap: 8-assignment tiles for the mma.sync kernels and, when
+// `wide` is set, wide tiles (experts with more than kTileTokens assignments) for the
+// tensor-core kernels; such experts then get no 8-assignment tiles.
+struct TileOut {
+    ExpertTile *tiles;
+    int *n_tiles;
+    WideTile *wide_tiles;   // nullptr: every expert gets 8-assignment tiles
+    int *n_wide;
+};
 cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
-                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
-                                        int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl);
-cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos,
-                           ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl);
+                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M,
+                                        int E, int k, cudaStream_t s, bool pdl);
+cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
+                           int M, int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
                                int *status, int E, int k, cudaStream_t s);
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
@@ -160,6 +192,13 @@ cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, co
                         float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
                         bool pdl);
 cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl);
+cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __half *x_perm, int n, int H, int k,
+                               cudaStream_t s, bool pdl);
+cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap &smap, const CUtensorMap &bmap,
+                        const WideTile *tiles, const int *n_tiles, int max_tiles, const int32_t *sorted_ids,
+                        const float *topk_w, __half *h, float *y, int *status, int32_t *status_out, int H, int I,
+                        cudaStream_t s, bool pdl);
+int wide_smem_bytes();
 
 // Row blocks of the down projection per token (one arrival counter each).
 __host__ __device__ inline int down_row_blocks(int H) { return (H + kItemRows - 1) / kItemRows; }

@@ -7,8 +7,7 @@ namespace moe {
 // Route remap of given topk_ids (rank_and_scatter in rounds of kPermuteThreads assignments).
 __global__ void __launch_bounds__(kPermuteThreads, 1)
 permute_kernel(const int32_t *__restrict__ topk_ids, int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_ids,
-               int32_t *__restrict__ inv_pos, ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int n, int E,
-               int k)
+               int32_t *__restrict__ inv_pos, TileOut to, int n, int E, int k)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     int *s_e = reinterpret_cast<int *>(smem + permute_smem_bytes(E));   // [n]
@@ -30,7 +29,7 @@ permute_kernel(const int32_t *__restrict__ topk_ids, int32_t *__restrict__ offse
         }
     }
     __syncthreads();
-    rank_and_scatter(s_e, n, E, k, rank_smem(smem, E), offsets, sorted_ids, inv_pos, tiles, n_tiles);
+    rank_and_scatter(s_e, n, E, k, rank_smem(smem, E), offsets, sorted_ids, inv_pos, to);
 }
 
 // Expert tiles from given offsets / sorted ids; also resets the call's status word.
@@ -45,21 +44,23 @@ __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__r
         status[0] = kStatusOk;
         status[kQueueGateUp] = 0;
         status[kQueueDown] = 0;
+        status[kQueueGateUpWide] = 0;
+        status[kQueueDownWide] = 0;
     }
     for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
     emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
 }
 
-cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos,
-                           ExpertTile *tiles, int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl)
+cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
+                           int M, int E, int k, cudaStream_t s, bool pdl)
 {
     const int n = M * k;
     const int smem = permute_smem_bytes(E) + n * static_cast<int>(sizeof(int));
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(permute_kernel), smem);
     if (e != cudaSuccess) return e;
-    return launch_ex(permute_kernel, dim3(1), dim3(kPermuteThreads), smem, s, pdl, ids, offsets, sorted_ids, inv_pos,
-                     tiles, n_tiles, n, E, k);
+    return launch_ex(permute_kernel, dim3(1), dim3(kPermuteThreads), smem, s, pdl, ids, offsets, sorted_ids, inv_pos, to,
+                     n, E, k);
 }
 
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,

@@ -50,11 +50,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &t
 }
 
 // Shared memory of the ranking, carved from one dynamic buffer of permute_smem_bytes(E) bytes:
-// wc at 0, pref at 64 E, the int arrays at 128 E, the scan buffer at 144 E (+132 bytes).
+// wc at 0, pref at 64 E, the five int arrays at 128 E, the scan buffer at 148 E (+132 bytes).
 struct RankSmem {
     uint16_t *wc;     // [32][E] counts of the current round's warps
     uint16_t *pref;   // [32][E] their prefix counts (with earlier rounds)
-    int *cnt, *off, *tb, *base;   // [E] count, offset, first tile, assignments ranked so far
+    int *cnt, *off, *tb, *base, *wb;   // [E] count, offset, first tile, ranked so far, first wide tile
     int *scan;        // 33
 };
 
@@ -69,7 +69,8 @@ __device__ __forceinline__ RankSmem rank_smem(uint8_t *raw, int E)
     r.off = ints + E;
     r.tb = ints + 2 * E;
     r.base = ints + 3 * E;
-    r.scan = ints + 4 * E;
+    r.wb = ints + 4 * E;
+    r.scan = ints + 5 * E;
     return r;
 }
 
@@ -80,9 +81,9 @@ __device__ __forceinline__ RankSmem rank_smem(uint8_t *raw, int E)
 // index past an array.  Called by every thread of a kPermuteThreads-thread CTA.
 __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, RankSmem sm,
                                         int32_t *__restrict__ offsets, int32_t *__restrict__ sorted_ids,
-                                        int32_t *__restrict__ inv_pos, ExpertTile *__restrict__ tiles,
-                                        int *__restrict__ n_tiles)
+                                        int32_t *__restrict__ inv_pos, TileOut to)
 {
+    ExpertTile *__restrict__ tiles = to.tiles;
     constexpr int kW = kPermuteThreads / 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // only the warps that hold assignments in some round use table rows
@@ -98,8 +99,11 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
         if (e >= 0 && e < E) atomicAdd(&sm.cnt[e], 1);
     }
     __syncthreads();
-    // offsets and tile bases: (tiles << 16) | count per expert, one scan (counts <= 16384)
-    const int mine = tid < E ? (((sm.cnt[tid] + kTileTokens - 1) / kTileTokens) << 16) | sm.cnt[tid] : 0;
+    // offsets and tile bases: (tiles << 16) | count per expert, one scan (counts <= 16384); an
+    // expert with at least kWideMinTokens assignments takes wide tiles instead, when enabled
+    const int my_cnt = tid < E ? sm.cnt[tid] : 0;
+    const bool my_wide = to.wide_tiles != nullptr && my_cnt >= kWideMinTokens;
+    const int mine = tid < E ? ((my_wide ? 0 : (my_cnt + kTileTokens - 1) / kTileTokens) << 16) | my_cnt : 0;
     int total = 0;
     const int base = block_exclusive_scan(mine, sm.scan, total);   // ends with a block barrier
     if (tid < E) {
@@ -109,7 +113,14 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
     }
     if (tid == 0) {
         offsets[E] = total & 0xFFFF;
-        if (tiles) *n_tiles = total >> 16;
+        if (tiles) *to.n_tiles = total >> 16;
+    }
+    if (to.wide_tiles != nullptr) {
+        __syncthreads();   // every thread has read the first scan's totals before the buffer is reused
+        int wtotal = 0;
+        const int wbase = block_exclusive_scan(my_wide ? (my_cnt + kWideTokens - 1) / kWideTokens : 0, sm.scan, wtotal);
+        if (tid < E) sm.wb[tid] = wbase;
+        if (tid == 0) *to.n_wide = wtotal;
     }
     for (int r0 = 0; r0 < n; r0 += kPermuteThreads) {
         const int f = r0 + tid;
@@ -142,8 +153,16 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
             const int pos = sm.off[e] + rank;
             sorted_ids[pos] = f;
             inv_pos[f] = pos;
-            if (tiles) {
-                const int cnt = sm.cnt[e];
+            const int cnt = sm.cnt[e];
+            if (to.wide_tiles != nullptr && cnt >= kWideMinTokens) {
+                if (rank % kWideTokens == 0) {
+                    WideTile *wp = to.wide_tiles + sm.wb[e] + rank / kWideTokens;
+                    wp->expert = e;
+                    wp->p0 = pos;
+                    wp->count = min(kWideTokens, cnt - rank);
+                    wp->pad = 0;
+                }
+            } else if (tiles) {
                 const int slot = rank % kTileTokens, tile_first = rank - slot;
                 ExpertTile *tp = tiles + sm.tb[e] + rank / kTileTokens;
                 const int t = f / k;
@@ -168,10 +187,12 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
 // per-expert count, whose leader then advances it; one warp scan of (tiles << 16 | count)
 // over the experts gives offsets and tile bases.  Only __syncwarp, no block barrier.
 __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k, int *cnt, int *off, int *tb,
-                                             int *rank, int32_t *__restrict__ offsets,
+                                             int *wb, int *rank, int32_t *__restrict__ offsets,
                                              int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
-                                             ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles)
+                                             TileOut to)
 {
+    ExpertTile *__restrict__ tiles = to.tiles;
+    const bool wide_on = to.wide_tiles != nullptr;
     const int lane = threadIdx.x & 31;
     for (int e = lane; e < E; e += 32) cnt[e] = 0;
     __syncwarp();
@@ -191,25 +212,42 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
     // lane l scans the contiguous experts [l * per, (l + 1) * per)
     const int per = (E + 31) / 32;
     const int ea = min(E, lane * per), eb = min(E, ea + per);
-    int local = 0;
-    for (int e = ea; e < eb; ++e) local += (((cnt[e] + kTileTokens - 1) / kTileTokens) << 16) | cnt[e];
-    int incl = local;
+    // per expert: (8-assignment tiles << 16) | count, and wide tiles (experts with kWideMinTokens or more
+    // when the wide path is on); lane l scans the contiguous experts [l * per, (l + 1) * per)
+    auto packed = [&](int c) {
+        return (((wide_on && c >= kWideMinTokens) ? 0 : (c + kTileTokens - 1) / kTileTokens) << 16) | c;
+    };
+    auto wide_n = [&](int c) { return (wide_on && c >= kWideMinTokens) ? (c + kWideTokens - 1) / kWideTokens : 0; };
+    int local = 0, wlocal = 0;
+    for (int e = ea; e < eb; ++e) {
+        local += packed(cnt[e]);
+        wlocal += wide_n(cnt[e]);
+    }
+    int incl = local, wincl = wlocal;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += o;
+        const int wo = __shfl_up_sync(0xffffffffu, wincl, d);
+        if (lane >= d) {
+            incl += o;
+            wincl += wo;
+        }
     }
     const int total = __shfl_sync(0xffffffffu, incl, 31);
-    int run = incl - local;
+    const int wtotal = __shfl_sync(0xffffffffu, wincl, 31);
+    int run = incl - local, wrun = wincl - wlocal;
     for (int e = ea; e < eb; ++e) {
         off[e] = run & 0xFFFF;
         tb[e] = run >> 16;
+        wb[e] = wrun;
         offsets[e] = run & 0xFFFF;
-        run += (((cnt[e] + kTileTokens - 1) / kTileTokens) << 16) | cnt[e];
+        run += packed(cnt[e]);
+        wrun += wide_n(cnt[e]);
     }
     if (lane == 0) {
         offsets[E] = total & 0xFFFF;
-        *n_tiles = total >> 16;
+        *to.n_tiles = total >> 16;
+        if (wide_on) *to.n_wide = wtotal;
     }
     __syncwarp();
     for (int f = lane; f < n; f += 32) {
@@ -219,6 +257,16 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
         sorted_ids[pos] = f;
         inv_pos[f] = pos;
         const int c = cnt[e];
+        if (wide_on && c >= kWideMinTokens) {
+            if (r % kWideTokens == 0) {
+                WideTile *wp = to.wide_tiles + wb[e] + r / kWideTokens;
+                wp->expert = e;
+                wp->p0 = pos;
+                wp->count = min(kWideTokens, c - r);
+                wp->pad = 0;
+            }
+            continue;
+        }
         const int slot = r % kTileTokens, tile_first = r - slot;
         ExpertTile *tp = tiles + tb[e] + r / kTileTokens;
         const int t = f / k;

@@ -87,6 +87,8 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
             status[0] = kStatusOk;
             status[kQueueGateUp] = 0;
             status[kQueueDown] = 0;
+            status[kQueueGateUpWide] = 0;
+            status[kQueueDownWide] = 0;
         }
         if (status_out) *status_out = kStatusOk;
     }
@@ -295,14 +297,14 @@ template <int kPerLane>
 __global__ void __launch_bounds__(kPermuteThreads, 1)
 route_select_permute_kernel(const float *__restrict__ partial, int splits, const float *__restrict__ bias,
                             int32_t *__restrict__ ids, float *__restrict__ wout, int32_t *__restrict__ offsets,
-                            int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
-                            ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles, int M, int E, int k)
+                            int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos, TileOut to, int M,
+                            int E, int k)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_e[kPermuteThreads];      // expert of assignment f
     __shared__ int s_rank[kPermuteThreads];   // its rank inside the expert
     float *s_log = reinterpret_cast<float *>(smem);                      // [M][E]
-    int *s_cnt = reinterpret_cast<int *>(smem) + M * E;                   // [E] x 3
+    int *s_cnt = reinterpret_cast<int *>(smem) + M * E;                   // [E] x 4
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_wait();
     pdl_trigger();
@@ -331,8 +333,8 @@ route_select_permute_kernel(const float *__restrict__ partial, int splits, const
     }
     __syncthreads();
     if (warp != 0) return;
-    warp_rank_and_scatter(s_e, M * k, E, k, s_cnt, s_cnt + E, s_cnt + 2 * E, s_rank, offsets, sorted_ids, inv_pos,
-                          tiles, n_tiles);
+    warp_rank_and_scatter(s_e, M * k, E, k, s_cnt, s_cnt + E, s_cnt + 2 * E, s_cnt + 3 * E, s_rank, offsets,
+                          sorted_ids, inv_pos, to);
 }
 
 __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
@@ -392,22 +394,21 @@ cudaError_t launch_route_topk(const float *partial, int splits, const float *bia
 
 template <int P>
 static cudaError_t select_permute_p(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
-                                    int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
-                                    int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl)
+                                    int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M, int E,
+                                    int k, cudaStream_t s, bool pdl)
 {
-    const int smem = (M * E + 3 * E) * static_cast<int>(sizeof(float));
+    const int smem = (M * E + 4 * E) * static_cast<int>(sizeof(float));
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>), smem);
     if (e != cudaSuccess) return e;
     return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kPermuteThreads), smem, s, pdl, partial, splits,
-                     bias, ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, E, k);
+                     bias, ids, w, offsets, sorted_ids, inv_pos, to, M, E, k);
 }
 
 cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
-                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, ExpertTile *tiles,
-                                        int *n_tiles, int M, int E, int k, cudaStream_t s, bool pdl)
+                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M,
+                                        int E, int k, cudaStream_t s, bool pdl)
 {
-#define MOE_SEL(P) select_permute_p<P>(partial, splits, bias, ids, w, offsets, sorted_ids, inv_pos, tiles, n_tiles, M, \
-                                       E, k, s, pdl)
+#define MOE_SEL(P) select_permute_p<P>(partial, splits, bias, ids, w, offsets, sorted_ids, inv_pos, to, M, E, k, s, pdl)
     if (E <= 32) return MOE_SEL(1);
     if (E <= 64) return MOE_SEL(2);
     if (E <= 128) return MOE_SEL(4);

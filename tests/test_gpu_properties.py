@@ -124,6 +124,30 @@ def test_ragged_shapes_against_oracle(moe, H, I, E, k, M):
     U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "ragged %s" % ((H, I, E, k, M),))
 
 
+@pytest.mark.parametrize("H,I,E,k,M", [
+    (1024, 512, 4, 2, 80),    # ~40 assignments per expert: three of four experts on the tensor-core path
+    (512, 512, 4, 2, 300),    # ~150 per expert: two wide tiles per expert, the second partial
+    (512, 1024, 16, 4, 160),  # ~40 per expert, spread: wide and 8-assignment tiles in the same call
+])
+def test_wide_tiles_against_oracle(moe, H, I, E, k, M):
+    # experts with more than 8 assignments take the tcgen05 path (H, I multiples of 512)
+    shape = gen.LayerShape("wide", H, I, E, k, (M,))
+    inp = gen.make_inputs(0, M, shape=shape, seed=7 * H + I + E + k + M)
+    d = U.device_inputs(inp)
+    ids = torch.empty((M, k), dtype=torch.int32, device="cuda")
+    st = torch.full((1,), 123, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.moe_workspace_bytes(M, H, I, E, k), dtype=torch.uint8, device="cuda")
+    out = moe.moe_mxfp4_forward_ex(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], k, ws,
+                                   topk_ids_out=ids, status_out=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == moe.MOE_OK
+    r = U.oracle_forward(inp)
+    counts = np.bincount(r["topk_ids"].reshape(-1), minlength=E)
+    assert counts.max() >= 32                    # the case does reach the wide path
+    assert np.array_equal(ids.cpu().numpy(), r["topk_ids"])
+    U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "wide %s" % ((H, I, E, k, M),))
+
+
 def test_zero_tokens_is_a_no_op(moe):
     inp = gen.make_inputs(0, 2)
     d = U.device_inputs(inp)
