@@ -228,7 +228,7 @@ static int library_workspace(cudaStream_t s, size_t need, char **out)
 // ------------------------------------------------------------------ step bodies (arguments already validated)
 
 static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const ExpertTile *tiles,
-                       const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E,
+                       const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E, int k,
                        int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
@@ -242,7 +242,7 @@ static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x1
                             kItemRows / 2);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, max_tiles, s, pdl));
+    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, k, max_tiles, s, pdl));
     return MOE_OK;
 }
 
@@ -258,8 +258,7 @@ struct Marks {
         if (m) MOE_TRY((m)->mark(s));                   \
     } while (0)
 
-static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
-                    const float *topk_w, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
                     int32_t *status_out, int H, int I, int E, int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
@@ -270,8 +269,7 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
         rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_down(map, smap, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, y, status, status_out, H, I, max_tiles,
-                        s, pdl));
+    MOE_TRY(launch_down(map, smap, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, max_tiles, s, pdl));
     return MOE_OK;
 }
 
@@ -279,7 +277,7 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
 // expert-grouped order -> h; down: h -> y).  Weight boxes of 64 rows x 128 bytes, scale boxes
 // of 64 rows x 16 bytes (one 512-element stage), activation boxes of 16 rows x 64 elements.
 static int run_wide(bool gate_up, const void *wq, const uint8_t *ws_, const __half *act, const WideTile *wtiles,
-                    const int *n_wide, int max_wide, const int32_t *sorted_ids, const float *topk_w, __half *h, float *y,
+                    const int *n_wide, int max_wide, const int32_t *sorted_ids, __half *h, float *y,
                     int *status, int32_t *status_out, int M, int H, int I, int E, int k, cudaStream_t s, bool pdl)
 {
     CUtensorMap wmap, smap, bmap;
@@ -289,8 +287,8 @@ static int run_wide(bool gate_up, const void *wq, const uint8_t *ws_, const __ha
     if (rc == MOE_OK) rc = make_scale_map(&smap, ws_, rows, K / 32, 64, kWideStageK / 32);
     if (rc == MOE_OK) rc = make_act_map(&bmap, act, static_cast<uint64_t>(M) * k, K);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_wide(gate_up, wmap, smap, bmap, wtiles, n_wide, max_wide, sorted_ids, topk_w, h, y, status,
-                        status_out, H, I, s, pdl));
+    MOE_TRY(launch_wide(gate_up, wmap, smap, bmap, wtiles, n_wide, max_wide, sorted_ids, h, y, status, status_out, H,
+                        I, s, pdl));
     return MOE_OK;
 }
 
@@ -335,24 +333,24 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     }
     MOE_MARK(marks, s);
     // gate_up: the 8-assignment tiles on mma.sync, then (large M) the wide tiles on tcgen05
-    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, L.max_tiles, s, pdl);
+    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, k, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
     if (L.wide) {
         MOE_TRY(launch_gather_rows(x16, sorted_ids, x_perm, M * k, H, k, s, pdl));
-        rc = run_wide(true, w13_q, w13_s, x_perm, wtiles, n_wide, L.max_wide, sorted_ids, tw, h, y, status, status_out,
+        rc = run_wide(true, w13_q, w13_s, x_perm, wtiles, n_wide, L.max_wide, sorted_ids, h, y, status, status_out,
                       M, H, I, E, k, s, pdl);
         if (rc != MOE_OK) return rc;
     }
     MOE_MARK(marks, s);
     // down likewise, then the weighted top-k combine
-    rc = run_down(w2_q, w2_s, h, sorted_ids, tw, tiles, n_tiles, y, status, status_out, H, I, E, L.max_tiles, s, pdl);
+    rc = run_down(w2_q, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, E, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
     if (L.wide) {
-        rc = run_wide(false, w2_q, w2_s, h, wtiles, n_wide, L.max_wide, sorted_ids, tw, h, y, status, status_out, M, H, I,
+        rc = run_wide(false, w2_q, w2_s, h, wtiles, n_wide, L.max_wide, sorted_ids, h, y, status, status_out, M, H, I,
                       E, k, s, pdl);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_combine(y, out, M, H, k, s, pdl));
+    MOE_TRY(launch_combine(y, tw, out, M, H, k, s, pdl));
     MOE_MARK(marks, s);
     return MOE_OK;
 }
@@ -462,7 +460,7 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
-    return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E,
+    return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E, k,
                        L.max_tiles, stream, false);
 }
 
@@ -487,10 +485,10 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
-    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, topk_w, tiles, n_tiles, y, status,
-                  nullptr, H, I, E, L.max_tiles, stream, false);
+    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), tiles, n_tiles, y, status, nullptr, H, I, E,
+                  L.max_tiles, stream, false);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_combine(y, out_bf16, M, H, k, stream, false));
+    MOE_TRY(launch_combine(y, topk_w, out_bf16, M, H, k, stream, false));
     return MOE_OK;
 }
 

@@ -36,8 +36,9 @@
 //    E8M0 scale is applied once to the fp32 partial sum.  At the end of an item a
 //    warp parks its partial sums in a double-buffered reduction area and moves on.
 //  * 2 epilogue warps sum the 8 K slots in slot order, then gate_up applies
-//    clamp-SwiGLU and stores h; down applies the routing weight and stores the
-//    fp32 row of the assignment -- off the compute path.  The weighted top-k
+//    clamp-SwiGLU and stores h; down stores the unweighted fp32 row of each
+//    assignment -- off the compute path.  The item's positions and flat assignment
+//    ids reach them from the producer through shared memory.  The weighted top-k
 //    combine that follows is its own small kernel (combine_kernel).
 // Activations (x or h) are read as binary16; bf16 x converts exactly for
 // 2^-17 <= |x| <= 65504, h is stored scaled by 2^10 (exact for |h| >= 2^-27,
@@ -75,7 +76,7 @@ __host__ __device__ inline SmemPlan smem_plan(int K)
     p.sbuf_bytes = per_stage_scales(K) ? 0 : (kItemRows * (K / 32) + 127) / 128 * 128;
     p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
     p.bars_off = p.red_off + kRedBufs * kRedFloats * 4;
-    p.total = p.bars_off + (2 * kStages + 8) * 8 + (kItemQ + 2) * 4 + 1024;   // + alignment slack
+    p.total = p.bars_off + (2 * kStages + 8) * 8 + (3 + kTileTokens) * (kItemQ + kRedBufs) * 4 + 1024;   // + slack
     return p;
 }
 
@@ -96,10 +97,9 @@ template <bool kGateUp>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
-                     const int32_t *__restrict__ sorted_ids, const float *__restrict__ topk_w,
                      const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
                      __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out,
-                     int *queue, int K, int I, int H)
+                     int *queue, int K, int I, int H, int k)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -113,8 +113,17 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bars_off);
     uint64_t *full = bars, *empty = bars + kStages;
     uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
-    volatile int *item_q = reinterpret_cast<volatile int *>(bars + 2 * kStages + 8);   // [kItemQ] producer -> compute
-    volatile int *red_item = item_q + kItemQ;                                         // [2] compute -> epilogue
+    // per item in flight: id, first expert-grouped position, assignment count and the slots'
+    // flat assignment ids (producer -> compute warps -> epilogue warps), so that no consumer
+    // reads the tile list from global memory
+    volatile int *item_q = reinterpret_cast<volatile int *>(bars + 2 * kStages + 8);   // [kItemQ]
+    volatile int *item_p0 = item_q + kItemQ;                                          // [kItemQ]
+    volatile int *item_cnt = item_p0 + kItemQ;                                        // [kItemQ]
+    volatile int *item_flat = item_cnt + kItemQ;                                      // [kItemQ][kTileTokens]
+    volatile int *red_item = item_flat + kItemQ * kTileTokens;                        // [kRedBufs]
+    volatile int *red_p0 = red_item + kRedBufs;                                       // [kRedBufs]
+    volatile int *red_cnt = red_p0 + kRedBufs;                                        // [kRedBufs]
+    volatile int *red_flat = red_cnt + kRedBufs;                                      // [kRedBufs][kTileTokens]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
@@ -166,14 +175,14 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         int stage_ctr = 0, item_ctr = 0;
         int stages_issued = 0, scales_issued = 0;   // copies in flight must land before exit
         // the next item's descriptor, loaded one item ahead so that no copy waits on it
-        int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_tok = 0;
+        int nx_e = 0, nx_p0 = 0, nx_cnt = 1, nx_flat = 0;
         auto fetch = [&](int it) {
             if (it < n_items) {
                 const ExpertTile *tp = tiles + it / row_blocks;
                 nx_e = __ldcg(&tp->expert);
                 nx_p0 = __ldcg(&tp->p0);
                 nx_cnt = __ldcg(&tp->count);
-                nx_tok = __ldcg(&tp->tok[lane & (kTileTokens - 1)]);
+                nx_flat = __ldcg(&tp->flat[lane & (kTileTokens - 1)]);
             }
         };
         // down: h copies of the first stages, held back until gate_up has completed
@@ -219,17 +228,22 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         for (;; ++item_ctr) {
             const int item = next_id;
             if (item >= n_items) break;
-            const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, tok = nx_tok;
+            const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, flat = nx_flat;
             next_id = take();
             fetch(next_id);
-            if (lane == 0) item_q[item_ctr % kItemQ] = item;   // published by the first stage's arrival
+            if (lane == 0) {   // published by the first stage's arrival
+                item_q[item_ctr % kItemQ] = item;
+                item_p0[item_ctr % kItemQ] = p0;
+                item_cnt[item_ctr % kItemQ] = cnt;
+            }
+            if (!kGateUp && lane < kTileTokens) item_flat[(item_ctr % kItemQ) * kTileTokens + lane] = flat;
             const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
             const int row_b = row_a + I;                               // gate_up only
             const int valid_rows = kGateUp ? kItemRows : min(kItemRows, H - rb * kItemRows);
-            // this lane's activation row (gate_up: the token's x row; down: the h row)
-            const __half *arow = kGateUp ? act + static_cast<size_t>(tok) * K
+            // this lane's activation row (gate_up: the x row of the slot's token; down: the h row)
+            const __half *arow = kGateUp ? act + static_cast<size_t>(flat / k) * K
                                          : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
             if (!stage_scales) {
                 const int b = item_ctr & 1;
@@ -334,9 +348,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             if (aborted) break;
             const int item = red_item[b];   // -1: no further item
             if (item < 0) break;
-            const ExpertTile *tp = tiles + item / row_blocks;
             const int rb = item % row_blocks;
-            const int cnt = tp->count, p0 = tp->p0;
+            const int cnt = red_cnt[b], p0 = red_p0[b];
             float4 sums[2];
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
@@ -367,20 +380,19 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     if (li1 < cnt)
                         hout[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
                 } else {
-                    // remove e8m0_times2's factor 2 and h's 2^10 storage scale
+                    // remove e8m0_times2's factor 2 and h's 2^10 storage scale; the routing weight
+                    // is applied by the combine
                     const float unscale = 0.5f / kHScale;
                     const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
                     if (li0 < cnt) {
-                        const int f = sorted_ids[p0 + li0];
-                        const float w = topk_w[f] * unscale;
-                        if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.x;
-                        if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.z;
+                        float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokens + li0]) * H;
+                        if (ra < rows_total) yr[ra] = unscale * sum.x;
+                        if (rbw < rows_total) yr[rbw] = unscale * sum.z;
                     }
                     if (li1 < cnt) {
-                        const int f = sorted_ids[p0 + li1];
-                        const float w = topk_w[f] * unscale;
-                        if (ra < rows_total) yout[static_cast<size_t>(f) * H + ra] = w * sum.y;
-                        if (rbw < rows_total) yout[static_cast<size_t>(f) * H + rbw] = w * sum.w;
+                        float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokens + li1]) * H;
+                        if (ra < rows_total) yr[ra] = unscale * sum.y;
+                        if (rbw < rows_total) yr[rbw] = unscale * sum.w;
                     }
                 }
             }
@@ -482,7 +494,13 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         for (int m = 0; m < kWarpMTiles; ++m)
             *reinterpret_cast<float4 *>(rbuf + ((kslot * kItemMTiles + mgrp * kWarpMTiles + m) * 32 + lane) * 4) =
                 make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
-        if (warp == 0 && lane == 0) red_item[rb] = item_q[item_ctr % kItemQ];
+        if (warp == 0 && lane == 0) {
+            red_item[rb] = item_q[item_ctr % kItemQ];
+            red_p0[rb] = item_p0[item_ctr % kItemQ];
+            red_cnt[rb] = item_cnt[item_ctr % kItemQ];
+        }
+        if (!kGateUp && warp == 0 && lane < kTileTokens)
+            red_flat[rb * kTileTokens + lane] = item_flat[(item_ctr % kItemQ) * kTileTokens + lane];
         __syncwarp();
         if (lane == 0) mbar_arrive(&rfull[rb]);
     }
@@ -496,9 +514,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     }
 }
 
-// out[t] = bf16( sum_j y[t*k + j] ), slots j ascending (a fixed order, no atomics); y already
-// carries the routing weight.  Four outputs per thread.
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, __nv_bfloat16 *__restrict__ out,
+// out[t] = bf16( sum_j w[t*k + j] * y[t*k + j] ), slots j ascending (a fixed order, no atomics);
+// y holds the unweighted down-projection row of every assignment.  Four outputs per thread.
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, const float *__restrict__ topk_w,
+                                                      __nv_bfloat16 *__restrict__ out,
                                                       int M, int H, int k)
 {
     pdl_wait();
@@ -509,11 +528,13 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     const int c = static_cast<int>(idx - static_cast<size_t>(t) * per_row) * 4;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
-        const float4 v = *reinterpret_cast<const float4 *>(y + (static_cast<size_t>(t) * k + j) * H + c);
-        a.x += v.x;
-        a.y += v.y;
-        a.z += v.z;
-        a.w += v.w;
+        const int f = t * k + j;
+        const float w = topk_w[f];
+        const float4 v = *reinterpret_cast<const float4 *>(y + static_cast<size_t>(f) * H + c);
+        a.x = fmaf(w, v.x, a.x);
+        a.y = fmaf(w, v.y, a.y);
+        a.z = fmaf(w, v.z, a.z);
+        a.w = fmaf(w, v.w, a.w);
     }
     __nv_bfloat162 o[2] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w)};
     *reinterpret_cast<uint2 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint2 *>(o);
@@ -521,9 +542,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 
 template <bool kGateUp>
 static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
-                                  const __half *act, const int32_t *sorted_ids, const float *topk_w,
-                                  const ExpertTile *tiles, const int *n_tiles, __half *h, float *y, int *status,
-                                  int32_t *status_out, int K, int I, int H, int max_tiles, cudaStream_t s, bool pdl)
+                                  const __half *act, const ExpertTile *tiles, const int *n_tiles, __half *h, float *y,
+                                  int *status, int32_t *status_out, int K, int I, int H, int k, int max_tiles,
+                                  cudaStream_t s, bool pdl)
 {
     const SmemPlan plan = smem_plan(K);
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
@@ -534,33 +555,34 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &sma
     if (grid < 1) grid = 1;
     int *queue = status + (kGateUp ? kQueueGateUp : kQueueDown);
     return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, smap,
-                     scales, act, sorted_ids, topk_w, tiles, n_tiles, h, y, status, status_out, queue, K, I, H);
+                     scales, act, tiles, n_tiles, h, y, status, status_out, queue, K, I, H, k);
 }
 
 int grouped_smem_bytes(int K) { return smem_plan(K).total; }
 
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
                            const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
-                           int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl)
+                           int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl)
 {
-    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, nullptr, nullptr, tiles, n_tiles, h, nullptr, status,
-                                status_out, H, I, H, max_tiles, s, pdl);
+    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, tiles, n_tiles, h, nullptr, status, status_out, H, I, H,
+                                k, max_tiles, s, pdl);
 }
 
 cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles, const int *n_tiles,
+                        const ExpertTile *tiles, const int *n_tiles,
                         float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
                         bool pdl)
 {
-    return launch_grouped<false>(w2_map, s2_map, w2_s, h, sorted_ids, topk_w, tiles, n_tiles, nullptr, y, status,
-                                 status_out, I, I, H, max_tiles, s, pdl);
+    return launch_grouped<false>(w2_map, s2_map, w2_s, h, tiles, n_tiles, nullptr, y, status, status_out, I, I, H, 1,
+                                 max_tiles, s, pdl);
 }
 
-cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl)
+cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
+                           bool pdl)
 {
     const size_t n = static_cast<size_t>(M) * H / 4;
     const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
-    return launch_ex(combine_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, y,
+    return launch_ex(combine_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, y, topk_w,
                      static_cast<__nv_bfloat16 *>(out), M, H, k);
 }
 

@@ -11,23 +11,28 @@
 //
 // One persistent CTA per SM, 16 warps:
 //  * warp 0 (weights producer): per 512-K stage, TMA copies of the item's packed E2M1 rows
-//    (128 rows x 256 bytes, 128-byte swizzle) and their E8M0 scales into a 3-stage ring;
+//    (128 rows x 256 bytes, 128-byte swizzle) and their E8M0 scales into a 4-stage ring;
 //    items come from the call's work queue, the ids reach the other warps through shared
 //    memory with the stage arrivals.
 //  * warp 2 (activations producer): per 64-K sub-tile, TMA copies of the item's activation
 //    rows (x gathered into expert-grouped order for gate_up, h for down), 16 rows per box,
-//    128-byte swizzle, into a 4-slot ring.  Rows past the tile are read and ignored.
+//    128-byte swizzle, into a 5-slot ring.  Rows past the tile are read and ignored.
 //  * warps 4..11 (dequant): per 64-K sub-tile, 256 threads each decode 32 weights of one row
 //    (hardware E2M1 -> f16x2), apply the row's E8M0 block scale in f16 (exact for scale bytes
 //    104..140: every scaled E2M1 value is then an f16 normal or subnormal; other bytes are
-//    flagged), and store them into a K-major 128-byte-swizzled A tile.  gate_up interleaves
-//    gate row i and up row i as A rows 2i, 2i+1, so one TMEM lane pair holds g and u.
-//  * warp 1 (MMA): one thread issues 4 tcgen05.mma kind::f16 (M 128, N = the tile's tokens
-//    rounded up to 16, K 16) per sub-tile into one of two TMEM accumulators and commits the
-//    consumed A and B buffers and, per item, the accumulator.
+//    flagged), and store them with tcgen05.st into an A buffer in tensor memory (TMEM lane =
+//    A row; a warp reaches the 32 lanes of its warp index mod 4, and warps 4..7 / 8..11 take
+//    the low / high 32 K of the sub-tile).  gate_up interleaves gate row i and up row i as A
+//    rows 2i, 2i+1, so one TMEM lane pair holds g and u.  A never passes through shared
+//    memory, which leaves shared-memory bandwidth to the TMA copies and the B operand.
+//  * warp 1 (MMA): one thread issues 4 tcgen05.mma kind::f16 (A from TMEM, B from shared
+//    memory; M 128, N = the tile's tokens rounded up to 16, K 16) per sub-tile into one of two
+//    TMEM accumulators and commits the consumed A and B buffers and, per item, the
+//    accumulator.
 //  * warps 12..15 (epilogue): tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //    32 (w % 4) ..); gate_up pairs g and u with one shuffle, applies clamp-SwiGLU and the bf16
-//    rounding and stores h; down applies the routing weight and stores the fp32 row of y.
+//    rounding and stores h; down stores the assignment's fp32 row of y (the combine applies
+//    the routing weight).
 // Every wait is bounded; after a timeout the kernel records MOE_ERR_TIMEOUT, drains the
 // copies it issued and frees its tensor memory.
 #include <cuda_bf16.h>
@@ -41,10 +46,10 @@ namespace moe {
 namespace wide {
 constexpr int kRows = 128;                               // weight rows per item (MMA M)
 constexpr int kStageK = kWideStageK;                     // 512 K per packed stage
-constexpr int kPStages = 3;                             // packed weight stages
+constexpr int kPStages = 4;                              // packed weight stages
 constexpr int kSubK = 64;                                // K per A/B sub-tile (one swizzle atom of f16)
 constexpr int kSubs = kStageK / kSubK;                   // 8
-constexpr int kABufs = 2, kBBufs = 4, kDBufs = 2;
+constexpr int kABufs = 4, kBBufs = 5, kDBufs = 2;
 constexpr int kItemQ = 8;
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
@@ -52,17 +57,18 @@ constexpr int kWProd = 0, kMma = 1, kBProd = 2, kDeq0 = 4, kDeqWarps = 8, kEpi0 
 constexpr int kPackedStage = kRows * kStageK / 2;        // 32 KB: 2 box columns x 128 rows x 128 B
 constexpr int kPackedCol = kRows * 128;                  // one box column (two 64-row boxes)
 constexpr int kScaleStage = kRows * kStageK / 32;        // 2 KB: 128 rows x 16 B
-constexpr int kATile = kRows * kSubK * 2;                // 16 KB
 constexpr int kBTile = kWideTokens * kSubK * 2;          // 16 KB
 constexpr int kBBox = 16 * kSubK * 2;                    // one 16-row activation box
-constexpr int kTmemCols = kDBufs * kWideTokens;          // 256
+constexpr int kACols = kSubK / 2;                        // TMEM columns of one A buffer (2 f16 per column)
+constexpr int kACol0 = kDBufs * kWideTokens;             // accumulators first, then the A buffers
+constexpr int kTmemCols = 512;                           // power of two >= kACol0 + kABufs * kACols
 constexpr int kOffPacked = 0;
 constexpr int kOffScale = kOffPacked + kPStages * kPackedStage;
-constexpr int kOffA = kOffScale + kPStages * kScaleStage;
-constexpr int kOffB = kOffA + kABufs * kATile;
+constexpr int kOffB = kOffScale + kPStages * kScaleStage;
 constexpr int kOffBars = kOffB + kBBufs * kBTile;
 constexpr int kSmemBytes = kOffBars + 512 + 1024;        // barriers and slots, + alignment slack
-static_assert(kOffA % 1024 == 0 && kOffB % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
+static_assert(kOffB % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
+static_assert(kACol0 + kABufs * kACols <= kTmemCols && kTmemCols <= 512, "TMEM budget");
 static_assert(kSmemBytes <= 227 * 1024, "fits one SM");
 }  // namespace wide
 
@@ -70,9 +76,8 @@ struct WideArgs {
     const WideTile *tiles;
     const int *n_tiles;
     const int32_t *sorted_ids;   // down: flat ids of the expert-grouped positions
-    const float *topk_w;         // down: routing weights by flat id
-    __half *h;                   // gate_up output [M*k][I] (binary16, h * 2^10)
-    float *y;                    // down output [M*k][H]
+    __half *h;                   // gate_up output [M*k][I] (binary16, h * 2^10), expert-grouped rows
+    float *y;                    // down output [M*k][H] by flat id, before the routing weight
     int *status_ws;
     int32_t *status_out;
     int *queue;
@@ -245,12 +250,15 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     }
     else if (warp >= kDeq0 && warp < kDeq0 + kDeqWarps) {
         // ------------------------------------------------------------ dequant warps
-        // thread t of the 256: weight row r = t / 2, K half h = t % 2 of each 64-K sub-tile
-        const int t = threadIdx.x - kDeq0 * 32;
-        const int r = t >> 1, h = t & 1;
-        // A row of weight row r: gate row i -> 2i, up row i -> 2i + 1 (gate_up); r (down)
-        const int ar = kGateUp ? (r < 64 ? 2 * r : 2 * (r - 64) + 1) : r;
+        // a warp stores TMEM lanes 32 (warp % 4) ..; its thread owns A row ar = that lane and the
+        // K half h (warps 4..7: low 32 K, 8..11: high 32 K) of each 64-K sub-tile
         const int dw = warp - kDeq0;
+        const int quarter = warp & 3, h = dw >> 2;
+        const int ar = 32 * quarter + lane;
+        // packed row of A row ar: A rows 2i, 2i + 1 = gate row i (box rows 0..63), up row i (box
+        // rows 64..127) for gate_up; row ar for down
+        const int r = kGateUp ? (ar >> 1) + (ar & 1) * 64 : ar;
+        const uint32_t a_lane = static_cast<uint32_t>(32 * quarter) << 16;
         bool bad_scale = false;
         int stage_ctr = 0, sub_ctr = 0;
         for (int item_ctr = 0;; ++item_ctr) {
@@ -270,6 +278,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     const int ab = sub_ctr % kABufs;
                     mbar_wait(&a_empty[ab], ((sub_ctr / kABufs) & 1) ^ 1, aborted, status);
                     if (aborted) break;
+                    tc_fence_after();   // the MMAs that read this A buffer are complete
                     if (item >= 0) {
                         // 16 packed bytes: box column j / 4, 16-byte chunk (j % 4) * 2 + h of row r
                         const int ch = (j & 3) * 2 + h;
@@ -291,14 +300,11 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                             v = __hmul2(v, s2);
                             f[i] = *reinterpret_cast<uint32_t *>(&v);
                         }
-                        uint8_t *at = smem + kOffA + ab * kATile;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)   // K 32h + 8i .. +7 of A row ar
-                            *reinterpret_cast<uint4 *>(at + sw128_offset(ar, 32 * h + 8 * i)) =
-                                make_uint4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
-                        fence_proxy_async_smem();
+                        // columns 16h .. 16h + 15 of the buffer: K 32h + 2i, 32h + 2i + 1 in column 16h + i
+                        tmem_st16(tmem + a_lane + static_cast<uint32_t>(kACol0 + ab * kACols + 16 * h), f);
                     }
                     if (dw == 0 && lane == 0) a_item[ab] = item;
+                    tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&a_full[ab]);
                 }
@@ -344,12 +350,12 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 if (aborted) break;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t a_addr = smem_u32(smem + kOffA + ab * kATile);
+                    const uint32_t a_tmem = tmem + static_cast<uint32_t>(kACol0 + ab * kACols);
                     const uint32_t b_addr = smem_u32(smem + kOffB + bb * kBTile);
 #pragma unroll
                     for (int ks = 0; ks < kSubK / 16; ++ks)
-                        umma_f16(d_tmem, umma_sdesc_sw128(a_addr + 32 * ks), umma_sdesc_sw128(b_addr + 32 * ks), idesc,
-                                 (j > 0 || ks > 0) ? 1u : 0u);
+                        umma_f16_tmem_a(d_tmem, a_tmem + 8 * ks, umma_sdesc_sw128(b_addr + 32 * ks), idesc,
+                                        (j > 0 || ks > 0) ? 1u : 0u);
                     umma_commit(smem_u32(&a_empty[ab]));
                     umma_commit(smem_u32(&b_empty[bb]));
                 }
@@ -397,15 +403,14 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                         }
                     }
                 } else {
+                    // h carries the 2^10 storage scale; the routing weight is applied by the combine
                     const int r = rb * kRows + row;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
+                    for (int j = 0; j < 16; ++j)
                         if (c + j < cnt) {
                             const int f = __ldcg(&a.sorted_ids[p0 + c + j]);
-                            const float w = __ldcg(&a.topk_w[f]) * (1.0f / kHScale);
-                            a.y[static_cast<size_t>(f) * H + r] = w * __uint_as_float(v[j]);
+                            a.y[static_cast<size_t>(f) * H + r] = __uint_as_float(v[j]) * (1.0f / kHScale);
                         }
-                    }
                 }
             }
             tc_fence_before();
@@ -446,14 +451,13 @@ cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __h
 
 cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap &smap, const CUtensorMap &bmap,
                         const WideTile *tiles, const int *n_tiles, int max_tiles, const int32_t *sorted_ids,
-                        const float *topk_w, __half *h, float *y, int *status, int32_t *status_out, int H, int I,
+                        __half *h, float *y, int *status, int32_t *status_out, int H, int I,
                         cudaStream_t s, bool pdl)
 {
     WideArgs a;
     a.tiles = tiles;
     a.n_tiles = n_tiles;
     a.sorted_ids = sorted_ids;
-    a.topk_w = topk_w;
     a.h = h;
     a.y = y;
     a.status_ws = status;

@@ -87,7 +87,7 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
     int p0;           // first position in the expert-grouped order
     int count;
     int pad;
-    int tok[kTileTokens];   // token of each assignment (sorted_ids[p0+i] / k); entries >= count repeat the last
+    int flat[kTileTokens];  // flat assignment id t*k + j of each slot (sorted_ids[p0+i]); entries >= count repeat the last
 };
 
 // Experts with at least kWideMinTokens assignments go to the tensor-core path (grouped_wide.cu)
@@ -186,17 +186,17 @@ cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
                            const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
-                           int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s, bool pdl);
+                           int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl);
 cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const int32_t *sorted_ids, const float *topk_w, const ExpertTile *tiles, const int *n_tiles,
-                        float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
+                        const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
                         bool pdl);
-cudaError_t launch_combine(const float *y, void *out, int M, int H, int k, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
+                           bool pdl);
 cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __half *x_perm, int n, int H, int k,
                                cudaStream_t s, bool pdl);
 cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap &smap, const CUtensorMap &bmap,
                         const WideTile *tiles, const int *n_tiles, int max_tiles, const int32_t *sorted_ids,
-                        const float *topk_w, __half *h, float *y, int *status, int32_t *status_out, int H, int I,
+                        __half *h, float *y, int *status, int32_t *status_out, int H, int I,
                         cudaStream_t s, bool pdl);
 int wide_smem_bytes();
 

@@ -165,16 +165,15 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
             } else if (tiles) {
                 const int slot = rank % kTileTokens, tile_first = rank - slot;
                 ExpertTile *tp = tiles + sm.tb[e] + rank / kTileTokens;
-                const int t = f / k;
-                tp->tok[slot] = t;
+                tp->flat[slot] = f;
                 if (slot == 0) {
                     tp->expert = e;
                     tp->p0 = sm.off[e] + tile_first;
                     tp->count = min(kTileTokens, cnt - tile_first);
                     tp->pad = 0;
                 }
-                if (rank == cnt - 1)   // the tile's last assignment repeats its token into the unused slots
-                    for (int j = slot + 1; j < kTileTokens; ++j) tp->tok[j] = t;
+                if (rank == cnt - 1)   // the tile's last assignment repeats into the unused slots
+                    for (int j = slot + 1; j < kTileTokens; ++j) tp->flat[j] = f;
             }
         }
     }
@@ -269,16 +268,15 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
         }
         const int slot = r % kTileTokens, tile_first = r - slot;
         ExpertTile *tp = tiles + tb[e] + r / kTileTokens;
-        const int t = f / k;
-        tp->tok[slot] = t;
+        tp->flat[slot] = f;
         if (slot == 0) {
             tp->expert = e;
             tp->p0 = off[e] + tile_first;
             tp->count = min(kTileTokens, c - tile_first);
             tp->pad = 0;
         }
-        if (r == c - 1)   // the tile's last assignment repeats its token into the unused slots
-            for (int j = slot + 1; j < kTileTokens; ++j) tp->tok[j] = t;
+        if (r == c - 1)   // the tile's last assignment repeats into the unused slots
+            for (int j = slot + 1; j < kTileTokens; ++j) tp->flat[j] = f;
     }
 }
 
@@ -303,7 +301,7 @@ __device__ inline void emit_tiles(const int *off, int E, int k, ExpertTile *tile
             tl.count = min(kTileTokens, cnt - i * kTileTokens);
             tl.pad = 0;
 #pragma unroll
-            for (int j = 0; j < kTileTokens; ++j) tl.tok[j] = sorted_flat(tl.p0 + min(j, tl.count - 1)) / k;
+            for (int j = 0; j < kTileTokens; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
             tiles[base++] = tl;
         }
     }

@@ -1,9 +1,10 @@
 // tcgen05.cuh -- 5th-generation tensor core (tcgen05) and tensor memory wrappers, sm_100a.
 //
 // Used by the wide-tile grouped kernel (grouped_wide.cu): a single thread issues
-// tcgen05.mma with both operands in shared memory (K-major, 128-byte swizzle) and the fp32
-// accumulator in tensor memory (TMEM); tcgen05.commit signals an mbarrier when the issued
-// MMAs are complete; tcgen05.ld moves accumulator columns to registers.
+// tcgen05.mma with B in shared memory (K-major, 128-byte swizzle), A in shared memory or in
+// tensor memory (TMEM), and the fp32 accumulator in TMEM; tcgen05.commit signals an mbarrier
+// when the issued MMAs are complete; tcgen05.st / tcgen05.ld move columns between registers
+// and TMEM.
 #pragma once
 
 #include <stdint.h>
@@ -67,6 +68,29 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
                  "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
                  : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, one kind::f16 instruction (K = 16).  A sits in TMEM with
+// lane i = row i and column c holding K elements 2c (low half) and 2c + 1 (high half), so one
+// K=16 step spans 8 columns.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane from registers (lane as in
+// tmem_ld16), then wait until the stores are done.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+                 "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // The mbarrier receives one arrival when every tcgen05 operation this thread issued before
