@@ -86,7 +86,8 @@ def algorithmic(shape, M, ids):
     gate_up = touched * (2 * I * H * 17 // 32) + M * H * 2 + M * k * I * 2
     down = touched * (I * H * 17 // 32) + M * k * I * 2 + M * H * 2
     return {"touched": touched, "bytes": total, "flops": flops, "weight_bytes": w_bytes,
-            "gate_up_bytes": gate_up, "down_bytes": down}
+            "gate_up_bytes": gate_up, "down_bytes": down,
+            "gate_up_flops": 4 * I * H * M * k, "down_flops": 2 * I * H * M * k}
 
 
 def kernel_source_hash():
@@ -358,7 +359,16 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     dom_bytes = {"gate_up_swiglu": work["gate_up_bytes"], "down_combine": work["down_bytes"]}.get(dominant)
     if dom_bytes is None:
         dom_bytes = work["bytes"]
-    achieved = dom_bytes / (kern_us[dominant] * 1e3)          # GB/s
+    dom_flops = {"gate_up_swiglu": work["gate_up_flops"], "down_combine": work["down_flops"]}.get(dominant,
+                                                                                                   work["flops"])
+    call_bound = "hbm" if work["bytes"] / hbm > work["flops"] / (tflops * 1e3) else "tensor"
+    if call_bound == "hbm":
+        roof = {"bound": "hbm", "achieved": dom_bytes / (kern_us[dominant] * 1e3), "peak": hbm, "unit": "GB/s",
+                "algorithmic_bytes_per_launch": dom_bytes}
+    else:   # the contraction binds: FLOPs against the sustained bf16 tensor peak
+        roof = {"bound": "tensor", "achieved": dom_flops / (kern_us[dominant] * 1e6), "peak": tflops,
+                "unit": "TFLOP/s", "algorithmic_flops_per_launch": dom_flops}
+    roof["frac"] = roof["achieved"] / roof["peak"]
     traffic = profiled_traffic() if (ci, M) == (1, 8) and dominant == "gate_up_swiglu" else None
     sorted_ms = sorted(step_ms)
     rec = {
@@ -369,18 +379,16 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
         "p10_us": sorted_ms[len(sorted_ms) // 10] * 1e3, "p50_us": statistics.median(step_ms) * 1e3,
         "p90_us": sorted_ms[(9 * len(sorted_ms)) // 10] * 1e3,
         "gbs": work["bytes"] / (mean_us * 1e3),
-        "roofline_call": {"bound": "hbm" if work["bytes"] / hbm > work["flops"] / (tflops * 1e3) else "tensor",
+        "roofline_call": {"bound": call_bound,
                           "roofline_us": roof_us, "frac": roof_us / mean_us, "peaks": peak_kind,
                           "roofline_us_nominal": roof_nominal_us, "frac_nominal": roof_nominal_us / mean_us,
                           "algorithmic_bytes": work["bytes"], "flops": work["flops"],
                           "touched_experts": work["touched"]},
         "kernels_us": kern_us,
-        "roofline": {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": dom_bytes},
+        "roofline": dict(kernel=dominant, traffic=traffic, peak_kind=peak_kind, **roof),
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": M * H * 2,
                 "path": "pinned host x -> moe_mxfp4_forward_ex (eager C-ABI call) -> pinned host out"},
-        "gpu_launches": (5 if M <= 64 else 6) * args.steps,
+        "gpu_launches": moe.moe_forward_launches(M, H, I, E, k) * args.steps,
         "clocks": clk,
     }
     if baselines and rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     MoEError,
     load,
     moe_down_combine,
+    moe_forward_launches,
     moe_gate_up_swiglu,
     moe_mxfp4_forward,
     moe_mxfp4_forward_ex,

@@ -21,7 +21,7 @@ MOE_ERR_TIMEOUT = -5
 # every symbol include/moe.h declares
 EXPORTS = (
     "moe_status_string", "moe_last_cuda_error", "moe_route", "moe_permute", "moe_gate_up_swiglu",
-    "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_mxfp4_forward_ex",
+    "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_forward_launches", "moe_mxfp4_forward_ex",
     "moe_mxfp4_forward_profile", "moe_route_noalloc",
 )
 H_STORAGE_SCALE = 1024.0   # moe_gate_up_swiglu stores binary16(h * 2^10)
@@ -67,6 +67,8 @@ def load():
     lib.moe_mxfp4_forward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P]
     lib.moe_workspace_bytes.restype = S
     lib.moe_workspace_bytes.argtypes = [I, I, I, I, I]
+    lib.moe_forward_launches.restype = I
+    lib.moe_forward_launches.argtypes = [I, I, I, I, I]
     lib.moe_mxfp4_forward_ex.restype = I
     lib.moe_mxfp4_forward_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, S, P]
     lib.moe_mxfp4_forward_profile.restype = I
@@ -102,6 +104,11 @@ def moe_status_string(status: int) -> str:
 
 def moe_workspace_bytes(M: int, H: int, I: int, E: int, k: int) -> int:
     return int(load().moe_workspace_bytes(M, H, I, E, k))
+
+
+def moe_forward_launches(M: int, H: int, I: int, E: int, k: int) -> int:
+    """Kernel launches of one layer call for this shape (negative MOE_* status if unsupported)."""
+    return int(load().moe_forward_launches(M, H, I, E, k))
 
 
 def moe_route(x, router_w, k: int, router_bias=None, stream=None):

@@ -14,7 +14,7 @@
 
 namespace moe {
 
-int grouped_smem_bytes(int K);
+int grouped_smem_bytes(int K, int width);
 
 static thread_local int g_last_cuda_error = 0;
 
@@ -58,8 +58,12 @@ Layout make_layout(int M, int H, int I, int E, int k)
 {
     Layout L;
     const size_t n = static_cast<size_t>(M) * k;
+    // 16-wide tiles when the experts average 4 or more assignments and their larger stages fit
+    L.width = tile_width(M, E, k);
+    if (L.width == 16 && (grouped_smem_bytes(H, 16) > 227 * 1024 || grouped_smem_bytes(I, 16) > 227 * 1024))
+        L.width = 8;
     L.max_tiles = static_cast<int>((n < static_cast<size_t>(E) ? n : static_cast<size_t>(E)) +
-                                   (n + kTileTokens - 1) / kTileTokens);
+                                   (n + L.width - 1) / L.width);
     size_t off = 0;
     auto take = [&](size_t bytes) {
         const size_t o = off;
@@ -80,8 +84,8 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.h = take(n * I * 2);
     L.y = take(n * H * sizeof(float));
     L.wide = wide_enabled(M, H, I);
-    L.max_wide = L.wide ? static_cast<int>((n / (kTileTokens + 1) < static_cast<size_t>(E) ? n / (kTileTokens + 1)
-                                                                                             : static_cast<size_t>(E)) +
+    L.max_wide = L.wide ? static_cast<int>((n / kWideMinTokens < static_cast<size_t>(E) ? n / kWideMinTokens
+                                                                                         : static_cast<size_t>(E)) +
                                            n / kWideTokens + 1)
                         : 0;
     L.wide_tiles = take(static_cast<size_t>(L.max_wide) * sizeof(WideTile));
@@ -105,7 +109,7 @@ int check_dims(int M, int H, int I, int E, int k, bool need_hi)
     if (need_hi) {
         if (static_cast<long long>(E) * 2 * I >= (1LL << 31) || static_cast<long long>(E) * H >= (1LL << 31))
             return MOE_ERR_UNSUPPORTED_SHAPE;
-        if (grouped_smem_bytes(H) > 227 * 1024 || grouped_smem_bytes(I) > 227 * 1024)
+        if (grouped_smem_bytes(H, 8) > 227 * 1024 || grouped_smem_bytes(I, 8) > 227 * 1024)
             return MOE_ERR_UNSUPPORTED_SHAPE;
     }
     return MOE_OK;
@@ -229,7 +233,7 @@ static int library_workspace(cudaStream_t s, size_t need, char **out)
 
 static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const ExpertTile *tiles,
                        const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E, int k,
-                       int max_tiles, cudaStream_t s, bool pdl)
+                       int width, int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
     // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
@@ -242,7 +246,8 @@ static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x1
                             kItemRows / 2);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, k, max_tiles, s, pdl));
+    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, k, width, max_tiles, s,
+                           pdl));
     return MOE_OK;
 }
 
@@ -259,7 +264,7 @@ struct Marks {
     } while (0)
 
 static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
-                    int32_t *status_out, int H, int I, int E, int max_tiles, cudaStream_t s, bool pdl)
+                    int32_t *status_out, int H, int I, int E, int width, int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
     int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kItemRows);
@@ -269,7 +274,7 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
         rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_down(map, smap, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, max_tiles, s, pdl));
+    MOE_TRY(launch_down(map, smap, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, width, max_tiles, s, pdl));
     return MOE_OK;
 }
 
@@ -312,7 +317,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     WideTile *wtiles = reinterpret_cast<WideTile *>(ws + L.wide_tiles);
     int *n_wide = reinterpret_cast<int *>(ws + L.n_wide);
     __half *x_perm = reinterpret_cast<__half *>(ws + L.x_perm);
-    const TileOut to{tiles, n_tiles, L.wide ? wtiles : nullptr, n_wide};
+    const TileOut to{tiles, n_tiles, L.wide ? wtiles : nullptr, n_wide, L.width};
     // The first kernel is ordered after everything before it on the stream; each later
     // kernel of the call is launched early (programmatic dependent launch) and waits on
     // device for its predecessor.  Event marks (profiling) break that overlap, so the
@@ -333,7 +338,8 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     }
     MOE_MARK(marks, s);
     // gate_up: the 8-assignment tiles on mma.sync, then (large M) the wide tiles on tcgen05
-    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, k, L.max_tiles, s, pdl);
+    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, k, L.width, L.max_tiles, s,
+                         pdl);
     if (rc != MOE_OK) return rc;
     if (L.wide) {
         MOE_TRY(launch_gather_rows(x16, sorted_ids, x_perm, M * k, H, k, s, pdl));
@@ -343,7 +349,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     }
     MOE_MARK(marks, s);
     // down likewise, then the weighted top-k combine
-    rc = run_down(w2_q, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, E, L.max_tiles, s, pdl);
+    rc = run_down(w2_q, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, E, L.width, L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
     if (L.wide) {
         rc = run_wide(false, w2_q, w2_s, h, wtiles, n_wide, L.max_wide, sorted_ids, h, y, status, status_out, M, H, I,
@@ -402,6 +408,15 @@ size_t moe_workspace_bytes(int M, int H, int I, int E, int k)
     return make_layout(M, H, I, E, k).total;
 }
 
+int moe_forward_launches(int M, int H, int I, int E, int k)
+{
+    const int rc = check_dims(M, H, I, E, k, true);
+    if (rc != MOE_OK) return rc;
+    if (M == 0) return 0;
+    // route_logits, select (+ permute), gate_up, down, combine; gather + two wide GEMMs
+    return (fused_select(M, E, k) ? 5 : 6) + (wide_enabled(M, H, I) ? 3 : 0);
+}
+
 int moe_route(const void *x_bf16, const float *router_w, const float *router_bias, int32_t *topk_ids, float *topk_w,
               int M, int H, int E, int k, cudaStream_t stream)
 {
@@ -434,7 +449,7 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
     if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
         return MOE_ERR_INVALID_ARG;
     if (M == 0) return MOE_OK;
-    const TileOut none{nullptr, nullptr, nullptr, nullptr};
+    const TileOut none{nullptr, nullptr, nullptr, nullptr, 8};
     MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, none, M, E, k, stream, false));
     return MOE_OK;
 }
@@ -459,9 +474,9 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, L.width, stream));
     return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E, k,
-                       L.max_tiles, stream, false);
+                       L.width, L.max_tiles, stream, false);
 }
 
 int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
@@ -484,8 +499,8 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, k, stream));
-    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), tiles, n_tiles, y, status, nullptr, H, I, E,
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, L.width, stream));
+    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), tiles, n_tiles, y, status, nullptr, H, I, E, L.width,
                   L.max_tiles, stream, false);
     if (rc != MOE_OK) return rc;
     MOE_TRY(launch_combine(y, topk_w, out_bf16, M, H, k, stream, false));

@@ -51,32 +51,52 @@
 
 namespace moe {
 
-constexpr int kThreads = (kComputeWarps + 1 + kEpilogueWarps) * 32;
 constexpr int kProducerWarp = kComputeWarps;
 constexpr int kFirstEpilogueWarp = kComputeWarps + 1;
-constexpr int kRedFloats = kKSlots * kItemMTiles * 32 * 4;   // one buffer: [kslot][m-tile][lane][4]
 constexpr int kBlocksPerStage = kChunkK / 32;
 constexpr int kBlocksPerWarp = kBlocksPerStage / kKSlots;
 constexpr int kItemQ = 8;   // item ids in flight between the producer and the compute warps (> kStages)
-constexpr int kRedBufs = 2; // K-slot partial-sum buffers between the compute and epilogue warps
 static_assert(kBlocksPerWarp * kKSlots == kBlocksPerStage, "stage blocks split evenly over K slots");
 static_assert(8 % kBlocksPerWarp == 0, "a warp's blocks stay inside one 128-byte box column");
+static_assert(kKSlots % 2 == 0, "K slots pair up");
+
+// Per tile width kN (8 or 16 assignments): kN / 8 MMA n-tiles share every decoded weight
+// fragment.  With 16, the K-slot partial sums are pre-reduced in pairs of warps (odd K slot into
+// its even neighbour) so that one buffer of them fits next to the 16-row activation stages.
+template <int kN>
+struct Tiling {
+    static constexpr int kHalves = kN / 8;
+    static constexpr bool kPairRed = kN == 16;
+    static constexpr int kRedSets = kPairRed ? kKSlots / 2 : kKSlots;   // partial sets per buffer
+    static constexpr int kRedBufs = kPairRed ? 1 : 2;
+    static constexpr int kRedFloats = kRedSets * kItemMTiles * 32 * 4 * kHalves;   // [set][m-tile][lane][4 kHalves]
+    static constexpr int kEpiWarps = kN == 16 ? 4 : 2;
+    static constexpr int kThreads = (kComputeWarps + 1 + kEpiWarps) * 32;
+    static constexpr int kActStageBytes = kN * kActPitch;
+    static constexpr int kRedArrivals = kPairRed ? kComputeWarps / 2 : kComputeWarps;   // warps that post partials
+    static_assert(kItemMTiles % kEpiWarps == 0, "m-tiles split evenly over the epilogue warps");
+};
 
 struct SmemPlan {
     int wst_off, act_off, sst_off, sbuf_off, sbuf_bytes, red_off, bars_off, total;
 };
 
+constexpr int kNumBars = 2 * kStages + 8 + kComputeWarps / 2;   // ring, scale buffers, partials, K-slot pairs
+constexpr int kMetaInts = (3 + kTileTokensMax) * (kItemQ + 2);  // item ids, positions, counts, flat ids
+
+template <int kN>
 __host__ __device__ inline SmemPlan smem_plan(int K)
 {
+    using T = Tiling<kN>;
     SmemPlan p;
     p.wst_off = 0;
     p.act_off = kStages * kStageBytes;
-    p.sst_off = p.act_off + kStages * kActStageBytes;
+    p.sst_off = p.act_off + kStages * T::kActStageBytes;
     p.sbuf_off = p.sst_off + kStages * kStageScaleBytes;
     p.sbuf_bytes = per_stage_scales(K) ? 0 : (kItemRows * (K / 32) + 127) / 128 * 128;
     p.red_off = p.sbuf_off + 2 * p.sbuf_bytes;
-    p.bars_off = p.red_off + kRedBufs * kRedFloats * 4;
-    p.total = p.bars_off + (2 * kStages + 8) * 8 + (3 + kTileTokens) * (kItemQ + kRedBufs) * 4 + 1024;   // + slack
+    p.bars_off = p.red_off + T::kRedBufs * T::kRedFloats * 4;
+    p.total = p.bars_off + kNumBars * 8 + kMetaInts * 4 + 1024;   // + alignment slack
     return p;
 }
 
@@ -93,8 +113,8 @@ __device__ __forceinline__ __half store_h(float v)
     return __float2half_rn(__bfloat162float(__float2bfloat16_rn(v)) * kHScale);
 }
 
-template <bool kGateUp>
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool kGateUp, int kN>
+__global__ void __launch_bounds__(Tiling<kN>::kThreads, 1)
 grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
                      const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
@@ -104,7 +124,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    const SmemPlan plan = smem_plan(K);
+    using T = Tiling<kN>;
+    constexpr int kRedBufs = T::kRedBufs;
+    constexpr int kActStageBytes = T::kActStageBytes;
+    const SmemPlan plan = smem_plan<kN>(K);
     uint8_t *wst = smem + plan.wst_off;
     uint8_t *ast = smem + plan.act_off;
     uint8_t *sst = smem + plan.sst_off;
@@ -113,17 +136,18 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + plan.bars_off);
     uint64_t *full = bars, *empty = bars + kStages;
     uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
+    uint64_t *pair = sfull + 8;   // [kComputeWarps / 2]: odd K slot's partials posted (pair reduction)
     // per item in flight: id, first expert-grouped position, assignment count and the slots'
     // flat assignment ids (producer -> compute warps -> epilogue warps), so that no consumer
     // reads the tile list from global memory
-    volatile int *item_q = reinterpret_cast<volatile int *>(bars + 2 * kStages + 8);   // [kItemQ]
+    volatile int *item_q = reinterpret_cast<volatile int *>(bars + kNumBars);         // [kItemQ]
     volatile int *item_p0 = item_q + kItemQ;                                          // [kItemQ]
     volatile int *item_cnt = item_p0 + kItemQ;                                        // [kItemQ]
-    volatile int *item_flat = item_cnt + kItemQ;                                      // [kItemQ][kTileTokens]
-    volatile int *red_item = item_flat + kItemQ * kTileTokens;                        // [kRedBufs]
-    volatile int *red_p0 = red_item + kRedBufs;                                       // [kRedBufs]
-    volatile int *red_cnt = red_p0 + kRedBufs;                                        // [kRedBufs]
-    volatile int *red_flat = red_cnt + kRedBufs;                                      // [kRedBufs][kTileTokens]
+    volatile int *item_flat = item_cnt + kItemQ;                                      // [kItemQ][kTileTokensMax]
+    volatile int *red_item = item_flat + kItemQ * kTileTokensMax;                     // [kRedBufs]
+    volatile int *red_p0 = red_item + 2;                                              // [kRedBufs]
+    volatile int *red_cnt = red_p0 + 2;                                               // [kRedBufs]
+    volatile int *red_flat = red_cnt + 2;                                             // [kRedBufs][kTileTokensMax]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
@@ -147,9 +171,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             mbar_init(&sempty[b], kComputeWarps);
         }
         for (int b = 0; b < kRedBufs; ++b) {
-            mbar_init(&rfull[b], kComputeWarps);
-            mbar_init(&rempty[b], kEpilogueWarps);
+            mbar_init(&rfull[b], T::kRedArrivals);
+            mbar_init(&rempty[b], T::kEpiWarps);
         }
+        for (int i = 0; i < kComputeWarps / 2; ++i) mbar_init(&pair[i], 1);
         fence_barrier_init();
     }
     __syncthreads();
@@ -182,7 +207,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 nx_e = __ldcg(&tp->expert);
                 nx_p0 = __ldcg(&tp->p0);
                 nx_cnt = __ldcg(&tp->count);
-                nx_flat = __ldcg(&tp->flat[lane & (kTileTokens - 1)]);
+                nx_flat = __ldcg(&tp->flat[lane & (kTileTokensMax - 1)]);
             }
         };
         // down: h copies of the first stages, held back until gate_up has completed
@@ -236,7 +261,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 item_p0[item_ctr % kItemQ] = p0;
                 item_cnt[item_ctr % kItemQ] = cnt;
             }
-            if (!kGateUp && lane < kTileTokens) item_flat[(item_ctr % kItemQ) * kTileTokens + lane] = flat;
+            if (!kGateUp && lane < kN) item_flat[(item_ctr % kItemQ) * kTileTokensMax + lane] = flat;
             const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
@@ -341,58 +366,68 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         // nothing for the epilogue before the first item's partial sums; the down kernel's
         // epilogue waits for gate_up here so that its plain loads see the current call's data
         if (!kGateUp) pdl_wait();
+        constexpr int kEpiMTiles = kItemMTiles / T::kEpiWarps;   // m-tiles ep, ep + kEpiWarps, ..
+        constexpr int kVals = 4 * T::kHalves;                    // partial floats per lane and m-tile
         for (int item_ctr = 0;; ++item_ctr) {
             const int b = item_ctr % kRedBufs;
-            const float *rbuf = red + b * kRedFloats;
+            const float *rbuf = red + b * T::kRedFloats;
             mbar_wait(&rfull[b], (item_ctr / kRedBufs) & 1, aborted, status);
             if (aborted) break;
             const int item = red_item[b];   // -1: no further item
             if (item < 0) break;
             const int rb = item % row_blocks;
             const int cnt = red_cnt[b], p0 = red_p0[b];
-            float4 sums[2];
+            // sums over the partial sets in set order (K slots, or K-slot pairs), per n-half
+            float4 sums[kEpiMTiles][T::kHalves];
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int j = ep + 2 * m;
-                float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int m = 0; m < kEpiMTiles; ++m) {
+                const int j = ep + T::kEpiWarps * m;
 #pragma unroll
-                for (int ks = 0; ks < kKSlots; ++ks) {
-                    const float4 v = *reinterpret_cast<const float4 *>(rbuf + ((ks * kItemMTiles + j) * 32 + lane) * 4);
-                    sum.x += v.x;
-                    sum.y += v.y;
-                    sum.z += v.z;
-                    sum.w += v.w;
+                for (int hf = 0; hf < T::kHalves; ++hf) {
+                    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int ks = 0; ks < T::kRedSets; ++ks) {
+                        const float4 v =
+                            *reinterpret_cast<const float4 *>(rbuf + ((ks * kItemMTiles + j) * 32 + lane) * kVals + 4 * hf);
+                        sum.x += v.x;
+                        sum.y += v.y;
+                        sum.z += v.z;
+                        sum.w += v.w;
+                    }
+                    sums[m][hf] = sum;
                 }
-                sums[m] = sum;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&rempty[b]);
-            const int li0 = 2 * q, li1 = li0 + 1;
 #pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int j = ep + 2 * m;
-                float4 sum = sums[m];
-                if (kGateUp) {
-                    // remove the factor 2 carried by e8m0_times2
-                    const int n = rb * 32 + 8 * j + g;
-                    if (li0 < cnt)
-                        hout[static_cast<size_t>(p0 + li0) * I + n] = store_h(clamp_swiglu(0.5f * sum.x, 0.5f * sum.z));
-                    if (li1 < cnt)
-                        hout[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
-                } else {
-                    // remove e8m0_times2's factor 2 and h's 2^10 storage scale; the routing weight
-                    // is applied by the combine
-                    const float unscale = 0.5f / kHScale;
-                    const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
-                    if (li0 < cnt) {
-                        float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokens + li0]) * H;
-                        if (ra < rows_total) yr[ra] = unscale * sum.x;
-                        if (rbw < rows_total) yr[rbw] = unscale * sum.z;
-                    }
-                    if (li1 < cnt) {
-                        float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokens + li1]) * H;
-                        if (ra < rows_total) yr[ra] = unscale * sum.y;
-                        if (rbw < rows_total) yr[rbw] = unscale * sum.w;
+            for (int m = 0; m < kEpiMTiles; ++m) {
+                const int j = ep + T::kEpiWarps * m;
+#pragma unroll
+                for (int hf = 0; hf < T::kHalves; ++hf) {
+                    const float4 sum = sums[m][hf];
+                    const int li0 = 8 * hf + 2 * q, li1 = li0 + 1;   // the fragment's two tile slots
+                    if (kGateUp) {
+                        // remove the factor 2 carried by e8m0_times2
+                        const int n = rb * 32 + 8 * j + g;
+                        if (li0 < cnt)
+                            hout[static_cast<size_t>(p0 + li0) * I + n] = store_h(clamp_swiglu(0.5f * sum.x, 0.5f * sum.z));
+                        if (li1 < cnt)
+                            hout[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
+                    } else {
+                        // remove e8m0_times2's factor 2 and h's 2^10 storage scale; the routing
+                        // weight is applied by the combine
+                        const float unscale = 0.5f / kHScale;
+                        const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
+                        if (li0 < cnt) {
+                            float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokensMax + li0]) * H;
+                            if (ra < rows_total) yr[ra] = unscale * sum.x;
+                            if (rbw < rows_total) yr[rbw] = unscale * sum.z;
+                        }
+                        if (li1 < cnt) {
+                            float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokensMax + li1]) * H;
+                            if (ra < rows_total) yr[ra] = unscale * sum.y;
+                            if (rbw < rows_total) yr[rbw] = unscale * sum.w;
+                        }
                     }
                 }
             }
@@ -430,6 +465,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     // scale addressing: per stage, row pitch kChunkK/32 bytes and block index within the stage;
     // per item, row pitch kblocks and the global block index
     const int s_pitch = stage_scales ? kChunkK / 32 : kblocks;
+    // pair reduction (kN == 16): the odd K slot posts its partials, the even one adds its own
+    const bool odd_slot = (kslot & 1) != 0;
+    const int pair_id = mgrp * (kKSlots / 2) + (kslot >> 1);
+    constexpr int kVals = 4 * T::kHalves;   // partial floats per lane and m-tile
 
     int stage_ctr = 0, item_ctr = 0;
     for (;; ++item_ctr) {
@@ -438,14 +477,16 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         mbar_wait(&full[stage_ctr % kStages], (stage_ctr / kStages) & 1, aborted, status);
         if (aborted) break;
         if (item_q[item_ctr % kItemQ] < 0) break;
+        // the second n-tile of a 16-wide tile only when it holds assignments (warp-uniform)
+        const bool two = kN == 16 && item_cnt[item_ctr % kItemQ] > 8;
         const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
         if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
 
-        float acc[kWarpMTiles][4];
+        float acc[kWarpMTiles][kVals];
 #pragma unroll
         for (int m = 0; m < kWarpMTiles; ++m)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) acc[m][r] = 0.f;
+            for (int r = 0; r < kVals; ++r) acc[m][r] = 0.f;
 
         for (int c = 0; c < n_chunks; ++c, ++stage_ctr) {
             const int s = stage_ctr % kStages;
@@ -459,6 +500,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             for (int bi = 0; bi < kBlocksPerWarp; ++bi) {
                 if (c * kBlocksPerStage + blk_base + bi >= kblocks) continue;
                 const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (blk_base + bi) + 8 * q) * 2);
+                uint4 xc = make_uint4(0u, 0u, 0u, 0u);   // token g + 8 (second n-tile)
+                if (kN == 16 && two)
+                    xc = *reinterpret_cast<const uint4 *>(xa + 8 * kActPitch + (32 * (blk_base + bi) + 8 * q) * 2);
                 const int sw = (((bb0 + bi) ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
 #pragma unroll
                 for (int m = 0; m < kWarpMTiles; ++m) {
@@ -478,6 +522,15 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     acc[m][1] = fmaf(tmp[1], st_scale, acc[m][1]);
                     acc[m][2] = fmaf(tmp[2], sb_scale, acc[m][2]);
                     acc[m][3] = fmaf(tmp[3], sb_scale, acc[m][3]);
+                    if (kN == 16 && two) {
+                        float tmq[4];
+                        mma_f16_16816(tmq, a0, xc.x, xc.y, zero4);
+                        mma_f16_16816(tmq, a1, xc.z, xc.w, tmq);
+                        acc[m][kVals - 4] = fmaf(tmq[0], st_scale, acc[m][kVals - 4]);
+                        acc[m][kVals - 3] = fmaf(tmq[1], st_scale, acc[m][kVals - 3]);
+                        acc[m][kVals - 2] = fmaf(tmq[2], sb_scale, acc[m][kVals - 2]);
+                        acc[m][kVals - 1] = fmaf(tmq[3], sb_scale, acc[m][kVals - 1]);
+                    }
                 }
             }
             __syncwarp();
@@ -486,25 +539,59 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         __syncwarp();
         if (!stage_scales && lane == 0) mbar_arrive(&sempty[b]);
 
-        // park the K-slot partial sums (and the item id) for the epilogue warps
+        // park the K-slot partial sums (and the item's ids) for the epilogue warps
         const int rb = item_ctr % kRedBufs;
-        mbar_wait(&rempty[rb], ((item_ctr / kRedBufs) & 1) ^ 1, aborted, status);
-        float *rbuf = red + rb * kRedFloats;
+        float *rbuf = red + rb * T::kRedFloats;
+        const int set = T::kPairRed ? kslot >> 1 : kslot;
+        if (T::kPairRed && odd_slot) {
+            // post this slot's partials into the pair's set; the even neighbour adds to them
+            mbar_wait(&rempty[rb], ((item_ctr / kRedBufs) & 1) ^ 1, aborted, status);
+            if (aborted) break;
+#pragma unroll
+            for (int m = 0; m < kWarpMTiles; ++m)
+#pragma unroll
+                for (int v = 0; v < kVals; v += 4)
+                    *reinterpret_cast<float4 *>(rbuf + ((set * kItemMTiles + mgrp * kWarpMTiles + m) * 32 + lane) * kVals + v) =
+                        make_float4(acc[m][v], acc[m][v + 1], acc[m][v + 2], acc[m][v + 3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pair[pair_id]);
+            continue;
+        }
+        if (T::kPairRed) {
+            // the odd neighbour's partials are posted (it waited for the buffer); even + odd
+            mbar_wait(&pair[pair_id], item_ctr & 1, aborted, status);
+        } else {
+            mbar_wait(&rempty[rb], ((item_ctr / kRedBufs) & 1) ^ 1, aborted, status);
+        }
+        if (aborted) break;
 #pragma unroll
         for (int m = 0; m < kWarpMTiles; ++m)
-            *reinterpret_cast<float4 *>(rbuf + ((kslot * kItemMTiles + mgrp * kWarpMTiles + m) * 32 + lane) * 4) =
-                make_float4(acc[m][0], acc[m][1], acc[m][2], acc[m][3]);
+#pragma unroll
+            for (int v = 0; v < kVals; v += 4) {
+                float4 *dst =
+                    reinterpret_cast<float4 *>(rbuf + ((set * kItemMTiles + mgrp * kWarpMTiles + m) * 32 + lane) * kVals + v);
+                float4 o = make_float4(acc[m][v], acc[m][v + 1], acc[m][v + 2], acc[m][v + 3]);
+                if (T::kPairRed) {
+                    const float4 p = *dst;
+                    o.x += p.x;
+                    o.y += p.y;
+                    o.z += p.z;
+                    o.w += p.w;
+                }
+                *dst = o;
+            }
         if (warp == 0 && lane == 0) {
             red_item[rb] = item_q[item_ctr % kItemQ];
             red_p0[rb] = item_p0[item_ctr % kItemQ];
             red_cnt[rb] = item_cnt[item_ctr % kItemQ];
         }
-        if (!kGateUp && warp == 0 && lane < kTileTokens)
-            red_flat[rb * kTileTokens + lane] = item_flat[(item_ctr % kItemQ) * kTileTokens + lane];
+        if (!kGateUp && warp == 0 && lane < kN)
+            red_flat[rb * kTileTokensMax + lane] = item_flat[(item_ctr % kItemQ) * kTileTokensMax + lane];
         __syncwarp();
         if (lane == 0) mbar_arrive(&rfull[rb]);
     }
-    // end marker for the epilogue warps
+    // end marker for the epilogue warps (from the warps that post partials)
+    if (T::kPairRed && odd_slot) return;
     const int rb = item_ctr % kRedBufs;
     mbar_wait(&rempty[rb], ((item_ctr / kRedBufs) & 1) ^ 1, aborted, status);
     if (!aborted) {
@@ -540,41 +627,48 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     *reinterpret_cast<uint2 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint2 *>(o);
 }
 
-template <bool kGateUp>
+template <bool kGateUp, int kN>
 static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
                                   const __half *act, const ExpertTile *tiles, const int *n_tiles, __half *h, float *y,
                                   int *status, int32_t *status_out, int K, int I, int H, int k, int max_tiles,
                                   cudaStream_t s, bool pdl)
 {
-    const SmemPlan plan = smem_plan(K);
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(grouped_mxfp4_kernel<kGateUp>), plan.total);
+    const SmemPlan plan = smem_plan<kN>(K);
+    auto kern = grouped_mxfp4_kernel<kGateUp, kN>;
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(kern), plan.total);
     if (e != cudaSuccess) return e;
     const long long row_blocks = kGateUp ? I / 32 : down_row_blocks(H);
     const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
     int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     if (grid < 1) grid = 1;
     int *queue = status + (kGateUp ? kQueueGateUp : kQueueDown);
-    return launch_ex(grouped_mxfp4_kernel<kGateUp>, dim3(grid), dim3(kThreads), plan.total, s, pdl, map, smap,
-                     scales, act, tiles, n_tiles, h, y, status, status_out, queue, K, I, H, k);
+    return launch_ex(kern, dim3(grid), dim3(Tiling<kN>::kThreads), plan.total, s, pdl, map, smap, scales, act, tiles,
+                     n_tiles, h, y, status, status_out, queue, K, I, H, k);
 }
 
-int grouped_smem_bytes(int K) { return smem_plan(K).total; }
+int grouped_smem_bytes(int K, int width) { return width == 16 ? smem_plan<16>(K).total : smem_plan<8>(K).total; }
 
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
                            const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
-                           int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl)
+                           int32_t *status_out, int H, int I, int k, int width, int max_tiles, cudaStream_t s,
+                           bool pdl)
 {
-    return launch_grouped<true>(w13_map, s13_map, w13_s, x16, tiles, n_tiles, h, nullptr, status, status_out, H, I, H,
-                                k, max_tiles, s, pdl);
+    if (width == 16)
+        return launch_grouped<true, 16>(w13_map, s13_map, w13_s, x16, tiles, n_tiles, h, nullptr, status, status_out, H,
+                                        I, H, k, max_tiles, s, pdl);
+    return launch_grouped<true, 8>(w13_map, s13_map, w13_s, x16, tiles, n_tiles, h, nullptr, status, status_out, H, I,
+                                   H, k, max_tiles, s, pdl);
 }
 
 cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const ExpertTile *tiles, const int *n_tiles,
-                        float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
-                        bool pdl)
+                        const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int32_t *status_out, int H,
+                        int I, int width, int max_tiles, cudaStream_t s, bool pdl)
 {
-    return launch_grouped<false>(w2_map, s2_map, w2_s, h, tiles, n_tiles, nullptr, y, status, status_out, I, I, H, 1,
-                                 max_tiles, s, pdl);
+    if (width == 16)
+        return launch_grouped<false, 16>(w2_map, s2_map, w2_s, h, tiles, n_tiles, nullptr, y, status, status_out, I, I,
+                                         H, 1, max_tiles, s, pdl);
+    return launch_grouped<false, 8>(w2_map, s2_map, w2_s, h, tiles, n_tiles, nullptr, y, status, status_out, I, I, H, 1,
+                                    max_tiles, s, pdl);
 }
 
 cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,

@@ -21,7 +21,8 @@ constexpr int kQueueGateUpWide = 24;
 constexpr int kQueueDownWide = 32;
 
 // Grouped GEMM tiling (both projections).
-constexpr int kTileTokens = 8;       // assignments per expert tile (one MMA n-tile)
+// An expert tile holds up to 8 or 16 assignments (tile_width): one or two MMA n-tiles of 8.
+constexpr int kTileTokensMax = 16;
 constexpr int kItemMTiles = 4;       // MMA m-tiles (16 weight rows each) per work item
 constexpr int kItemRows = 16 * kItemMTiles;
 constexpr int kChunkK = 1024;        // K elements per pipeline stage (512 bytes of E2M1 per row)
@@ -29,7 +30,6 @@ constexpr int kBoxCols = kChunkK / 256;              // 128-byte TMA box columns
 constexpr int kStageBytes = kItemRows * kChunkK / 2; // packed weights of one stage (32 KB)
 constexpr int kStageScaleBytes = kItemRows * kChunkK / 32;   // E8M0 bytes of one stage (per-stage mode)
 constexpr int kActPitch = kChunkK * 2 + 64;         // one token's binary16 chunk, padded against bank conflicts
-constexpr int kActStageBytes = kTileTokens * kActPitch;
 constexpr int kStages = 3;
 constexpr int kComputeWarps = 16;    // 2 m-tile pairs x 8 K slots
 constexpr int kWarpMTiles = 2;       // m-tiles per compute warp (the activation fragment serves both)
@@ -82,13 +82,23 @@ constexpr int kMaxE = 1024;
 constexpr int kMaxK = 32;
 constexpr int kMaxAssignments = 16384;
 
-struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignments
+struct ExpertTile {   // one expert's run of <= tile_width consecutive assignments
     int expert;
     int p0;           // first position in the expert-grouped order
     int count;
     int pad;
-    int flat[kTileTokens];  // flat assignment id t*k + j of each slot (sorted_ids[p0+i]); entries >= count repeat the last
+    int flat[kTileTokensMax];   // flat assignment id t*k + j of each slot (sorted_ids[p0+i]); entries >= count repeat the last
 };
+
+// Tile width of a call: 16 assignments (two n-tiles per decoded weight fragment) once the
+// experts average at least 6 assignments, else 8.  Wider tiles stream each expert's weights
+// once for up to 16 assignments at the price of twice the MMAs per decoded fragment, larger
+// per-item buffers and a single partial-sum buffer, which only pays when many experts hold
+// more than 8.
+__host__ __device__ inline int tile_width(int M, int E, int k)
+{
+    return static_cast<long long>(M) * k >= 6LL * E ? 16 : 8;
+}
 
 // Experts with at least kWideMinTokens assignments go to the tensor-core path (grouped_wide.cu)
 // as wide tiles of up to kWideTokens consecutive assignments; it needs H and I to be multiples
@@ -96,7 +106,7 @@ struct ExpertTile {   // one expert's run of <= kTileTokens consecutive assignme
 // never uses it.
 constexpr int kWideTokens = 128;
 constexpr int kWideStageK = 512;
-constexpr int kWideMinTokens = 32;   // fewer assignments stream faster as 8-assignment tiles
+constexpr int kWideMinTokens = 32;   // fewer assignments stream faster as mma.sync tiles
 struct WideTile {
     int expert;
     int p0;      // first position in the expert-grouped order
@@ -113,6 +123,7 @@ struct Layout {
     size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y;
     size_t wide_tiles, n_wide, x_perm, total;
     int splits;   // router partial-logit slices (route_plan)
+    int width;    // tile_width
     int max_tiles, max_wide;
     bool wide;    // wide_enabled for this shape
 };
@@ -167,14 +178,15 @@ cudaError_t launch_route_logits(const void *x, const float *router_w, float *par
                                 int32_t *status_out, int M, int H, int E, cudaStream_t s);
 cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
                               int E, int k, cudaStream_t s, bool pdl);
-// Tile outputs of the route remap: 8-assignment tiles for the mma.sync kernels and, when
-// `wide` is set, wide tiles (experts with more than kTileTokens assignments) for the
-// tensor-core kernels; such experts then get no 8-assignment tiles.
+// Tile outputs of the route remap: tiles of `width` (8 or 16) assignments for the mma.sync
+// kernels and, when wide_tiles is set, wide tiles (experts with at least kWideMinTokens
+// assignments) for the tensor-core kernels; such experts then get no mma.sync tiles.
 struct TileOut {
     ExpertTile *tiles;
     int *n_tiles;
-    WideTile *wide_tiles;   // nullptr: every expert gets 8-assignment tiles
+    WideTile *wide_tiles;   // nullptr: every expert gets mma.sync tiles
     int *n_wide;
+    int width;
 };
 cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
                                         int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M,
@@ -182,14 +194,15 @@ cudaError_t launch_route_select_permute(const float *partial, int splits, const 
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
                            int M, int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
-                               int *status, int E, int k, cudaStream_t s);
+                               int *status, int E, int width, cudaStream_t s);
 cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
                            const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
-                           int32_t *status_out, int H, int I, int k, int max_tiles, cudaStream_t s, bool pdl);
+                           int32_t *status_out, int H, int I, int k, int width, int max_tiles, cudaStream_t s,
+                           bool pdl);
 cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int32_t *status_out, int H, int I, int max_tiles, cudaStream_t s,
-                        bool pdl);
+                        const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int32_t *status_out, int H,
+                        int I, int width, int max_tiles, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
                            bool pdl);
 cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __half *x_perm, int n, int H, int k,

@@ -36,7 +36,7 @@ permute_kernel(const int32_t *__restrict__ topk_ids, int32_t *__restrict__ offse
 __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__restrict__ offsets,
                                                               const int32_t *__restrict__ sorted_ids,
                                                               ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles,
-                                                              int *status, int E, int k)
+                                                              int *status, int E, int width)
 {
     __shared__ int s_off[kMaxE + 1];
     __shared__ int scan_buf[33];
@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__r
     }
     for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
-    emit_tiles(s_off, E, k, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
+    emit_tiles(s_off, E, width, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
 }
 
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
@@ -64,9 +64,9 @@ cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted
 }
 
 cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
-                               int *status, int E, int k, cudaStream_t s)
+                               int *status, int E, int width, cudaStream_t s)
 {
-    build_tiles_kernel<<<1, 1024, 0, s>>>(offsets, sorted_ids, tiles, n_tiles, status, E, k);
+    build_tiles_kernel<<<1, 1024, 0, s>>>(offsets, sorted_ids, tiles, n_tiles, status, E, width);
     return cudaGetLastError();
 }
 

@@ -103,7 +103,8 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
     // expert with at least kWideMinTokens assignments takes wide tiles instead, when enabled
     const int my_cnt = tid < E ? sm.cnt[tid] : 0;
     const bool my_wide = to.wide_tiles != nullptr && my_cnt >= kWideMinTokens;
-    const int mine = tid < E ? ((my_wide ? 0 : (my_cnt + kTileTokens - 1) / kTileTokens) << 16) | my_cnt : 0;
+    const int W = to.width;
+    const int mine = tid < E ? ((my_wide ? 0 : (my_cnt + W - 1) / W) << 16) | my_cnt : 0;
     int total = 0;
     const int base = block_exclusive_scan(mine, sm.scan, total);   // ends with a block barrier
     if (tid < E) {
@@ -163,17 +164,17 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
                     wp->pad = 0;
                 }
             } else if (tiles) {
-                const int slot = rank % kTileTokens, tile_first = rank - slot;
-                ExpertTile *tp = tiles + sm.tb[e] + rank / kTileTokens;
+                const int slot = rank % W, tile_first = rank - slot;
+                ExpertTile *tp = tiles + sm.tb[e] + rank / W;
                 tp->flat[slot] = f;
                 if (slot == 0) {
                     tp->expert = e;
                     tp->p0 = sm.off[e] + tile_first;
-                    tp->count = min(kTileTokens, cnt - tile_first);
+                    tp->count = min(W, cnt - tile_first);
                     tp->pad = 0;
                 }
-                if (rank == cnt - 1)   // the tile's last assignment repeats into the unused slots
-                    for (int j = slot + 1; j < kTileTokens; ++j) tp->flat[j] = f;
+                if (rank == cnt - 1 || slot == W - 1)   // the last assignment repeats into the unused slots
+                    for (int j = slot + 1; j < kTileTokensMax; ++j) tp->flat[j] = f;
             }
         }
     }
@@ -211,11 +212,10 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
     // lane l scans the contiguous experts [l * per, (l + 1) * per)
     const int per = (E + 31) / 32;
     const int ea = min(E, lane * per), eb = min(E, ea + per);
-    // per expert: (8-assignment tiles << 16) | count, and wide tiles (experts with kWideMinTokens or more
-    // when the wide path is on); lane l scans the contiguous experts [l * per, (l + 1) * per)
-    auto packed = [&](int c) {
-        return (((wide_on && c >= kWideMinTokens) ? 0 : (c + kTileTokens - 1) / kTileTokens) << 16) | c;
-    };
+    // per expert: (mma.sync tiles << 16) | count, and wide tiles (experts with kWideMinTokens or
+    // more when the wide path is on); lane l scans the contiguous experts [l * per, (l + 1) * per)
+    const int W = to.width;
+    auto packed = [&](int c) { return (((wide_on && c >= kWideMinTokens) ? 0 : (c + W - 1) / W) << 16) | c; };
     auto wide_n = [&](int c) { return (wide_on && c >= kWideMinTokens) ? (c + kWideTokens - 1) / kWideTokens : 0; };
     int local = 0, wlocal = 0;
     for (int e = ea; e < eb; ++e) {
@@ -266,42 +266,43 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
             }
             continue;
         }
-        const int slot = r % kTileTokens, tile_first = r - slot;
-        ExpertTile *tp = tiles + tb[e] + r / kTileTokens;
+        const int slot = r % W, tile_first = r - slot;
+        ExpertTile *tp = tiles + tb[e] + r / W;
         tp->flat[slot] = f;
         if (slot == 0) {
             tp->expert = e;
             tp->p0 = off[e] + tile_first;
-            tp->count = min(kTileTokens, c - tile_first);
+            tp->count = min(W, c - tile_first);
             tp->pad = 0;
         }
-        if (r == c - 1)   // the tile's last assignment repeats into the unused slots
-            for (int j = slot + 1; j < kTileTokens; ++j) tp->flat[j] = f;
+        if (r == c - 1 || slot == W - 1)   // the last assignment repeats into the unused slots
+            for (int j = slot + 1; j < kTileTokensMax; ++j) tp->flat[j] = f;
     }
 }
 
-// sorted_flat(p) returns the flat assignment id at position p of the expert-grouped order.
-// Each thread owns a contiguous run of ceil(E / blockDim) experts.
+// Tiles of W assignments from expert offsets; sorted_flat(p) returns the flat assignment id at
+// position p of the expert-grouped order.  Each thread owns a contiguous run of ceil(E / blockDim)
+// experts.
 template <typename SortedFlat>
-__device__ inline void emit_tiles(const int *off, int E, int k, ExpertTile *tiles, int *n_tiles, int *scan_buf,
+__device__ inline void emit_tiles(const int *off, int E, int W, ExpertTile *tiles, int *n_tiles, int *scan_buf,
                                   SortedFlat sorted_flat)
 {
     const int per = (E + blockDim.x - 1) / blockDim.x;
     const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
     int mine = 0;
-    for (int e = e0; e < e1; ++e) mine += (off[e + 1] - off[e] + kTileTokens - 1) / kTileTokens;
+    for (int e = e0; e < e1; ++e) mine += (off[e + 1] - off[e] + W - 1) / W;
     int total = 0;
     int base = block_exclusive_scan(mine, scan_buf, total);
     for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
-        for (int i = 0; i * kTileTokens < cnt; ++i) {
+        for (int i = 0; i * W < cnt; ++i) {
             ExpertTile tl;
             tl.expert = e;
-            tl.p0 = off[e] + i * kTileTokens;
-            tl.count = min(kTileTokens, cnt - i * kTileTokens);
+            tl.p0 = off[e] + i * W;
+            tl.count = min(W, cnt - i * W);
             tl.pad = 0;
 #pragma unroll
-            for (int j = 0; j < kTileTokens; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
+            for (int j = 0; j < kTileTokensMax; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
             tiles[base++] = tl;
         }
     }

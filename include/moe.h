@@ -170,6 +170,14 @@ int moe_route_noalloc(const void *x_bf16, const float *router_w, const float *ro
 size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
 
 /*
+ * Kernel launches one moe_mxfp4_forward / moe_mxfp4_forward_ex call enqueues for this shape
+ * (router logits, top-k + permutation as one or two kernels, the grouped GEMMs, the gather and
+ * tensor-core GEMMs when experts can reach 32 assignments, the combine); 0 for M == 0 and a
+ * negative MOE_* status for an unsupported shape.  For sizing CUDA graphs and for accounting.
+ */
+int moe_forward_launches(int M, int H, int I, int E, int k);
+
+/*
  * Whole layer with a caller-owned workspace (>= moe_workspace_bytes, 256-byte
  * aligned; its contents need no initialisation and are overwritten), an optional
  * router bias, optional copies of the routing (topk_ids_out [M,k] int32,

@@ -84,7 +84,7 @@ def test_permute_edge_cases(moe):
 
 # ----------------------------------------------------------------------------- gate_up + clamp-SwiGLU
 
-@pytest.mark.parametrize("ci,M", [(0, 2), (1, 8), (1, 37), (2, 1), (2, 16)])
+@pytest.mark.parametrize("ci,M", [(0, 2), (1, 8), (1, 37), (1, 96), (2, 1), (2, 16)])
 def test_gate_up_swiglu(moe, ci, M):
     big = ci >= 2
     inp = gen.make_inputs(ci, M, weights="torch" if big else "numpy", device="cuda")
@@ -110,7 +110,7 @@ def test_gate_up_swiglu(moe, ci, M):
 
 # ----------------------------------------------------------------------------- down + combine
 
-@pytest.mark.parametrize("ci,M", [(0, 2), (1, 8), (1, 37)])
+@pytest.mark.parametrize("ci,M", [(0, 2), (1, 8), (1, 37), (1, 96)])
 def test_down_combine(moe, ci, M):
     inp = gen.make_inputs(ci, M)
     k, E = inp.shape.k, inp.shape.E
@@ -128,7 +128,8 @@ def test_down_combine(moe, ci, M):
 
 # ----------------------------------------------------------------------------- whole layer
 
-SMALL_FORWARD = [(0, 2), (1, 1), (1, 2), (1, 4), (1, 8), (1, 37)]
+# (1, 96): M*k >= 6E, so 16-assignment tiles (two MMA n-tiles per decoded weight fragment)
+SMALL_FORWARD = [(0, 2), (1, 1), (1, 2), (1, 4), (1, 8), (1, 37), (1, 96)]
 
 
 @pytest.mark.parametrize("ci,M", SMALL_FORWARD)

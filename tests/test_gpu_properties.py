@@ -108,7 +108,8 @@ def test_token_permutation_permutes_rows(moe):
     (96, 64, 3, 2, 5),        # tiny: one partial box, K tails in both projections
     (1056, 800, 16, 4, 9),    # H, I not multiples of the 512-element stage
     (256, 32, 1, 1, 3),       # a single expert: dense clamp-SwiGLU MLP
-    (512, 256, 8, 8, 40),     # k == E: every token uses every expert, 5 tiles per expert
+    (512, 256, 8, 8, 40),     # k == E: every token uses every expert, 16-wide tiles of 16, 16, 8
+    (1056, 800, 16, 4, 40),   # 16-wide tiles (M*k >= 4E) with K tails and per-item scale rows
 ])
 def test_ragged_shapes_against_oracle(moe, H, I, E, k, M):
     shape = gen.LayerShape("ragged", H, I, E, k, (M,))
@@ -130,7 +131,7 @@ def test_ragged_shapes_against_oracle(moe, H, I, E, k, M):
     (512, 1024, 16, 4, 160),  # ~40 per expert, spread: wide and 8-assignment tiles in the same call
 ])
 def test_wide_tiles_against_oracle(moe, H, I, E, k, M):
-    # experts with more than 8 assignments take the tcgen05 path (H, I multiples of 512)
+    # experts with 32 or more assignments take the tcgen05 path (H, I multiples of 512)
     shape = gen.LayerShape("wide", H, I, E, k, (M,))
     inp = gen.make_inputs(0, M, shape=shape, seed=7 * H + I + E + k + M)
     d = U.device_inputs(inp)
