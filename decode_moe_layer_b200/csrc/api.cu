@@ -263,7 +263,8 @@ struct Marks {
         if (m) MOE_TRY((m)->mark(s));                   \
     } while (0)
 
-static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+                    const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
                     int32_t *status_out, int H, int I, int E, int width, int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
@@ -274,7 +275,8 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
         rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_down(map, smap, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, width, max_tiles, s, pdl));
+    MOE_TRY(launch_down(map, smap, w2_s, h, sorted_ids, tiles, n_tiles, y, status, status_out, H, I, width, max_tiles, s,
+                        pdl));
     return MOE_OK;
 }
 
@@ -349,7 +351,8 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     }
     MOE_MARK(marks, s);
     // down likewise, then the weighted top-k combine
-    rc = run_down(w2_q, w2_s, h, tiles, n_tiles, y, status, status_out, H, I, E, L.width, L.max_tiles, s, pdl);
+    rc = run_down(w2_q, w2_s, h, sorted_ids, tiles, n_tiles, y, status, status_out, H, I, E, L.width, L.max_tiles, s,
+                  pdl);
     if (rc != MOE_OK) return rc;
     if (L.wide) {
         rc = run_wide(false, w2_q, w2_s, h, wtiles, n_wide, L.max_wide, sorted_ids, h, y, status, status_out, M, H, I,
@@ -500,8 +503,8 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
     float *y = reinterpret_cast<float *>(ws + L.y);
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, L.width, stream));
-    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), tiles, n_tiles, y, status, nullptr, H, I, E, L.width,
-                  L.max_tiles, stream, false);
+    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, tiles, n_tiles, y, status, nullptr, H, I,
+                  E, L.width, L.max_tiles, stream, false);
     if (rc != MOE_OK) return rc;
     MOE_TRY(launch_combine(y, topk_w, out_bf16, M, H, k, stream, false));
     return MOE_OK;

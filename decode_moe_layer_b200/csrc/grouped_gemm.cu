@@ -37,9 +37,10 @@
 //    warp parks its partial sums in a double-buffered reduction area and moves on.
 //  * 2 epilogue warps sum the 8 K slots in slot order, then gate_up applies
 //    clamp-SwiGLU and stores h; down stores the unweighted fp32 row of each
-//    assignment -- off the compute path.  The item's positions and flat assignment
-//    ids reach them from the producer through shared memory.  The weighted top-k
-//    combine that follows is its own small kernel (combine_kernel).
+//    assignment (at its flat id, from the expert-grouped order) -- off the compute
+//    path.  The item's position range reaches them from the producer through shared
+//    memory.  The weighted top-k combine that follows is its own small kernel
+//    (combine_kernel).
 // Activations (x or h) are read as binary16; bf16 x converts exactly for
 // 2^-17 <= |x| <= 65504, h is stored scaled by 2^10 (exact for |h| >= 2^-27,
 // |h| <= 49 so no overflow), E2M1 values are exact in binary16, and products
@@ -82,7 +83,7 @@ struct SmemPlan {
 };
 
 constexpr int kNumBars = 2 * kStages + 8 + kComputeWarps / 2;   // ring, scale buffers, partials, K-slot pairs
-constexpr int kMetaInts = (3 + kTileTokensMax) * (kItemQ + 2);  // item ids, positions, counts, flat ids
+constexpr int kMetaInts = 3 * (kItemQ + 2);                      // item ids, positions, counts
 
 template <int kN>
 __host__ __device__ inline SmemPlan smem_plan(int K)
@@ -117,7 +118,7 @@ template <bool kGateUp, int kN>
 __global__ void __launch_bounds__(Tiling<kN>::kThreads, 1)
 grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                      const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
-                     const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
+                     const int32_t *__restrict__ sorted_ids, const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
                      __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out,
                      int *queue, int K, int I, int H, int k)
 {
@@ -137,17 +138,14 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     uint64_t *full = bars, *empty = bars + kStages;
     uint64_t *sfull = bars + 2 * kStages, *sempty = sfull + 2, *rfull = sfull + 4, *rempty = sfull + 6;
     uint64_t *pair = sfull + 8;   // [kComputeWarps / 2]: odd K slot's partials posted (pair reduction)
-    // per item in flight: id, first expert-grouped position, assignment count and the slots'
-    // flat assignment ids (producer -> compute warps -> epilogue warps), so that no consumer
-    // reads the tile list from global memory
+    // per item in flight: id, first expert-grouped position and assignment count (producer ->
+    // compute warps -> epilogue warps), so that no consumer reads the tile list itself
     volatile int *item_q = reinterpret_cast<volatile int *>(bars + kNumBars);         // [kItemQ]
     volatile int *item_p0 = item_q + kItemQ;                                          // [kItemQ]
     volatile int *item_cnt = item_p0 + kItemQ;                                        // [kItemQ]
-    volatile int *item_flat = item_cnt + kItemQ;                                      // [kItemQ][kTileTokensMax]
-    volatile int *red_item = item_flat + kItemQ * kTileTokensMax;                     // [kRedBufs]
+    volatile int *red_item = item_cnt + kItemQ;                                       // [kRedBufs]
     volatile int *red_p0 = red_item + 2;                                              // [kRedBufs]
     volatile int *red_cnt = red_p0 + 2;                                               // [kRedBufs]
-    volatile int *red_flat = red_cnt + 2;                                             // [kRedBufs][kTileTokensMax]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
@@ -261,7 +259,6 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 item_p0[item_ctr % kItemQ] = p0;
                 item_cnt[item_ctr % kItemQ] = cnt;
             }
-            if (!kGateUp && lane < kN) item_flat[(item_ctr % kItemQ) * kTileTokensMax + lane] = flat;
             const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
@@ -419,12 +416,12 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                         const float unscale = 0.5f / kHScale;
                         const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
                         if (li0 < cnt) {
-                            float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokensMax + li0]) * H;
+                            float *yr = yout + static_cast<size_t>(sorted_ids[p0 + li0]) * H;
                             if (ra < rows_total) yr[ra] = unscale * sum.x;
                             if (rbw < rows_total) yr[rbw] = unscale * sum.z;
                         }
                         if (li1 < cnt) {
-                            float *yr = yout + static_cast<size_t>(red_flat[b * kTileTokensMax + li1]) * H;
+                            float *yr = yout + static_cast<size_t>(sorted_ids[p0 + li1]) * H;
                             if (ra < rows_total) yr[ra] = unscale * sum.y;
                             if (rbw < rows_total) yr[rbw] = unscale * sum.w;
                         }
@@ -585,8 +582,6 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             red_p0[rb] = item_p0[item_ctr % kItemQ];
             red_cnt[rb] = item_cnt[item_ctr % kItemQ];
         }
-        if (!kGateUp && warp == 0 && lane < kN)
-            red_flat[rb * kTileTokensMax + lane] = item_flat[(item_ctr % kItemQ) * kTileTokensMax + lane];
         __syncwarp();
         if (lane == 0) mbar_arrive(&rfull[rb]);
     }
@@ -629,9 +624,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 
 template <bool kGateUp, int kN>
 static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
-                                  const __half *act, const ExpertTile *tiles, const int *n_tiles, __half *h, float *y,
-                                  int *status, int32_t *status_out, int K, int I, int H, int k, int max_tiles,
-                                  cudaStream_t s, bool pdl)
+                                  const __half *act, const int32_t *sorted_ids, const ExpertTile *tiles,
+                                  const int *n_tiles, __half *h, float *y, int *status, int32_t *status_out, int K,
+                                  int I, int H, int k, int max_tiles, cudaStream_t s, bool pdl)
 {
     const SmemPlan plan = smem_plan<kN>(K);
     auto kern = grouped_mxfp4_kernel<kGateUp, kN>;
@@ -642,8 +637,8 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &sma
     int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
     if (grid < 1) grid = 1;
     int *queue = status + (kGateUp ? kQueueGateUp : kQueueDown);
-    return launch_ex(kern, dim3(grid), dim3(Tiling<kN>::kThreads), plan.total, s, pdl, map, smap, scales, act, tiles,
-                     n_tiles, h, y, status, status_out, queue, K, I, H, k);
+    return launch_ex(kern, dim3(grid), dim3(Tiling<kN>::kThreads), plan.total, s, pdl, map, smap, scales, act,
+                     sorted_ids, tiles, n_tiles, h, y, status, status_out, queue, K, I, H, k);
 }
 
 int grouped_smem_bytes(int K, int width) { return width == 16 ? smem_plan<16>(K).total : smem_plan<8>(K).total; }
@@ -654,21 +649,21 @@ cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_ma
                            bool pdl)
 {
     if (width == 16)
-        return launch_grouped<true, 16>(w13_map, s13_map, w13_s, x16, tiles, n_tiles, h, nullptr, status, status_out, H,
-                                        I, H, k, max_tiles, s, pdl);
-    return launch_grouped<true, 8>(w13_map, s13_map, w13_s, x16, tiles, n_tiles, h, nullptr, status, status_out, H, I,
-                                   H, k, max_tiles, s, pdl);
+        return launch_grouped<true, 16>(w13_map, s13_map, w13_s, x16, nullptr, tiles, n_tiles, h, nullptr, status,
+                                        status_out, H, I, H, k, max_tiles, s, pdl);
+    return launch_grouped<true, 8>(w13_map, s13_map, w13_s, x16, nullptr, tiles, n_tiles, h, nullptr, status,
+                                   status_out, H, I, H, k, max_tiles, s, pdl);
 }
 
 cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int32_t *status_out, int H,
-                        int I, int width, int max_tiles, cudaStream_t s, bool pdl)
+                        const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+                        int32_t *status_out, int H, int I, int width, int max_tiles, cudaStream_t s, bool pdl)
 {
     if (width == 16)
-        return launch_grouped<false, 16>(w2_map, s2_map, w2_s, h, tiles, n_tiles, nullptr, y, status, status_out, I, I,
-                                         H, 1, max_tiles, s, pdl);
-    return launch_grouped<false, 8>(w2_map, s2_map, w2_s, h, tiles, n_tiles, nullptr, y, status, status_out, I, I, H, 1,
-                                    max_tiles, s, pdl);
+        return launch_grouped<false, 16>(w2_map, s2_map, w2_s, h, sorted_ids, tiles, n_tiles, nullptr, y, status,
+                                         status_out, I, I, H, 1, max_tiles, s, pdl);
+    return launch_grouped<false, 8>(w2_map, s2_map, w2_s, h, sorted_ids, tiles, n_tiles, nullptr, y, status,
+                                    status_out, I, I, H, 1, max_tiles, s, pdl);
 }
 
 cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,

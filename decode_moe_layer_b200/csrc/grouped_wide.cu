@@ -1,5 +1,5 @@
 // grouped_wide.cu -- grouped MXFP4 expert GEMMs on the 5th-generation tensor cores, for the
-// experts that receive more than kTileTokens routed assignments ("wide" tiles of up to
+// experts that receive kWideMinTokens or more routed assignments ("wide" tiles of up to
 // kWideTokens assignments of one expert).
 //
 // "Compact routed MXFP4 GEMM" and "Routed clamp-SwiGLU" rows of "Post-Portfolio Device
@@ -7,16 +7,18 @@
 // the page's "Decision" section.  At large token counts the expert GEMMs become real dense
 // contractions: an expert with many assignments is streamed once for all of them (the narrow
 // kernel in grouped_gemm.cu re-streams it for every 8 assignments), and the MMA runs on
-// tcgen05 with the fp32 accumulator in tensor memory.
+// tcgen05 with the fp32 accumulator in tensor memory.  The kernel keeps a kWideTokens-wide tile of
+// one expert's assignments against 128 weight rows per item, and the wider the tile the more
+// work each MMA instruction does (their issue cost hardly depends on N).
 //
 // One persistent CTA per SM, 16 warps:
 //  * warp 0 (weights producer): per 512-K stage, TMA copies of the item's packed E2M1 rows
-//    (128 rows x 256 bytes, 128-byte swizzle) and their E8M0 scales into a 4-stage ring;
+//    (128 rows x 256 bytes, 128-byte swizzle) and their E8M0 scales into a 3-stage ring;
 //    items come from the call's work queue, the ids reach the other warps through shared
 //    memory with the stage arrivals.
 //  * warp 2 (activations producer): per 64-K sub-tile, TMA copies of the item's activation
 //    rows (x gathered into expert-grouped order for gate_up, h for down), 16 rows per box,
-//    128-byte swizzle, into a 5-slot ring.  Rows past the tile are read and ignored.
+//    128-byte swizzle, into a 4-slot ring.  Rows past the tile are read and ignored.
 //  * warps 4..11 (dequant): per 64-K sub-tile, 256 threads each decode 32 weights of one row
 //    (hardware E2M1 -> f16x2), apply the row's E8M0 block scale in f16 (exact for scale bytes
 //    104..140: every scaled E2M1 value is then an f16 normal or subnormal; other bytes are
@@ -46,10 +48,12 @@ namespace moe {
 namespace wide {
 constexpr int kRows = 128;                               // weight rows per item (MMA M)
 constexpr int kStageK = kWideStageK;                     // 512 K per packed stage
-constexpr int kPStages = 4;                              // packed weight stages
+constexpr int kPStages = 3;                              // packed weight stages
 constexpr int kSubK = 64;                                // K per A/B sub-tile (one swizzle atom of f16)
 constexpr int kSubs = kStageK / kSubK;                   // 8
-constexpr int kABufs = 4, kBBufs = 5, kDBufs = 2;
+// A tcgen05.mma costs about the same issue time for any N, so N is as large as TMEM allows:
+// two accumulators of kWideTokens columns plus the A buffers.
+constexpr int kABufs = 2, kBBufs = 4, kDBufs = 2;
 constexpr int kItemQ = 8;
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
@@ -57,7 +61,7 @@ constexpr int kWProd = 0, kMma = 1, kBProd = 2, kDeq0 = 4, kDeqWarps = 8, kEpi0 
 constexpr int kPackedStage = kRows * kStageK / 2;        // 32 KB: 2 box columns x 128 rows x 128 B
 constexpr int kPackedCol = kRows * 128;                  // one box column (two 64-row boxes)
 constexpr int kScaleStage = kRows * kStageK / 32;        // 2 KB: 128 rows x 16 B
-constexpr int kBTile = kWideTokens * kSubK * 2;          // 16 KB
+constexpr int kBTile = kWideTokens * kSubK * 2;          // 28 KB
 constexpr int kBBox = 16 * kSubK * 2;                    // one 16-row activation box
 constexpr int kACols = kSubK / 2;                        // TMEM columns of one A buffer (2 f16 per column)
 constexpr int kACol0 = kDBufs * kWideTokens;             // accumulators first, then the A buffers
@@ -67,7 +71,7 @@ constexpr int kOffScale = kOffPacked + kPStages * kPackedStage;
 constexpr int kOffB = kOffScale + kPStages * kScaleStage;
 constexpr int kOffBars = kOffB + kBBufs * kBTile;
 constexpr int kSmemBytes = kOffBars + 512 + 1024;        // barriers and slots, + alignment slack
-static_assert(kOffB % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
+static_assert(kOffB % 1024 == 0 && kBTile % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
 static_assert(kACol0 + kABufs * kACols <= kTmemCols && kTmemCols <= 512, "TMEM budget");
 static_assert(kSmemBytes <= 227 * 1024, "fits one SM");
 }  // namespace wide

@@ -87,7 +87,8 @@ struct ExpertTile {   // one expert's run of <= tile_width consecutive assignmen
     int p0;           // first position in the expert-grouped order
     int count;
     int pad;
-    int flat[kTileTokensMax];   // flat assignment id t*k + j of each slot (sorted_ids[p0+i]); entries >= count repeat the last
+    int flat[kTileTokensMax];   // flat assignment id t*k + j of each slot (sorted_ids[p0+i]); slots count..width-1
+                                // repeat the last, slots past the width are not written
 };
 
 // Tile width of a call: 16 assignments (two n-tiles per decoded weight fragment) once the
@@ -104,7 +105,7 @@ __host__ __device__ inline int tile_width(int M, int E, int k)
 // as wide tiles of up to kWideTokens consecutive assignments; it needs H and I to be multiples
 // of its 512-element packed stage.  No expert can exceed M assignments, so M < kWideMinTokens
 // never uses it.
-constexpr int kWideTokens = 128;
+constexpr int kWideTokens = 224;   // MMA N: two accumulators of 224 columns + A buffers fill TMEM
 constexpr int kWideStageK = 512;
 constexpr int kWideMinTokens = 32;   // fewer assignments stream faster as mma.sync tiles
 struct WideTile {
@@ -201,8 +202,8 @@ cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_ma
                            int32_t *status_out, int H, int I, int k, int width, int max_tiles, cudaStream_t s,
                            bool pdl);
 cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const ExpertTile *tiles, const int *n_tiles, float *y, int *status, int32_t *status_out, int H,
-                        int I, int width, int max_tiles, cudaStream_t s, bool pdl);
+                        const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
+                        int32_t *status_out, int H, int I, int width, int max_tiles, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
                            bool pdl);
 cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __half *x_perm, int n, int H, int k,

@@ -103,8 +103,8 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
     // expert with at least kWideMinTokens assignments takes wide tiles instead, when enabled
     const int my_cnt = tid < E ? sm.cnt[tid] : 0;
     const bool my_wide = to.wide_tiles != nullptr && my_cnt >= kWideMinTokens;
-    const int W = to.width;
-    const int mine = tid < E ? ((my_wide ? 0 : (my_cnt + W - 1) / W) << 16) | my_cnt : 0;
+    const int W = to.width, wsh = W == 16 ? 4 : 3;   // 8 or 16 assignments per tile
+    const int mine = tid < E ? ((my_wide ? 0 : (my_cnt + W - 1) >> wsh) << 16) | my_cnt : 0;
     int total = 0;
     const int base = block_exclusive_scan(mine, sm.scan, total);   // ends with a block barrier
     if (tid < E) {
@@ -164,8 +164,8 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
                     wp->pad = 0;
                 }
             } else if (tiles) {
-                const int slot = rank % W, tile_first = rank - slot;
-                ExpertTile *tp = tiles + sm.tb[e] + rank / W;
+                const int slot = rank & (W - 1), tile_first = rank - slot;
+                ExpertTile *tp = tiles + sm.tb[e] + (rank >> wsh);
                 tp->flat[slot] = f;
                 if (slot == 0) {
                     tp->expert = e;
@@ -173,8 +173,8 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
                     tp->count = min(W, cnt - tile_first);
                     tp->pad = 0;
                 }
-                if (rank == cnt - 1 || slot == W - 1)   // the last assignment repeats into the unused slots
-                    for (int j = slot + 1; j < kTileTokensMax; ++j) tp->flat[j] = f;
+                if (rank == cnt - 1)   // the last assignment repeats into the unused slots
+                    for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
             }
         }
     }
@@ -214,8 +214,8 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
     const int ea = min(E, lane * per), eb = min(E, ea + per);
     // per expert: (mma.sync tiles << 16) | count, and wide tiles (experts with kWideMinTokens or
     // more when the wide path is on); lane l scans the contiguous experts [l * per, (l + 1) * per)
-    const int W = to.width;
-    auto packed = [&](int c) { return (((wide_on && c >= kWideMinTokens) ? 0 : (c + W - 1) / W) << 16) | c; };
+    const int W = to.width, wsh = W == 16 ? 4 : 3;   // 8 or 16 assignments per tile
+    auto packed = [&](int c) { return (((wide_on && c >= kWideMinTokens) ? 0 : (c + W - 1) >> wsh) << 16) | c; };
     auto wide_n = [&](int c) { return (wide_on && c >= kWideMinTokens) ? (c + kWideTokens - 1) / kWideTokens : 0; };
     int local = 0, wlocal = 0;
     for (int e = ea; e < eb; ++e) {
@@ -266,8 +266,8 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
             }
             continue;
         }
-        const int slot = r % W, tile_first = r - slot;
-        ExpertTile *tp = tiles + tb[e] + r / W;
+        const int slot = r & (W - 1), tile_first = r - slot;
+        ExpertTile *tp = tiles + tb[e] + (r >> wsh);
         tp->flat[slot] = f;
         if (slot == 0) {
             tp->expert = e;
@@ -275,8 +275,8 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
             tp->count = min(W, c - tile_first);
             tp->pad = 0;
         }
-        if (r == c - 1 || slot == W - 1)   // the last assignment repeats into the unused slots
-            for (int j = slot + 1; j < kTileTokensMax; ++j) tp->flat[j] = f;
+        if (r == c - 1)   // the last assignment repeats into the unused slots
+            for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
     }
 }
 
@@ -296,13 +296,12 @@ __device__ inline void emit_tiles(const int *off, int E, int W, ExpertTile *tile
     for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
         for (int i = 0; i * W < cnt; ++i) {
-            ExpertTile tl;
+            ExpertTile tl{};
             tl.expert = e;
             tl.p0 = off[e] + i * W;
             tl.count = min(W, cnt - i * W);
             tl.pad = 0;
-#pragma unroll
-            for (int j = 0; j < kTileTokensMax; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
+            for (int j = 0; j < W; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
             tiles[base++] = tl;
         }
     }

@@ -127,7 +127,7 @@ def test_ragged_shapes_against_oracle(moe, H, I, E, k, M):
 
 @pytest.mark.parametrize("H,I,E,k,M", [
     (1024, 512, 4, 2, 80),    # ~40 assignments per expert: three of four experts on the tensor-core path
-    (512, 512, 4, 2, 300),    # ~150 per expert: two wide tiles per expert, the second partial
+    (512, 512, 4, 2, 600),    # ~300 per expert: two wide tiles per expert (224 + the rest)
     (512, 1024, 16, 4, 160),  # ~40 per expert, spread: wide and 8-assignment tiles in the same call
 ])
 def test_wide_tiles_against_oracle(moe, H, I, E, k, M):
