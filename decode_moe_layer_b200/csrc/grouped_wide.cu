@@ -69,7 +69,8 @@ constexpr int kTmemCols = 512;                           // power of two >= kACo
 constexpr int kOffPacked = 0;
 constexpr int kOffScale = kOffPacked + kPStages * kPackedStage;
 constexpr int kOffB = kOffScale + kPStages * kScaleStage;
-constexpr int kOffBars = kOffB + kBBufs * kBTile;
+constexpr int kOffIds = kOffB + kBBufs * kBTile;         // down: each epilogue warp's copy of the tile's flat ids
+constexpr int kOffBars = kOffIds + kEpiWarps * kWideTokens * 4;
 constexpr int kSmemBytes = kOffBars + 512 + 1024;        // barriers and slots, + alignment slack
 static_assert(kOffB % 1024 == 0 && kBTile % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
 static_assert(kACol0 + kABufs * kACols <= kTmemCols && kTmemCols <= 512, "TMEM budget");
@@ -390,6 +391,12 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int rb = item % row_blocks;
             const int p0 = __ldcg(&tp->p0), cnt = __ldcg(&tp->count);
             const uint32_t taddr = tmem + static_cast<uint32_t>(db * kWideTokens) + (static_cast<uint32_t>(32 * quarter) << 16);
+            // down: the tile's flat ids, loaded once per item (independent loads) into this warp's copy
+            int *ids = reinterpret_cast<int *>(smem + kOffIds) + (warp - kEpi0) * kWideTokens;
+            if (!kGateUp) {
+                for (int i = lane; i < cnt; i += 32) ids[i] = __ldcg(&a.sorted_ids[p0 + i]);
+                __syncwarp();
+            }
             for (int c = 0; c < cnt; c += 16) {
                 uint32_t v[16];
                 tmem_ld16(taddr + c, v);
@@ -411,10 +418,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     const int r = rb * kRows + row;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c + j < cnt) {
-                            const int f = __ldcg(&a.sorted_ids[p0 + c + j]);
-                            a.y[static_cast<size_t>(f) * H + r] = __uint_as_float(v[j]) * (1.0f / kHScale);
-                        }
+                        if (c + j < cnt) a.y[static_cast<size_t>(ids[c + j]) * H + r] = __uint_as_float(v[j]) * (1.0f / kHScale);
                 }
             }
             tc_fence_before();
