@@ -180,47 +180,30 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
     }
 }
 
-// The same stable order, offsets, sorted ids, inverse positions and tiles, computed by ONE
-// warp (the calling warp) for n assignments whose experts are s_e[0..n) (shared memory; the
-// experts of a fused top-k, all in [0, E)).  Shared scratch: cnt, off, tb [E] and rank [n].
-// Rounds of 32 assignments: each round's matching lanes get their rank from the running
-// per-expert count, whose leader then advances it; one warp scan of (tiles << 16 | count)
-// over the experts gives offsets and tile bases.  Only __syncwarp, no block barrier.
-__device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k, int *cnt, int *off, int *tb,
-                                             int *wb, int *rank, int32_t *__restrict__ offsets,
-                                             int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos,
-                                             TileOut to)
+// Route remap of the fused router select (M <= 64 tokens), in two helpers.  Every token picks
+// each expert at most once, so the stable rank of assignment f = t*k + j on its expert e is the
+// number of earlier tokens that chose e: with mask[e] = the set of tokens that chose e (one bit
+// per token), rank = popc(mask[e] & (2^t - 1)) and count = popc(mask[e]).
+
+// One warp (the calling warp): per expert, (mma.sync tiles << 16) | count and the wide tiles
+// (experts with kWideMinTokens or more when the wide path is on), one warp scan over the experts
+// (lane l takes the contiguous experts [l * per, (l + 1) * per)); writes off, tb, wb (shared) and
+// expert_offsets, the tile counts (global).
+__device__ inline void warp_scan_experts(const unsigned long long *mask, int E, TileOut to, int *off, int *tb, int *wb,
+                                         int32_t *__restrict__ offsets)
 {
-    ExpertTile *__restrict__ tiles = to.tiles;
     const bool wide_on = to.wide_tiles != nullptr;
     const int lane = threadIdx.x & 31;
-    for (int e = lane; e < E; e += 32) cnt[e] = 0;
-    __syncwarp();
-    for (int r0 = 0; r0 < n; r0 += 32) {
-        const int f = r0 + lane;
-        const int e = f < n ? s_e[f] : -1;
-        const unsigned same = __match_any_sync(0xffffffffu, e);
-        const int rank_w = __popc(same & ((1u << lane) - 1u));
-        const int before = e >= 0 ? cnt[e] : 0;
-        __syncwarp();
-        if (e >= 0) {
-            rank[f] = before + rank_w;
-            if (rank_w == 0) cnt[e] = before + __popc(same);
-        }
-        __syncwarp();
-    }
-    // lane l scans the contiguous experts [l * per, (l + 1) * per)
-    const int per = (E + 31) / 32;
-    const int ea = min(E, lane * per), eb = min(E, ea + per);
-    // per expert: (mma.sync tiles << 16) | count, and wide tiles (experts with kWideMinTokens or
-    // more when the wide path is on); lane l scans the contiguous experts [l * per, (l + 1) * per)
     const int W = to.width, wsh = W == 16 ? 4 : 3;   // 8 or 16 assignments per tile
     auto packed = [&](int c) { return (((wide_on && c >= kWideMinTokens) ? 0 : (c + W - 1) >> wsh) << 16) | c; };
     auto wide_n = [&](int c) { return (wide_on && c >= kWideMinTokens) ? (c + kWideTokens - 1) / kWideTokens : 0; };
+    const int per = (E + 31) / 32;
+    const int ea = min(E, lane * per), eb = min(E, ea + per);
     int local = 0, wlocal = 0;
     for (int e = ea; e < eb; ++e) {
-        local += packed(cnt[e]);
-        wlocal += wide_n(cnt[e]);
+        const int c = __popcll(mask[e]);
+        local += packed(c);
+        wlocal += wide_n(c);
     }
     int incl = local, wincl = wlocal;
 #pragma unroll
@@ -236,48 +219,51 @@ __device__ inline void warp_rank_and_scatter(const int *s_e, int n, int E, int k
     const int wtotal = __shfl_sync(0xffffffffu, wincl, 31);
     int run = incl - local, wrun = wincl - wlocal;
     for (int e = ea; e < eb; ++e) {
+        const int c = __popcll(mask[e]);
         off[e] = run & 0xFFFF;
         tb[e] = run >> 16;
         wb[e] = wrun;
         offsets[e] = run & 0xFFFF;
-        run += packed(cnt[e]);
-        wrun += wide_n(cnt[e]);
+        run += packed(c);
+        wrun += wide_n(c);
     }
     if (lane == 0) {
         offsets[E] = total & 0xFFFF;
         *to.n_tiles = total >> 16;
         if (wide_on) *to.n_wide = wtotal;
     }
-    __syncwarp();
-    for (int f = lane; f < n; f += 32) {
-        const int e = s_e[f];
-        const int r = rank[f];
-        const int pos = off[e] + r;
-        sorted_ids[pos] = f;
-        inv_pos[f] = pos;
-        const int c = cnt[e];
-        if (wide_on && c >= kWideMinTokens) {
-            if (r % kWideTokens == 0) {
-                WideTile *wp = to.wide_tiles + wb[e] + r / kWideTokens;
-                wp->expert = e;
-                wp->p0 = pos;
-                wp->count = min(kWideTokens, c - r);
-                wp->pad = 0;
-            }
-            continue;
+}
+
+// Assignment f (token t, expert e, rank r among the expert's c assignments): its position, the
+// inverse map and its slot of an mma.sync tile or a wide tile (off, tb, wb from warp_scan_experts).
+__device__ inline void scatter_assignment(int f, int e, int r, int c, const int *off, const int *tb, const int *wb,
+                                          int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos, TileOut to)
+{
+    const int pos = off[e] + r;
+    sorted_ids[pos] = f;
+    inv_pos[f] = pos;
+    if (to.wide_tiles != nullptr && c >= kWideMinTokens) {
+        if (r % kWideTokens == 0) {
+            WideTile *wp = to.wide_tiles + wb[e] + r / kWideTokens;
+            wp->expert = e;
+            wp->p0 = pos;
+            wp->count = min(kWideTokens, c - r);
+            wp->pad = 0;
         }
-        const int slot = r & (W - 1), tile_first = r - slot;
-        ExpertTile *tp = tiles + tb[e] + (r >> wsh);
-        tp->flat[slot] = f;
-        if (slot == 0) {
-            tp->expert = e;
-            tp->p0 = off[e] + tile_first;
-            tp->count = min(W, c - tile_first);
-            tp->pad = 0;
-        }
-        if (r == c - 1)   // the last assignment repeats into the unused slots
-            for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
+        return;
     }
+    const int W = to.width, wsh = W == 16 ? 4 : 3;
+    const int slot = r & (W - 1), tile_first = r - slot;
+    ExpertTile *tp = to.tiles + tb[e] + (r >> wsh);
+    tp->flat[slot] = f;
+    if (slot == 0) {
+        tp->expert = e;
+        tp->p0 = off[e] + tile_first;
+        tp->count = min(W, c - tile_first);
+        tp->pad = 0;
+    }
+    if (r == c - 1)   // the last assignment repeats into the unused slots
+        for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
 }
 
 // Tiles of W assignments from expert offsets; sorted_flat(p) returns the flat assignment id at

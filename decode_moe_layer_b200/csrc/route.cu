@@ -290,9 +290,10 @@ __device__ __forceinline__ void stage_logits(const float *__restrict__ partial, 
 }
 
 // Top-k of every token and the route remap, in one CTA of kPermuteThreads threads, when
-// fused_select(M, E, k): all threads sum the partial-logit slices into shared memory, warps
-// take the tokens' top-k, then warp 0 alone ranks and scatters the M*k assignments
-// (warp_rank_and_scatter) while the other warps exit.
+// fused_select(M, E, k) (M <= 64): all threads sum the partial-logit slices into shared memory,
+// warps take the tokens' top-k and mark each chosen expert's token mask, warp 0 scans the
+// experts' counts into offsets and tile bases, then every thread places assignments (stable rank
+// = earlier tokens in the expert's mask).
 template <int kPerLane>
 __global__ void __launch_bounds__(kPermuteThreads, 1)
 route_select_permute_kernel(const float *__restrict__ partial, int splits, const float *__restrict__ bias,
@@ -301,13 +302,14 @@ route_select_permute_kernel(const float *__restrict__ partial, int splits, const
                             int E, int k)
 {
     extern __shared__ __align__(16) uint8_t smem[];
-    __shared__ int s_e[kPermuteThreads];      // expert of assignment f
-    __shared__ int s_rank[kPermuteThreads];   // its rank inside the expert
-    float *s_log = reinterpret_cast<float *>(smem);                      // [M][E]
-    int *s_cnt = reinterpret_cast<int *>(smem) + M * E;                   // [E] x 4
+    __shared__ int s_e[kPermuteThreads];                    // expert of assignment f
+    __shared__ unsigned long long s_mask[kMaxE];            // bit t: token t chose the expert
+    __shared__ int s_off[kMaxE], s_tb[kMaxE], s_wb[kMaxE];  // first position, first tile, first wide tile
+    float *s_log = reinterpret_cast<float *>(smem);         // [M][E]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_wait();
     pdl_trigger();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_mask[e] = 0ull;
     const int n_log = M * E;
     if (n_log <= kPermuteThreads)
         stage_logits<1, 32>(partial, splits, bias, n_log, E, s_log);
@@ -329,12 +331,19 @@ route_select_permute_kernel(const float *__restrict__ partial, int splits, const
             ids[f] = sel_e;
             wout[f] = sel_w;
             s_e[f] = sel_e;
+            atomicOr(&s_mask[sel_e], 1ull << t);
         }
     }
     __syncthreads();
-    if (warp != 0) return;
-    warp_rank_and_scatter(s_e, M * k, E, k, s_cnt, s_cnt + E, s_cnt + 2 * E, s_cnt + 3 * E, s_rank, offsets,
-                          sorted_ids, inv_pos, to);
+    if (warp == 0) warp_scan_experts(s_mask, E, to, s_off, s_tb, s_wb, offsets);
+    __syncthreads();
+    const int n = M * k;
+    for (int f = threadIdx.x; f < n; f += blockDim.x) {
+        const int e = s_e[f], t = f / k;
+        const unsigned long long mk = s_mask[e];
+        scatter_assignment(f, e, __popcll(mk & ((1ull << t) - 1ull)), __popcll(mk), s_off, s_tb, s_wb, sorted_ids,
+                           inv_pos, to);
+    }
 }
 
 __global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
@@ -397,7 +406,7 @@ static cudaError_t select_permute_p(const float *partial, int splits, const floa
                                     int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M, int E,
                                     int k, cudaStream_t s, bool pdl)
 {
-    const int smem = (M * E + 4 * E) * static_cast<int>(sizeof(float));
+    const int smem = M * E * static_cast<int>(sizeof(float));
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>), smem);
     if (e != cudaSuccess) return e;
     return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kPermuteThreads), smem, s, pdl, partial, splits,
