@@ -53,7 +53,7 @@ constexpr int kRouteWarps = 8;
 constexpr int kPlanSMs = 148;
 struct RoutePlan {
     int tiles;    // MMA n-tiles (8 tokens) per token block: 1 or 4
-    int steps;    // 16-K MMA steps per pass: 2 or 8
+    int steps;    // 16-K MMA steps per pass: 2 or 4
     int splits;   // CTAs per (expert group, token block), each a partial-logit slice
     int passes;   // K ranges per warp
     int blocks_t; // token blocks
@@ -62,12 +62,12 @@ __host__ __device__ inline RoutePlan route_plan(int M, int H, int E)
 {
     RoutePlan p;
     p.tiles = M <= 8 ? 1 : 4;
-    p.steps = M <= 8 ? 2 : 8;
+    p.steps = M <= 8 ? 2 : 4;   // 4: two CTAs' registers fit one SM
     p.blocks_t = (M + 8 * p.tiles - 1) / (8 * p.tiles);
     const int gx = (E + kRouteExperts - 1) / kRouteExperts;
     const int units = (H + kRouteWarps * 16 * p.steps - 1) / (kRouteWarps * 16 * p.steps);
     const long long base = static_cast<long long>(gx) * p.blocks_t;
-    const int cap = (p.tiles == 1 ? 4 : 1) * kPlanSMs;   // light CTAs share SMs, heavy ones do not
+    const int cap = (p.tiles == 1 ? 4 : 2) * kPlanSMs;   // resident CTAs per SM: 4 light ones, 2 heavy ones
     if (base * units <= cap) {
         p.splits = units;
     } else {

@@ -377,8 +377,8 @@ cudaError_t launch_route_logits(const void *x, const float *router_w, float *par
     const RoutePlan plan = route_plan(M, H, E);
     if (plan.tiles == 1 && plan.steps == 2)
         return logits_launch<2, 1>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
-    if (plan.tiles == 4 && plan.steps == 8)
-        return logits_launch<8, 4>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
+    if (plan.tiles == 4 && plan.steps == 4)
+        return logits_launch<4, 4>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
     return cudaErrorInvalidConfiguration;   // route_plan yields only the two shapes above
 }
 
