@@ -80,6 +80,19 @@ def test_permute_edge_cases(moe):
         assert np.array_equal(off.cpu().numpy(), roff), (M, k)
         assert np.array_equal(srt.cpu().numpy(), rsrt), (M, k)
         assert np.array_equal(inv.cpu().numpy(), rinv), (M, k)
+    # tokens that repeat an expert (the token-mask ranking must hand over to the exact one), and
+    # masks too large for shared memory (E * ceil(M/32) words above 64 KB)
+    for M, k, E2, repeat in [(300, 4, 16, True), (700, 2, 1024, False)]:
+        if repeat:
+            ids = rng.integers(0, E2, size=(M, k)).astype(np.int32)
+            assert any(len(set(r)) < k for r in ids.tolist())
+        else:
+            ids = np.stack([rng.choice(E2, k, replace=False) for _ in range(M)]).astype(np.int32)
+        off, srt, inv = moe.moe_permute(torch.from_numpy(ids).cuda(), E2)
+        roff, rsrt, rinv = oracle.permute(ids, E2)
+        assert np.array_equal(off.cpu().numpy(), roff), (M, k, E2)
+        assert np.array_equal(srt.cpu().numpy(), rsrt), (M, k, E2)
+        assert np.array_equal(inv.cpu().numpy(), rinv), (M, k, E2)
 
 
 # ----------------------------------------------------------------------------- gate_up + clamp-SwiGLU
