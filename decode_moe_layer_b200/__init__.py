@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     moe_permute,
     moe_route,
     moe_route_noalloc,
+    moe_selftest_wait_timeout,
     moe_status_string,
     moe_workspace_bytes,
 )

@@ -22,7 +22,7 @@ MOE_ERR_TIMEOUT = -5
 EXPORTS = (
     "moe_status_string", "moe_last_cuda_error", "moe_route", "moe_permute", "moe_gate_up_swiglu",
     "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_forward_launches", "moe_mxfp4_forward_ex",
-    "moe_mxfp4_forward_profile", "moe_route_noalloc",
+    "moe_mxfp4_forward_profile", "moe_route_noalloc", "moe_selftest_wait_timeout",
 )
 H_STORAGE_SCALE = 1024.0   # moe_gate_up_swiglu stores binary16(h * 2^10)
 PROFILE_KERNELS = ("route_logits", "route_select", "permute", "gate_up_swiglu", "down_combine")
@@ -73,6 +73,8 @@ def load():
     lib.moe_mxfp4_forward_ex.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, S, P]
     lib.moe_mxfp4_forward_profile.restype = I
     lib.moe_mxfp4_forward_profile.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, S, P, P]
+    lib.moe_selftest_wait_timeout.restype = I
+    lib.moe_selftest_wait_timeout.argtypes = [P, P]
     _lib = lib
     return lib
 
@@ -109,6 +111,12 @@ def moe_workspace_bytes(M: int, H: int, I: int, E: int, k: int) -> int:
 def moe_forward_launches(M: int, H: int, I: int, E: int, k: int) -> int:
     """Kernel launches of one layer call for this shape (negative MOE_* status if unsupported)."""
     return int(load().moe_forward_launches(M, H, I, E, k))
+
+
+def moe_selftest_wait_timeout(status_out, stream=None):
+    """Launch the bounded-wait self-test: writes MOE_ERR_TIMEOUT into status_out (int32 [1], CUDA)."""
+    _need(status_out, torch.int32, "status_out")
+    _check(load().moe_selftest_wait_timeout(_ptr(status_out), _stream(stream)), "moe_selftest_wait_timeout")
 
 
 def moe_route(x, router_w, k: int, router_bias=None, stream=None):

@@ -411,6 +411,13 @@ size_t moe_workspace_bytes(int M, int H, int I, int E, int k)
     return make_layout(M, H, I, E, k).total;
 }
 
+int moe_selftest_wait_timeout(int32_t *status_out, cudaStream_t stream)
+{
+    if (!status_out || !aligned(status_out, 4)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(launch_wait_timeout_selftest(status_out, stream));
+    return MOE_OK;
+}
+
 int moe_forward_launches(int M, int H, int I, int E, int k)
 {
     const int rc = check_dims(M, H, I, E, k, true);

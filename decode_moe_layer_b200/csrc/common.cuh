@@ -87,14 +87,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 
 // Bounded wait for the phase with the given parity to complete.  Once a wait
 // has timed out (`aborted` set) later waits return at once, so every thread
-// still reaches every CTA barrier and the kernel ends.
+// still reaches every CTA barrier and the kernel ends.  kLimit is in SM clock
+// cycles (the kernels use kWaitLimitCycles; the wait self-test a short limit).
+template <long long kLimit = kWaitLimitCycles>
 __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &aborted, const StatusPtrs &st)
 {
     if (aborted) return;
     if (mbar_try_wait(bar, parity)) return;
     long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > kLimit) {
             aborted = true;
             record_timeout(st);
             return;

@@ -213,6 +213,7 @@ cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap
                         __half *h, float *y, int *status, int32_t *status_out, int H, int I,
                         cudaStream_t s, bool pdl);
 int wide_smem_bytes();
+cudaError_t launch_wait_timeout_selftest(int32_t *status_out, cudaStream_t s);
 
 // Row blocks of the down projection per token (one arrival counter each).
 __host__ __device__ inline int down_row_blocks(int H) { return (H + kItemRows - 1) / kItemRows; }

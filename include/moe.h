@@ -178,6 +178,18 @@ size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
 int moe_forward_launches(int M, int H, int I, int E, int k);
 
 /*
+ * Self-test of the device-side failure path.  Every producer/consumer wait inside the layer's
+ * kernels is bounded: when it runs out, the kernel records MOE_ERR_TIMEOUT in the call's status
+ * (moe_mxfp4_forward_ex's status_out), skips its remaining waits and ends, so the CUDA context
+ * stays usable.  This call launches one small kernel that waits, through the same bounded wait
+ * with a limit of about 10 ms, on a barrier that nothing ever completes.  It writes
+ * MOE_ERR_TIMEOUT (int32) to status_out, a 4-byte-aligned DEVICE pointer, which the caller reads
+ * after synchronising `stream`.  Returns MOE_ERR_INVALID_ARG for a null or misaligned pointer,
+ * MOE_ERR_CUDA if the launch fails, else MOE_OK.  It faults nothing and touches no other memory.
+ */
+int moe_selftest_wait_timeout(int32_t *status_out, cudaStream_t stream);
+
+/*
  * Whole layer with a caller-owned workspace (>= moe_workspace_bytes, 256-byte
  * aligned; its contents need no initialisation and are overwritten), an optional
  * router bias, optional copies of the routing (topk_ids_out [M,k] int32,

@@ -91,3 +91,23 @@ def test_step_validation():
     assert lib.moe_down_combine(a, a, a, a, a, a, None, 4, 2048, 768, 128, 8, None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_down_combine(a, a, a, a, a, a, a, 0, 2048, 768, 128, 8, None) == moe.MOE_OK
     assert lib.moe_mxfp4_forward(a, a, a, a, a, a, a, 4, 2048, 768, 128, 8, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_selftest_validation():
+    # argument checks only (no launch): null and misaligned status pointers are refused
+    lib = moe.load()
+    assert lib.moe_selftest_wait_timeout(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(P(0x1002), None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_forward_launch_counts():
+    # 5 launches at decode sizes (fused select), 6 with the separate top-k + permutation, and 3
+    # more once experts can reach the tensor-core tile size (M >= 32, H and I multiples of 512)
+    lib = moe.load()
+    assert lib.moe_forward_launches(0, 2048, 768, 128, 8) == 0
+    assert lib.moe_forward_launches(8, 2048, 768, 128, 8) == 5
+    assert lib.moe_forward_launches(1, 7168, 2048, 256, 8) == 5
+    assert lib.moe_forward_launches(96, 2048, 768, 128, 8) == 6
+    assert lib.moe_forward_launches(256, 7168, 2048, 256, 8) == 9
+    assert lib.moe_forward_launches(1024, 4096, 1536, 128, 8) == 9
+    assert lib.moe_forward_launches(8, 2048, 100, 128, 8) == moe.MOE_ERR_UNSUPPORTED_SHAPE

@@ -169,6 +169,25 @@ def test_status_out_reports_ok(moe):
     assert int(st.item()) == moe.MOE_OK
 
 
+def test_bounded_wait_gives_up_with_timeout_status(moe):
+    # A wait that nothing completes runs out, reports MOE_ERR_TIMEOUT and ends the kernel; the
+    # context stays usable and the next layer call reports MOE_OK with the same output as before.
+    inp = gen.make_inputs(0, 2)
+    d = U.device_inputs(inp)
+    ws = torch.empty(moe.moe_workspace_bytes(2, 1024, 512, 16, 4), dtype=torch.uint8, device="cuda")
+    before = moe.moe_mxfp4_forward_ex(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], 4, ws)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    moe.moe_selftest_wait_timeout(st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == moe.MOE_ERR_TIMEOUT
+    st2 = torch.full((1,), -99, dtype=torch.int32, device="cuda")
+    after = moe.moe_mxfp4_forward_ex(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], 4, ws,
+                                     status_out=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == moe.MOE_OK
+    assert np.array_equal(_bits(before), _bits(after))
+
+
 def test_generator_device_streams_match_host(moe):
     # the integer weight streams are bit-identical when generated on the device
     inp = gen.make_inputs(1, 2, weights="torch", device="cuda")
