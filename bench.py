@@ -90,9 +90,14 @@ def algorithmic(shape, M, ids):
             "gate_up_flops": 4 * I * H * M * k, "down_flops": 2 * I * H * M * k}
 
 
-def kernel_source_hash():
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def kernel_code_hash(path=None):
+    """sha256[:16] of the dominant kernel's source with comments and blank space removed: any change
+    to its code changes it, a change to its comments or layout does not."""
+    with open(path or KERNEL_SRC) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()[:16]
 
 
 def profiled_traffic():
@@ -100,9 +105,9 @@ def profiled_traffic():
     if not os.path.exists(TRAFFIC_PROFILE):
         return None
     text = open(TRAFFIC_PROFILE).read()
-    h = re.search(r"kernel source sha256\[:16\]:\s*([0-9a-f]+)", text)
+    h = re.search(r"kernel code sha256\[:16\]:\s*([0-9a-f]+)", text)
     t = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", text)
-    if not h or not t or h.group(1) != kernel_source_hash():
+    if not h or not t or h.group(1) != kernel_code_hash():
         return None
     return float(t.group(1))
 

@@ -10,14 +10,17 @@
 // HBM bandwidth ("The Systematic Optimization Campaign", chunk 8.0).
 //
 // Design (one persistent CTA per SM, warp specialised):
-//  * Work item = (expert tile of <= 8 assignments, 64 weight rows).  gate_up:
-//    gate rows n0..n0+31 and the matching up rows I+n0..; down: W2 rows
-//    r0..r0+63.  The item is 4 MMA m-tiles of 16 rows; for gate_up an m-tile
+//  * Work item = (expert tile of <= 8 or <= 16 assignments -- the call's tile
+//    width -- and 64 weight rows).  gate_up: gate rows n0..n0+31 and the
+//    matching up rows I+n0..; down: W2 rows r0..r0+63.  The item is 4 MMA
+//    m-tiles of 16 rows; for gate_up an m-tile
 //    holds 8 gate rows (fragment rows 0-7) and the same 8 up rows (fragment rows
 //    8-15), so every thread ends with g and u of one output row and applies
-//    clamp-SwiGLU and the bf16 rounding in registers.  Each CTA takes a
-//    contiguous run of items in (tile, row block) order, so it streams adjacent
-//    32 KB weight regions of one expert back to back (DRAM page locality).
+//    clamp-SwiGLU and the bf16 rounding in registers.  Items are numbered in
+//    (tile, row block) order; with few items per CTA each CTA first takes a
+//    contiguous run of them (adjacent 32 KB weight regions of one expert back
+//    to back, for DRAM page locality), then single items or small groups from
+//    the call's work queue, so faster SMs take more.
 //  * Producer warp: per 1024-K stage, TMA 2-D tiled copies of the item's packed
 //    E2M1 bytes -- 4 column boxes of 32 or 64 rows x 128 bytes per row block,
 //    issued together so that each row's 512 contiguous bytes are read at once --
@@ -33,10 +36,13 @@
 //    and runs two m16n8k16 f16 MMAs per block.  Inside a block the K order is
 //    permuted (thread q's word covers K 8q..8q+7) identically for A and for the
 //    activation fragment, so each MMA pair spans exactly one scale block and the
-//    E8M0 scale is applied once to the fp32 partial sum.  At the end of an item a
-//    warp parks its partial sums in a double-buffered reduction area and moves on.
-//  * 2 epilogue warps sum the 8 K slots in slot order, then gate_up applies
-//    clamp-SwiGLU and stores h; down stores the unweighted fp32 row of each
+//    E8M0 scale is applied once to the fp32 partial sum.  With 16-assignment tiles
+//    each decoded fragment feeds two MMA n-tiles.  At the end of an item a warp
+//    parks its partial sums in a reduction area (two buffers for 8-wide tiles; one
+//    for 16-wide, where the K slots first add up in pairs) and moves on.
+//  * 2 epilogue warps (4 for 16-wide tiles) sum the K-slot partials in slot
+//    order, then gate_up applies clamp-SwiGLU and stores h; down stores the
+//    unweighted fp32 row of each
 //    assignment (at its flat id, from the expert-grouped order) -- off the compute
 //    path.  The item's position range reaches them from the producer through shared
 //    memory.  The weighted top-k combine that follows is its own small kernel
