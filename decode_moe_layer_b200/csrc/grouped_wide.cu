@@ -6,7 +6,7 @@
 // Attribution" ("MTP1 Post-Portfolio Eager-Cycle Profile"), with the fused gate/up producer of
 // the page's "Decision" section.  At large token counts the expert GEMMs become real dense
 // contractions: an expert with many assignments is streamed once for all of them (the narrow
-// kernel in grouped_gemm.cu re-streams it for every 8 assignments), and the MMA runs on
+// kernel in grouped_gemm.cu re-streams it for every 8 or 16 assignments), and the MMA runs on
 // tcgen05 with the fp32 accumulator in tensor memory.  The kernel keeps a kWideTokens-wide tile of
 // one expert's assignments against 128 weight rows per item, and the wider the tile the more
 // work each MMA instruction does (their issue cost hardly depends on N).
