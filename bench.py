@@ -275,6 +275,14 @@ def main():
     return 0
 
 
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of every rank's values; all ranks get it (a step's time is its slowest rank's)."""
+    import torch
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
 def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind, baselines):
     H, I, E, k = shape.H, shape.I, shape.E, shape.k
     inp = gen.make_inputs(ci, M, weights="torch", device=dev)
@@ -363,9 +371,7 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     mean_us = statistics.mean(step_ms) * 1e3
     e2e_us = statistics.mean(e2e_ms) * 1e3
     if world > 1:
-        t = torch.tensor([mean_us, e2e_us], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_us, e2e_us = float(t[0]), float(t[1])
+        mean_us, e2e_us = max_over_ranks(dist, [mean_us, e2e_us], dev)
 
     hbm = peaks["hbm_gbs"]
     tflops = peaks["bf16_tflops_sustained"]
