@@ -294,7 +294,9 @@ def test_single_expert_reduces_to_dense_mlp():
         xv = bf16_of_bits(x[t])
         g = W13[:I] @ xv
         u = W13[I:] @ xv
-        assert np.abs(g).max() > 7 and np.abs(u).max() > 7   # the clamps are exercised
+        # the clamps are exercised: g above 7 (clamped) and below -7 (not clamped: silu's
+        # negative tail is kept), u beyond both bounds
+        assert g.max() > 7 and g.min() < -7 and u.max() > 7 and u.min() < -7
         a = np.minimum(g, 7.0)
         hv = _bf16_nearest_vec(a * scipy.special.expit(a) * np.clip(u, -7.0, 7.0))
         assert np.array_equal(bf16_of_bits(r["h"][t]), hv)
