@@ -202,9 +202,10 @@ def run_reference(args):
     shape = gen.CONFIGS[args.config]
     M = args.M
     inp = gen.make_inputs(args.config, M, weights="none")
-    # each step: one full layer call of the workload (all M tokens).  A token subset would not do:
-    # the oracle decodes each touched expert once per call, a cost the tokens share.  The timed
-    # steps stop once REF_MAX_SECONDS have passed, so that a large --steps still ends in minutes.
+    # each step: one full layer call of the workload (all M tokens).  A one-token step scaled by M
+    # would not do: the oracle spreads a call over its assignments and tokens, so one token leaves
+    # most host cores idle.  The timed steps stop once REF_MAX_SECONDS have passed, so that a large
+    # --steps still ends in minutes.
     full = [list(range(M))]
     for _ in range(min(args.warmup, 3)):
         time_oracle(inp, full, 0.0, 1)
