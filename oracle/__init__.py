@@ -17,23 +17,35 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+# MOE_ORACLE_LIB: load another build of the same interface instead (the pins' mutation test loads
+# copies of the oracle with one planted mistake each this way)
+_LIB_OVERRIDE = os.environ.get("MOE_ORACLE_LIB")
 _lib = None
+
+
+def compile_lib(src: str, out: str) -> str:
+    """gcc -O2 -fopenmp of one oracle source into a shared library (IEEE fp64, no fast-math)."""
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-Wall", "-shared", "-fPIC", src, "-o", tmp, "-lm"])
+    os.replace(tmp, out)
+    return out
 
 
 def build(force: bool = False) -> str:
     """Compile moe_oracle.c into liboracle.so (gcc, -O2, OpenMP, IEEE fp64)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-Wall", "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"])
-        os.replace(tmp, _LIB)
+        compile_lib(_SRC, _LIB)
     return _LIB
 
 
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = ctypes.CDLL(_LIB)
+        if _LIB_OVERRIDE:
+            lib = ctypes.CDLL(_LIB_OVERRIDE)
+        else:
+            build()
+            lib = ctypes.CDLL(_LIB)
         P = ctypes.c_void_p
         i = ctypes.c_int
         lib.oracle_e2m1_value.restype = ctypes.c_double
