@@ -18,7 +18,7 @@ Legs of the default run (one JSON line on rank 0):
     the out download inside the timed region;
   * cpu_baseline: the fp64 oracle on the host cores (rank 0, N=1), on a bounded
     sample of the same workload.
-`--impl reference` times the oracle alone (the reference arm of this build).
+`--impl reference` is the reference arm: the fp64 oracle alone, full layer calls on the host cores.
 With N>1 (torchrun) every rank runs an independent replica of the layer call.
 """
 from __future__ import annotations
