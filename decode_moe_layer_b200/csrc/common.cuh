@@ -137,13 +137,6 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
 
-// ------------------------------------------------------------------ named barriers
-
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // ------------------------------------------------------------------ MMA + decode
 
 // D = A(16x16, row) * B(16x8, col) + C, f16 inputs, f32 accumulate.
