@@ -4,8 +4,9 @@ calls into the oracle for the same inputs, and the tolerance checks.
 Tolerances (derivations in the design notes):
   * routing ids, expert offsets, sorted ids, inverse positions: bit-exact;
   * routing weights: |w - w_oracle| <= 1e-5 (fp32 logits and softmax vs fp64);
-  * h: each element equal to the oracle's bf16 value or one bf16 ulp away
-    (fp32 vs fp64 accumulation may flip a rounding), flips counted;
+  * h: within one bf16 ulp of the oracle's bf16 value plus h's sensitivity to a
+    worst-case fp32 accumulation error and the binary16 storage of h * 2^10
+    (check_h_bound), flips counted;
   * out: relative L2 error <= 5e-3 and max abs error <= 2e-2 * rms, both against
     the oracle's fp64 out64.
 """
@@ -140,20 +141,4 @@ def check_h_bound(gpu_h, ref_bits, g, u, x_row_bits, w13_q_e, w13_s_e, what=""):
         what, int(bad.sum()), float((diff - tol).max()), float(ref[np.argmax(diff - tol)]))
     flips = int((diff > 0).sum())
     FLIP_LOG.append((what, flips, diff.size))
-    return flips
-
-
-def check_h(gpu_h: np.ndarray, ref_bits: np.ndarray, what="", max_flip_frac=0.3):
-    """gpu_h: float64 values (binary16-stored bf16 values); ref_bits: oracle bf16 bit patterns.
-    Every element must be within one bf16 ulp; the share of flipped roundings is recorded
-    (FLIP_LOG), with only a loose ceiling against gross errors."""
-    ref = gen.bf16_bits_to_f64(ref_bits)
-    diff = np.abs(gpu_h - ref)
-    tol = np.maximum(bf16_ulp(np.maximum(np.abs(gpu_h), np.abs(ref))), 2.0 ** -24)
-    bad = diff > tol
-    assert not bad.any(), "%s: %d elements differ by more than one bf16 ulp (worst %.3e)" % (
-        what, int(bad.sum()), float(diff.max()))
-    flips = int((diff > 0).sum())
-    FLIP_LOG.append((what, flips, diff.size))
-    assert flips <= max_flip_frac * diff.size + 1, "%s: %d of %d elements flipped" % (what, flips, diff.size)
     return flips
