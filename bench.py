@@ -193,6 +193,7 @@ def time_oracle(inp, tokens_per_step, min_seconds, max_steps, max_seconds=float(
 
 
 REF_MAX_SECONDS = 120
+REF_MAX_WARMUP_SECONDS = 20
 
 
 def run_reference(args):
@@ -207,19 +208,19 @@ def run_reference(args):
     # most host cores idle.  The timed steps stop once REF_MAX_SECONDS have passed, so that a large
     # --steps still ends in minutes.
     full = [list(range(M))]
-    for _ in range(min(args.warmup, 3)):
-        time_oracle(inp, full, 0.0, 1)
+    warm = time_oracle(inp, full, float("inf"), args.warmup, REF_MAX_WARMUP_SECONDS)[0] if args.warmup > 0 else []
     times, cores = time_oracle(inp, full, float("inf"), args.steps, REF_MAX_SECONDS)
     us_call = statistics.mean(times) * 1e6
     rec = {
         "impl": "reference", "metric": METRIC, "value": us_call, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": len(times), "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3,
+        "steps": len(times), "warmup": len(warm), "ms_per_step": statistics.mean(times) * 1e3,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(workload_config(shape, M), timing="fp64 oracle on the host cores, wall clock"),
         "cpu_baseline": {"value": us_call, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": "%d full layer calls (all %d tokens) of the same workload, one per step "
-                                   "(%d requested; timed steps stop after %d s)"
-                                   % (len(times), M, args.steps, REF_MAX_SECONDS)},
+                         "sample": "%d full layer calls (all %d tokens) of the same workload, one per step, "
+                                   "after %d untimed ones (%d and %d requested; timed steps stop after %d s, "
+                                   "warm-up after %d s)" % (len(times), M, len(warm), args.steps, args.warmup,
+                                                            REF_MAX_SECONDS, REF_MAX_WARMUP_SECONDS)},
         "e2e": {"value": us_call, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(rec))
