@@ -58,7 +58,7 @@ Layout make_layout(int M, int H, int I, int E, int k)
 {
     Layout L;
     const size_t n = static_cast<size_t>(M) * k;
-    // 16-wide tiles when the experts average 4 or more assignments and their larger stages fit
+    // 16-wide tiles when the experts average 6 or more assignments (tile_width) and their larger stages fit
     L.width = tile_width(M, E, k);
     if (L.width == 16 && (grouped_smem_bytes(H, 16) > 227 * 1024 || grouped_smem_bytes(I, 16) > 227 * 1024))
         L.width = 8;
