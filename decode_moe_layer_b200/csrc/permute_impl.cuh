@@ -5,16 +5,20 @@
 // Post-Portfolio Eager-Cycle Profile").  The expert-grouped order is the stable
 // counting sort of the assignments f = t*k + j by expert: position(f) =
 // offset[e_f] + rank(f), rank(f) = the number of earlier assignments on the same
-// expert.  One thread per assignment, in rounds of blockDim assignments:
-//  * a warp's lanes that share an expert find each other with __match_any_sync
-//    (rank inside the warp = matching lanes below it);
-//  * the lowest of them records the warp's count of that expert in a
-//    [warp][expert] table, one pass per expert turns the table into prefix counts
-//    (plus the counts of earlier rounds) and the thread reads its rank back.
-// Counts per expert come first (shared-memory atomics: order-free), then one block
-// scan of (tiles << 16 | count) gives every expert offset and tile base at once.
-// Two block barriers per round, no sort; every result is unique, so the bytes do
-// not depend on scheduling.
+// expert.  Two ways to rank:
+//  * the fused router select (M <= 64) keeps one 64-bit token mask per expert (see
+//    warp_scan_experts / scatter_assignment below);
+//  * rank_and_scatter (the stand-alone permutation, any M) takes one thread per
+//    assignment, in rounds of blockDim assignments:
+//    - a warp's lanes that share an expert find each other with __match_any_sync
+//      (rank inside the warp = matching lanes below it);
+//    - the lowest of them records the warp's count of that expert in a
+//      [warp][expert] table, one pass per expert turns the table into prefix counts
+//      (plus the counts of earlier rounds) and the thread reads its rank back;
+//    - counts per expert come first (shared-memory atomics: order-free), then one
+//      block scan of (tiles << 16 | count) gives every expert offset and tile base
+//      at once; two block barriers per round, no sort.
+// Every result is unique, so the bytes do not depend on scheduling.
 #pragma once
 
 #include "common.cuh"
