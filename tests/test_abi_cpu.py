@@ -4,6 +4,7 @@ paths, so they run without a GPU)."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -111,3 +112,34 @@ def test_forward_launch_counts():
     assert lib.moe_forward_launches(256, 7168, 2048, 256, 8) == 9
     assert lib.moe_forward_launches(1024, 4096, 1536, 128, 8) == 9
     assert lib.moe_forward_launches(8, 2048, 100, 128, 8) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    # include/moe.h compiles as strict C99, every declared function resolves against libmoe.so, and
+    # the host-only entry points answer from a C program (no torch, no GPU)
+    names = sorted(declared_functions())
+    checks = ("    typedef void (*fn)(void);\n    fn volatile table[] = {%s};\n"
+              "    for (unsigned i = 0; i < sizeof(table) / sizeof(table[0]); ++i)\n"
+              "        if (!table[i]) return 2;" % ", ".join("(fn)%s" % n for n in names))
+    src = tmp_path / "abi.c"
+    src.write_text("""#include "moe.h"
+#include <stdio.h>
+#include <string.h>
+int main(void)
+{
+%s
+    if (strcmp(moe_status_string(MOE_ERR_TIMEOUT), "MOE_ERR_TIMEOUT") != 0) return 3;
+    if (moe_workspace_bytes(8, 2048, 768, 128, 8) == 0) return 4;
+    if (moe_forward_launches(8, 2048, 768, 128, 8) != 5) return 5;
+    if (moe_forward_launches(8, 2047, 768, 128, 8) != MOE_ERR_UNSUPPORTED_SHAPE) return 6;
+    printf("ok\\n");
+    return 0;
+}
+""" % checks)
+    exe = str(tmp_path / "abi")
+    libdir = os.path.dirname(moe.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                           "-I", os.path.join(ROOT, "include"), str(src), "-o", exe,
+                           "-L", libdir, "-lmoe", "-Wl,-rpath," + libdir])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
