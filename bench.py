@@ -1,19 +1,23 @@
 #!/usr/bin/env python
 """Benchmark: microseconds per routed MXFP4 MoE layer call on B200.
 
-Default workload: the decode-width Qwen3-MoE-like layer (H=2048, I=768, E=128,
-top-8) at M=8 tokens, the c8 decode point that "row/QUANT-CT-MXFP4-C8-DIFF"
-(vllm.cpp PR #52) traces.  Synthetic seeded inputs (moe_inputs), weights resident
-in HBM, L2 flushed (512 MB write) before every timed call.
+Headline workload: the largest single-GPU configuration, the DeepSeek-V3-class routed layer
+(H=7168, I=2048, E=256, top-8, ~6 GB of MXFP4 weights) at M=512 tokens, where nearly every expert
+is hit and the tensor-core path runs.  Before it, one line per other workload (the tiny layer, the
+decode-width layer at M=1..8, the DeepSeek-class layer at M=1..32 and 256, the skewed layer at
+M=1024) from the same run; the driver reads the last line.  Synthetic seeded inputs (moe_inputs),
+weights resident in HBM, L2 flushed before every timed call by reading a 512 MB buffer (a read
+leaves no dirty lines for the layer's kernels to write back).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config C] [--M M] [--sweep]
+                    [--config C] [--M M] [--sweep] [--headline-only]
 
-Legs of the default run (one JSON line on rank 0):
+Legs of the headline (one JSON line on rank 0):
   * timed: K CUDA-graph replays of one moe_mxfp4_forward_ex call, each bracketed
     by CUDA events on the replay stream; value = mean us/call (max over ranks);
-  * kernel roofline: per-kernel event times from moe_mxfp4_forward_profile; the
-    dominant kernel's algorithmic bytes / time against the measured HBM peak;
+  * kernel roofline: per-launch event times from moe_mxfp4_forward_profile; the
+    dominant launch's algorithmic bytes (or FLOPs, when the call is tensor-bound) / time
+    against the measured peak;
   * e2e: the same call through the C ABI from pinned HOST buffers, the x upload and
     the out download inside the timed region;
   * cpu_baseline: the fp64 oracle on the host cores (rank 0, N=1), on a bounded
@@ -48,8 +52,17 @@ NOMINAL_HBM_GBS = 8000.0
 NOMINAL_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 512 << 20
-KERNEL_SRC = os.path.join(ROOT, "decode_moe_layer_b200", "csrc", "grouped_gemm.cu")
-TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "grouped_mxfp4_decode_h2048_i768_e128_k8_M8.md")
+CSRC = os.path.join(ROOT, "decode_moe_layer_b200", "csrc")
+# committed ncu summaries that give a launch's DRAM bytes for a workload, with the hash of the
+# kernel source they were taken on: (workload name, launch) -> (kernel source, summary)
+TRAFFIC_PROFILES = {
+    ("dsv3_wide_h7168_i2048_e256_k8 M=512", "gate_up_tc_small"):
+        (os.path.join(CSRC, "grouped_wide.cu"),
+         os.path.join(ROOT, "profiles", "grouped_wide_dsv3_h7168_i2048_e256_k8_M512.md")),
+    ("decode_h2048_i768_e128_k8 M=8", "gate_up"):
+        (os.path.join(CSRC, "grouped_gemm.cu"),
+         os.path.join(ROOT, "profiles", "grouped_mxfp4_decode_h2048_i768_e128_k8_M8.md")),
+}
 
 
 def parse_args():
@@ -58,9 +71,11 @@ def parse_args():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--config", type=int, default=1)
-    p.add_argument("--M", type=int, default=8)
+    p.add_argument("--config", type=int, default=3)
+    p.add_argument("--M", type=int, default=512)
     p.add_argument("--sweep", action="store_true", help="one line per (config, M) of the workloads, no baselines")
+    p.add_argument("--headline-only", action="store_true", help="skip the other workloads' lines")
+    p.add_argument("--other-steps", type=int, default=20, help="timed steps of the non-headline lines")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
 
@@ -76,38 +91,74 @@ def load_peaks():
 
 # --------------------------------------------------------------------------- algorithmic work
 
-def algorithmic(shape, M, ids):
-    """Bytes and FLOPs the method must move/do for one call, from the realised routing."""
+# The library's split of an expert's assignments (moe_internal.h): tensor-core tiles when H and I are
+# multiples of 512, M >= 9 and the experts average >= 4.5 assignments, for the experts with 9 or
+# more (small tiles up to 64, large tiles above); mma.sync tiles for the others.
+WIDE_MIN_TOKENS, WIDE_SMALL_MAX = 9, 64
+
+
+def expert_classes(shape, M, ids):
+    """Per-expert assignment counts and class ('narrow', 'small', 'large') from the realised routing."""
     H, I, E, k = shape.H, shape.I, shape.E, shape.k
-    touched = len(np.unique(ids))
+    counts = np.bincount(np.asarray(ids).reshape(-1), minlength=E)
+    wide_on = M >= WIDE_MIN_TOKENS and H % 512 == 0 and I % 512 == 0 and 2 * M * k >= WIDE_MIN_TOKENS * E
+    cls = {}
+    for e in range(E):
+        c = int(counts[e])
+        if c == 0:
+            continue
+        if wide_on and c >= WIDE_MIN_TOKENS:
+            cls[e] = "small" if c <= WIDE_SMALL_MAX else "large"
+        else:
+            cls[e] = "narrow"
+    return counts, cls
+
+
+def algorithmic(shape, M, ids):
+    """Bytes and FLOPs the method must move/do for one call, from the realised routing, in total
+    and per launch (the launches of moe_mxfp4_forward_profile)."""
+    H, I, E, k = shape.H, shape.I, shape.E, shape.k
+    counts, cls = expert_classes(shape, M, ids)
+    touched = len(cls)
     w_bytes = touched * (51 * I * H // 32)
     total = w_bytes + E * H * 4 + 2 * M * H * 2 + M * k * 8
     flops = 6 * I * H * M * k + 2 * M * E * H
-    gate_up = touched * (2 * I * H * 17 // 32) + M * H * 2 + M * k * I * 2
-    down = touched * (I * H * 17 // 32) + M * k * I * 2 + M * H * 2
-    return {"touched": touched, "bytes": total, "flops": flops, "weight_bytes": w_bytes,
-            "gate_up_bytes": gate_up, "down_bytes": down,
-            "gate_up_flops": 4 * I * H * M * k, "down_flops": 2 * I * H * M * k}
+    per = {"route_logits": {"bytes": E * H * 4 + M * H * 2, "flops": 2 * M * E * H}}
+    for name, kind in (("gate_up", "narrow"), ("gate_up_tc_small", "small"), ("gate_up_tc_large", "large"),
+                       ("down", "narrow"), ("down_tc_small", "small"), ("down_tc_large", "large")):
+        ex = [e for e, c in cls.items() if c == kind]
+        n_assign = int(sum(counts[e] for e in ex))
+        if name.startswith("gate_up"):
+            b = len(ex) * (2 * I * H * 17 // 32) + n_assign * H * 2 + n_assign * I * 2
+            f = 4 * I * H * n_assign
+        else:
+            b = len(ex) * (I * H * 17 // 32) + n_assign * I * 2 + n_assign * H * 4
+            f = 2 * I * H * n_assign
+        per[name] = {"bytes": b, "flops": f, "experts": len(ex), "assignments": n_assign}
+    per["combine"] = {"bytes": M * k * H * 4 + M * k * 4 + M * H * 2, "flops": 0}
+    return {"touched": touched, "bytes": total, "flops": flops, "weight_bytes": w_bytes, "per_launch": per,
+            "classes": {kind: sum(1 for c in cls.values() if c == kind) for kind in ("narrow", "small", "large")}}
 
 
-def kernel_code_hash(path=None):
-    """sha256[:16] of the dominant kernel's source with comments and blank space removed: any change
-    to its code changes it, a change to its comments or layout does not."""
-    with open(path or KERNEL_SRC) as f:
+def kernel_code_hash(path):
+    """sha256[:16] of a kernel's source with comments and blank space removed: any change to its
+    code changes it, a change to its comments or layout does not."""
+    with open(path) as f:
         src = f.read()
     src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
     src = re.sub(r"//[^\n]*", " ", src)
     return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()[:16]
 
 
-def profiled_traffic():
-    """dram bytes per launch of the dominant kernel from the committed ncu summary, if the kernel is unchanged."""
-    if not os.path.exists(TRAFFIC_PROFILE):
+def profiled_traffic(workload, launch):
+    """DRAM bytes of one launch from the committed ncu summary, if the kernel is unchanged since."""
+    src, path = TRAFFIC_PROFILES.get((workload, launch), (None, None))
+    if path is None or not os.path.exists(path):
         return None
-    text = open(TRAFFIC_PROFILE).read()
+    text = open(path).read()
     h = re.search(r"kernel code sha256\[:16\]:\s*([0-9a-f]+)", text)
     t = re.search(r"dram bytes per launch:\s*([0-9.eE+]+)", text)
-    if not h or not t or h.group(1) != kernel_code_hash():
+    if not h or not t or h.group(1) != kernel_code_hash(src):
         return None
     return float(t.group(1))
 
@@ -173,9 +224,7 @@ def time_oracle(inp, tokens_per_step, min_seconds, max_steps, max_seconds=float(
     import oracle
     shape = inp.shape
     ids, _, _ = oracle.route(inp.x, inp.router_w, inp.router_bias, shape.k)
-    need = sorted(set(int(e) for e in ids.ravel()))
-    ex = {e: inp.expert_weights(e) for e in need}
-    tabs = [{e: v[i] for e, v in ex.items()} for i in range(4)]
+    tabs = [{}, {}, {}, {}]
     times = []
     t_start = time.perf_counter()
     step = 0
@@ -184,6 +233,11 @@ def time_oracle(inp, tokens_per_step, min_seconds, max_steps, max_seconds=float(
         if step >= 2 and (elapsed >= min_seconds or elapsed >= max_seconds):
             break
         toks = tokens_per_step[step % len(tokens_per_step)]
+        # the experts this step's tokens use, regenerated on the host (outside the step's timer)
+        for e in sorted(set(int(e) for t in toks for e in ids[t])):
+            if e not in tabs[0]:
+                for i, v in enumerate(inp.expert_weights(e)):
+                    tabs[i][e] = v
         t0 = time.perf_counter()
         oracle.forward(inp.x, inp.router_w, inp.router_bias, tabs[0], tabs[1], tabs[2], tabs[3], shape.k,
                        tokens=toks, I=shape.I)
@@ -203,24 +257,22 @@ def run_reference(args):
     shape = gen.CONFIGS[args.config]
     M = args.M
     inp = gen.make_inputs(args.config, M, weights="none")
-    # each step: one full layer call of the workload (all M tokens).  A one-token step scaled by M
-    # would not do: the oracle spreads a call over its assignments and tokens, so one token leaves
-    # most host cores idle.  The timed steps stop once REF_MAX_SECONDS have passed, so that a large
-    # --steps still ends in minutes.
-    full = [list(range(M))]
-    warm = time_oracle(inp, full, float("inf"), args.warmup, REF_MAX_WARMUP_SECONDS)[0] if args.warmup > 0 else []
-    times, cores = time_oracle(inp, full, float("inf"), args.steps, REF_MAX_SECONDS)
-    us_call = statistics.mean(times) * 1e6
+    # each step: the oracle on one group of tokens (the whole call when M is small; else enough tokens
+    # to keep every host core busy, the time scaled by M / tokens), so that a step of the largest
+    # workload takes seconds, not minutes.  The timed steps stop once REF_MAX_SECONDS have passed.
+    subsets, n_tok = oracle_token_sample(M, shape.k)
+    warm = time_oracle(inp, subsets, float("inf"), args.warmup, REF_MAX_WARMUP_SECONDS)[0] if args.warmup > 0 else []
+    times, cores = time_oracle(inp, subsets, float("inf"), args.steps, REF_MAX_SECONDS)
+    us_call = statistics.mean(times) * 1e6 * M / n_tok
     rec = {
         "impl": "reference", "metric": METRIC, "value": us_call, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": len(times), "warmup": len(warm), "ms_per_step": statistics.mean(times) * 1e3,
+        "steps": len(times), "warmup": len(warm), "ms_per_step": us_call / 1e3,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(workload_config(shape, M), timing="fp64 oracle on the host cores, wall clock"),
         "cpu_baseline": {"value": us_call, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": "%d full layer calls (all %d tokens) of the same workload, one per step, "
-                                   "after %d untimed ones (%d and %d requested; timed steps stop after %d s, "
-                                   "warm-up after %d s)" % (len(times), M, len(warm), args.steps, args.warmup,
-                                                            REF_MAX_SECONDS, REF_MAX_WARMUP_SECONDS)},
+                         "sample": oracle_sample_text(len(times), n_tok, M) +
+                         ", after %d untimed ones (%d and %d requested; timed steps stop after %d s, warm-up after "
+                         "%d s)" % (len(warm), args.steps, args.warmup, REF_MAX_SECONDS, REF_MAX_WARMUP_SECONDS)},
         "e2e": {"value": us_call, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(rec))
@@ -229,7 +281,7 @@ def run_reference(args):
 
 def workload_config(shape, M):
     return {"workload": "%s M=%d" % (shape.name, M), "M": M, "H": shape.H, "I": shape.I, "E": shape.E,
-            "top_k": shape.k, "weights": "MXFP4 (E2M1 + E8M0 per 32)", "l2": "flushed (512 MB write) before each call",
+            "top_k": shape.k, "weights": "MXFP4 (E2M1 + E8M0 per 32)", "l2": "flushed (512 MB read) before each call",
             "timing": "CUDA-graph replay of one moe_mxfp4_forward_ex call, CUDA events"}
 
 
@@ -262,16 +314,23 @@ def main():
 
     peaks, peak_kind = load_peaks()
 
-    cases = [(args.config, args.M)]
+    every = [(ci, M) for ci, s in enumerate(gen.CONFIGS) for M in s.Ms]
+    headline = (args.config, args.M)
     if args.sweep:
-        cases = [(ci, M) for ci, s in enumerate(gen.CONFIGS) for M in s.Ms]
+        cases = [(c, False) for c in every]
+    elif args.headline_only:
+        cases = [(headline, True)]
+    else:   # the other workloads first (fewer steps, no baselines), the headline last
+        cases = [(c, False) for c in every if c != headline] + [(headline, True)]
 
-    for ci, M in cases:
+    for (ci, M), is_headline in cases:
         shape = gen.CONFIGS[ci]
+        steps = args.steps if (is_headline or args.sweep) else min(args.steps, args.other_steps)
         rec = run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind,
-                       baselines=not args.sweep)
+                       baselines=is_headline, steps=steps)
         if rank == 0:
             print(json.dumps(rec), flush=True)
+        torch.cuda.empty_cache()
     if world > 1:
         dist.destroy_process_group()
     return 0
@@ -285,7 +344,7 @@ def max_over_ranks(dist, values, device):
     return [float(v) for v in t]
 
 
-def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind, baselines):
+def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind, baselines, steps):
     H, I, E, k = shape.H, shape.I, shape.E, shape.k
     inp = gen.make_inputs(ci, M, weights="torch", device=dev)
     xb = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -295,7 +354,12 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     ws = torch.empty(moe.moe_workspace_bytes(M, H, I, E, k), dtype=torch.uint8, device=dev)
     out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
     ids = torch.empty((M, k), dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def flush_l2():
+        # reads 512 MB (four L2 capacities): the layer's weights and activations leave L2, and the
+        # lines the read brings in are clean, so no kernel of the call pays a write-back for them
+        torch.sum(flush)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -323,13 +387,13 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
                 graph.replay()
             stream.synchronize()
         for i in range(args.warmup):
-            flush.fill_(i & 0xFF)
+            flush_l2()
             graph.replay()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+              for _ in range(steps)]
         barrier()
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+        for i in range(steps):
+            flush_l2()
             ev[i][0].record(stream)
             graph.replay()
             ev[i][1].record(stream)
@@ -340,8 +404,8 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     # ------------------------------------------------------------------ per-kernel attribution
     prof = {n: [] for n in moe.PROFILE_KERNELS}
     with torch.cuda.stream(stream):
-        for i in range(max(10, min(args.steps, 50))):
-            flush.fill_(i & 0xFF)
+        for i in range(max(10, min(steps, 50))):
+            flush_l2()
             # a short device-side sleep queued first lets the host enqueue every kernel and
             # event of the call before the GPU reaches them: event gaps then hold device time only
             torch.cuda._sleep(2_000_000)
@@ -357,8 +421,8 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     x_dev = torch.empty_like(xb)
     e2e_ms = []
     with torch.cuda.stream(stream):
-        for i in range(args.warmup + args.steps):
-            flush.fill_(i & 0xFF)
+        for i in range(args.warmup + steps):
+            flush_l2()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             x_dev.copy_(x_host, non_blocking=True)
@@ -379,26 +443,24 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
     tflops = peaks["bf16_tflops_sustained"]
     roof_us = max(work["bytes"] / (hbm * 1e3), work["flops"] / (tflops * 1e6))
     roof_nominal_us = max(work["bytes"] / (NOMINAL_HBM_GBS * 1e3), work["flops"] / (NOMINAL_BF16_TFLOPS * 1e6))
-    dominant = max(kern_us, key=kern_us.get)
-    dom_bytes = {"gate_up_swiglu": work["gate_up_bytes"], "down_combine": work["down_bytes"]}.get(dominant)
-    if dom_bytes is None:
-        dom_bytes = work["bytes"]
-    dom_flops = {"gate_up_swiglu": work["gate_up_flops"], "down_combine": work["down_flops"]}.get(dominant,
-                                                                                                   work["flops"])
     call_bound = "hbm" if work["bytes"] / hbm > work["flops"] / (tflops * 1e3) else "tensor"
+    # the dominant launch and its own algorithmic work (route_select / permute / gather have none
+    # in this accounting; they are never dominant at these sizes)
+    dominant = max(kern_us, key=kern_us.get)
+    dom = work["per_launch"].get(dominant, {"bytes": work["bytes"], "flops": work["flops"]})
     if call_bound == "hbm":
-        roof = {"bound": "hbm", "achieved": dom_bytes / (kern_us[dominant] * 1e3), "peak": hbm, "unit": "GB/s",
-                "algorithmic_bytes_per_launch": dom_bytes}
+        roof = {"bound": "hbm", "achieved": dom["bytes"] / (kern_us[dominant] * 1e3), "peak": hbm, "unit": "GB/s",
+                "algorithmic_bytes_per_launch": dom["bytes"]}
     else:   # the contraction binds: FLOPs against the sustained bf16 tensor peak
-        roof = {"bound": "tensor", "achieved": dom_flops / (kern_us[dominant] * 1e6), "peak": tflops,
-                "unit": "TFLOP/s", "algorithmic_flops_per_launch": dom_flops}
+        roof = {"bound": "tensor", "achieved": dom["flops"] / (kern_us[dominant] * 1e6), "peak": tflops,
+                "unit": "TFLOP/s", "algorithmic_flops_per_launch": dom["flops"]}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    traffic = profiled_traffic() if (ci, M) == (1, 8) and dominant == "gate_up_swiglu" else None
+    traffic = profiled_traffic(workload_config(shape, M)["workload"], dominant)
     sorted_ms = sorted(step_ms)
     rec = {
-        "metric": METRIC, "value": mean_us, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": mean_us, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": mean_us / 1e3, "higher_is_better": False, "scaling": "weak",
-        "vs_baseline": None, "dtype": "mxfp4 weights x f16 activations, fp32 accumulate", "data": "synthetic",
+        "vs_baseline": None, "dtype": "bf16 (MXFP4 weights decoded exactly to bf16), fp32 accumulate", "data": "synthetic",
         "config": dict(workload_config(shape, M), parallelism="replicas" if world > 1 else "1 GPU"),
         "p10_us": sorted_ms[len(sorted_ms) // 10] * 1e3, "p50_us": statistics.median(step_ms) * 1e3,
         "p90_us": sorted_ms[(9 * len(sorted_ms)) // 10] * 1e3,
@@ -408,20 +470,40 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
                           "roofline_us_nominal": roof_nominal_us, "frac_nominal": roof_nominal_us / mean_us,
                           "algorithmic_bytes": work["bytes"], "flops": work["flops"],
                           "touched_experts": work["touched"]},
-        "kernels_us": kern_us,
+        "kernels_us": {n: v for n, v in kern_us.items() if v > 0},
+        "expert_tiles": work["classes"],
         "roofline": dict(kernel=dominant, traffic=traffic, peak_kind=peak_kind, **roof),
         "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": M * H * 2,
                 "path": "pinned host x -> moe_mxfp4_forward_ex (eager C-ABI call) -> pinned host out"},
-        "gpu_launches": moe.moe_forward_launches(M, H, I, E, k) * args.steps,
+        "gpu_launches": moe.moe_forward_launches(M, H, I, E, k) * steps,
         "clocks": clk,
     }
     if baselines and rank == 0 and world == 1 and not args.no_cpu_baseline:
         host = gen.make_inputs(ci, M, weights="none")
-        subsets = [list(range(M))]
-        times, cores = time_oracle(host, subsets, 10.0, 30)
-        rec["cpu_baseline"] = {"value": statistics.mean(times) * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
-                               "sample": "%d full layer calls (all %d tokens) of the same workload" % (len(times), M)}
+        subsets, n_tok = oracle_token_sample(M, k)
+        times, cores = time_oracle(host, subsets, 10.0, 30, 30.0)
+        rec["cpu_baseline"] = {"value": statistics.mean(times) * 1e6 * M / n_tok, "unit": UNIT, "cores": cores,
+                               "kind": "oracle", "sample": oracle_sample_text(len(times), n_tok, M)}
     return rec
+
+
+def oracle_token_sample(M, k, cores=None):
+    """Token subsets for timing the oracle: the whole call when M is small, else disjoint groups of
+    enough tokens (4 assignments per host core) to keep every core busy, each step's time scaled by
+    M / tokens per step."""
+    import oracle
+    cores = cores or oracle.num_threads()
+    n = min(M, max(1, -(-4 * cores // k)))
+    groups = [list(range(i, min(M, i + n))) for i in range(0, M, n)]
+    groups = [g for g in groups if len(g) == n] or [list(range(M))]
+    return groups, n
+
+
+def oracle_sample_text(steps, n_tok, M):
+    if n_tok >= M:
+        return "%d full layer calls (all %d tokens) of the same workload" % (steps, M)
+    return ("%d oracle calls on disjoint groups of %d of the workload's %d tokens (all their %d assignments "
+            "and the full routing), each scaled by %d/%d to one call" % (steps, n_tok, M, n_tok * 8, M, n_tok))
 
 
 if __name__ == "__main__":

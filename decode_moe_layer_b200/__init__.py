@@ -6,7 +6,6 @@ the library and fails loudly if it has not been built.
 """
 from ._lib import (  # noqa: F401
     EXPORTS,
-    H_STORAGE_SCALE,
     LIB_PATH,
     MOE_ERR_CUDA,
     MOE_ERR_INVALID_ARG,

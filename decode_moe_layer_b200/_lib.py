@@ -24,8 +24,8 @@ EXPORTS = (
     "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_forward_launches", "moe_mxfp4_forward_ex",
     "moe_mxfp4_forward_profile", "moe_route_noalloc", "moe_selftest_wait_timeout",
 )
-H_STORAGE_SCALE = 1024.0   # moe_gate_up_swiglu stores binary16(h * 2^10)
-PROFILE_KERNELS = ("route_logits", "route_select", "permute", "gate_up_swiglu", "down_combine")
+PROFILE_KERNELS = ("route_logits", "route_select", "permute", "gate_up", "gather", "gate_up_tc_small",
+                   "gate_up_tc_large", "down", "down_tc_small", "down_tc_large", "combine")
 
 _lib = None
 
@@ -160,12 +160,12 @@ def moe_permute(topk_ids, E: int, stream=None):
 
 
 def moe_gate_up_swiglu(x, w13_q, w13_s, expert_offsets, sorted_ids, k: int, stream=None):
-    """-> h binary16 [M*k, I] in expert-grouped order, element = bf16_rne(h) * 2^10."""
+    """-> h bf16 [M*k, I] in expert-grouped order (row p = assignment sorted_ids[p])."""
     _need(x, torch.bfloat16, "x")
     M, H = x.shape
     E, I2, _ = w13_q.shape
     I = I2 // 2
-    h = torch.empty((M * k, I), dtype=torch.float16, device=x.device)
+    h = torch.empty((M * k, I), dtype=torch.bfloat16, device=x.device)
     rc = load().moe_gate_up_swiglu(_ptr(x), _ptr(w13_q), _ptr(w13_s), _ptr(expert_offsets), _ptr(sorted_ids),
                                    _ptr(h), M, H, I, E, k, _stream(stream))
     _check(rc, "moe_gate_up_swiglu")
@@ -173,8 +173,8 @@ def moe_gate_up_swiglu(x, w13_q, w13_s, expert_offsets, sorted_ids, k: int, stre
 
 
 def moe_down_combine(h, w2_q, w2_s, topk_w, expert_offsets, sorted_ids, M: int, k: int, stream=None):
-    """h binary16 [M*k, I] (expert-grouped, element = h * 2^10) -> out bf16 [M, H]."""
-    _need(h, torch.float16, "h")
+    """h bf16 [M*k, I] (expert-grouped, as moe_gate_up_swiglu writes it) -> out bf16 [M, H]."""
+    _need(h, torch.bfloat16, "h")
     E, H, _ = w2_q.shape
     I = h.shape[1]
     out = torch.empty((M, H), dtype=torch.bfloat16, device=h.device)

@@ -73,7 +73,7 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.status = take(256);
     L.splits = route_plan(M, H, E).splits;
     L.partial = take(static_cast<size_t>(L.splits) * M * E * sizeof(float));
-    L.x16 = take(static_cast<size_t>(M) * H * 2);
+    L.x_p4 = take(static_cast<size_t>(M) * H * 2);
     L.topk_ids = take(n * 4);
     L.topk_w = take(n * 4);
     L.offsets = take(static_cast<size_t>(E + 1) * 4);
@@ -83,13 +83,17 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.n_tiles = take(4);
     L.h = take(n * I * 2);
     L.y = take(n * H * sizeof(float));
-    L.wide = wide_enabled(M, H, I);
-    L.max_wide = L.wide ? static_cast<int>((n / kWideMinTokens < static_cast<size_t>(E) ? n / kWideMinTokens
-                                                                                         : static_cast<size_t>(E)) +
-                                           n / kWideTokens + 1)
-                        : 0;
-    L.wide_tiles = take(static_cast<size_t>(L.max_wide) * sizeof(WideTile));
-    L.n_wide = take(4);
+    L.wide = wide_enabled(M, H, I, E, k);
+    // small tensor-core tiles: one per expert with kWideMinTokens .. kWideSmallMax assignments;
+    // large: the experts with more, in tiles of up to kWideTokens
+    const size_t ne = static_cast<size_t>(E);
+    const size_t n_small = n / kWideMinTokens, n_big = n / (kWideSmallMax + 1);
+    L.max_small = L.wide ? static_cast<int>(n_small < ne ? n_small : ne) : 0;
+    L.max_large = L.wide ? static_cast<int>((n_big < ne ? n_big : ne) + n / kWideTokens + 1) : 0;
+    L.wide_small = take(static_cast<size_t>(L.max_small) * sizeof(WideTile));
+    L.n_wide_small = take(4);
+    L.wide_large = take(static_cast<size_t>(L.max_large) * sizeof(WideTile));
+    L.n_wide_large = take(4);
     L.x_perm = take(L.wide ? n * H * 2 : 0);
     L.total = off;
     return L;
@@ -175,8 +179,8 @@ static int make_scale_map(CUtensorMap *map, const void *base, uint64_t rows, uin
     return MOE_OK;
 }
 
-// binary16 activation rows [rows][K] (expert-grouped x or h) for the wide kernel: boxes of 16 rows
-// x 64 elements (128 bytes), 128-byte swizzle, the K-major operand layout of tcgen05.mma.
+// bf16 activation rows [rows][K] (expert-grouped x or h, P4 K order) for the wide kernel: boxes
+// of 16 rows x 64 elements (128 bytes), 128-byte swizzle, the K-major operand layout of tcgen05.mma.
 static int make_act_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t K)
 {
     EncodeTiledFn fn = encode_fn();
@@ -185,7 +189,7 @@ static int make_act_map(CUtensorMap *map, const void *base, uint64_t rows, uint6
     const cuuint64_t strides[1] = {K * 2};
     const cuuint32_t box[2] = {64, 16};
     const cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
@@ -231,9 +235,9 @@ static int library_workspace(cudaStream_t s, size_t need, char **out)
 
 // ------------------------------------------------------------------ step bodies (arguments already validated)
 
-static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x16, const ExpertTile *tiles,
-                       const int *n_tiles, __half *h, int *status, int32_t *status_out, int H, int I, int E, int k,
-                       int width, int max_tiles, cudaStream_t s, bool pdl)
+static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __nv_bfloat16 *x, const ExpertTile *tiles,
+                       const int *n_tiles, __nv_bfloat16 *h, bool h_p4, int *status, int32_t *status_out, int H,
+                       int I, int E, int k, int width, int max_tiles, cudaStream_t s, bool pdl)
 {
     CUtensorMap map, smap;
     // gate rows and up rows of an item are two boxes of kItemRows / 2 rows
@@ -246,24 +250,38 @@ static int run_gate_up(const void *w13_q, const uint8_t *w13_s, const __half *x1
                             kItemRows / 2);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_gate_up(map, smap, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, k, width, max_tiles, s,
-                           pdl));
+    MOE_TRY(launch_gate_up(map, smap, w13_s, x, tiles, n_tiles, h, h_p4, status, status_out, H, I, k, width, max_tiles,
+                           s, pdl));
     return MOE_OK;
 }
 
-// Optional per-launch event marks (profiling entry point only).
+// Optional per-launch event marks (profiling entry point only): an event before the first launch
+// and one after every launch, each launch's slot (moe.h, moe_mxfp4_forward_profile) remembering
+// the event that closes it.
 struct Marks {
     cudaEvent_t ev[MOE_PROFILE_KERNELS + 1];
+    int slot[MOE_PROFILE_KERNELS] = {};   // index of the event after the slot's launch; 0: not launched
     int n = 0;
-    cudaError_t mark(cudaStream_t s) { return cudaEventRecord(ev[n++], s); }
+    cudaError_t start(cudaStream_t s) { return cudaEventRecord(ev[n++], s); }
+    cudaError_t after(cudaStream_t s, int k)
+    {
+        slot[k] = n;
+        return cudaEventRecord(ev[n++], s);
+    }
 };
 
-#define MOE_MARK(m, s)                                  \
+enum ProfileSlot {
+    kProfLogits = 0, kProfSelect, kProfPermute, kProfGateUp, kProfGather, kProfGateUpTcSmall, kProfGateUpTcLarge,
+    kProfDown, kProfDownTcSmall, kProfDownTcLarge, kProfCombine
+};
+static_assert(kProfCombine + 1 == MOE_PROFILE_KERNELS, "one slot per launch kind");
+
+#define MOE_AFTER(m, s, k)                              \
     do {                                                \
-        if (m) MOE_TRY((m)->mark(s));                   \
+        if (m) MOE_TRY((m)->after((s), (k)));           \
     } while (0)
 
-static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, const int32_t *sorted_ids,
+static int run_down(const void *w2_q, const uint8_t *w2_s, const __nv_bfloat16 *h_p4, const int32_t *sorted_ids,
                     const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
                     int32_t *status_out, int H, int I, int E, int width, int max_tiles, cudaStream_t s, bool pdl)
 {
@@ -275,17 +293,18 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __half *h, cons
         rc = make_scale_map(&smap, w2_s, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 32, kItemRows);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_down(map, smap, w2_s, h, sorted_ids, tiles, n_tiles, y, status, status_out, H, I, width, max_tiles, s,
-                        pdl));
+    MOE_TRY(launch_down(map, smap, w2_s, h_p4, sorted_ids, tiles, n_tiles, y, status, status_out, H, I, width,
+                        max_tiles, s, pdl));
     return MOE_OK;
 }
 
 // The tensor-core path for the wide tiles of one projection (gate_up: x rows gathered into
-// expert-grouped order -> h; down: h -> y).  Weight boxes of 64 rows x 128 bytes, scale boxes
-// of 64 rows x 16 bytes (one 512-element stage), activation boxes of 16 rows x 64 elements.
-static int run_wide(bool gate_up, const void *wq, const uint8_t *ws_, const __half *act, const WideTile *wtiles,
-                    const int *n_wide, int max_wide, const int32_t *sorted_ids, __half *h, float *y,
-                    int *status, int32_t *status_out, int M, int H, int I, int E, int k, cudaStream_t s, bool pdl)
+// expert-grouped P4 order -> h; down: h (P4) -> y).  Weight boxes of 64 rows x 128 bytes, scale
+// boxes of 64 rows x 16 bytes (one 512-element stage), activation boxes of 16 rows x 64 elements.
+static int run_wide(bool gate_up, const void *wq, const uint8_t *ws_, const __nv_bfloat16 *act,
+                    const WideLists &wl, const int32_t *sorted_ids, __nv_bfloat16 *h, bool h_p4, float *y,
+                    int *status, int32_t *status_out, int M, int H, int I, int E, int k, cudaStream_t s, bool pdl,
+                    Marks *marks = nullptr)
 {
     CUtensorMap wmap, smap, bmap;
     const uint64_t rows = gate_up ? static_cast<uint64_t>(E) * 2 * I : static_cast<uint64_t>(E) * H;
@@ -294,9 +313,26 @@ static int run_wide(bool gate_up, const void *wq, const uint8_t *ws_, const __ha
     if (rc == MOE_OK) rc = make_scale_map(&smap, ws_, rows, K / 32, 64, kWideStageK / 32);
     if (rc == MOE_OK) rc = make_act_map(&bmap, act, static_cast<uint64_t>(M) * k, K);
     if (rc != MOE_OK) return rc;
-    MOE_TRY(launch_wide(gate_up, wmap, smap, bmap, wtiles, n_wide, max_wide, sorted_ids, h, y, status, status_out, H,
-                        I, s, pdl));
+    // small tiles, then large ones (two launches: each kernel splits tensor memory for its tile size)
+    MOE_TRY(launch_wide(gate_up, true, wmap, smap, bmap, wl.small, wl.n_small, wl.max_small, sorted_ids, h, h_p4, y,
+                        status, status_out, H, I, s, pdl));
+    MOE_AFTER(marks, s, gate_up ? kProfGateUpTcSmall : kProfDownTcSmall);
+    MOE_TRY(launch_wide(gate_up, false, wmap, smap, bmap, wl.large, wl.n_large, wl.max_large, sorted_ids, h, h_p4, y,
+                        status, status_out, H, I, s, pdl));
+    MOE_AFTER(marks, s, gate_up ? kProfGateUpTcLarge : kProfDownTcLarge);
     return MOE_OK;
+}
+
+static WideLists wide_lists(char *ws, const Layout &L)
+{
+    WideLists wl;
+    wl.small = reinterpret_cast<WideTile *>(ws + L.wide_small);
+    wl.n_small = reinterpret_cast<int *>(ws + L.n_wide_small);
+    wl.large = reinterpret_cast<WideTile *>(ws + L.wide_large);
+    wl.n_large = reinterpret_cast<int *>(ws + L.n_wide_large);
+    wl.max_small = L.max_small;
+    wl.max_large = L.max_large;
+    return wl;
 }
 
 static int forward_impl(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
@@ -306,7 +342,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
 {
     int *status = reinterpret_cast<int *>(ws + L.status);
     float *partial = reinterpret_cast<float *>(ws + L.partial);
-    __half *x16 = reinterpret_cast<__half *>(ws + L.x16);
+    __nv_bfloat16 *x_p4 = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_p4);   // x in P4 K order (router)
     int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(ws + L.topk_ids);
     float *tw = topk_w_out ? topk_w_out : reinterpret_cast<float *>(ws + L.topk_w);
     int32_t *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
@@ -314,53 +350,54 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     int32_t *inv_pos = reinterpret_cast<int32_t *>(ws + L.inv_pos);
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
-    __half *h = reinterpret_cast<__half *>(ws + L.h);
+    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(ws + L.h);   // P4 K order
     float *y = reinterpret_cast<float *>(ws + L.y);
-    WideTile *wtiles = reinterpret_cast<WideTile *>(ws + L.wide_tiles);
-    int *n_wide = reinterpret_cast<int *>(ws + L.n_wide);
-    __half *x_perm = reinterpret_cast<__half *>(ws + L.x_perm);
-    const TileOut to{tiles, n_tiles, L.wide ? wtiles : nullptr, n_wide, L.width};
+    const WideLists wl = wide_lists(ws, L);
+    __nv_bfloat16 *x_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_perm);
+    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width};
     // The first kernel is ordered after everything before it on the stream; each later
     // kernel of the call is launched early (programmatic dependent launch) and waits on
     // device for its predecessor.  Event marks (profiling) break that overlap, so the
     // profiling entry point launches without it.
     const bool pdl = (marks == nullptr);
 
-    MOE_MARK(marks, s);
-    MOE_TRY(launch_route_logits(x, router_w, partial, x16, status, status_out, M, H, E, s));
-    MOE_MARK(marks, s);
+    if (marks) MOE_TRY(marks->start(s));
+    MOE_TRY(launch_route_logits(x, router_w, partial, x_p4, status, status_out, M, H, E, s));
+    MOE_AFTER(marks, s, kProfLogits);
     if (fused_select(M, E, k)) {
         MOE_TRY(launch_route_select_permute(partial, L.splits, router_bias, ids, tw, offsets, sorted_ids, inv_pos, to, M,
                                             E, k, s, pdl));
-        MOE_MARK(marks, s);
+        MOE_AFTER(marks, s, kProfSelect);
     } else {
         MOE_TRY(launch_route_topk(partial, L.splits, router_bias, ids, tw, M, E, k, s, pdl));
-        MOE_MARK(marks, s);
+        MOE_AFTER(marks, s, kProfSelect);
         MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, to, M, E, k, s, pdl));
+        MOE_AFTER(marks, s, kProfPermute);
     }
-    MOE_MARK(marks, s);
-    // gate_up: the 8-assignment tiles on mma.sync, then (large M) the wide tiles on tcgen05
-    int rc = run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, h, status, status_out, H, I, E, k, L.width, L.max_tiles, s,
-                         pdl);
+    // gate_up: the 8/16-assignment tiles on mma.sync, then (large M) the tensor-core tiles
+    int rc = run_gate_up(w13_q, w13_s, x_p4, tiles, n_tiles, h, true, status, status_out, H, I, E, k, L.width,
+                         L.max_tiles, s, pdl);
     if (rc != MOE_OK) return rc;
+    MOE_AFTER(marks, s, kProfGateUp);
     if (L.wide) {
-        MOE_TRY(launch_gather_rows(x16, sorted_ids, x_perm, M * k, H, k, s, pdl));
-        rc = run_wide(true, w13_q, w13_s, x_perm, wtiles, n_wide, L.max_wide, sorted_ids, h, y, status, status_out,
-                      M, H, I, E, k, s, pdl);
+        MOE_TRY(launch_gather_wide_rows(x_p4, sorted_ids, wl, x_perm, H, k, s, pdl));
+        MOE_AFTER(marks, s, kProfGather);
+        rc = run_wide(true, w13_q, w13_s, x_perm, wl, sorted_ids, h, true, y, status, status_out, M, H, I, E, k, s,
+                      pdl, marks);
         if (rc != MOE_OK) return rc;
     }
-    MOE_MARK(marks, s);
     // down likewise, then the weighted top-k combine
     rc = run_down(w2_q, w2_s, h, sorted_ids, tiles, n_tiles, y, status, status_out, H, I, E, L.width, L.max_tiles, s,
                   pdl);
     if (rc != MOE_OK) return rc;
+    MOE_AFTER(marks, s, kProfDown);
     if (L.wide) {
-        rc = run_wide(false, w2_q, w2_s, h, wtiles, n_wide, L.max_wide, sorted_ids, h, y, status, status_out, M, H, I,
-                      E, k, s, pdl);
+        rc = run_wide(false, w2_q, w2_s, h, wl, sorted_ids, nullptr, true, y, status, status_out, M, H, I, E, k, s,
+                      pdl, marks);
         if (rc != MOE_OK) return rc;
     }
     MOE_TRY(launch_combine(y, tw, out, M, H, k, s, pdl));
-    MOE_MARK(marks, s);
+    MOE_AFTER(marks, s, kProfCombine);
     return MOE_OK;
 }
 
@@ -423,8 +460,8 @@ int moe_forward_launches(int M, int H, int I, int E, int k)
     const int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
     if (M == 0) return 0;
-    // route_logits, select (+ permute), gate_up, down, combine; gather + two wide GEMMs
-    return (fused_select(M, E, k) ? 5 : 6) + (wide_enabled(M, H, I) ? 3 : 0);
+    // route_logits, select (+ permute), gate_up, down, combine; gather + four tensor-core GEMMs
+    return (fused_select(M, E, k) ? 5 : 6) + (wide_enabled(M, H, I, E, k) ? 5 : 0);
 }
 
 int moe_route(const void *x_bf16, const float *router_w, const float *router_bias, int32_t *topk_ids, float *topk_w,
@@ -459,48 +496,59 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
     if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
         return MOE_ERR_INVALID_ARG;
     if (M == 0) return MOE_OK;
-    const TileOut none{nullptr, nullptr, nullptr, nullptr, 8};
+    const TileOut none{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 8};
     MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, none, M, E, k, stream, false));
     return MOE_OK;
 }
 
 int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *w13_s, const int32_t *expert_offsets,
-                       const int32_t *sorted_ids, void *h_f16, int M, int H, int I, int E, int k, cudaStream_t stream)
+                       const int32_t *sorted_ids, void *h_bf16, int M, int H, int I, int E, int k, cudaStream_t stream)
 {
     int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
     if (M == 0) return MOE_OK;
-    if (!x_bf16 || !w13_q || !w13_s || !expert_offsets || !sorted_ids || !h_f16) return MOE_ERR_INVALID_ARG;
-    if (!aligned(x_bf16, 16) || !aligned(w13_q, 16) || !aligned(w13_s, 16) || !aligned(h_f16, 16) ||
+    if (!x_bf16 || !w13_q || !w13_s || !expert_offsets || !sorted_ids || !h_bf16) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(w13_q, 16) || !aligned(w13_s, 16) || !aligned(h_bf16, 16) ||
         !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4))
         return MOE_ERR_INVALID_ARG;
-    if (M == 0) return MOE_OK;
     const Layout L = make_layout(M, H, I, E, k);
     char *ws = nullptr;
     rc = library_workspace(stream, L.total, &ws);
     if (rc != MOE_OK) return rc;
     int *status = reinterpret_cast<int *>(ws + L.status);
-    __half *x16 = reinterpret_cast<__half *>(ws + L.x16);
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
-    MOE_TRY(launch_convert_x(x_bf16, x16, status, M, H, stream));
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, L.width, stream));
-    return run_gate_up(w13_q, w13_s, x16, tiles, n_tiles, static_cast<__half *>(h_f16), status, nullptr, H, I, E, k,
-                       L.width, L.max_tiles, stream, false);
+    const WideLists wl = wide_lists(ws, L);
+    __nv_bfloat16 *x_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_perm);
+    __nv_bfloat16 *x_p4 = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_p4);
+    __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(h_bf16);
+    // the same tiles as a whole-layer call (mma.sync tiles, and tensor-core tiles)
+    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width};
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, to, status, E, stream));
+    // x into the P4 K order the grouped GEMMs read (the whole layer's router writes it)
+    MOE_TRY(launch_rows_to_p4(static_cast<const __nv_bfloat16 *>(x_bf16), x_p4, static_cast<size_t>(M), H, stream));
+    rc = run_gate_up(w13_q, w13_s, x_p4, tiles, n_tiles, h, false, status, nullptr, H, I, E, k, L.width, L.max_tiles,
+                     stream, false);
+    if (rc != MOE_OK) return rc;
+    if (L.wide) {
+        MOE_TRY(launch_gather_wide_rows(x_p4, sorted_ids, wl, x_perm, H, k, stream, false));
+        rc = run_wide(true, w13_q, w13_s, x_perm, wl, sorted_ids, h, false, nullptr, status, nullptr, M, H, I, E, k,
+                      stream, false);
+    }
+    return rc;
 }
 
-int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
+int moe_down_combine(const void *h_bf16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
                      const int32_t *expert_offsets, const int32_t *sorted_ids, void *out_bf16, int M, int H, int I,
                      int E, int k, cudaStream_t stream)
 {
     int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
     if (M == 0) return MOE_OK;
-    if (!h_f16 || !w2_q || !w2_s || !topk_w || !expert_offsets || !sorted_ids || !out_bf16) return MOE_ERR_INVALID_ARG;
-    if (!aligned(h_f16, 16) || !aligned(w2_q, 16) || !aligned(w2_s, 16) || !aligned(out_bf16, 16) ||
+    if (!h_bf16 || !w2_q || !w2_s || !topk_w || !expert_offsets || !sorted_ids || !out_bf16) return MOE_ERR_INVALID_ARG;
+    if (!aligned(h_bf16, 16) || !aligned(w2_q, 16) || !aligned(w2_s, 16) || !aligned(out_bf16, 16) ||
         !aligned(topk_w, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4))
         return MOE_ERR_INVALID_ARG;
-    if (M == 0) return MOE_OK;
     const Layout L = make_layout(M, H, I, E, k);
     char *ws = nullptr;
     rc = library_workspace(stream, L.total, &ws);
@@ -508,11 +556,22 @@ int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s
     int *status = reinterpret_cast<int *>(ws + L.status);
     ExpertTile *tiles = reinterpret_cast<ExpertTile *>(ws + L.tiles);
     int *n_tiles = reinterpret_cast<int *>(ws + L.n_tiles);
+    const WideLists wl = wide_lists(ws, L);
+    __nv_bfloat16 *h_p4 = reinterpret_cast<__nv_bfloat16 *>(ws + L.h);
     float *y = reinterpret_cast<float *>(ws + L.y);
-    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, tiles, n_tiles, status, E, L.width, stream));
-    rc = run_down(w2_q, w2_s, static_cast<const __half *>(h_f16), sorted_ids, tiles, n_tiles, y, status, nullptr, H, I,
-                  E, L.width, L.max_tiles, stream, false);
+    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width};
+    MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, to, status, E, stream));
+    // the caller's h rows (natural K order) into the P4 order the down kernels read
+    MOE_TRY(launch_rows_to_p4(static_cast<const __nv_bfloat16 *>(h_bf16), h_p4, static_cast<size_t>(M) * k, I,
+                              stream));
+    rc = run_down(w2_q, w2_s, h_p4, sorted_ids, tiles, n_tiles, y, status, nullptr, H, I, E, L.width, L.max_tiles,
+                  stream, false);
     if (rc != MOE_OK) return rc;
+    if (L.wide) {
+        rc = run_wide(false, w2_q, w2_s, h_p4, wl, sorted_ids, nullptr, true, y, status, nullptr, M, H, I, E, k,
+                      stream, false);
+        if (rc != MOE_OK) return rc;
+    }
     MOE_TRY(launch_combine(y, topk_w, out_bf16, M, H, k, stream, false));
     return MOE_OK;
 }
@@ -555,9 +614,10 @@ int moe_mxfp4_forward_profile(const void *x, const float *router_w, const float 
         rc = forward_impl(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, topk_ids_out,
                           topk_w_out, status_out, static_cast<char *>(workspace), L, stream, &marks);
         if (rc == MOE_OK) {
-            e = cudaEventSynchronize(marks.ev[MOE_PROFILE_KERNELS]);
+            e = cudaEventSynchronize(marks.ev[marks.n - 1]);
             for (int i = 0; i < MOE_PROFILE_KERNELS && e == cudaSuccess; ++i)
-                e = cudaEventElapsedTime(&kernel_ms[i], marks.ev[i], marks.ev[i + 1]);
+                if (marks.slot[i] > 0)
+                    e = cudaEventElapsedTime(&kernel_ms[i], marks.ev[marks.slot[i] - 1], marks.ev[marks.slot[i]]);
         }
     } else {
         --created;

@@ -27,16 +27,18 @@
 //    with a 128-byte swizzle into a 3-stage ring of 32 KB; in the same stage a TMA
 //    box of the matching E8M0 scales (when scale rows are 16-byte multiples, else
 //    the item's scale rows once per item), and one 1-D bulk copy per tile token of
-//    its binary16 activation chunk (the routed gather: x rows for gate_up, h rows
+//    its bf16 activation chunk (the routed gather: x rows for gate_up, h rows
 //    for down).
 //  * 16 compute warps = 2 m-tile pairs x 8 K slots.  Per stage a warp takes 4 of
 //    the 32 blocks of 32 K for its 2 m-tiles: a thread reads the 32-bit word q of
-//    its rows' 16-byte block (conflict-free thanks to the swizzle), decodes it with
-//    the hardware E2M1 -> f16x2 conversion straight into MMA A-fragment registers,
-//    and runs two m16n8k16 f16 MMAs per block.  Inside a block the K order is
-//    permuted (thread q's word covers K 8q..8q+7) identically for A and for the
-//    activation fragment, so each MMA pair spans exactly one scale block and the
-//    E8M0 scale is applied once to the fp32 partial sum.  With 16-assignment tiles
+//    its rows' 16-byte block (conflict-free thanks to the swizzle), decodes it
+//    exactly to bf16 (e2m1x8_to_bf16x2_p4) straight into MMA A-fragment registers,
+//    and runs two m16n8k16 bf16 MMAs per block.  Inside a block the K order is
+//    permuted identically for A and for the activation fragment: thread q's word
+//    covers K 8q..8q+7, its registers pair K 8q+i with 8q+i+4, and the activation
+//    rows are stored in that same P4 order (x by the router, h by gate_up).  So
+//    each MMA pair spans exactly one scale block, and the E8M0 scale multiplies the
+//    block's fp32 partial once (exact: a power of two).  With 16-assignment tiles
 //    each decoded fragment feeds two MMA n-tiles.  At the end of an item a warp
 //    parks its partial sums in a reduction area (two buffers for 8-wide tiles; one
 //    for 16-wide, where the K slots first add up in pairs) and moves on.
@@ -47,10 +49,9 @@
 //    path.  The item's position range reaches them from the producer through shared
 //    memory.  The weighted top-k combine that follows is its own small kernel
 //    (combine_kernel).
-// Activations (x or h) are read as binary16; bf16 x converts exactly for
-// 2^-17 <= |x| <= 65504, h is stored scaled by 2^10 (exact for |h| >= 2^-27,
-// |h| <= 49 so no overflow), E2M1 values are exact in binary16, and products
-// accumulate in fp32.
+// Both MMA operands are bf16: x as the caller gives it and h as gate_up rounds it (both
+// stored in the P4 K order of common.cuh), and the weights decoded exactly (every E2M1
+// value is a bf16 value); products accumulate in fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -114,19 +115,13 @@ __device__ __forceinline__ float clamp_swiglu(float g, float u)
     return a / (1.0f + expf(-a)) * c;
 }
 
-// bf16 round-to-nearest-even, then the exact move into binary16 with the 2^10 storage scale
-__device__ __forceinline__ __half store_h(float v)
-{
-    return __float2half_rn(__bfloat162float(__float2bfloat16_rn(v)) * kHScale);
-}
-
 template <bool kGateUp, int kN>
 __global__ void __launch_bounds__(Tiling<kN>::kThreads, 1)
 grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
-                     const uint8_t *__restrict__ wscale, const __half *__restrict__ act,
+                     const uint8_t *__restrict__ wscale, const __nv_bfloat16 *__restrict__ act,
                      const int32_t *__restrict__ sorted_ids, const ExpertTile *__restrict__ tiles, const int *__restrict__ n_tiles_ptr,
-                     __half *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out,
-                     int *queue, int K, int I, int H, int k)
+                     __nv_bfloat16 *__restrict__ hout, float *__restrict__ yout, int *status_ws, int32_t *status_out,
+                     int *queue, int K, int I, int H, int k, int h_p4)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -216,7 +211,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         };
         // down: h copies of the first stages, held back until gate_up has completed
         bool h_ready = kGateUp;
-        const __half *pend_src[kStages];
+        const __nv_bfloat16 *pend_src[kStages];
         uint32_t pend_bytes[kStages];
 #pragma unroll
         for (int i = 0; i < kStages; ++i) pend_bytes[i] = 0;
@@ -271,7 +266,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
             const int row_b = row_a + I;                               // gate_up only
             const int valid_rows = kGateUp ? kItemRows : min(kItemRows, H - rb * kItemRows);
             // this lane's activation row (gate_up: the x row of the slot's token; down: the h row)
-            const __half *arow = kGateUp ? act + static_cast<size_t>(flat / k) * K
+            const __nv_bfloat16 *arow = kGateUp ? act + static_cast<size_t>(flat / k) * K
                                          : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
             if (!stage_scales) {
                 const int b = item_ctr & 1;
@@ -321,7 +316,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     if (kGateUp) tma_load_2d(ss + kScaleBoxBytes, &smap, kc / 32, row_b, &full[s]);
                 }
                 if (lane >= 16 && lane - 16 < cnt) {
-                    const __half *src = (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc;
+                    const __nv_bfloat16 *src = (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc;
                     if (h_ready) {
                         bulk_load(ast + s * kActStageBytes + (lane - 16) * kActPitch, src, act_bytes, &full[s]);
                     } else {
@@ -410,26 +405,25 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     const float4 sum = sums[m][hf];
                     const int li0 = 8 * hf + 2 * q, li1 = li0 + 1;   // the fragment's two tile slots
                     if (kGateUp) {
-                        // remove the factor 2 carried by e8m0_times2
+                        // h rounded to bf16 once, at column n (P4 storage order for the down kernels)
                         const int n = rb * 32 + 8 * j + g;
+                        const int col = h_p4 ? p4_pos(n) : n;
                         if (li0 < cnt)
-                            hout[static_cast<size_t>(p0 + li0) * I + n] = store_h(clamp_swiglu(0.5f * sum.x, 0.5f * sum.z));
+                            hout[static_cast<size_t>(p0 + li0) * I + col] = __float2bfloat16_rn(clamp_swiglu(sum.x, sum.z));
                         if (li1 < cnt)
-                            hout[static_cast<size_t>(p0 + li1) * I + n] = store_h(clamp_swiglu(0.5f * sum.y, 0.5f * sum.w));
+                            hout[static_cast<size_t>(p0 + li1) * I + col] = __float2bfloat16_rn(clamp_swiglu(sum.y, sum.w));
                     } else {
-                        // remove e8m0_times2's factor 2 and h's 2^10 storage scale; the routing
-                        // weight is applied by the combine
-                        const float unscale = 0.5f / kHScale;
+                        // the unweighted row; the routing weight is applied by the combine
                         const int ra = rb * kItemRows + 16 * j + g, rbw = ra + 8;
                         if (li0 < cnt) {
                             float *yr = yout + static_cast<size_t>(sorted_ids[p0 + li0]) * H;
-                            if (ra < rows_total) yr[ra] = unscale * sum.x;
-                            if (rbw < rows_total) yr[rbw] = unscale * sum.z;
+                            if (ra < rows_total) yr[ra] = sum.x;
+                            if (rbw < rows_total) yr[rbw] = sum.z;
                         }
                         if (li1 < cnt) {
                             float *yr = yout + static_cast<size_t>(sorted_ids[p0 + li1]) * H;
-                            if (ra < rows_total) yr[ra] = unscale * sum.y;
-                            if (rbw < rows_total) yr[rbw] = unscale * sum.w;
+                            if (ra < rows_total) yr[ra] = sum.y;
+                            if (rbw < rows_total) yr[rbw] = sum.w;
                         }
                     }
                 }
@@ -444,8 +438,8 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     const int mgrp = warp % kGroups;        // m-tiles mgrp*kWarpMTiles ..
     const int kslot = warp / kGroups;       // blocks kslot*kBlocksPerWarp .. of every stage
     const int col = (kslot * kBlocksPerWarp) >> 3;
-    const int bb0 = (kslot * kBlocksPerWarp) & 7;
     const float zero4[4] = {0.f, 0.f, 0.f, 0.f};
+    const int bb0 = (kslot * kBlocksPerWarp) & 7;
 
     // per m-tile: smem byte offsets (inside a stage) of the top/bottom rows' 16-byte blocks,
     // and scale-row indices (rows of the item's 64 weight rows)
@@ -502,6 +496,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 #pragma unroll
             for (int bi = 0; bi < kBlocksPerWarp; ++bi) {
                 if (c * kBlocksPerStage + blk_base + bi >= kblocks) continue;
+                // K 8q..8q+7 of token g (and g + 8), stored in P4 order like the decoded weights
                 const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (blk_base + bi) + 8 * q) * 2);
                 uint4 xc = make_uint4(0u, 0u, 0u, 0u);   // token g + 8 (second n-tile)
                 if (kN == 16 && two)
@@ -511,24 +506,27 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 for (int m = 0; m < kWarpMTiles; ++m) {
                     const uint32_t wt = *reinterpret_cast<const uint32_t *>(st + top_off[m] + sw);
                     const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_off[m] + sw);
-                    const float st_scale = e8m0_times2(sc_base[top_sr[m] * s_pitch + sc_col0 + bi]);
-                    const float sb_scale = e8m0_times2(sc_base[bot_sr[m] * s_pitch + sc_col0 + bi]);
-                    uint32_t t0, t1, t2, t3, u0, u1, u2, u3;
-                    e2m1x8_to_f16x2(wt, t0, t1, t2, t3);
-                    e2m1x8_to_f16x2(wb, u0, u1, u2, u3);
-                    const uint32_t a0[4] = {t0, u0, t1, u1};
-                    const uint32_t a1[4] = {t2, u2, t3, u3};
+                    const float st_scale = e8m0_scale(sc_base[top_sr[m] * s_pitch + sc_col0 + bi]);
+                    const float sb_scale = e8m0_scale(sc_base[bot_sr[m] * s_pitch + sc_col0 + bi]);
+                    uint32_t t[4], u[4];
+                    e2m1x8_to_bf16x2_p4(wt, t);
+                    e2m1x8_to_bf16x2_p4(wb, u);
+                    // registers i = K (8q+i, 8q+i+4): the first MMA takes i = 0, 1, the second 2, 3.
+                    // Each block's MMA pair starts from zero (no dependence on the previous block's
+                    // MMAs) and its fp32 partial times the block scale (exact) joins the K slot's sums.
+                    const uint32_t a0[4] = {t[0], u[0], t[1], u[1]};
+                    const uint32_t a1[4] = {t[2], u[2], t[3], u[3]};
                     float tmp[4];
-                    mma_f16_16816(tmp, a0, xb.x, xb.y, zero4);
-                    mma_f16_16816(tmp, a1, xb.z, xb.w, tmp);
+                    mma_bf16_16816(tmp, a0, xb.x, xb.y, zero4);
+                    mma_bf16_16816(tmp, a1, xb.z, xb.w, tmp);
                     acc[m][0] = fmaf(tmp[0], st_scale, acc[m][0]);
                     acc[m][1] = fmaf(tmp[1], st_scale, acc[m][1]);
                     acc[m][2] = fmaf(tmp[2], sb_scale, acc[m][2]);
                     acc[m][3] = fmaf(tmp[3], sb_scale, acc[m][3]);
                     if (kN == 16 && two) {
                         float tmq[4];
-                        mma_f16_16816(tmq, a0, xc.x, xc.y, zero4);
-                        mma_f16_16816(tmq, a1, xc.z, xc.w, tmq);
+                        mma_bf16_16816(tmq, a0, xc.x, xc.y, zero4);
+                        mma_bf16_16816(tmq, a1, xc.z, xc.w, tmq);
                         acc[m][kVals - 4] = fmaf(tmq[0], st_scale, acc[m][kVals - 4]);
                         acc[m][kVals - 3] = fmaf(tmq[1], st_scale, acc[m][kVals - 3]);
                         acc[m][kVals - 2] = fmaf(tmq[2], sb_scale, acc[m][kVals - 2]);
@@ -630,9 +628,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
 
 template <bool kGateUp, int kN>
 static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &smap, const uint8_t *scales,
-                                  const __half *act, const int32_t *sorted_ids, const ExpertTile *tiles,
-                                  const int *n_tiles, __half *h, float *y, int *status, int32_t *status_out, int K,
-                                  int I, int H, int k, int max_tiles, cudaStream_t s, bool pdl)
+                                  const __nv_bfloat16 *act, const int32_t *sorted_ids, const ExpertTile *tiles,
+                                  const int *n_tiles, __nv_bfloat16 *h, float *y, int *status, int32_t *status_out,
+                                  int K, int I, int H, int k, int h_p4, int max_tiles, cudaStream_t s, bool pdl)
 {
     const SmemPlan plan = smem_plan<kN>(K);
     auto kern = grouped_mxfp4_kernel<kGateUp, kN>;
@@ -644,32 +642,33 @@ static cudaError_t launch_grouped(const CUtensorMap &map, const CUtensorMap &sma
     if (grid < 1) grid = 1;
     int *queue = status + (kGateUp ? kQueueGateUp : kQueueDown);
     return launch_ex(kern, dim3(grid), dim3(Tiling<kN>::kThreads), plan.total, s, pdl, map, smap, scales, act,
-                     sorted_ids, tiles, n_tiles, h, y, status, status_out, queue, K, I, H, k);
+                     sorted_ids, tiles, n_tiles, h, y, status, status_out, queue, K, I, H, k, h_p4);
 }
 
 int grouped_smem_bytes(int K, int width) { return width == 16 ? smem_plan<16>(K).total : smem_plan<8>(K).total; }
 
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
-                           const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
-                           int32_t *status_out, int H, int I, int k, int width, int max_tiles, cudaStream_t s,
-                           bool pdl)
+                           const __nv_bfloat16 *x, const ExpertTile *tiles, const int *n_tiles, __nv_bfloat16 *h,
+                           bool h_p4, int *status, int32_t *status_out, int H, int I, int k, int width, int max_tiles,
+                           cudaStream_t s, bool pdl)
 {
     if (width == 16)
-        return launch_grouped<true, 16>(w13_map, s13_map, w13_s, x16, nullptr, tiles, n_tiles, h, nullptr, status,
-                                        status_out, H, I, H, k, max_tiles, s, pdl);
-    return launch_grouped<true, 8>(w13_map, s13_map, w13_s, x16, nullptr, tiles, n_tiles, h, nullptr, status,
-                                   status_out, H, I, H, k, max_tiles, s, pdl);
+        return launch_grouped<true, 16>(w13_map, s13_map, w13_s, x, nullptr, tiles, n_tiles, h, nullptr, status,
+                                        status_out, H, I, H, k, h_p4 ? 1 : 0, max_tiles, s, pdl);
+    return launch_grouped<true, 8>(w13_map, s13_map, w13_s, x, nullptr, tiles, n_tiles, h, nullptr, status,
+                                   status_out, H, I, H, k, h_p4 ? 1 : 0, max_tiles, s, pdl);
 }
 
-cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
-                        int32_t *status_out, int H, int I, int width, int max_tiles, cudaStream_t s, bool pdl)
+cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s,
+                        const __nv_bfloat16 *h_p4, const int32_t *sorted_ids, const ExpertTile *tiles,
+                        const int *n_tiles, float *y, int *status, int32_t *status_out, int H, int I, int width,
+                        int max_tiles, cudaStream_t s, bool pdl)
 {
     if (width == 16)
-        return launch_grouped<false, 16>(w2_map, s2_map, w2_s, h, sorted_ids, tiles, n_tiles, nullptr, y, status,
-                                         status_out, I, I, H, 1, max_tiles, s, pdl);
-    return launch_grouped<false, 8>(w2_map, s2_map, w2_s, h, sorted_ids, tiles, n_tiles, nullptr, y, status,
-                                    status_out, I, I, H, 1, max_tiles, s, pdl);
+        return launch_grouped<false, 16>(w2_map, s2_map, w2_s, h_p4, sorted_ids, tiles, n_tiles, nullptr, y, status,
+                                         status_out, I, I, H, 1, 1, max_tiles, s, pdl);
+    return launch_grouped<false, 8>(w2_map, s2_map, w2_s, h_p4, sorted_ids, tiles, n_tiles, nullptr, y, status,
+                                    status_out, I, I, H, 1, 1, max_tiles, s, pdl);
 }
 
 cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,

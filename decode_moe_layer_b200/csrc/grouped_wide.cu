@@ -7,38 +7,50 @@
 // the page's "Decision" section.  At large token counts the expert GEMMs become real dense
 // contractions: an expert with many assignments is streamed once for all of them (the narrow
 // kernel in grouped_gemm.cu re-streams it for every 8 or 16 assignments), and the MMA runs on
-// tcgen05 with the fp32 accumulator in tensor memory.  The kernel keeps a kWideTokens-wide tile of
-// one expert's assignments against 128 weight rows per item, and the wider the tile the more
-// work each MMA instruction does (their issue cost hardly depends on N).
+// tcgen05 with the fp32 accumulator in tensor memory.  An item is one tile of an expert's
+// assignments against 128 weight rows.
 //
-// One persistent CTA per SM, 16 warps:
+// Measured on this part (one CTA per SM issuing back to back): a kind::f16 MMA of 128 x N x 16
+// with A in tensor memory takes about 40-50 cycles for N <= 64 and N / 2 above; every
+// tcgen05.commit costs the issuing thread about 80 cycles and every mbarrier wait about 185, even
+// on a completed phase.  So the dequant warps hand the MMA warp large A units (a wait and a commit
+// cover 8 or 16 MMAs), and the tensor memory is split by tile size (two kernels):
+//  * small tiles (kWideMinTokens .. kWideSmallMax assignments): two 64-column accumulators and
+//    three A units of 256 K (128 columns each);
+//  * large tiles (up to kWideTokens): two 192-column accumulators and two A units of 128 K.
+//
+// One persistent CTA per SM, 20 warps:
 //  * warp 0 (weights producer): per 512-K stage, TMA copies of the item's packed E2M1 rows
 //    (128 rows x 256 bytes, 128-byte swizzle) and their E8M0 scales into a 3-stage ring;
 //    items come from the call's work queue, the ids reach the other warps through shared
 //    memory with the stage arrivals.
-//  * warp 2 (activations producer): per 64-K sub-tile, TMA copies of the item's activation
-//    rows (x gathered into expert-grouped order for gate_up, h for down), 16 rows per box,
-//    128-byte swizzle, into a 4-slot ring.  Rows past the tile are read and ignored.
-//  * warps 4..11 (dequant): per 64-K sub-tile, 256 threads each decode 32 weights of one row
-//    (hardware E2M1 -> f16x2), apply the row's E8M0 block scale in f16 (exact for scale bytes
-//    104..140: every scaled E2M1 value is then an f16 normal or subnormal; other bytes are
-//    flagged), and store them with tcgen05.st into an A buffer in tensor memory (TMEM lane =
-//    A row; a warp reaches the 32 lanes of its warp index mod 4, and warps 4..7 / 8..11 take
-//    the low / high 32 K of the sub-tile).  gate_up interleaves gate row i and up row i as A
-//    rows 2i, 2i+1, so one TMEM lane pair holds g and u.  A never passes through shared
-//    memory, which leaves shared-memory bandwidth to the TMA copies and the B operand.
-//  * warp 1 (MMA): one thread issues 4 tcgen05.mma kind::f16 (A from TMEM, B from shared
-//    memory; M 128, N = the tile's tokens rounded up to 16, K 16) per sub-tile into one of two
-//    TMEM accumulators and commits the consumed A and B buffers and, per item, the
+//  * warp 2 (activations producer): TMA copies of the item's activation rows (x gathered into
+//    expert-grouped order for gate_up, h for down), 16 rows x 64 K per box, 128-byte swizzle,
+//    into a 4-slot ring; a slot takes 1 to 8 consecutive 64-K sub-tiles, as many as fit, so
+//    that narrow tiles keep many sub-tiles in flight against the copies' latency.  Rows past
+//    the tile are read and ignored.
+//  * warps 4..15 (dequant, three groups of four): a group decodes a whole A unit, each thread
+//    the weights of one row, to bf16 with the row's E8M0 block scales folded in
+//    (mxfp4x8_to_bf16x2_p4: exact for every scale byte whose scaled values are bf16 values),
+//    and stores them with tcgen05.st into the unit's A buffer in tensor memory (TMEM lane = A
+//    row; a warp reaches the 32 lanes of its warp index mod 4).  The groups take units in turn
+//    (group g always unit g), so one group's store latency overlaps the others' decoding.  The decode pairs K 8j+i with
+//    8j+i+4 in a TMEM column, so the activation rows are stored in the matching P4 K order
+//    (common.cuh): x by the router (gathered into x_perm by gather_wide_rows_kernel), h by the
+//    gate_up epilogues.  gate_up interleaves gate row i and up row i as A rows 2i, 2i+1, so one
+//    TMEM lane pair holds g and u.  A never passes through shared memory, which leaves
+//    shared-memory bandwidth to the TMA copies and the B operand.
+//  * warp 1 (MMA): one thread issues the unit's tcgen05.mma kind::f16 with bf16 operands (A
+//    from TMEM, B from shared memory; M 128, N = the tile's tokens rounded up to 16, K 16) into
+//    one of two TMEM accumulators, commits the consumed A unit and B slots and, per item, the
 //    accumulator.
-//  * warps 12..15 (epilogue): tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//  * warps 16..19 (epilogue): tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //    32 (w % 4) ..); gate_up pairs g and u with one shuffle, applies clamp-SwiGLU and the bf16
-//    rounding and stores h; down stores the assignment's fp32 row of y (the combine applies
-//    the routing weight).
+//    rounding and stores h (bf16); down stores the assignment's fp32 row of y (the combine
+//    applies the routing weight).
 // Every wait is bounded; after a timeout the kernel records MOE_ERR_TIMEOUT, drains the
 // copies it issued and frees its tensor memory.
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "tcgen05.cuh"
@@ -49,31 +61,59 @@ namespace wide {
 constexpr int kRows = 128;                               // weight rows per item (MMA M)
 constexpr int kStageK = kWideStageK;                     // 512 K per packed stage
 constexpr int kPStages = 3;                              // packed weight stages
-constexpr int kSubK = 64;                                // K per A/B sub-tile (one swizzle atom of f16)
+constexpr int kSubK = 64;                                // K per B sub-tile (one 128-byte swizzle atom of bf16)
 constexpr int kSubs = kStageK / kSubK;                   // 8
-// A tcgen05.mma costs about the same issue time for any N, so N is as large as TMEM allows:
-// two accumulators of kWideTokens columns plus the A buffers.
-constexpr int kABufs = 2, kBBufs = 4, kDBufs = 2;
+constexpr int kBBufs = 4, kDBufs = 2;
 constexpr int kItemQ = 8;
-constexpr int kWarps = 16;
+// Warps: 0 weights producer, 1 MMA issuer, 2 activations producer, 3 idle, 4..15 dequant (three
+// groups of four: a group covers the 128 TMEM lanes and decodes whole A units, the groups taking
+// units in turn), 16..19 epilogue.
+constexpr int kWarps = 20;
 constexpr int kThreads = kWarps * 32;
-constexpr int kWProd = 0, kMma = 1, kBProd = 2, kDeq0 = 4, kDeqWarps = 8, kEpi0 = 12, kEpiWarps = 4;
+constexpr int kWProd = 0, kMma = 1, kBProd = 2, kDeq0 = 4, kDeqGroups = 3, kDeqWarps = 4 * kDeqGroups;
+constexpr int kEpi0 = kDeq0 + kDeqWarps, kEpiWarps = 4;
+static_assert(kDeq0 % 4 == 0 && kEpi0 % 4 == 0, "a group of four warps reaches all 128 TMEM lanes");
 constexpr int kPackedStage = kRows * kStageK / 2;        // 32 KB: 2 box columns x 128 rows x 128 B
 constexpr int kPackedCol = kRows * 128;                  // one box column (two 64-row boxes)
 constexpr int kScaleStage = kRows * kStageK / 32;        // 2 KB: 128 rows x 16 B
-constexpr int kBTile = kWideTokens * kSubK * 2;          // 28 KB
-constexpr int kBBox = 16 * kSubK * 2;                    // one 16-row activation box
-constexpr int kACols = kSubK / 2;                        // TMEM columns of one A buffer (2 f16 per column)
-constexpr int kACol0 = kDBufs * kWideTokens;             // accumulators first, then the A buffers
-constexpr int kTmemCols = 512;                           // power of two >= kACol0 + kABufs * kACols
+constexpr int kBTile = kWideTokens * kSubK * 2;          // one activation slot: 24 KB
+constexpr int kBBox = 16 * kSubK * 2;                    // one 16-row activation box (2 KB)
+constexpr int kBoxesPerSlot = kBTile / kBBox;            // 12
+// A slot holds `spb` consecutive sub-tiles of a tile with nbox 16-row boxes each: as many as fit,
+// a power of two up to 8 (so that the sub-tiles of an item, a multiple of 8, split into whole
+// slots).  Narrow tiles thus keep up to 32 sub-tiles of activations in flight, wide ones 4.
+__host__ __device__ constexpr int subs_per_slot(int nbox)
+{
+    return 8 * nbox <= kBoxesPerSlot ? 8 : (4 * nbox <= kBoxesPerSlot ? 4 : (2 * nbox <= kBoxesPerSlot ? 2 : 1));
+}
+// Tensor-memory partition of a tile class (512 columns): accumulators first, then the A units.
+template <bool kSmall>
+struct Part {
+    static constexpr int kAccCols = kSmall ? kWideSmallMax : kWideTokens;   // max N of the class
+    static constexpr int kUnitK = kSmall ? 256 : 128;                       // K per A unit
+    static constexpr int kUnitSubs = kUnitK / kSubK;
+    static constexpr int kACols = kUnitK / 2;                               // 2 bf16 per column
+    static constexpr int kABufs = kSmall ? 3 : 2;
+    // Units rotate over as many dequant groups as there are A units, so that a group always
+    // refills the same unit and waits on its barrier phases in order (a parity wait cannot tell a
+    // phase from the one two before it); the large class leaves its third group idle.
+    static constexpr int kGroups = kABufs;
+    static constexpr int kACol0 = kDBufs * kAccCols;
+    static_assert(kACol0 + kABufs * kACols <= 512, "TMEM budget");
+    static_assert(kGroups <= kDeqGroups, "enough dequant groups");
+    static_assert(kStageK % kUnitK == 0, "units tile a stage");
+};
+constexpr int kTmemCols = 512;
+constexpr int kMaxABufs = 3;
 constexpr int kOffPacked = 0;
 constexpr int kOffScale = kOffPacked + kPStages * kPackedStage;
 constexpr int kOffB = kOffScale + kPStages * kScaleStage;
 constexpr int kOffIds = kOffB + kBBufs * kBTile;         // down: each epilogue warp's copy of the tile's flat ids
 constexpr int kOffBars = kOffIds + kEpiWarps * kWideTokens * 4;
 constexpr int kSmemBytes = kOffBars + 512 + 1024;        // barriers and slots, + alignment slack
-static_assert(kOffB % 1024 == 0 && kBTile % 1024 == 0, "swizzled tiles sit on 1024-byte boundaries");
-static_assert(kACol0 + kABufs * kACols <= kTmemCols && kTmemCols <= 512, "TMEM budget");
+static_assert(kOffB % 1024 == 0 && kBTile % 1024 == 0 && kBBox % 1024 == 0,
+              "swizzled tiles sit on 1024-byte boundaries");
+static_assert(kWideTokens % 16 == 0 && kWideTokens / 16 <= kBoxesPerSlot, "a sub-tile of the widest tile fits a slot");
 static_assert(kSmemBytes <= 227 * 1024, "fits one SM");
 }  // namespace wide
 
@@ -81,12 +121,13 @@ struct WideArgs {
     const WideTile *tiles;
     const int *n_tiles;
     const int32_t *sorted_ids;   // down: flat ids of the expert-grouped positions
-    __half *h;                   // gate_up output [M*k][I] (binary16, h * 2^10), expert-grouped rows
+    __nv_bfloat16 *h;            // gate_up output [M*k][I] bf16, expert-grouped rows (P4 K order if h_p4)
     float *y;                    // down output [M*k][H] by flat id, before the routing weight
     int *status_ws;
     int32_t *status_out;
     int *queue;
     int H, I;
+    int h_p4;                    // gate_up: store h in P4 K order (the down kernels' operand layout)
 };
 
 __device__ __forceinline__ float wide_clamp_swiglu(float g, float u)
@@ -96,31 +137,26 @@ __device__ __forceinline__ float wide_clamp_swiglu(float g, float u)
     return a / (1.0f + expf(-a)) * c;
 }
 
-__device__ __forceinline__ void record_status(const StatusPtrs &st, int code)
-{
-    if (st.ws) atomicExch(st.ws, code);
-    if (st.out) atomicExch(st.out, code);
-}
-
-template <bool kGateUp>
+template <bool kGateUp, bool kSmall>
 __global__ void __launch_bounds__(wide::kThreads, 1)
 grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
                     const __grid_constant__ CUtensorMap bmap, const __grid_constant__ WideArgs a)
 {
     using namespace wide;
+    using P = Part<kSmall>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
     uint64_t *full_p = bars, *empty_p = bars + kPStages;                       // packed stages
-    uint64_t *a_full = bars + 2 * kPStages, *a_empty = a_full + kABufs;        // A tiles
-    uint64_t *b_full = a_empty + kABufs, *b_empty = b_full + kBBufs;          // B tiles
+    uint64_t *a_full = bars + 2 * kPStages, *a_empty = a_full + kMaxABufs;     // A units
+    uint64_t *b_full = a_empty + kMaxABufs, *b_empty = b_full + kBBufs;       // B slots
     uint64_t *d_full = b_empty + kBBufs, *d_empty = d_full + kDBufs;          // accumulators
     uint64_t *pub = d_empty + kDBufs;                                         // [kItemQ] item ids published
     uint64_t *mma_done = pub + kItemQ;                                        // final drain of the MMAs
     volatile int *item_q = reinterpret_cast<volatile int *>(mma_done + 1);   // [kItemQ]
-    volatile int *a_item = item_q + kItemQ;                                   // [kABufs]
-    volatile int *d_item = a_item + kABufs;                                   // [kDBufs]
+    volatile int *a_item = item_q + kItemQ;                                   // [kMaxABufs]
+    volatile int *d_item = a_item + kMaxABufs;                                // [kDBufs]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<int *>(d_item + kDBufs));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -128,6 +164,8 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     const int H = a.H, I = a.I;
     const int K = kGateUp ? H : I;
     const int n_stages = K / kStageK;
+    const int n_units = K / P::kUnitK;
+    constexpr int kUnitsPerStage = kStageK / P::kUnitK;
     const int row_blocks = kGateUp ? I / 64 : H / kRows;
 
     if (threadIdx.x == 0) {
@@ -135,8 +173,8 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             mbar_init(&full_p[s], 1);
             mbar_init(&empty_p[s], kDeqWarps);
         }
-        for (int b = 0; b < kABufs; ++b) {
-            mbar_init(&a_full[b], kDeqWarps);
+        for (int b = 0; b < P::kABufs; ++b) {
+            mbar_init(&a_full[b], 4);   // the four warps of the group that decoded the unit
             mbar_init(&a_empty[b], 1);
         }
         for (int b = 0; b < kBBufs; ++b) {
@@ -191,11 +229,12 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 mbar_wait(&empty_p[s], ((stage_ctr / kPStages) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);
                 if (aborted) break;
-                if (lane == 0) {
+                uint8_t *pk = smem + kOffPacked + s * kPackedStage;
+                uint8_t *sc = smem + kOffScale + s * kScaleStage;
+                const int kb = st * (kStageK / 2);
+                if (elect_one()) {
                     mbar_arrive_expect_tx(&full_p[s], kPackedStage + kScaleStage);
-                    uint8_t *pk = smem + kOffPacked + s * kPackedStage;
-                    uint8_t *sc = smem + kOffScale + s * kScaleStage;
-                    const int kb = st * (kStageK / 2);
+#pragma unroll
                     for (int c = 0; c < 2; ++c) {
                         tma_load_2d(pk + c * kPackedCol, &wmap, kb + 128 * c, row_a, &full_p[s]);
                         tma_load_2d(pk + c * kPackedCol + 64 * 128, &wmap, kb + 128 * c, row_b, &full_p[s]);
@@ -225,7 +264,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     } else if (warp == kBProd) {
         // ------------------------------------------------------------ activations producer
         if (lane == 0) prefetch_tensormap(&bmap);
-        int sub_ctr = 0, issued = 0;
+        int bload = 0, issued = 0;   // slot loads so far / issued (a prefix of them)
         for (int item_ctr = 0;; ++item_ctr) {
             mbar_wait(&pub[item_ctr % kItemQ], (item_ctr / kItemQ) & 1, aborted, status);
             aborted = __any_sync(0xffffffffu, aborted);
@@ -235,15 +274,22 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const WideTile *tp = a.tiles + item / row_blocks;
             const int p0 = __ldcg(&tp->p0), cnt = __ldcg(&tp->count);
             const int nbox = (cnt + 15) / 16;
-            for (int j = 0; j < n_stages * kSubs; ++j, ++sub_ctr) {
-                const int bb = sub_ctr % kBBufs;
-                mbar_wait(&b_empty[bb], ((sub_ctr / kBBufs) & 1) ^ 1, aborted, status);
+            const int spb = subs_per_slot(nbox);
+            for (int j0 = 0; j0 < n_stages * kSubs; j0 += spb, ++bload) {
+                const int bb = bload % kBBufs;
+                mbar_wait(&b_empty[bb], ((bload / kBBufs) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);
                 if (aborted) break;
-                if (lane == 0) mbar_arrive_expect_tx(&b_full[bb], static_cast<uint32_t>(nbox * kBBox));
+                // box (sub-tile u, rows 16 b..) -> slot offset (u * nbox + b) boxes
+                uint8_t *slot = smem + kOffB + bb * kBTile;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&b_full[bb], static_cast<uint32_t>(spb * nbox * kBBox));
+                    for (int u = 0; u < spb; ++u)
+                        for (int bx = 0; bx < nbox; ++bx)
+                            tma_load_2d(slot + (u * nbox + bx) * kBBox, &bmap, (j0 + u) * kSubK, p0 + 16 * bx,
+                                        &b_full[bb]);
+                }
                 __syncwarp();
-                if (lane < nbox)
-                    tma_load_2d(smem + kOffB + bb * kBTile + lane * kBBox, &bmap, j * kSubK, p0 + 16 * lane, &b_full[bb]);
                 ++issued;
             }
             if (aborted) break;
@@ -252,26 +298,38 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int sc = issued - 1 - i;
             mbar_wait_drain(&b_full[sc % kBBufs], (sc / kBBufs) & 1, status);
         }
-    }
-    else if (warp >= kDeq0 && warp < kDeq0 + kDeqWarps) {
+    } else if (warp >= kDeq0 && warp < kDeq0 + kDeqWarps) {
         // ------------------------------------------------------------ dequant warps
-        // a warp stores TMEM lanes 32 (warp % 4) ..; its thread owns A row ar = that lane and the
-        // K half h (warps 4..7: low 32 K, 8..11: high 32 K) of each 64-K sub-tile
-        const int dw = warp - kDeq0;
-        const int quarter = warp & 3, h = dw >> 2;
+        // group grp takes the units whose running index is grp mod P::kGroups (so always A unit
+        // grp); a warp stores TMEM lanes 32 (warp % 4) ..; its thread owns A row ar = that lane,
+        // all K of the unit.  Groups past P::kGroups take no unit but release every stage.
+        const int grp = (warp - kDeq0) >> 2;
+        const int quarter = warp & 3;
         const int ar = 32 * quarter + lane;
         // packed row of A row ar: A rows 2i, 2i + 1 = gate row i (box rows 0..63), up row i (box
         // rows 64..127) for gate_up; row ar for down
         const int r = kGateUp ? (ar >> 1) + (ar & 1) * 64 : ar;
         const uint32_t a_lane = static_cast<uint32_t>(32 * quarter) << 16;
-        bool bad_scale = false;
-        int stage_ctr = 0, sub_ctr = 0;
+        int stage_ctr = 0, unit_ctr = 0;   // every group counts every stage and unit
         for (int item_ctr = 0;; ++item_ctr) {
             // the item's first stage (or the end marker) names the item
             mbar_wait(&full_p[stage_ctr % kPStages], (stage_ctr / kPStages) & 1, aborted, status);
             if (aborted) break;
             const int item = item_q[item_ctr % kItemQ];
-            for (int st = 0; st < (item < 0 ? 1 : n_stages); ++st) {
+            if (item < 0) {
+                // the end marker reaches the MMA warp as one more unit, from the group whose turn it is
+                if (unit_ctr % P::kGroups == grp) {
+                    const int ab = unit_ctr % P::kABufs;
+                    mbar_wait(&a_empty[ab], ((unit_ctr / P::kABufs) & 1) ^ 1, aborted, status);
+                    if (!aborted) {
+                        if (quarter == 0 && lane == 0) a_item[ab] = -1;
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&a_full[ab]);
+                    }
+                }
+                break;
+            }
+            for (int st = 0; st < n_stages; ++st) {
                 const int s = stage_ctr % kPStages;
                 if (st > 0) {
                     mbar_wait(&full_p[s], (stage_ctr / kPStages) & 1, aborted, status);
@@ -279,56 +337,51 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 }
                 const uint8_t *pk = smem + kOffPacked + s * kPackedStage;
                 const uint8_t *sc = smem + kOffScale + s * kScaleStage;
-                for (int j = 0; j < (item < 0 ? 1 : kSubs); ++j, ++sub_ctr) {
-                    const int ab = sub_ctr % kABufs;
-                    mbar_wait(&a_empty[ab], ((sub_ctr / kABufs) & 1) ^ 1, aborted, status);
+                for (int uu = 0; uu < kUnitsPerStage; ++uu, ++unit_ctr) {
+                    if (unit_ctr % P::kGroups != grp) continue;
+                    const int ab = unit_ctr % P::kABufs;
+                    mbar_wait(&a_empty[ab], ((unit_ctr / P::kABufs) & 1) ^ 1, aborted, status);
                     if (aborted) break;
-                    tc_fence_after();   // the MMAs that read this A buffer are complete
-                    if (item >= 0) {
-                        // 16 packed bytes: box column j / 4, 16-byte chunk (j % 4) * 2 + h of row r
-                        const int ch = (j & 3) * 2 + h;
-                        const uint4 w = *reinterpret_cast<const uint4 *>(pk + (j >> 2) * kPackedCol + r * 128 +
-                                                                         ((ch ^ (r & 7)) << 4));
-                        const uint32_t sbyte = sc[r * 16 + 2 * j + h];
-                        bad_scale |= (sbyte < 104u) | (sbyte > 140u);
-                        // 2^(sbyte - 127) as f16 (exact for 103 <= sbyte <= 142), in both halves
-                        const __half s16 = __float2half_rn(__int_as_float(static_cast<int>(sbyte << 23)));
-                        const __half2 s2 = __halves2half2(s16, s16);
-                        uint32_t f[16];
-                        e2m1x8_to_f16x2(w.x, f[0], f[1], f[2], f[3]);
-                        e2m1x8_to_f16x2(w.y, f[4], f[5], f[6], f[7]);
-                        e2m1x8_to_f16x2(w.z, f[8], f[9], f[10], f[11]);
-                        e2m1x8_to_f16x2(w.w, f[12], f[13], f[14], f[15]);
+                    tc_fence_after();   // the MMAs that read this A unit are complete
+                    for (int c = 0; c < P::kUnitSubs; ++c) {
+                        const int j = uu * P::kUnitSubs + c;   // 64-K sub-tile within the stage
+                        // 32 packed bytes of row r: box column j / 4, 16-byte chunks (j % 4) * 2 + h
+                        uint32_t f[32];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            __half2 v = *reinterpret_cast<__half2 *>(&f[i]);
-                            v = __hmul2(v, s2);
-                            f[i] = *reinterpret_cast<uint32_t *>(&v);
+                        for (int h = 0; h < 2; ++h) {
+                            const int ch = (j & 3) * 2 + h;
+                            const uint4 w = *reinterpret_cast<const uint4 *>(pk + (j >> 2) * kPackedCol + r * 128 +
+                                                                             ((ch ^ (r & 7)) << 4));
+                            const uint32_t sbyte = sc[r * 16 + 2 * j + h];
+                            const bool large = __any_sync(0xffffffffu, sbyte > 128u);
+                            mxfp4x8_to_bf16x2_p4(w.x, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h]));
+                            mxfp4x8_to_bf16x2_p4(w.y, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h + 4]));
+                            mxfp4x8_to_bf16x2_p4(w.z, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h + 8]));
+                            mxfp4x8_to_bf16x2_p4(w.w, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h + 12]));
                         }
-                        // columns 16h .. 16h + 15 of the buffer: K 32h + 2i, 32h + 2i + 1 in column 16h + i
-                        tmem_st16(tmem + a_lane + static_cast<uint32_t>(kACol0 + ab * kACols + 16 * h), f);
+                        // column 32c + 16h + 4u + i of the unit holds K 64c + 32h + 8u + i (low half) and
+                        // 64c + 32h + 8u + i + 4 (high half): MMA K positions 2 col, 2 col + 1 in P4 order
+                        tmem_st32(tmem + a_lane + static_cast<uint32_t>(P::kACol0 + ab * P::kACols + 32 * c), f);
                     }
-                    if (dw == 0 && lane == 0) a_item[ab] = item;
+                    if (quarter == 0 && lane == 0) a_item[ab] = item;
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&a_full[ab]);
                 }
                 if (aborted) break;
-                if (item < 0) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty_p[s]);
                 ++stage_ctr;
             }
-            if (aborted || item < 0) break;
+            if (aborted) break;
         }
-        if (__any_sync(0xffffffffu, bad_scale) && lane == 0) record_status(status, kStatusUnsupported);
     } else if (warp == kMma) {
         // ------------------------------------------------------------ MMA issuer
-        int sub_ctr = 0, bsub = 0;
+        int unit_ctr = 0, bload = 0;
         for (int item_ctr = 0;; ++item_ctr) {
             const int db = item_ctr % kDBufs;
-            int ab = sub_ctr % kABufs;
-            mbar_wait(&a_full[ab], (sub_ctr / kABufs) & 1, aborted, status);
+            int ab = unit_ctr % P::kABufs;
+            mbar_wait(&a_full[ab], (unit_ctr / P::kABufs) & 1, aborted, status);
             if (aborted) break;
             const int item = a_item[ab];
             // the accumulator's previous item must have left the epilogue (also before the end
@@ -344,39 +397,52 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             }
             if (lane == 0) d_item[db] = item;
             const WideTile *tp = a.tiles + item / row_blocks;
-            const int n_mma = ((__ldcg(&tp->count) + 15) / 16) * 16;
-            const uint32_t idesc = umma_idesc_f16(kRows, n_mma);
-            const uint32_t d_tmem = tmem + static_cast<uint32_t>(db * kWideTokens);
-            for (int j = 0; j < n_stages * kSubs; ++j, ++sub_ctr, ++bsub) {
-                ab = sub_ctr % kABufs;
-                const int bb = bsub % kBBufs;
-                if (j > 0) mbar_wait(&a_full[ab], (sub_ctr / kABufs) & 1, aborted, status);
-                mbar_wait(&b_full[bb], (bsub / kBBufs) & 1, aborted, status);
+            const int nbox = (__ldcg(&tp->count) + 15) / 16;
+            const int spb = subs_per_slot(nbox);
+            const uint32_t idesc = umma_idesc_bf16(kRows, 16 * nbox);
+            const uint32_t d_tmem = tmem + static_cast<uint32_t>(db * P::kAccCols);
+            for (int u = 0; u < n_units; ++u, ++unit_ctr) {
+                ab = unit_ctr % P::kABufs;
+                if (u > 0) mbar_wait(&a_full[ab], (unit_ctr / P::kABufs) & 1, aborted, status);
                 if (aborted) break;
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t a_tmem = tmem + static_cast<uint32_t>(kACol0 + ab * kACols);
-                    const uint32_t b_addr = smem_u32(smem + kOffB + bb * kBTile);
-#pragma unroll
-                    for (int ks = 0; ks < kSubK / 16; ++ks)
-                        umma_f16_tmem_a(d_tmem, a_tmem + 8 * ks, umma_sdesc_sw128(b_addr + 32 * ks), idesc,
-                                        (j > 0 || ks > 0) ? 1u : 0u);
-                    umma_commit(smem_u32(&a_empty[ab]));
-                    umma_commit(smem_u32(&b_empty[bb]));
+                for (int c = 0; c < P::kUnitSubs; ++c) {
+                    const int j = u * P::kUnitSubs + c;
+                    const int bb = bload % kBBufs, uo = j % spb;
+                    if (uo == 0) {
+                        mbar_wait(&b_full[bb], (bload / kBBufs) & 1, aborted, status);
+                        if (aborted) break;
+                        tc_fence_after();
+                    }
+                    // operands computed by the whole warp; one elected lane issues
+                    const uint32_t a_tmem = tmem + static_cast<uint32_t>(P::kACol0 + ab * P::kACols + 32 * c);
+                    const uint64_t b_desc = umma_sdesc_sw128(smem_u32(smem + kOffB + bb * kBTile + uo * nbox * kBBox));
+                    const uint32_t first = (j == 0) ? 0u : 1u;
+                    if (elect_one()) {
+                        // K steps of 16 advance A by 8 columns and B by 32 bytes (2 in the descriptor)
+                        umma_f16_tmem_a(d_tmem, a_tmem, b_desc, idesc, first);
+                        umma_f16_tmem_a(d_tmem, a_tmem + 8, b_desc + 2, idesc, 1u);
+                        umma_f16_tmem_a(d_tmem, a_tmem + 16, b_desc + 4, idesc, 1u);
+                        umma_f16_tmem_a(d_tmem, a_tmem + 24, b_desc + 6, idesc, 1u);
+                        if (uo == spb - 1) umma_commit(smem_u32(&b_empty[bb]));   // the slot's last sub-tile
+                    }
+                    __syncwarp();
+                    if (uo == spb - 1) ++bload;
                 }
+                if (aborted) break;
+                if (elect_one()) umma_commit(smem_u32(&a_empty[ab]));
                 __syncwarp();
             }
             if (aborted) break;
-            if (lane == 0) umma_commit(smem_u32(&d_full[db]));
+            if (elect_one()) umma_commit(smem_u32(&d_full[db]));
             __syncwarp();
         }
-        // every MMA this thread issued is complete before the tensor memory can be freed
-        if (lane == 0) umma_commit(smem_u32(mma_done));
+        // every MMA this warp issued is complete before the tensor memory can be freed
+        if (elect_one()) umma_commit(smem_u32(mma_done));
         __syncwarp();
         bool gave_up = false;
         mbar_wait(mma_done, 0, gave_up, status);
-    }
-    else if (warp >= kEpi0) {
+    } else if (warp >= kEpi0) {
         // ------------------------------------------------------------ epilogue warps
         const int quarter = warp & 3;                    // TMEM lanes 32 * quarter .. + 31
         const int row = 32 * quarter + lane;             // accumulator row (A row)
@@ -390,7 +456,8 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const WideTile *tp = a.tiles + item / row_blocks;
             const int rb = item % row_blocks;
             const int p0 = __ldcg(&tp->p0), cnt = __ldcg(&tp->count);
-            const uint32_t taddr = tmem + static_cast<uint32_t>(db * kWideTokens) + (static_cast<uint32_t>(32 * quarter) << 16);
+            const uint32_t taddr =
+                tmem + static_cast<uint32_t>(db * P::kAccCols) + (static_cast<uint32_t>(32 * quarter) << 16);
             // down: the tile's flat ids, loaded once per item (independent loads) into this warp's copy
             int *ids = reinterpret_cast<int *>(smem + kOffIds) + (warp - kEpi0) * kWideTokens;
             if (!kGateUp) {
@@ -403,22 +470,20 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 if (kGateUp) {
                     // even rows hold g, odd rows u of output column n
                     const int n = rb * 64 + (row >> 1);
+                    const int col = a.h_p4 ? p4_pos(n) : n;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const float mine = __uint_as_float(v[j]);
                         const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                        if (!(lane & 1) && c + j < cnt) {
-                            const float hv = wide_clamp_swiglu(mine, other);
-                            a.h[static_cast<size_t>(p0 + c + j) * I + n] =
-                                __float2half_rn(__bfloat162float(__float2bfloat16_rn(hv)) * kHScale);
-                        }
+                        if (!(lane & 1) && c + j < cnt)
+                            a.h[static_cast<size_t>(p0 + c + j) * I + col] = __float2bfloat16_rn(wide_clamp_swiglu(mine, other));
                     }
                 } else {
-                    // h carries the 2^10 storage scale; the routing weight is applied by the combine
+                    // the unweighted row; the routing weight is applied by the combine
                     const int r = rb * kRows + row;
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c + j < cnt) a.y[static_cast<size_t>(ids[c + j]) * H + r] = __uint_as_float(v[j]) * (1.0f / kHScale);
+                        if (c + j < cnt) a.y[static_cast<size_t>(ids[c + j]) * H + r] = __uint_as_float(v[j]);
                 }
             }
             tc_fence_before();
@@ -433,34 +498,58 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     if (warp == kMma) tmem_dealloc(tmem, kTmemCols);
 }
 
-// x_perm[p] = x16[sorted_ids[p] / k]: the activation rows in expert-grouped order, so that the
-// wide kernel's activation boxes are plain TMA tiles.  One warp per row, 16-byte copies.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const __half *__restrict__ x16,
-                                                          const int32_t *__restrict__ sorted_ids,
-                                                          __half *__restrict__ x_perm, int n, int H, int k)
+// x_perm[p] = x_p4[sorted_ids[p] / k] (rows already in P4 K order), for the positions p of the
+// wide tiles only (the rows the wide kernels' activation boxes read; the other rows of x_perm are
+// never read).  CTA (w, c) copies rows 8c .. 8c + 7 of wide tile w -- tiles [0, max_small) of the
+// small-tile list, then those of the large-tile list -- one warp per row, 16 bytes a lane.
+__global__ void __launch_bounds__(256) gather_wide_rows_kernel(const __nv_bfloat16 *__restrict__ x_p4,
+                                                               const int32_t *__restrict__ sorted_ids, WideLists wl,
+                                                               __nv_bfloat16 *__restrict__ x_perm, int H, int k)
 {
     pdl_wait();
     pdl_trigger();
-    const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (p >= n) return;
-    const int t = sorted_ids[p] / k;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x16 + static_cast<size_t>(t) * H);
+    const bool small = static_cast<int>(blockIdx.x) < wl.max_small;
+    const int w = small ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - wl.max_small;
+    if (w >= __ldcg(small ? wl.n_small : wl.n_large)) return;
+    const WideTile *tp = (small ? wl.small : wl.large) + w;
+    const int p0 = __ldcg(&tp->p0), cnt = __ldcg(&tp->count);
+    const int i = blockIdx.y * 8 + (threadIdx.x >> 5);
+    if (i >= cnt) return;
+    const int p = p0 + i;
+    const int t = __ldcg(&sorted_ids[p]) / k;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x_p4 + static_cast<size_t>(t) * H);
     uint4 *dst = reinterpret_cast<uint4 *>(x_perm + static_cast<size_t>(p) * H);
-    for (int i = threadIdx.x & 31; i < H / 8; i += 32) dst[i] = src[i];
+    for (int g = threadIdx.x & 31; g < H / 8; g += 32) dst[g] = __ldcg(&src[g]);
 }
 
 int wide_smem_bytes() { return wide::kSmemBytes; }
 
-cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __half *x_perm, int n, int H, int k,
-                               cudaStream_t s, bool pdl)
+cudaError_t launch_gather_wide_rows(const __nv_bfloat16 *x_p4, const int32_t *sorted_ids, const WideLists &wl,
+                                    __nv_bfloat16 *x_perm, int H, int k, cudaStream_t s, bool pdl)
 {
-    return launch_ex(gather_rows_kernel, dim3((n + 7) / 8), dim3(256), 0, s, pdl, x16, sorted_ids, x_perm, n, H, k);
+    const int n = wl.max_small + wl.max_large;
+    const dim3 grid(n > 0 ? n : 1, (kWideTokens + 7) / 8);
+    return launch_ex(gather_wide_rows_kernel, grid, dim3(256), 0, s, pdl, x_p4, sorted_ids, wl, x_perm, H, k);
 }
 
-cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap &smap, const CUtensorMap &bmap,
-                        const WideTile *tiles, const int *n_tiles, int max_tiles, const int32_t *sorted_ids,
-                        __half *h, float *y, int *status, int32_t *status_out, int H, int I,
-                        cudaStream_t s, bool pdl)
+template <bool kGateUp, bool kSmall>
+static cudaError_t launch_wide_t(const CUtensorMap &wmap, const CUtensorMap &smap, const CUtensorMap &bmap,
+                                 const WideArgs &a, int max_tiles, cudaStream_t s, bool pdl)
+{
+    auto kern = grouped_wide_kernel<kGateUp, kSmall>;
+    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(kern), wide::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const long long row_blocks = kGateUp ? a.I / 64 : a.H / wide::kRows;
+    const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
+    int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
+    if (grid < 1) grid = 1;
+    return launch_ex(kern, dim3(grid), dim3(wide::kThreads), wide::kSmemBytes, s, pdl, wmap, smap, bmap, a);
+}
+
+cudaError_t launch_wide(bool gate_up, bool small, const CUtensorMap &wmap, const CUtensorMap &smap,
+                        const CUtensorMap &bmap, const WideTile *tiles, const int *n_tiles, int max_tiles,
+                        const int32_t *sorted_ids, __nv_bfloat16 *h, bool h_p4, float *y, int *status,
+                        int32_t *status_out, int H, int I, cudaStream_t s, bool pdl)
 {
     WideArgs a;
     a.tiles = tiles;
@@ -470,17 +559,16 @@ cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap
     a.y = y;
     a.status_ws = status;
     a.status_out = status_out;
-    a.queue = status + (gate_up ? kQueueGateUpWide : kQueueDownWide);
+    a.queue = status + (gate_up ? (small ? kQueueGateUpWide : kQueueGateUpWideL)
+                                : (small ? kQueueDownWide : kQueueDownWideL));
     a.H = H;
     a.I = I;
-    auto kern = gate_up ? grouped_wide_kernel<true> : grouped_wide_kernel<false>;
-    cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(kern), wide::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    const long long row_blocks = gate_up ? I / 64 : H / wide::kRows;
-    const long long max_items = static_cast<long long>(max_tiles) * row_blocks;
-    int grid = static_cast<int>(max_items < num_sms() ? max_items : num_sms());
-    if (grid < 1) grid = 1;
-    return launch_ex(kern, dim3(grid), dim3(wide::kThreads), wide::kSmemBytes, s, pdl, wmap, smap, bmap, a);
+    a.h_p4 = h_p4 ? 1 : 0;
+    if (gate_up)
+        return small ? launch_wide_t<true, true>(wmap, smap, bmap, a, max_tiles, s, pdl)
+                     : launch_wide_t<true, false>(wmap, smap, bmap, a, max_tiles, s, pdl);
+    return small ? launch_wide_t<false, true>(wmap, smap, bmap, a, max_tiles, s, pdl)
+                 : launch_wide_t<false, false>(wmap, smap, bmap, a, max_tiles, s, pdl);
 }
 
 }  // namespace moe

@@ -3,7 +3,7 @@
 #pragma once
 
 #include <cuda.h>
-#include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -12,13 +12,14 @@ namespace moe {
 
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = -5;
-constexpr int kStatusUnsupported = -2;   // MOE_ERR_UNSUPPORTED_SHAPE: an input outside a kernel's exact range
 // The call's 256-byte status block: word 0 is the status; words kQueueGateUp and kQueueDown
 // are the grouped kernels' work-queue counters, zeroed by the first kernel of the call.
 constexpr int kQueueGateUp = 8;
 constexpr int kQueueDown = 16;
-constexpr int kQueueGateUpWide = 24;
+constexpr int kQueueGateUpWide = 24;    // tensor-core launches: small tiles
 constexpr int kQueueDownWide = 32;
+constexpr int kQueueGateUpWideL = 40;   // and large tiles
+constexpr int kQueueDownWideL = 48;
 
 // Grouped GEMM tiling (both projections).
 // An expert tile holds up to 8 or 16 assignments (tile_width): one or two MMA n-tiles of 8.
@@ -29,13 +30,12 @@ constexpr int kChunkK = 1024;        // K elements per pipeline stage (512 bytes
 constexpr int kBoxCols = kChunkK / 256;              // 128-byte TMA box columns per stage
 constexpr int kStageBytes = kItemRows * kChunkK / 2; // packed weights of one stage (32 KB)
 constexpr int kStageScaleBytes = kItemRows * kChunkK / 32;   // E8M0 bytes of one stage (per-stage mode)
-constexpr int kActPitch = kChunkK * 2 + 64;         // one token's binary16 chunk, padded against bank conflicts
+constexpr int kActPitch = kChunkK * 2 + 64;         // one token's bf16 chunk, padded against bank conflicts
 constexpr int kStages = 3;
 constexpr int kComputeWarps = 16;    // 2 m-tile pairs x 8 K slots
 constexpr int kWarpMTiles = 2;       // m-tiles per compute warp (the activation fragment serves both)
 constexpr int kKSlots = kComputeWarps * kWarpMTiles / kItemMTiles;
 constexpr int kEpilogueWarps = 2;
-constexpr float kHScale = 1024.0f;   // h is stored as binary16(h * 2^10): exact for |h| >= 2^-27
 
 // E8M0 scales travel with each stage (a TMA box of the scale matrix) when a scale row is a
 // multiple of 16 bytes; otherwise the item's scale rows are copied once per item.
@@ -101,31 +101,49 @@ __host__ __device__ inline int tile_width(int M, int E, int k)
     return static_cast<long long>(M) * k >= 6LL * E ? 16 : 8;
 }
 
-// Experts with at least kWideMinTokens assignments go to the tensor-core path (grouped_wide.cu)
-// as wide tiles of up to kWideTokens consecutive assignments; it needs H and I to be multiples
-// of its 512-element packed stage.  No expert can exceed M assignments, so M < kWideMinTokens
-// never uses it.
-constexpr int kWideTokens = 224;   // MMA N: two accumulators of 224 columns + A buffers fill TMEM
+// Experts with at least kWideMinTokens assignments go to the tensor-core path (grouped_wide.cu),
+// when the call enables it: one small tile if they have at most kWideSmallMax, else large tiles
+// of up to kWideTokens consecutive assignments.  The path is enabled
+// (wide_enabled): H and I multiples of its 512-element packed stage, M >= kWideMinTokens (no
+// expert can exceed M assignments), and on average at least kWideMinTokens / 2 assignments per
+// expert, so that decode-size calls, whose experts hold one or two assignments, skip its three
+// launches.  Every other expert streams its weights as mma.sync tiles of 8 or 16 assignments
+// (grouped_gemm.cu).
+constexpr int kWideTokens = 192;   // the large-tile kernel's MMA N: two 192-column accumulators + A units fill TMEM
+constexpr int kWideSmallMax = 64;  // an expert with up to this many assignments is one small tile
 constexpr int kWideStageK = 512;
-constexpr int kWideMinTokens = 32;   // fewer assignments stream faster as mma.sync tiles
+constexpr int kWideMinTokens = 9;
 struct WideTile {
     int expert;
     int p0;      // first position in the expert-grouped order
     int count;   // assignments, 1 .. kWideTokens
     int pad;
 };
-__host__ __device__ inline bool wide_enabled(int M, int H, int I)
+// The two tensor-core tile lists of a call (small: one tile per expert with kWideMinTokens ..
+// kWideSmallMax assignments; large: tiles of up to kWideTokens of the experts with more).
+struct WideLists {
+    WideTile *small;
+    int *n_small;
+    WideTile *large;
+    int *n_large;
+    int max_small, max_large;
+};
+__host__ __device__ inline bool wide_small_expert(int c) { return c >= kWideMinTokens && c <= kWideSmallMax; }
+__host__ __device__ inline bool wide_large_expert(int c) { return c > kWideSmallMax; }
+__host__ __device__ inline int wide_large_tiles(int c) { return (c + kWideTokens - 1) / kWideTokens; }
+__host__ __device__ inline bool wide_enabled(int M, int H, int I, int E, int k)
 {
-    return M >= kWideMinTokens && H % kWideStageK == 0 && I % kWideStageK == 0;
+    return M >= kWideMinTokens && H % kWideStageK == 0 && I % kWideStageK == 0 &&
+           2LL * M * k >= static_cast<long long>(kWideMinTokens) * E;
 }
 
 // Byte offsets of every buffer inside one call's workspace (256-byte aligned).
 struct Layout {
-    size_t status, partial, x16, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y;
-    size_t wide_tiles, n_wide, x_perm, total;
+    size_t status, partial, x_p4, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y;
+    size_t wide_small, n_wide_small, wide_large, n_wide_large, x_perm, total;
     int splits;   // router partial-logit slices (route_plan)
     int width;    // tile_width
-    int max_tiles, max_wide;
+    int max_tiles, max_small, max_large;
     bool wide;    // wide_enabled for this shape
 };
 
@@ -168,14 +186,15 @@ __host__ __device__ inline bool fused_select(int M, int E, int k)
            static_cast<long long>(M) * E <= kFusedSelectMaxLogits;
 }
 // Dynamic shared memory of the ranking (rank_smem): two [warp][expert] u16 tables (counts and
-// prefix counts), five int arrays over E and a 33-int scan buffer.
+// prefix counts), six int arrays over E and a 33-int scan buffer.
 __host__ __device__ inline int permute_smem_bytes(int E)
 {
-    return 2 * (kPermuteThreads / 32) * E * 2 + 5 * E * 4 + 64 * 4;
+    return 2 * (kPermuteThreads / 32) * E * 2 + 6 * E * 4 + 64 * 4;
 }
 
 // Kernel launchers (return cudaError_t of the launch).
-cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
+// x_p4 (nullable): x [M, H] rewritten in P4 K order for the grouped GEMMs.
+cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, void *x_p4, int *status,
                                 int32_t *status_out, int M, int H, int E, cudaStream_t s);
 cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
                               int E, int k, cudaStream_t s, bool pdl);
@@ -185,8 +204,10 @@ cudaError_t launch_route_topk(const float *partial, int splits, const float *bia
 struct TileOut {
     ExpertTile *tiles;
     int *n_tiles;
-    WideTile *wide_tiles;   // nullptr: every expert gets mma.sync tiles
+    WideTile *wide_tiles;   // small tensor-core tiles; nullptr: every expert gets mma.sync tiles
     int *n_wide;
+    WideTile *wide_large;   // large tensor-core tiles (set whenever wide_tiles is)
+    int *n_wide_large;
     int width;
 };
 cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
@@ -194,24 +215,28 @@ cudaError_t launch_route_select_permute(const float *partial, int splits, const 
                                         int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
                            int M, int E, int k, cudaStream_t s, bool pdl);
-cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
-                               int *status, int E, int width, cudaStream_t s);
-cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s);
+// Tiles of both kinds from given expert offsets and sorted ids (the step-level entry points);
+// also resets the call's status words.
+cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, TileOut to, int *status, int E,
+                               cudaStream_t s);
+// Rows [n_rows, cols] in natural K order -> P4 order (the grouped GEMMs' activation layout).
+cudaError_t launch_rows_to_p4(const __nv_bfloat16 *src, __nv_bfloat16 *dst, size_t n_rows, int cols, cudaStream_t s);
 cudaError_t launch_gate_up(const CUtensorMap &w13_map, const CUtensorMap &s13_map, const uint8_t *w13_s,
-                           const __half *x16, const ExpertTile *tiles, const int *n_tiles, __half *h, int *status,
-                           int32_t *status_out, int H, int I, int k, int width, int max_tiles, cudaStream_t s,
-                           bool pdl);
-cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s, const __half *h,
-                        const int32_t *sorted_ids, const ExpertTile *tiles, const int *n_tiles, float *y, int *status,
-                        int32_t *status_out, int H, int I, int width, int max_tiles, cudaStream_t s, bool pdl);
+                           const __nv_bfloat16 *x, const ExpertTile *tiles, const int *n_tiles, __nv_bfloat16 *h,
+                           bool h_p4, int *status, int32_t *status_out, int H, int I, int k, int width, int max_tiles,
+                           cudaStream_t s, bool pdl);
+cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, const uint8_t *w2_s,
+                        const __nv_bfloat16 *h_p4, const int32_t *sorted_ids, const ExpertTile *tiles,
+                        const int *n_tiles, float *y, int *status, int32_t *status_out, int H, int I, int width,
+                        int max_tiles, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
                            bool pdl);
-cudaError_t launch_gather_rows(const __half *x16, const int32_t *sorted_ids, __half *x_perm, int n, int H, int k,
-                               cudaStream_t s, bool pdl);
-cudaError_t launch_wide(bool gate_up, const CUtensorMap &wmap, const CUtensorMap &smap, const CUtensorMap &bmap,
-                        const WideTile *tiles, const int *n_tiles, int max_tiles, const int32_t *sorted_ids,
-                        __half *h, float *y, int *status, int32_t *status_out, int H, int I,
-                        cudaStream_t s, bool pdl);
+cudaError_t launch_gather_wide_rows(const __nv_bfloat16 *x_p4, const int32_t *sorted_ids, const WideLists &wl,
+                                    __nv_bfloat16 *x_perm, int H, int k, cudaStream_t s, bool pdl);
+cudaError_t launch_wide(bool gate_up, bool small, const CUtensorMap &wmap, const CUtensorMap &smap,
+                        const CUtensorMap &bmap, const WideTile *tiles, const int *n_tiles, int max_tiles,
+                        const int32_t *sorted_ids, __nv_bfloat16 *h, bool h_p4, float *y, int *status,
+                        int32_t *status_out, int H, int I, cudaStream_t s, bool pdl);
 int wide_smem_bytes();
 cudaError_t launch_wait_timeout_selftest(int32_t *status_out, cudaStream_t s);
 

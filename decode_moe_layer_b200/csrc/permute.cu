@@ -1,5 +1,6 @@
 // permute.cu -- stand-alone route remap kernel (rank_and_scatter of permute_impl.cuh
-// over given topk_ids) and the expert-tile builder used by the step-level entry points.
+// over given topk_ids), and the expert-tile builder and h reordering used by the step-level
+// entry points.
 #include "permute_impl.cuh"
 
 namespace moe {
@@ -32,11 +33,10 @@ permute_kernel(const int32_t *__restrict__ topk_ids, int32_t *__restrict__ offse
     rank_and_scatter(s_e, n, E, k, rank_smem(smem, E), offsets, sorted_ids, inv_pos, to);
 }
 
-// Expert tiles from given offsets / sorted ids; also resets the call's status word.
+// Expert tiles (both kinds) from given offsets / sorted ids; also resets the call's status words.
 __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__restrict__ offsets,
-                                                              const int32_t *__restrict__ sorted_ids,
-                                                              ExpertTile *__restrict__ tiles, int *__restrict__ n_tiles,
-                                                              int *status, int E, int width)
+                                                              const int32_t *__restrict__ sorted_ids, TileOut to,
+                                                              int *status, int E)
 {
     __shared__ int s_off[kMaxE + 1];
     __shared__ int scan_buf[33];
@@ -46,10 +46,20 @@ __global__ void __launch_bounds__(1024, 1) build_tiles_kernel(const int32_t *__r
         status[kQueueDown] = 0;
         status[kQueueGateUpWide] = 0;
         status[kQueueDownWide] = 0;
+        status[kQueueGateUpWideL] = 0;
+        status[kQueueDownWideL] = 0;
     }
     for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = offsets[e];
     __syncthreads();
-    emit_tiles(s_off, E, width, tiles, n_tiles, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
+    emit_tiles(s_off, E, to, scan_buf, [&](int p) { return static_cast<int>(sorted_ids[p]); });
+}
+
+// dst[r] = src[r] with every 8-element group moved from natural to P4 K order (common.cuh).
+__global__ void __launch_bounds__(256) rows_to_p4_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst,
+                                                         size_t n_groups)
+{
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i < n_groups) dst[i] = p4_from_natural(src[i]);
 }
 
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
@@ -63,10 +73,19 @@ cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted
                      n, E, k);
 }
 
-cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, ExpertTile *tiles, int *n_tiles,
-                               int *status, int E, int width, cudaStream_t s)
+cudaError_t launch_build_tiles(const int32_t *offsets, const int32_t *sorted_ids, TileOut to, int *status, int E,
+                               cudaStream_t s)
 {
-    build_tiles_kernel<<<1, 1024, 0, s>>>(offsets, sorted_ids, tiles, n_tiles, status, E, width);
+    build_tiles_kernel<<<1, 1024, 0, s>>>(offsets, sorted_ids, to, status, E);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rows_to_p4(const __nv_bfloat16 *src, __nv_bfloat16 *dst, size_t n_rows, int cols, cudaStream_t s)
+{
+    const size_t n_groups = n_rows * static_cast<size_t>(cols) / 8;
+    const unsigned blocks = static_cast<unsigned>((n_groups + 255) / 256);
+    rows_to_p4_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(reinterpret_cast<const uint4 *>(src),
+                                                               reinterpret_cast<uint4 *>(dst), n_groups);
     return cudaGetLastError();
 }
 

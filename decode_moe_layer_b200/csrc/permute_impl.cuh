@@ -54,11 +54,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int *warp_tot, int &t
 }
 
 // Shared memory of the ranking, carved from one dynamic buffer of permute_smem_bytes(E) bytes:
-// wc at 0, pref at 64 E, the five int arrays at 128 E, the scan buffer at 148 E (+132 bytes).
+// wc at 0, pref at 64 E, the six int arrays at 128 E, the scan buffer at 152 E (+132 bytes).
 struct RankSmem {
     uint16_t *wc;     // [32][E] counts of the current round's warps
     uint16_t *pref;   // [32][E] their prefix counts (with earlier rounds)
-    int *cnt, *off, *tb, *base, *wb;   // [E] count, offset, first tile, ranked so far, first wide tile
+    int *cnt, *off, *tb, *base, *wb, *wbl;   // [E] count, offset, first tile, ranked so far, small / large wide tile
     int *scan;        // 33
 };
 
@@ -74,7 +74,8 @@ __device__ __forceinline__ RankSmem rank_smem(uint8_t *raw, int E)
     r.tb = ints + 2 * E;
     r.base = ints + 3 * E;
     r.wb = ints + 4 * E;
-    r.scan = ints + 5 * E;
+    r.wbl = ints + 5 * E;
+    r.scan = ints + 6 * E;
     return r;
 }
 
@@ -104,11 +105,13 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
     }
     __syncthreads();
     // offsets and tile bases: (tiles << 16) | count per expert, one scan (counts <= 16384); an
-    // expert with at least kWideMinTokens assignments takes wide tiles instead, when enabled
+    // expert with at least kWideMinTokens assignments takes tensor-core tiles instead, when enabled
     const int my_cnt = tid < E ? sm.cnt[tid] : 0;
-    const bool my_wide = to.wide_tiles != nullptr && my_cnt >= kWideMinTokens;
+    const bool wide_on = to.wide_tiles != nullptr;
+    const bool my_small = wide_on && wide_small_expert(my_cnt);
+    const bool my_large = wide_on && wide_large_expert(my_cnt);
     const int W = to.width, wsh = W == 16 ? 4 : 3;   // 8 or 16 assignments per tile
-    const int mine = tid < E ? ((my_wide ? 0 : (my_cnt + W - 1) >> wsh) << 16) | my_cnt : 0;
+    const int mine = tid < E ? (((my_small || my_large) ? 0 : (my_cnt + W - 1) >> wsh) << 16) | my_cnt : 0;
     int total = 0;
     const int base = block_exclusive_scan(mine, sm.scan, total);   // ends with a block barrier
     if (tid < E) {
@@ -120,12 +123,17 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
         offsets[E] = total & 0xFFFF;
         if (tiles) *to.n_tiles = total >> 16;
     }
-    if (to.wide_tiles != nullptr) {
+    if (wide_on) {
         __syncthreads();   // every thread has read the first scan's totals before the buffer is reused
         int wtotal = 0;
-        const int wbase = block_exclusive_scan(my_wide ? (my_cnt + kWideTokens - 1) / kWideTokens : 0, sm.scan, wtotal);
+        const int wbase = block_exclusive_scan(my_small ? 1 : 0, sm.scan, wtotal);
         if (tid < E) sm.wb[tid] = wbase;
         if (tid == 0) *to.n_wide = wtotal;
+        __syncthreads();
+        int ltotal = 0;
+        const int lbase = block_exclusive_scan(my_large ? wide_large_tiles(my_cnt) : 0, sm.scan, ltotal);
+        if (tid < E) sm.wbl[tid] = lbase;
+        if (tid == 0) *to.n_wide_large = ltotal;
     }
     for (int r0 = 0; r0 < n; r0 += kPermuteThreads) {
         const int f = r0 + tid;
@@ -159,9 +167,17 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
             sorted_ids[pos] = f;
             inv_pos[f] = pos;
             const int cnt = sm.cnt[e];
-            if (to.wide_tiles != nullptr && cnt >= kWideMinTokens) {
+            if (wide_on && wide_small_expert(cnt)) {
+                if (rank == 0) {
+                    WideTile *wp = to.wide_tiles + sm.wb[e];
+                    wp->expert = e;
+                    wp->p0 = pos;
+                    wp->count = cnt;
+                    wp->pad = 0;
+                }
+            } else if (wide_on && wide_large_expert(cnt)) {
                 if (rank % kWideTokens == 0) {
-                    WideTile *wp = to.wide_tiles + sm.wb[e] + rank / kWideTokens;
+                    WideTile *wp = to.wide_large + sm.wbl[e] + rank / kWideTokens;
                     wp->expert = e;
                     wp->p0 = pos;
                     wp->count = min(kWideTokens, cnt - rank);
@@ -189,66 +205,89 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
 // number of earlier tokens that chose e: with mask[e] = the set of tokens that chose e (one bit
 // per token), rank = popc(mask[e] & (2^t - 1)) and count = popc(mask[e]).
 
-// One warp (the calling warp): per expert, (mma.sync tiles << 16) | count and the wide tiles
-// (experts with kWideMinTokens or more when the wide path is on), one warp scan over the experts
-// (lane l takes the contiguous experts [l * per, (l + 1) * per)); writes off, tb, wb (shared) and
+// One warp (the calling warp): per expert, (mma.sync tiles << 16) | count and the small and large
+// tensor-core tiles (when the wide path is on), one warp scan over the experts (lane l takes the
+// contiguous experts [l * per, (l + 1) * per)); writes off, tb, wb, wbl (shared) and
 // expert_offsets, the tile counts (global).
 __device__ inline void warp_scan_experts(const unsigned long long *mask, int E, TileOut to, int *off, int *tb, int *wb,
-                                         int32_t *__restrict__ offsets)
+                                         int *wbl, int32_t *__restrict__ offsets)
 {
     const bool wide_on = to.wide_tiles != nullptr;
     const int lane = threadIdx.x & 31;
     const int W = to.width, wsh = W == 16 ? 4 : 3;   // 8 or 16 assignments per tile
-    auto packed = [&](int c) { return (((wide_on && c >= kWideMinTokens) ? 0 : (c + W - 1) >> wsh) << 16) | c; };
-    auto wide_n = [&](int c) { return (wide_on && c >= kWideMinTokens) ? (c + kWideTokens - 1) / kWideTokens : 0; };
+    auto narrow = [&](int c) { return !wide_on || c < kWideMinTokens; };
+    auto packed = [&](int c) { return ((narrow(c) ? (c + W - 1) >> wsh : 0) << 16) | c; };
+    auto small_n = [&](int c) { return (wide_on && wide_small_expert(c)) ? 1 : 0; };
+    auto large_n = [&](int c) { return (wide_on && wide_large_expert(c)) ? wide_large_tiles(c) : 0; };
     const int per = (E + 31) / 32;
     const int ea = min(E, lane * per), eb = min(E, ea + per);
-    int local = 0, wlocal = 0;
+    int local = 0, wlocal = 0, llocal = 0;
     for (int e = ea; e < eb; ++e) {
         const int c = __popcll(mask[e]);
         local += packed(c);
-        wlocal += wide_n(c);
+        wlocal += small_n(c);
+        llocal += large_n(c);
     }
-    int incl = local, wincl = wlocal;
+    int incl = local, wincl = wlocal, lincl = llocal;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
         const int o = __shfl_up_sync(0xffffffffu, incl, d);
         const int wo = __shfl_up_sync(0xffffffffu, wincl, d);
+        const int lo = __shfl_up_sync(0xffffffffu, lincl, d);
         if (lane >= d) {
             incl += o;
             wincl += wo;
+            lincl += lo;
         }
     }
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     const int wtotal = __shfl_sync(0xffffffffu, wincl, 31);
-    int run = incl - local, wrun = wincl - wlocal;
+    const int ltotal = __shfl_sync(0xffffffffu, lincl, 31);
+    int run = incl - local, wrun = wincl - wlocal, lrun = lincl - llocal;
     for (int e = ea; e < eb; ++e) {
         const int c = __popcll(mask[e]);
         off[e] = run & 0xFFFF;
         tb[e] = run >> 16;
         wb[e] = wrun;
+        wbl[e] = lrun;
         offsets[e] = run & 0xFFFF;
         run += packed(c);
-        wrun += wide_n(c);
+        wrun += small_n(c);
+        lrun += large_n(c);
     }
     if (lane == 0) {
         offsets[E] = total & 0xFFFF;
         *to.n_tiles = total >> 16;
-        if (wide_on) *to.n_wide = wtotal;
+        if (wide_on) {
+            *to.n_wide = wtotal;
+            *to.n_wide_large = ltotal;
+        }
     }
 }
 
 // Assignment f (token t, expert e, rank r among the expert's c assignments): its position, the
-// inverse map and its slot of an mma.sync tile or a wide tile (off, tb, wb from warp_scan_experts).
+// inverse map and its slot of an mma.sync tile or a tensor-core tile (off, tb, wb, wbl from
+// warp_scan_experts).
 __device__ inline void scatter_assignment(int f, int e, int r, int c, const int *off, const int *tb, const int *wb,
-                                          int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos, TileOut to)
+                                          const int *wbl, int32_t *__restrict__ sorted_ids,
+                                          int32_t *__restrict__ inv_pos, TileOut to)
 {
     const int pos = off[e] + r;
     sorted_ids[pos] = f;
     inv_pos[f] = pos;
-    if (to.wide_tiles != nullptr && c >= kWideMinTokens) {
+    if (to.wide_tiles != nullptr && wide_small_expert(c)) {
+        if (r == 0) {
+            WideTile *wp = to.wide_tiles + wb[e];
+            wp->expert = e;
+            wp->p0 = pos;
+            wp->count = c;
+            wp->pad = 0;
+        }
+        return;
+    }
+    if (to.wide_tiles != nullptr && wide_large_expert(c)) {
         if (r % kWideTokens == 0) {
-            WideTile *wp = to.wide_tiles + wb[e] + r / kWideTokens;
+            WideTile *wp = to.wide_large + wbl[e] + r / kWideTokens;
             wp->expert = e;
             wp->p0 = pos;
             wp->count = min(kWideTokens, c - r);
@@ -270,21 +309,52 @@ __device__ inline void scatter_assignment(int f, int e, int r, int c, const int 
         for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
 }
 
-// Tiles of W assignments from expert offsets; sorted_flat(p) returns the flat assignment id at
-// position p of the expert-grouped order.  Each thread owns a contiguous run of ceil(E / blockDim)
-// experts.
+// Tiles from expert offsets (the step-level entry points, whose caller gives the permutation):
+// mma.sync tiles of to.width assignments and, when to.wide_tiles is set, small and large
+// tensor-core tiles (the same split as the route remap kernels make).  sorted_flat(p) returns the
+// flat assignment id at position p of the expert-grouped order.  Each thread owns a contiguous run
+// of ceil(E / blockDim) experts.
 template <typename SortedFlat>
-__device__ inline void emit_tiles(const int *off, int E, int W, ExpertTile *tiles, int *n_tiles, int *scan_buf,
-                                  SortedFlat sorted_flat)
+__device__ inline void emit_tiles(const int *off, int E, TileOut to, int *scan_buf, SortedFlat sorted_flat)
 {
+    const int W = to.width;
+    const bool wide_on = to.wide_tiles != nullptr;
     const int per = (E + blockDim.x - 1) / blockDim.x;
-    const int e0 = threadIdx.x * per, e1 = min(E, e0 + per);
-    int mine = 0;
-    for (int e = e0; e < e1; ++e) mine += (off[e + 1] - off[e] + W - 1) / W;
-    int total = 0;
-    int base = block_exclusive_scan(mine, scan_buf, total);
+    const int e0 = min(E, static_cast<int>(threadIdx.x) * per), e1 = min(E, e0 + per);
+    int mine = 0, smine = 0, lmine = 0;
     for (int e = e0; e < e1; ++e) {
         const int cnt = off[e + 1] - off[e];
+        if (wide_on && wide_small_expert(cnt))
+            ++smine;
+        else if (wide_on && wide_large_expert(cnt))
+            lmine += wide_large_tiles(cnt);
+        else
+            mine += (cnt + W - 1) / W;
+    }
+    int total = 0, stotal = 0, ltotal = 0;
+    int base = block_exclusive_scan(mine, scan_buf, total);
+    __syncthreads();   // every thread has read a scan's totals before the buffer is reused
+    int sbase = block_exclusive_scan(smine, scan_buf, stotal);
+    __syncthreads();
+    int lbase = block_exclusive_scan(lmine, scan_buf, ltotal);
+    for (int e = e0; e < e1; ++e) {
+        const int cnt = off[e + 1] - off[e];
+        if (wide_on && (wide_small_expert(cnt) || wide_large_expert(cnt))) {
+            const bool small = wide_small_expert(cnt);
+            const int step = small ? cnt : kWideTokens;
+            for (int i = 0; i * step < cnt; ++i) {
+                WideTile wt;
+                wt.expert = e;
+                wt.p0 = off[e] + i * step;
+                wt.count = min(step, cnt - i * step);
+                wt.pad = 0;
+                if (small)
+                    to.wide_tiles[sbase++] = wt;
+                else
+                    to.wide_large[lbase++] = wt;
+            }
+            continue;
+        }
         for (int i = 0; i * W < cnt; ++i) {
             ExpertTile tl{};
             tl.expert = e;
@@ -292,10 +362,16 @@ __device__ inline void emit_tiles(const int *off, int E, int W, ExpertTile *tile
             tl.count = min(W, cnt - i * W);
             tl.pad = 0;
             for (int j = 0; j < W; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
-            tiles[base++] = tl;
+            to.tiles[base++] = tl;
         }
     }
-    if (threadIdx.x == 0) *n_tiles = total;
+    if (threadIdx.x == 0) {
+        *to.n_tiles = total;
+        if (wide_on) {
+            *to.n_wide = stotal;
+            *to.n_wide_large = ltotal;
+        }
+    }
 }
 
 }  // namespace moe

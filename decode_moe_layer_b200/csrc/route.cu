@@ -11,8 +11,8 @@
 //     runs it against every token tile.  The 8 warp partials are summed in warp
 //     order in shared memory and the CTA writes its slice of partial logits
 //     [split][M][E]; the top-k adds the slices in split order.  The CTAs of expert
-//     group 0 also write the binary16 copy of x that the grouped GEMM consumes; the
-//     first CTA resets the call's status words.
+//     group 0 also write x in the P4 K order (common.cuh) that the grouped GEMMs read;
+//     the first CTA resets the call's status words.
 //  2. top-k per token, one warp per token: sum the slices, add the bias, select the
 //     top k by k rounds of a warp arg-max (warp max of order-preserving logit keys,
 //     then warp min of the ids holding it: value desc, expert id asc), and
@@ -23,7 +23,6 @@
 //     shared memory with all its threads.
 // Every reduction has a fixed order, so ids and weights are bitwise reproducible.
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "permute_impl.cuh"
@@ -32,12 +31,6 @@ namespace moe {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v)
-{
-    __half2 h = __floats2half2_rn(bf16_lo(v), bf16_hi(v));
-    return *reinterpret_cast<uint32_t *>(&h);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
@@ -69,7 +62,8 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 template <int kSteps, int kTiles>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr, float *__restrict__ partial,
-                    __half *__restrict__ x16, int *status, int32_t *status_out, int M, int H, int E, int passes)
+                    uint16_t *__restrict__ x_p4, int *status, int32_t *status_out, int M, int H, int E,
+                    int passes)
 {
     constexpr int kPassK = 16 * kSteps;
     constexpr int kTokens = 8 * kTiles;
@@ -80,7 +74,7 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
     const int e0 = blockIdx.x * kRouteExperts;
     const int split = blockIdx.y;
     const int t0 = blockIdx.z * kTokens;
-    const bool write_x16 = (blockIdx.x == 0) && (x16 != nullptr);
+    const bool write_p4 = (blockIdx.x == 0) && (x_p4 != nullptr);
     pdl_trigger();
     if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) {
         if (status) {
@@ -89,6 +83,8 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
             status[kQueueDown] = 0;
             status[kQueueGateUpWide] = 0;
             status[kQueueDownWide] = 0;
+            status[kQueueGateUpWideL] = 0;
+            status[kQueueDownWideL] = 0;
         }
         if (status_out) *status_out = kStatusOk;
     }
@@ -134,16 +130,23 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
                 mma_bf16_16816(acc[j], lo, xv[j][s].x, xv[j][s].y);
             }
         }
-        if (write_x16) {
+        if (write_p4) {
+            // lanes q and q ^ 1 hold elements 0..3 and 4..7 of an 8-element group: the even lane
+            // writes the group's P4 words 0, 1 = (x0,x4), (x1,x5), the odd one words 2, 3
 #pragma unroll
             for (int s = 0; s < kSteps; ++s) {
                 const int kk = kw + 16 * s + 4 * q;
 #pragma unroll
                 for (int j = 0; j < kTiles; ++j) {
+                    const uint2 mine = xv[j][s];
+                    const uint2 other = make_uint2(__shfl_xor_sync(0xffffffffu, mine.x, 1),
+                                                   __shfl_xor_sync(0xffffffffu, mine.y, 1));
+                    const bool odd = (q & 1) != 0;
+                    const uint32_t lo = odd ? other.y : mine.x, hi = odd ? mine.y : other.x;
                     const int t = t0 + 8 * j + g;
                     if (kk < H && t < M)
-                        *reinterpret_cast<uint2 *>(x16 + static_cast<size_t>(t) * H + kk) =
-                            make_uint2(bf16x2_to_f16x2(xv[j][s].x), bf16x2_to_f16x2(xv[j][s].y));
+                        *reinterpret_cast<uint2 *>(x_p4 + static_cast<size_t>(t) * H + (kk & ~7) + (odd ? 4 : 0)) =
+                            make_uint2(prmt(lo, hi, 0x5410u), prmt(lo, hi, 0x7632u));
                 }
             }
         }
@@ -304,7 +307,8 @@ route_select_permute_kernel(const float *__restrict__ partial, int splits, const
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_e[kPermuteThreads];                    // expert of assignment f
     __shared__ unsigned long long s_mask[kMaxE];            // bit t: token t chose the expert
-    __shared__ int s_off[kMaxE], s_tb[kMaxE], s_wb[kMaxE];  // first position, first tile, first wide tile
+    __shared__ int s_off[kMaxE], s_tb[kMaxE];                // first position, first mma.sync tile
+    __shared__ int s_wb[kMaxE], s_wbl[kMaxE];                // first small / large tensor-core tile
     float *s_log = reinterpret_cast<float *>(smem);         // [M][E]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_wait();
@@ -335,50 +339,37 @@ route_select_permute_kernel(const float *__restrict__ partial, int splits, const
         }
     }
     __syncthreads();
-    if (warp == 0) warp_scan_experts(s_mask, E, to, s_off, s_tb, s_wb, offsets);
+    if (warp == 0) warp_scan_experts(s_mask, E, to, s_off, s_tb, s_wb, s_wbl, offsets);
     __syncthreads();
     const int n = M * k;
     for (int f = threadIdx.x; f < n; f += blockDim.x) {
         const int e = s_e[f], t = f / k;
         const unsigned long long mk = s_mask[e];
-        scatter_assignment(f, e, __popcll(mk & ((1ull << t) - 1ull)), __popcll(mk), s_off, s_tb, s_wb, sorted_ids,
-                           inv_pos, to);
+        scatter_assignment(f, e, __popcll(mk & ((1ull << t) - 1ull)), __popcll(mk), s_off, s_tb, s_wb, s_wbl,
+                           sorted_ids, inv_pos, to);
     }
 }
 
-__global__ void convert_x_kernel(const uint16_t *__restrict__ x, __half *__restrict__ x16, int *status, size_t n8)
-{
-    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i == 0 && status) *status = kStatusOk;
-    if (i >= n8) return;
-    uint4 v = reinterpret_cast<const uint4 *>(x)[i];
-    uint4 o;
-    o.x = bf16x2_to_f16x2(v.x);
-    o.y = bf16x2_to_f16x2(v.y);
-    o.z = bf16x2_to_f16x2(v.z);
-    o.w = bf16x2_to_f16x2(v.w);
-    reinterpret_cast<uint4 *>(x16)[i] = o;
-}
-
 template <int kSteps, int kTiles>
-static cudaError_t logits_launch(const void *x, const float *router_w, float *partial, __half *x16, int *status,
+static cudaError_t logits_launch(const void *x, const float *router_w, float *partial, void *x_p4, int *status,
                                  int32_t *status_out, int M, int H, int E, const RoutePlan &plan, cudaStream_t s)
 {
     const dim3 grid((E + kRouteExperts - 1) / kRouteExperts, plan.splits, plan.blocks_t);
     // first kernel of a call: fully ordered after whatever precedes it in the stream
     route_logits_kernel<kSteps, kTiles><<<grid, kRouteWarps * 32, 0, s>>>(
-        static_cast<const uint16_t *>(x), router_w, partial, x16, status, status_out, M, H, E, plan.passes);
+        static_cast<const uint16_t *>(x), router_w, partial, static_cast<uint16_t *>(x_p4), status, status_out, M, H,
+        E, plan.passes);
     return cudaGetLastError();
 }
 
-cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, __half *x16, int *status,
+cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, void *x_p4, int *status,
                                 int32_t *status_out, int M, int H, int E, cudaStream_t s)
 {
     const RoutePlan plan = route_plan(M, H, E);
     if (plan.tiles == 1 && plan.steps == 2)
-        return logits_launch<2, 1>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
+        return logits_launch<2, 1>(x, router_w, partial, x_p4, status, status_out, M, H, E, plan, s);
     if (plan.tiles == 4 && plan.steps == 4)
-        return logits_launch<4, 4>(x, router_w, partial, x16, status, status_out, M, H, E, plan, s);
+        return logits_launch<4, 4>(x, router_w, partial, x_p4, status, status_out, M, H, E, plan, s);
     return cudaErrorInvalidConfiguration;   // route_plan yields only the two shapes above
 }
 
@@ -425,15 +416,6 @@ cudaError_t launch_route_select_permute(const float *partial, int splits, const 
     if (E <= 512) return MOE_SEL(16);
     return MOE_SEL(32);
 #undef MOE_SEL
-}
-
-cudaError_t launch_convert_x(const void *x, __half *x16, int *status, int M, int H, cudaStream_t s)
-{
-    const size_t n8 = static_cast<size_t>(M) * H / 8;
-    const int threads = 256;
-    const unsigned blocks = static_cast<unsigned>((n8 + threads - 1) / threads);
-    convert_x_kernel<<<blocks > 0 ? blocks : 1, threads, 0, s>>>(static_cast<const uint16_t *>(x), x16, status, n8);
-    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -12,7 +12,7 @@
 namespace moe {
 
 // Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzle layout: rows of
-// 64 f16 (128 bytes), atoms of 8 rows (1024 bytes) stacked along M/N.  Fields: start address
+// 64 16-bit elements (128 bytes), atoms of 8 rows (1024 bytes) stacked along M/N.  Fields: start address
 // >> 4 (bits 0-13), leading byte offset >> 4 (16-29; unused for this layout, 16 bytes), stride
 // byte offset >> 4 (32-45: 1024 bytes between 8-row atoms), descriptor version 1 (46-47),
 // layout 2 = 128-byte swizzle (61-63).  Advancing K by 16 elements inside the atom adds 32
@@ -27,14 +27,16 @@ __device__ __forceinline__ uint64_t umma_sdesc_sw128(uint32_t smem_addr)
     return d;
 }
 
-// Instruction descriptor of kind::f16: f32 accumulator (bits 4-5 = 1), A and B f16 (bits 7-9,
-// 10-12 = 0), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-__host__ __device__ inline uint32_t umma_idesc_f16(int m, int n)
+// Instruction descriptor of kind::f16 with bf16 operands: f32 accumulator (bits 4-5 = 1), A and
+// B bf16 (bits 7-9 and 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22,
+// M >> 4 in bits 24-28.
+__host__ __device__ inline uint32_t umma_idesc_bf16(int m, int n)
 {
-    return (1u << 4) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+    return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+           (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-// Byte offset of f16 element (row r, k) in a K-major 128-byte-swizzled tile of 64-element rows
+// Byte offset of 16-bit element (row r, k) in a K-major 128-byte-swizzled tile of 64-element rows
 // (the layout umma_sdesc_sw128 describes and a 128B-swizzled TMA box produces).
 __host__ __device__ inline uint32_t sw128_offset(int r, int k)
 {
@@ -69,13 +71,16 @@ __device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
                  : "memory");
 }
 
-// 16 consecutive 32-bit columns of this thread's TMEM lane from registers (lane as in
-// tmem_ld16), then wait until the stores are done.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16])
+// 32 consecutive 32-bit columns of this thread's TMEM lane (lane as in tmem_ld16) from registers,
+// then wait until the stores are done.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
 {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
                  ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-                 "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+                 "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+                 "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
+                 "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
                  : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

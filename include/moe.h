@@ -26,9 +26,8 @@
  *   weight value      E2M1(code) * 2^(scale - 127)
  *   topk_ids / topk_w int32 / fp32 [M, k], slot j in descending router probability
  *   expert_offsets    int32 [E+1];  sorted_ids, inv_pos int32 [M*k]
- *   h                 binary16 [M*k, I] in expert-grouped order (row p holds the
- *                     assignment sorted_ids[p]); element = bf16_rne(h) * 2^10,
- *                     exact in binary16 for |h| >= 2^-27 (|h| <= 49, so no overflow)
+ *   h                 bf16 [M*k, I] in expert-grouped order (row p holds the
+ *                     assignment sorted_ids[p])
  *
  * Conventions for every entry point:
  *   - Pointers are device pointers the caller owns; the library keeps none after
@@ -43,8 +42,13 @@
  *   - Supported shapes: H % 32 == 0, I % 32 == 0, H,I >= 32, H <= 16384,
  *     1 <= k <= min(E, 32), E <= 1024, M*k <= 16384.  Others return
  *     MOE_ERR_UNSUPPORTED_SHAPE.
- *   - Out of contract (undefined output, no fault): NaN/Inf or |x| > 65504 in x,
- *     E8M0 scale bytes 254 and 255.
+ *   - Arithmetic: bf16 x and the exactly decoded bf16 weights multiply into fp32
+ *     accumulators; h is rounded to bf16 once; out is rounded to bf16 once.
+ *   - Out of contract (undefined output, no fault): NaN/Inf in x, E8M0 scale
+ *     byte 255 (NaN), and values beyond the fp32 range: a weight value of 2^128 or
+ *     more (scale byte 253 or 254 with a large code) or a dot product, logit or
+ *     output that overflows fp32.  Products that fall below fp32's normal range
+ *     (weights and activations both far below 1) lose relative precision.
  *   - Determinism: for a given device and inputs, every output is bitwise
  *     reproducible (no floating-point atomics; fixed reduction orders).
  *
@@ -114,24 +118,25 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
  * For each position p of the expert-grouped order, f = sorted_ids[p], t = f / k,
  * e = the expert whose offsets range holds p:
  *   g = W_gate,e x[t], u = W_up,e x[t] (bf16 products, fp32 accumulation),
- *   h[p] = bf16_rne(silu(min(g,7)) * clamp(u,-7,7)), stored as binary16(h[p] * 2^10).
- * expert_offsets/sorted_ids are moe_permute's outputs.  Uses the library-owned
+ *   h[p] = bf16_rne(silu(min(g,7)) * clamp(u,-7,7))  (bf16 [M*k, I], h_bf16).
+ * expert_offsets/sorted_ids are moe_permute's outputs.  The experts' assignments are
+ * split into tiles exactly as in moe_mxfp4_forward.  Uses the library-owned
  * workspace of `stream`.
  */
 int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *w13_s,
-                       const int32_t *expert_offsets, const int32_t *sorted_ids, void *h_f16,
+                       const int32_t *expert_offsets, const int32_t *sorted_ids, void *h_bf16,
                        int M, int H, int I, int E, int k, cudaStream_t stream);
 
 /*
  * Down GEMM with the weighted top-k combine fused behind it.  Defined by the
- * down half of the "Compact routed MXFP4 GEMM" row of the same table (h in the
- * binary16(h * 2^10) format moe_gate_up_swiglu writes):
+ * down half of the "Compact routed MXFP4 GEMM" row of the same table (h bf16
+ * [M*k, I] in expert-grouped order, as moe_gate_up_swiglu writes it):
  *   y[f] = W2_e h[inv position of f] (fp32 accumulation),
  *   out[t] = bf16_rne( sum_{j=0..k-1} topk_w[t,j] * y[t*k+j] ), summed in slot
  *   order j with no atomics.
  * Uses the library-owned workspace of `stream` for the fp32 per-assignment rows.
  */
-int moe_down_combine(const void *h_f16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
+int moe_down_combine(const void *h_bf16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
                      const int32_t *expert_offsets, const int32_t *sorted_ids, void *out_bf16,
                      int M, int H, int I, int E, int k, cudaStream_t stream);
 
@@ -154,7 +159,7 @@ int moe_mxfp4_forward(const void *x, const float *router_w, const uint8_t *w13_q
  * library-owned workspace.
  *   - Limit: 256 + S * M * E * 4 bytes must fit in 4 MiB, where S is the number of
  *     H slices the router splits each expert group into: ceil(H / 256) for M <= 8,
- *     ceil(H / 1024) for larger M, reduced toward 1 as M * E grows (for example
+ *     ceil(H / 512) for larger M, reduced toward 1 as M * E grows (for example
  *     33 KB at M = 8, H = 2048, E = 128; 1 MB at M = 1024, H = 7168, E = 256).
  *     Larger shapes return MOE_ERR_WORKSPACE and enqueue nothing.
  *   - The first call on a device looks the array's device address up (once per
@@ -172,7 +177,7 @@ size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
 /*
  * Kernel launches one moe_mxfp4_forward / moe_mxfp4_forward_ex call enqueues for this shape
  * (router logits, top-k + permutation as one or two kernels, the grouped GEMMs, the gather and
- * tensor-core GEMMs when experts can reach 32 assignments, the combine); 0 for M == 0 and a
+ * tensor-core GEMMs when the call can give experts 9 or more assignments, the combine); 0 for M == 0 and a
  * negative MOE_* status for an unsupported shape.  For sizing CUDA graphs and for accounting.
  */
 int moe_forward_launches(int M, int H, int I, int E, int k);
@@ -204,18 +209,20 @@ int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *rout
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Entries of moe_mxfp4_forward_profile's output. */
-#define MOE_PROFILE_KERNELS 5
+#define MOE_PROFILE_KERNELS 11
 
 /*
- * Per-kernel device-time attribution of one layer call, in the manner of the
- * per-kernel buckets of "Post-Portfolio Device Attribution" ("MTP1 Post-Portfolio
- * Eager-Cycle Profile").  Same arguments and results as moe_mxfp4_forward_ex;
- * additionally records a CUDA event between consecutive launches, WAITS for the
- * stream to finish (host synchronisation: not for use under stream capture) and
- * writes into the HOST array kernel_ms the event-to-event milliseconds of:
- *   [0] router logits, [1] router top-k (fused with the route remap when
- *   M <= 64), [2] route remap (0 when fused), [3] gate_up + clamp-SwiGLU,
- *   [4] down and the weighted combine (two kernels).
+ * Per-launch device-time attribution of one layer call, in the manner of the per-kernel
+ * buckets of "Post-Portfolio Device Attribution" ("MTP1 Post-Portfolio Eager-Cycle
+ * Profile").  Same arguments and results as moe_mxfp4_forward_ex; additionally records a
+ * CUDA event before the first launch and after every launch, WAITS for the stream to finish
+ * (host synchronisation: not for use under stream capture) and writes into the HOST array
+ * kernel_ms the milliseconds of each launch (0 for a launch this shape does not make):
+ *   [0] router logits, [1] router top-k (fused with the route remap when M <= 64),
+ *   [2] route remap (0 when fused), [3] gate_up + clamp-SwiGLU on mma.sync tiles,
+ *   [4] gather of the tensor-core tiles' x rows, [5] / [6] gate_up + clamp-SwiGLU on small /
+ *   large tensor-core tiles, [7] down on mma.sync tiles, [8] / [9] down on small / large
+ *   tensor-core tiles, [10] the weighted top-k combine.
  * Kernels run back to back here instead of overlapping their launches as in
  * moe_mxfp4_forward_ex, so the sum exceeds a normal call's time.
  */

@@ -55,10 +55,18 @@ int main()
             }
         }
         for (int H : Hs)
-            for (int I : Hs) {
-                // the tensor-core path needs whole 512-element stages and at least 32 assignments
-                if (wide_enabled(M, H, I)) CHECK(M >= 32 && H % 512 == 0 && I % 512 == 0, M, H, 0, I);
-            }
+            for (int I : Hs)
+                for (int E : Es)
+                    for (int k : Ks) {
+                        if (k > E) continue;
+                        // the tensor-core path needs whole 512-element stages, calls in which an
+                        // expert can reach kWideMinTokens assignments, and experts averaging at
+                        // least half that
+                        if (wide_enabled(M, H, I, E, k))
+                            CHECK(M >= kWideMinTokens && H % 512 == 0 && I % 512 == 0 &&
+                                      2LL * M * k >= 1LL * kWideMinTokens * E,
+                                  M, H, E, I);
+                    }
     }
     for (int H = 32; H <= 16384; H += 32) {
         CHECK(down_row_blocks(H) * kItemRows >= H && (down_row_blocks(H) - 1) * kItemRows < H, 0, H, 0, 0);
@@ -67,7 +75,7 @@ int main()
     CHECK(permute_smem_bytes(kMaxE) <= 227 * 1024, 0, 0, kMaxE, 0);
     // the fused select's static arrays (token masks, offsets, tile bases, assignment experts)
     // plus its staged logits
-    CHECK(kMaxE * (8 + 3 * 4) + kPermuteThreads * 4 + kFusedSelectMaxLogits * 4 <= 227 * 1024, 0, 0, kMaxE, 0);
+    CHECK(kMaxE * (8 + 4 * 4) + kPermuteThreads * 4 + kFusedSelectMaxLogits * 4 <= 227 * 1024, 0, 0, kMaxE, 0);
     if (fails) {
         std::printf("%d failures\n", fails);
         return 1;

@@ -102,15 +102,18 @@ def test_selftest_validation():
 
 
 def test_forward_launch_counts():
-    # 5 launches at decode sizes (fused select), 6 with the separate top-k + permutation, and 3
-    # more once experts can reach the tensor-core tile size (M >= 32, H and I multiples of 512)
+    # 5 launches at decode sizes (fused select), 6 with the separate top-k + permutation, and 5
+    # more (the gather and the small- and large-tile tensor-core GEMMs of both projections) once the
+    # tensor-core path is on: H and I multiples of 512, M >= 9 and experts averaging >= 4.5
+    # assignments
     lib = moe.load()
     assert lib.moe_forward_launches(0, 2048, 768, 128, 8) == 0
     assert lib.moe_forward_launches(8, 2048, 768, 128, 8) == 5
     assert lib.moe_forward_launches(1, 7168, 2048, 256, 8) == 5
+    assert lib.moe_forward_launches(32, 7168, 2048, 256, 8) == 5
     assert lib.moe_forward_launches(96, 2048, 768, 128, 8) == 6
-    assert lib.moe_forward_launches(256, 7168, 2048, 256, 8) == 9
-    assert lib.moe_forward_launches(1024, 4096, 1536, 128, 8) == 9
+    assert lib.moe_forward_launches(256, 7168, 2048, 256, 8) == 11
+    assert lib.moe_forward_launches(1024, 4096, 1536, 128, 8) == 11
     assert lib.moe_forward_launches(8, 2048, 100, 128, 8) == moe.MOE_ERR_UNSUPPORTED_SHAPE
 
 

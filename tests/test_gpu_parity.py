@@ -108,7 +108,7 @@ def test_gate_up_swiglu(moe, ci, M):
     h = moe.moe_gate_up_swiglu(d["x"], d["w13_q"], d["w13_s"], torch.from_numpy(roff).cuda(),
                                torch.from_numpy(rsrt).cuda(), k)
     torch.cuda.synchronize()
-    h_flat = h.float().cpu().numpy().astype(np.float64)[rinv] / moe.H_STORAGE_SCALE   # flat order t*k+j
+    h_flat = U.bf16_tensor_to_f64(h)[rinv]   # flat order t*k+j
     toks = list(range(M)) if not big else [0, M - 1]
     for t in toks:
         for j in range(k):
@@ -132,8 +132,8 @@ def test_down_combine(moe, ci, M):
     rids, rw = r["topk_ids"], r["topk_w"]
     roff, rsrt, rinv = oracle.permute(rids, E)
     h_bits = r["h"][rsrt]                                         # oracle h in expert-grouped order
-    h16 = torch.from_numpy((gen.bf16_bits_to_f64(h_bits) * moe.H_STORAGE_SCALE).astype(np.float16)).cuda()
-    out = moe.moe_down_combine(h16, d["w2_q"], d["w2_s"], torch.from_numpy(rw.astype(np.float32)).cuda(),
+    hb = U.bits_to_bf16_tensor(h_bits)
+    out = moe.moe_down_combine(hb, d["w2_q"], d["w2_s"], torch.from_numpy(rw.astype(np.float32)).cuda(),
                                torch.from_numpy(roff).cuda(), torch.from_numpy(rsrt).cuda(), M, k)
     torch.cuda.synchronize()
     U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "down_combine c%d M=%d" % (ci, M))
@@ -206,13 +206,108 @@ def test_forward_large_sampled(moe, large_weights, ci, M):
     rids, rw, _ = oracle.route(inp.x, inp.router_w, inp.router_bias, k)
     assert np.array_equal(ids.cpu().numpy(), rids)                 # whole routing, bit-exact
     assert np.abs(tw.cpu().numpy() - rw).max() <= U.W_TOL
-    rng = np.random.default_rng(M)
-    toks = sorted(set([0, M - 1] + list(rng.choice(M, min(M, 2), replace=False))))
-    if ci == 4:
-        # the most-loaded expert's tokens exercise the longest tile runs
-        heavy = np.nonzero((rids == 0).any(axis=1))[0]
-        toks = sorted(set(toks + [int(heavy[0]), int(heavy[-1])]))
+    # every token when M <= 64; else at least 64 that cover every mma.sync tile slot and fill
+    # count, the first and last assignment of tensor-core tiles, and random ones
+    toks, desc = U.sample_tokens(rids, inp.shape.E, inp.shape.H, inp.shape.I, seed=M)
+    print("c%d M=%d compared: %s" % (ci, M, desc))
     r = U.oracle_forward(inp, tokens=toks)
     got = U.bf16_tensor_to_f64(out)
-    U.check_out(got[toks], r["out64"][toks], "forward c%d M=%d tokens %s" % (ci, M, toks))
+    U.check_out(got[toks], r["out64"][toks], "forward c%d M=%d (%s)" % (ci, M, desc))
     assert np.all(np.isfinite(got))
+
+
+# ----------------------------------------------------------------------------- tensor-core tiles, step by step
+
+WIDE_STEP_SHAPES = [
+    (1024, 512, 4, 2, 80),    # ~40 assignments per expert: tensor-core tiles for every expert
+    (512, 1024, 16, 4, 160),  # ~40 per expert, spread: tensor-core and mma.sync tiles in one call
+]
+
+
+@pytest.mark.parametrize("H,I,E,k,M", WIDE_STEP_SHAPES)
+def test_gate_up_and_down_steps_on_tensor_core_tiles(moe, H, I, E, k, M):
+    # the step entry points take the same tile split as the whole layer, wide tiles included
+    assert U.wide_path_on(M, H, I, E, k)
+    shape = gen.LayerShape("wide_step", H, I, E, k, (M,))
+    inp = gen.make_inputs(0, M, shape=shape, seed=3 * H + I + E + k + M)
+    d = U.device_inputs(inp)
+    r = U.oracle_forward(inp)
+    rids, rw = r["topk_ids"], r["topk_w"]
+    roff, rsrt, rinv = oracle.permute(rids, E)
+    assert np.diff(roff).max() >= U.WIDE_MIN_TOKENS
+    h = moe.moe_gate_up_swiglu(d["x"], d["w13_q"], d["w13_s"], torch.from_numpy(roff).cuda(),
+                               torch.from_numpy(rsrt).cuda(), k)
+    torch.cuda.synchronize()
+    h_flat = U.bf16_tensor_to_f64(h)[rinv]
+    for t in range(M):
+        for j in range(k):
+            e = int(rids[t, j])
+            g, u, hb = oracle.expert_swiglu(inp.x[t], inp.w13_q[e], inp.w13_s[e])
+            U.check_h_bound(h_flat[t * k + j], hb, g, u, inp.x[t], inp.w13_q[e], inp.w13_s[e],
+                            "wide step %s h[t=%d,j=%d]" % ((H, I, E, k, M), t, j))
+    out = moe.moe_down_combine(U.bits_to_bf16_tensor(r["h"][rsrt]), d["w2_q"], d["w2_s"],
+                               torch.from_numpy(rw.astype(np.float32)).cuda(), torch.from_numpy(roff).cuda(),
+                               torch.from_numpy(rsrt).cuda(), M, k)
+    torch.cuda.synchronize()
+    U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "wide step down %s" % ((H, I, E, k, M),))
+
+
+# ----------------------------------------------------------------------------- inputs across the bf16 range
+
+def _wide_range_inputs(H, I, E, k, M, seed):
+    """Every x row mixes magnitudes above 65504 and below 2^-17 (each element of a seeded
+    workload scaled by 2^d, d uniform over -40..24: exact in bf16), and every E8M0 byte is drawn
+    from 90..150 (weights from 2^-38 to 6 * 2^23)."""
+    shape = gen.LayerShape("wide_range", H, I, E, k, (M,))
+    inp = gen.make_inputs(0, M, shape=shape, seed=seed)
+    rng = np.random.default_rng(seed)
+    inp.w13_s = rng.integers(90, 151, size=inp.w13_s.shape).astype(np.uint8)
+    inp.w2_s = rng.integers(90, 151, size=inp.w2_s.shape).astype(np.uint8)
+    base = gen.bf16_bits_to_f64(inp.x)
+    for _ in range(100):
+        xv = base * np.exp2(rng.integers(-40, 25, size=base.shape).astype(np.float64))
+        bits = gen._bf16_bits_rne(xv)
+        if gen.margin_ok(bits, inp.router_w, inp.router_bias, k).all():
+            break
+    else:
+        raise RuntimeError("no draw met the routing margin")
+    assert np.array_equal(gen.bf16_bits_to_f64(bits), xv)
+    assert (np.abs(xv) > 65504).any(axis=1).all()
+    assert ((np.abs(xv) < 2.0 ** -17) & (xv != 0)).any(axis=1).all()
+    inp.x = bits
+    return inp
+
+
+@pytest.mark.parametrize("H,I,E,k,M", [
+    (1024, 512, 16, 4, 6),    # mma.sync tiles only
+    (1024, 512, 4, 2, 80),    # tensor-core tiles (scale bytes above 128 take the two-multiply decode)
+])
+def test_wide_range_x_and_scale_bytes(moe, H, I, E, k, M):
+    inp = _wide_range_inputs(H, I, E, k, M, seed=11 * H + I + E + k + M)
+    d = U.device_inputs(inp)
+    ids = torch.empty((M, k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((M, k), dtype=torch.float32, device="cuda")
+    st = torch.full((1,), 123, dtype=torch.int32, device="cuda")
+    ws = torch.empty(moe.moe_workspace_bytes(M, H, I, E, k), dtype=torch.uint8, device="cuda")
+    out = moe.moe_mxfp4_forward_ex(d["x"], d["router_w"], d["w13_q"], d["w13_s"], d["w2_q"], d["w2_s"], k, ws,
+                                   topk_ids_out=ids, topk_w_out=tw, status_out=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == moe.MOE_OK
+    r = U.oracle_forward(inp)
+    assert np.array_equal(ids.cpu().numpy(), r["topk_ids"])
+    assert np.abs(tw.cpu().numpy() - r["topk_w"]).max() <= U.W_TOL
+    # outputs here span many binades (x scaled by up to 2^24): the bar adds each element's own rounding
+    U.check_out_heavy_tailed(U.bf16_tensor_to_f64(out), r["out64"], "wide-range forward %s" % ((H, I, E, k, M),))
+    # h element by element through the step entry point
+    rids = r["topk_ids"]
+    roff, rsrt, rinv = oracle.permute(rids, E)
+    h = moe.moe_gate_up_swiglu(d["x"], d["w13_q"], d["w13_s"], torch.from_numpy(roff).cuda(),
+                               torch.from_numpy(rsrt).cuda(), k)
+    torch.cuda.synchronize()
+    h_flat = U.bf16_tensor_to_f64(h)[rinv]
+    for t in range(M):
+        for j in range(k):
+            e = int(rids[t, j])
+            g, u, hb = oracle.expert_swiglu(inp.x[t], inp.w13_q[e], inp.w13_s[e])
+            U.check_h_bound(h_flat[t * k + j], hb, g, u, inp.x[t], inp.w13_q[e], inp.w13_s[e],
+                            "wide-range h[t=%d,j=%d]" % (t, j))

@@ -126,12 +126,14 @@ def test_ragged_shapes_against_oracle(moe, H, I, E, k, M):
 
 
 @pytest.mark.parametrize("H,I,E,k,M", [
-    (1024, 512, 4, 2, 80),    # ~40 assignments per expert: three of four experts on the tensor-core path
-    (512, 512, 4, 2, 600),    # ~300 per expert: two wide tiles per expert (224 + the rest)
-    (512, 1024, 16, 4, 160),  # ~40 per expert, spread: wide and 8-assignment tiles in the same call
+    (1024, 512, 4, 2, 80),    # ~40 assignments per expert: every expert on the tensor-core path
+    (512, 512, 4, 2, 600),    # ~300 per expert: two wide tiles per expert (192 + the rest)
+    (512, 1024, 16, 4, 160),  # ~40 per expert with I > H
+    (512, 512, 64, 4, 160),   # 3..19 per expert: mma.sync tiles and tensor-core tiles of N = 16 and 32
 ])
 def test_wide_tiles_against_oracle(moe, H, I, E, k, M):
-    # experts with 32 or more assignments take the tcgen05 path (H, I multiples of 512)
+    # experts with U.WIDE_MIN_TOKENS or more assignments take the tcgen05 path (H, I multiples of 512)
+    assert U.wide_path_on(M, H, I, E, k)
     shape = gen.LayerShape("wide", H, I, E, k, (M,))
     inp = gen.make_inputs(0, M, shape=shape, seed=7 * H + I + E + k + M)
     d = U.device_inputs(inp)
@@ -144,7 +146,7 @@ def test_wide_tiles_against_oracle(moe, H, I, E, k, M):
     assert int(st.item()) == moe.MOE_OK
     r = U.oracle_forward(inp)
     counts = np.bincount(r["topk_ids"].reshape(-1), minlength=E)
-    assert counts.max() >= 32                    # the case does reach the wide path
+    assert counts.max() >= U.WIDE_MIN_TOKENS     # the case does reach the wide path
     assert np.array_equal(ids.cpu().numpy(), r["topk_ids"])
     U.check_out(U.bf16_tensor_to_f64(out), r["out64"], "wide %s" % ((H, I, E, k, M),))
 
