@@ -23,7 +23,10 @@ Legs of the headline (one JSON line on rank 0):
   * cpu_baseline: the fp64 oracle on the host cores (rank 0, N=1), on a bounded
     sample of the same workload.
 `--impl reference` is the reference arm: the fp64 oracle alone, full layer calls on the host cores.
-With N>1 (torchrun) every rank runs an independent replica of the layer call.
+With N>1 (torchrun) the layer is split over the N GPUs along the expert intermediate dimension
+(decode_moe_layer_b200.sharded): each rank streams I/N of every expert, the ranks all-gather their
+fp32 [M,H] shares over NCCL and each reduces them in rank order; one step = the whole split call,
+timed eagerly (the collective sits inside it), max over ranks, strong scaling.
 """
 from __future__ import annotations
 
@@ -57,10 +60,13 @@ CSRC = os.path.join(ROOT, "decode_moe_layer_b200", "csrc")
 # kernel source they were taken on: (workload name, launch) -> (kernel source, summary)
 TRAFFIC_PROFILES = {
     ("dsv3_wide_h7168_i2048_e256_k8 M=512", "gate_up_tc_small"):
-        (os.path.join(CSRC, "grouped_wide.cu"),
+        ([os.path.join(CSRC, f) for f in ("grouped_wide.cu", "common.cuh", "tcgen05.cuh", "moe_internal.h")],
          os.path.join(ROOT, "profiles", "grouped_wide_dsv3_h7168_i2048_e256_k8_M512.md")),
+    ("dsv3_h7168_i2048_e256_k8 M=32", "gate_up"):
+        ([os.path.join(CSRC, f) for f in ("grouped_gemm.cu", "common.cuh", "moe_internal.h")],
+         os.path.join(ROOT, "profiles", "grouped_mxfp4_dsv3_h7168_i2048_e256_k8_M32.md")),
     ("decode_h2048_i768_e128_k8 M=8", "gate_up"):
-        (os.path.join(CSRC, "grouped_gemm.cu"),
+        ([os.path.join(CSRC, f) for f in ("grouped_gemm.cu", "common.cuh", "moe_internal.h")],
          os.path.join(ROOT, "profiles", "grouped_mxfp4_decode_h2048_i768_e128_k8_M8.md")),
 }
 
@@ -140,14 +146,18 @@ def algorithmic(shape, M, ids):
             "classes": {kind: sum(1 for c in cls.values() if c == kind) for kind in ("narrow", "small", "large")}}
 
 
-def kernel_code_hash(path):
-    """sha256[:16] of a kernel's source with comments and blank space removed: any change to its
-    code changes it, a change to its comments or layout does not."""
-    with open(path) as f:
-        src = f.read()
-    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
-    src = re.sub(r"//[^\n]*", " ", src)
-    return hashlib.sha256(" ".join(src.split()).encode()).hexdigest()[:16]
+def kernel_code_hash(paths):
+    """sha256[:16] of a kernel's sources (its file and the headers it includes, in order) with
+    comments and blank space removed: any change to their code changes it, a change to their
+    comments or layout does not."""
+    code = []
+    for path in paths:
+        with open(path) as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        code.append(" ".join(src.split()))
+    return hashlib.sha256("\n".join(code).encode()).hexdigest()[:16]
 
 
 def profiled_traffic(workload, launch):
@@ -326,8 +336,12 @@ def main():
     for (ci, M), is_headline in cases:
         shape = gen.CONFIGS[ci]
         steps = args.steps if (is_headline or args.sweep) else min(args.steps, args.other_steps)
-        rec = run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind,
-                       baselines=is_headline, steps=steps)
+        if world > 1:
+            rec = run_case_sharded(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks,
+                                   peak_kind, steps=steps)
+        else:
+            rec = run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind,
+                           baselines=is_headline, steps=steps)
         if rank == 0:
             print(json.dumps(rec), flush=True)
         torch.cuda.empty_cache()
@@ -485,6 +499,108 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
         rec["cpu_baseline"] = {"value": statistics.mean(times) * 1e6 * M / n_tok, "unit": UNIT, "cores": cores,
                                "kind": "oracle", "sample": oracle_sample_text(len(times), n_tok, M)}
     return rec
+
+
+def run_case_sharded(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind, steps):
+    """One workload on N GPUs, I-sharded: every rank holds its I/N slice of every expert, and a step
+    is this rank's share, the all-gather of the shares and the fixed-order reduction."""
+    from decode_moe_layer_b200 import sharded
+    H, I, E, k = shape.H, shape.I, shape.E, shape.k
+    inp = gen.make_inputs(ci, M, weights="torch", device=dev)
+    layer = sharded.IShardedLayer(inp.w13_q, inp.w13_s, inp.w2_q, inp.w2_s, k, device=dev)
+    inp.w13_q = inp.w13_s = inp.w2_q = inp.w2_s = None
+    torch.cuda.empty_cache()
+    Is = layer.I_shard
+    part_shape = gen.LayerShape(shape.name, H, Is, E, k, shape.Ms, shape.skew_bias)
+    xb = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).to(dev).view(torch.bfloat16)
+    wr = torch.from_numpy(inp.router_w).to(dev)
+    bias = None if inp.router_bias is None else torch.from_numpy(inp.router_bias).to(dev)
+    out = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    ids = torch.empty((M, k), dtype=torch.int32, device=dev)
+    flush = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def step(x=xb, o=out):
+        return layer.forward(x, wr, router_bias=bias, out=o)
+
+    layer.partial(xb, wr, router_bias=bias, topk_ids_out=ids)
+    torch.cuda.synchronize()
+    work = algorithmic(part_shape, M, ids.cpu().numpy())
+    clocks = ClockSampler(dev.index)
+    for _ in range(args.warmup):
+        torch.sum(flush)
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    for i in range(steps):
+        torch.sum(flush)
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    clk = clocks.stop()
+
+    # per-kernel attribution of this rank's share (the same kernels; the profile form rounds out)
+    ws = layer.workspace(M)
+    prof = {n: [] for n in moe.PROFILE_KERNELS}
+    for _ in range(10):
+        torch.sum(flush)
+        torch.cuda._sleep(2_000_000)
+        _, ms = moe.moe_mxfp4_forward_profile(xb, wr, layer.w13_q, layer.w13_s, layer.w2_q, layer.w2_s, k, ws,
+                                              router_bias=bias)
+        for n, v in ms.items():
+            prof[n].append(v)
+    kern_us = {n: statistics.mean(v) * 1e3 for n, v in prof.items()}
+
+    x_host = torch.empty((M, H), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(xb.cpu())
+    out_host = torch.empty((M, H), dtype=torch.bfloat16, pin_memory=True)
+    x_dev = torch.empty_like(xb)
+    e2e_ms = []
+    for i in range(args.warmup + steps):
+        torch.sum(flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x=x_dev)
+        out_host.copy_(out, non_blocking=True)
+        b.record()
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    barrier()
+    mean_us, e2e_us = max_over_ranks(dist, [statistics.mean(step_ms) * 1e3, statistics.mean(e2e_ms) * 1e3], dev)
+
+    hbm = peaks["hbm_gbs"]
+    tflops = peaks["bf16_tflops_sustained"]
+    # every rank streams its own slice at the same time: one rank's work sets the roofline
+    roof_us = max(work["bytes"] / (hbm * 1e3), work["flops"] / (tflops * 1e6))
+    call_bound = "hbm" if work["bytes"] / hbm > work["flops"] / (tflops * 1e3) else "tensor"
+    dominant = max(kern_us, key=kern_us.get)
+    dom = work["per_launch"].get(dominant, {"bytes": work["bytes"], "flops": work["flops"]})
+    if call_bound == "hbm":
+        roof = {"bound": "hbm", "achieved": dom["bytes"] / (kern_us[dominant] * 1e3), "peak": hbm, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": dom["flops"] / (kern_us[dominant] * 1e6), "peak": tflops,
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    exchange = M * H * 4 * (world - 1)
+    return {
+        "metric": METRIC, "value": mean_us, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": mean_us / 1e3, "higher_is_better": False, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16 (MXFP4 weights decoded exactly to bf16), fp32 accumulate",
+        "data": "synthetic",
+        "config": dict(workload_config(shape, M), parallelism="I-shard %d (I/%d = %d per GPU)" % (world, world, Is)),
+        "roofline_call": {"bound": call_bound, "roofline_us": roof_us, "frac": roof_us / mean_us,
+                          "peaks": peak_kind, "algorithmic_bytes_per_gpu": work["bytes"],
+                          "exchange_bytes_per_gpu": exchange, "touched_experts": work["touched"]},
+        "kernels_us": {n: v for n, v in kern_us.items() if v > 0},
+        "roofline": dict(kernel=dominant, traffic=None, peak_kind=peak_kind, **roof),
+        "e2e": {"value": e2e_us, "unit": UNIT, "h2d_bytes_per_step": M * H * 2, "d2h_bytes_per_step": M * H * 2,
+                "path": "pinned host x -> IShardedLayer.forward (share, NCCL all-gather, reduce) -> pinned host out"},
+        "gpu_launches": (moe.moe_forward_launches(M, H, Is, E, k) + 1) * steps,
+        "clocks": clk,
+    }
 
 
 def oracle_token_sample(M, k, cores=None):

@@ -20,9 +20,11 @@ from ._lib import (  # noqa: F401
     moe_gate_up_swiglu,
     moe_mxfp4_forward,
     moe_mxfp4_forward_ex,
+    moe_mxfp4_forward_partial,
     moe_mxfp4_forward_profile,
     PROFILE_KERNELS,
     moe_permute,
+    moe_reduce_partials,
     moe_route,
     moe_route_noalloc,
     moe_selftest_wait_timeout,

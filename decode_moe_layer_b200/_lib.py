@@ -22,7 +22,8 @@ MOE_ERR_TIMEOUT = -5
 EXPORTS = (
     "moe_status_string", "moe_last_cuda_error", "moe_route", "moe_permute", "moe_gate_up_swiglu",
     "moe_down_combine", "moe_mxfp4_forward", "moe_workspace_bytes", "moe_forward_launches", "moe_mxfp4_forward_ex",
-    "moe_mxfp4_forward_profile", "moe_route_noalloc", "moe_selftest_wait_timeout",
+    "moe_mxfp4_forward_profile", "moe_route_noalloc", "moe_selftest_wait_timeout", "moe_mxfp4_forward_partial",
+    "moe_reduce_partials",
 )
 PROFILE_KERNELS = ("route_logits", "route_select", "permute", "gate_up", "gather", "gate_up_tc_small",
                    "gate_up_tc_large", "down", "down_tc_small", "down_tc_large", "combine")
@@ -75,6 +76,10 @@ def load():
     lib.moe_mxfp4_forward_profile.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, S, P, P]
     lib.moe_selftest_wait_timeout.restype = I
     lib.moe_selftest_wait_timeout.argtypes = [P, P]
+    lib.moe_mxfp4_forward_partial.restype = I
+    lib.moe_mxfp4_forward_partial.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, P, P, S, P]
+    lib.moe_reduce_partials.restype = I
+    lib.moe_reduce_partials.argtypes = [P, I, P, I, I, P]
     _lib = lib
     return lib
 
@@ -211,6 +216,37 @@ def moe_mxfp4_forward_ex(x, router_w, w13_q, w13_s, w2_q, w2_s, k: int, workspac
                                      0 if workspace is None else workspace.numel() * workspace.element_size(),
                                      _stream(stream))
     _check(rc, "moe_mxfp4_forward_ex")
+    return out
+
+
+def moe_mxfp4_forward_partial(x, router_w, w13_q, w13_s, w2_q, w2_s, k: int, workspace, router_bias=None,
+                              partial_out=None, topk_ids_out=None, topk_w_out=None, status_out=None, stream=None):
+    """One rank's fp32 share [M,H] of an I-sharded layer; the weights are the rank's slices
+    (w13 [E, 2*I_shard, H/2], w2 [E, H, I_shard/2], as sharded.shard_weights returns them)."""
+    _need(x, torch.bfloat16, "x")
+    M, H = x.shape
+    E, I2, _ = w13_q.shape
+    if partial_out is None:
+        partial_out = torch.empty((M, H), dtype=torch.float32, device=x.device)
+    _need(partial_out, torch.float32, "partial_out")
+    rc = load().moe_mxfp4_forward_partial(_ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(w13_q), _ptr(w13_s),
+                                          _ptr(w2_q), _ptr(w2_s), _ptr(partial_out), M, H, I2 // 2, E, k,
+                                          _ptr(topk_ids_out), _ptr(topk_w_out), _ptr(status_out), _ptr(workspace),
+                                          0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                          _stream(stream))
+    _check(rc, "moe_mxfp4_forward_partial")
+    return partial_out
+
+
+def moe_reduce_partials(partials, out=None, stream=None):
+    """out [M,H] bf16 = bf16(sum over g ascending of partials[g]) for partials [G,M,H] fp32."""
+    _need(partials, torch.float32, "partials")
+    G, M, H = partials.shape
+    if out is None:
+        out = torch.empty((M, H), dtype=torch.bfloat16, device=partials.device)
+    _need(out, torch.bfloat16, "out")
+    rc = load().moe_reduce_partials(_ptr(partials), G, _ptr(out), M, H, _stream(stream))
+    _check(rc, "moe_reduce_partials")
     return out
 
 

@@ -338,7 +338,7 @@ static WideLists wide_lists(char *ws, const Layout &L)
 static int forward_impl(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
                         const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M, int H,
                         int I, int E, int k, int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
-                        char *ws, const Layout &L, cudaStream_t s, Marks *marks = nullptr)
+                        char *ws, const Layout &L, cudaStream_t s, Marks *marks = nullptr, bool f32_out = false)
 {
     int *status = reinterpret_cast<int *>(ws + L.status);
     float *partial = reinterpret_cast<float *>(ws + L.partial);
@@ -396,7 +396,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
                       pdl, marks);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_combine(y, tw, out, M, H, k, s, pdl));
+    MOE_TRY(launch_combine(y, tw, out, f32_out, M, H, k, s, pdl));
     MOE_AFTER(marks, s, kProfCombine);
     return MOE_OK;
 }
@@ -404,7 +404,7 @@ static int forward_impl(const void *x, const float *router_w, const float *route
 static int check_forward_args(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,
                               const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s, void *out, int M,
                               int H, int I, int E, int k, const int32_t *topk_ids_out, const float *topk_w_out,
-                              const int32_t *status_out)
+                              const int32_t *status_out, size_t out_elem_bytes = 2)
 {
     int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
@@ -417,7 +417,7 @@ static int check_forward_args(const void *x, const float *router_w, const float 
         (topk_w_out && !aligned(topk_w_out, 4)) || (status_out && !aligned(status_out, 4)))
         return MOE_ERR_INVALID_ARG;
     const size_t xbytes = static_cast<size_t>(M) * H * 2;
-    if (M > 0 && overlaps(x, xbytes, out, xbytes)) return MOE_ERR_INVALID_ARG;
+    if (M > 0 && overlaps(x, xbytes, out, static_cast<size_t>(M) * H * out_elem_bytes)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
@@ -572,7 +572,7 @@ int moe_down_combine(const void *h_bf16, const uint8_t *w2_q, const uint8_t *w2_
                       stream, false);
         if (rc != MOE_OK) return rc;
     }
-    MOE_TRY(launch_combine(y, topk_w, out_bf16, M, H, k, stream, false));
+    MOE_TRY(launch_combine(y, topk_w, out_bf16, false, M, H, k, stream, false));
     return MOE_OK;
 }
 
@@ -590,6 +590,36 @@ int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *rout
     if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
     return forward_impl(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, out, M, H, I, E, k, topk_ids_out,
                         topk_w_out, status_out, static_cast<char *>(workspace), L, stream);
+}
+
+int moe_mxfp4_forward_partial(const void *x, const float *router_w, const float *router_bias,
+                              const uint8_t *w13_q, const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s,
+                              float *partial_out, int M, int H, int I_shard, int E, int k, int32_t *topk_ids_out,
+                              float *topk_w_out, int32_t *status_out, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream)
+{
+    int rc = check_forward_args(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, partial_out, M, H, I_shard, E, k,
+                                topk_ids_out, topk_w_out, status_out, 4);
+    if (rc != MOE_OK) return rc;
+    if (M == 0) return MOE_OK;
+    const Layout L = make_layout(M, H, I_shard, E, k);
+    if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE;
+    return forward_impl(x, router_w, router_bias, w13_q, w13_s, w2_q, w2_s, partial_out, M, H, I_shard, E, k,
+                        topk_ids_out, topk_w_out, status_out, static_cast<char *>(workspace), L, stream, nullptr,
+                        true);
+}
+
+int moe_reduce_partials(const float *partials, int G, void *out_bf16, int M, int H, cudaStream_t stream)
+{
+    if (G <= 0 || M < 0 || H <= 0) return MOE_ERR_INVALID_ARG;
+    if (H % 4 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0) return MOE_OK;
+    if (!partials || !out_bf16 || !aligned(partials, 16) || !aligned(out_bf16, 16)) return MOE_ERR_INVALID_ARG;
+    const size_t pbytes = static_cast<size_t>(G) * M * H * 4;
+    if (overlaps(partials, pbytes, out_bf16, static_cast<size_t>(M) * H * 2)) return MOE_ERR_INVALID_ARG;
+    MOE_TRY(launch_reduce_partials(partials, G, out_bf16, M, H, stream));
+    return MOE_OK;
 }
 
 int moe_mxfp4_forward_profile(const void *x, const float *router_w, const float *router_bias, const uint8_t *w13_q,

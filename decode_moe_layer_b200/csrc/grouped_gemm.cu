@@ -209,18 +209,24 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 nx_flat = __ldcg(&tp->flat[lane & (kTileTokensMax - 1)]);
             }
         };
-        // down: h copies of the first stages, held back until gate_up has completed
+        // down: h copies of the first stages, held back until gate_up has completed (the rows of
+        // a down tile are consecutive in h, so a stage's copies are its first row, row count,
+        // K offset and bytes per row)
         bool h_ready = kGateUp;
-        const __nv_bfloat16 *pend_src[kStages];
+        int pend_p0[kStages], pend_cnt[kStages], pend_kc[kStages];
         uint32_t pend_bytes[kStages];
 #pragma unroll
-        for (int i = 0; i < kStages; ++i) pend_bytes[i] = 0;
+        for (int i = 0; i < kStages; ++i) pend_p0[i] = pend_cnt[i] = pend_kc[i] = 0, pend_bytes[i] = 0;
         auto release_h = [&]() {
             pdl_wait();
+            if (elect_one()) {
 #pragma unroll
-            for (int i = 0; i < kStages; ++i)
-                if (pend_bytes[i] != 0)
-                    bulk_load(ast + i * kActStageBytes + (lane - 16) * kActPitch, pend_src[i], pend_bytes[i], &full[i]);
+                for (int i = 0; i < kStages; ++i)
+                    for (int j = 0; j < pend_cnt[i]; ++j)
+                        bulk_load(ast + i * kActStageBytes + j * kActPitch,
+                                  act + static_cast<size_t>(pend_p0[i] + j) * K + pend_kc[i], pend_bytes[i], &full[i]);
+            }
+            __syncwarp();
             h_ready = true;
         };
         // Items come from the call's work queue (an atomic counter, zeroed by the first kernel of
@@ -260,14 +266,15 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 item_p0[item_ctr % kItemQ] = p0;
                 item_cnt[item_ctr % kItemQ] = cnt;
             }
+            __syncwarp();   // orders these stores before the arrival of whichever lane issues it
             const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
             const int row_a = kGateUp ? e * 2 * I + rb * 32 : e * H + rb * kItemRows;
             const int row_b = row_a + I;                               // gate_up only
             const int valid_rows = kGateUp ? kItemRows : min(kItemRows, H - rb * kItemRows);
-            // this lane's activation row (gate_up: the x row of the slot's token; down: the h row)
-            const __nv_bfloat16 *arow = kGateUp ? act + static_cast<size_t>(flat / k) * K
-                                         : act + static_cast<size_t>(p0 + min(lane, cnt - 1)) * K;
+            // gate_up: lane j < cnt holds the element offset of the x row of the tile's token j
+            // (down reads h rows p0 .. p0 + cnt - 1)
+            const long long xrow = kGateUp ? static_cast<long long>(flat / k) * K : 0;
             if (!stage_scales) {
                 const int b = item_ctr & 1;
                 // the scale buffer frees only when compute has finished item_ctr - 2, which may
@@ -275,7 +282,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 if (!h_ready && item_ctr >= 2) release_h();
                 mbar_wait(&sempty[b], ((item_ctr >> 1) & 1) ^ 1, aborted, status);
                 aborted = __any_sync(0xffffffffu, aborted);   // keep the warp's control flow uniform
-                if (!aborted && lane == 0) {
+                if (!aborted && elect_one()) {
                     uint8_t *dst = sbuf + b * plan.sbuf_bytes;
                     mbar_arrive_expect_tx(&sfull[b], static_cast<uint32_t>(valid_rows * kblocks));
                     if (kGateUp) {
@@ -302,32 +309,43 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 const int halves = kGateUp ? 2 : 1;
                 const uint32_t bytes = halves * (ncols * kBoxBytes + (stage_scales ? kScaleBoxBytes : 0)) +
                                        cnt * act_bytes;
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes);
-                __syncwarp();
+                // One elected lane issues every copy of the stage: copies issued from several lanes
+                // of a divergent branch are serialised anyway, and slowly while the compute warps
+                // keep the SM's issue slots busy.  Gate_up boxes: columns of the gate rows, then
+                // columns of the up rows; down: columns.
                 uint8_t *st = wst + s * kStageBytes;
-                // gate_up boxes: columns of the gate rows, then columns of the up rows; down: columns
-                if (lane < ncols) {
-                    tma_load_2d(st + lane * kBoxBytes, &wmap, kb + 128 * lane, row_a, &full[s]);
-                    if (kGateUp) tma_load_2d(st + (kBoxCols + lane) * kBoxBytes, &wmap, kb + 128 * lane, row_b, &full[s]);
-                }
-                if (stage_scales && lane == 8) {
-                    uint8_t *ss = sst + s * kStageScaleBytes;
-                    tma_load_2d(ss, &smap, kc / 32, row_a, &full[s]);
-                    if (kGateUp) tma_load_2d(ss + kScaleBoxBytes, &smap, kc / 32, row_b, &full[s]);
-                }
-                if (lane >= 16 && lane - 16 < cnt) {
-                    const __nv_bfloat16 *src = (kGateUp ? arow : act + static_cast<size_t>(p0 + lane - 16) * K) + kc;
-                    if (h_ready) {
-                        bulk_load(ast + s * kActStageBytes + (lane - 16) * kActPitch, src, act_bytes, &full[s]);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < kStages; ++i)   // stage_ctr < kStages here, so s == stage_ctr
-                            if (i == s) {
-                                pend_src[i] = src;
-                                pend_bytes[i] = act_bytes;
-                            }
+                uint8_t *sa = ast + s * kActStageBytes;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[s], bytes);
+                    for (int col = 0; col < ncols; ++col) {
+                        tma_load_2d(st + col * kBoxBytes, &wmap, kb + 128 * col, row_a, &full[s]);
+                        if (kGateUp) tma_load_2d(st + (kBoxCols + col) * kBoxBytes, &wmap, kb + 128 * col, row_b, &full[s]);
                     }
+                    if (stage_scales) {
+                        uint8_t *ss = sst + s * kStageScaleBytes;
+                        tma_load_2d(ss, &smap, kc / 32, row_a, &full[s]);
+                        if (kGateUp) tma_load_2d(ss + kScaleBoxBytes, &smap, kc / 32, row_b, &full[s]);
+                    }
+                    if (!kGateUp && h_ready)
+                        for (int j = 0; j < cnt; ++j)
+                            bulk_load(sa + j * kActPitch, act + static_cast<size_t>(p0 + j) * K + kc, act_bytes, &full[s]);
                 }
+                if (kGateUp) {
+                    for (int j = 0; j < cnt; ++j) {
+                        const long long row = __shfl_sync(0xffffffffu, xrow, j);
+                        if (elect_one()) bulk_load(sa + j * kActPitch, act + row + kc, act_bytes, &full[s]);
+                    }
+                } else if (!h_ready) {
+#pragma unroll
+                    for (int i = 0; i < kStages; ++i)   // stage_ctr < kStages here, so s == stage_ctr
+                        if (i == s) {
+                            pend_p0[i] = p0;
+                            pend_cnt[i] = cnt;
+                            pend_kc[i] = kc;
+                            pend_bytes[i] = act_bytes;
+                        }
+                }
+                __syncwarp();
                 ++stages_issued;
             }
         }
@@ -602,9 +620,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 
 // out[t] = bf16( sum_j w[t*k + j] * y[t*k + j] ), slots j ascending (a fixed order, no atomics);
 // y holds the unweighted down-projection row of every assignment.  Four outputs per thread.
+// kF32: the same sum stored unrounded in fp32 (one rank's share of an I-sharded layer).
+template <bool kF32>
 __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y, const float *__restrict__ topk_w,
-                                                      __nv_bfloat16 *__restrict__ out,
-                                                      int M, int H, int k)
+                                                      void *__restrict__ out, int M, int H, int k)
 {
     pdl_wait();
     const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -622,8 +641,34 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
         a.z = fmaf(w, v.z, a.z);
         a.w = fmaf(w, v.w, a.w);
     }
-    __nv_bfloat162 o[2] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w)};
-    *reinterpret_cast<uint2 *>(out + static_cast<size_t>(t) * H + c) = *reinterpret_cast<uint2 *>(o);
+    const size_t o = static_cast<size_t>(t) * H + c;
+    if (kF32) {
+        *reinterpret_cast<float4 *>(static_cast<float *>(out) + o) = a;
+    } else {
+        __nv_bfloat162 b[2] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w)};
+        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(out) + o) = *reinterpret_cast<uint2 *>(b);
+    }
+}
+
+// out[i] = bf16( sum_g partials[g][i] ), g = 0 .. G-1 ascending: the fixed-order reduction of the
+// ranks' fp32 shares of an I-sharded layer (the same bits on every rank and in every run).  Four
+// outputs per thread; n4 = M * H / 4.
+__global__ void __launch_bounds__(256) reduce_partials_kernel(const float *__restrict__ partials, int G, size_t n4,
+                                                              __nv_bfloat16 *__restrict__ out)
+{
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    const float4 *p = reinterpret_cast<const float4 *>(partials);
+    float4 a = __ldg(p + i);
+    for (int g = 1; g < G; ++g) {
+        const float4 v = __ldg(p + static_cast<size_t>(g) * n4 + i);
+        a.x += v.x;
+        a.y += v.y;
+        a.z += v.z;
+        a.w += v.w;
+    }
+    __nv_bfloat162 b[2] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w)};
+    reinterpret_cast<uint2 *>(out)[i] = *reinterpret_cast<uint2 *>(b);
 }
 
 template <bool kGateUp, int kN>
@@ -671,13 +716,24 @@ cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, co
                                     status_out, I, I, H, 1, 1, max_tiles, s, pdl);
 }
 
-cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
-                           bool pdl)
+cudaError_t launch_combine(const float *y, const float *topk_w, void *out, bool f32_out, int M, int H, int k,
+                           cudaStream_t s, bool pdl)
 {
     const size_t n = static_cast<size_t>(M) * H / 4;
     const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
-    return launch_ex(combine_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, y, topk_w,
-                     static_cast<__nv_bfloat16 *>(out), M, H, k);
+    if (f32_out)
+        return launch_ex(combine_kernel<true>, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, y, topk_w, out, M,
+                         H, k);
+    return launch_ex(combine_kernel<false>, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, s, pdl, y, topk_w, out, M, H,
+                     k);
+}
+
+cudaError_t launch_reduce_partials(const float *partials, int G, void *out, int M, int H, cudaStream_t s)
+{
+    const size_t n4 = static_cast<size_t>(M) * H / 4;
+    const unsigned blocks = static_cast<unsigned>((n4 + 255) / 256);
+    reduce_partials_kernel<<<blocks > 0 ? blocks : 1, 256, 0, s>>>(partials, G, n4, static_cast<__nv_bfloat16 *>(out));
+    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -229,8 +229,9 @@ cudaError_t launch_down(const CUtensorMap &w2_map, const CUtensorMap &s2_map, co
                         const __nv_bfloat16 *h_p4, const int32_t *sorted_ids, const ExpertTile *tiles,
                         const int *n_tiles, float *y, int *status, int32_t *status_out, int H, int I, int width,
                         int max_tiles, cudaStream_t s, bool pdl);
-cudaError_t launch_combine(const float *y, const float *topk_w, void *out, int M, int H, int k, cudaStream_t s,
-                           bool pdl);
+cudaError_t launch_combine(const float *y, const float *topk_w, void *out, bool f32_out, int M, int H, int k,
+                           cudaStream_t s, bool pdl);
+cudaError_t launch_reduce_partials(const float *partials, int G, void *out, int M, int H, cudaStream_t s);
 cudaError_t launch_gather_wide_rows(const __nv_bfloat16 *x_p4, const int32_t *sorted_ids, const WideLists &wl,
                                     __nv_bfloat16 *x_perm, int H, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_wide(bool gate_up, bool small, const CUtensorMap &wmap, const CUtensorMap &smap,

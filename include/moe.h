@@ -208,6 +208,37 @@ int moe_mxfp4_forward_ex(const void *x, const float *router_w, const float *rout
                          int32_t *topk_ids_out, float *topk_w_out, int32_t *status_out,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * One rank's share of the layer split over G GPUs along the expert intermediate dimension
+ * ("I-sharding"; the pages' multi-GPU data point, expert parallelism over 8 GPUs in "The
+ * Systematic Optimization Campaign", chunk 8.0, ran slower than one GPU at low concurrency and
+ * failed under load, so the split here keeps every expert on every rank instead).
+ * Rank r of G holds, for every expert, gate rows [r*I_shard, (r+1)*I_shard) followed by the
+ * same up rows, as w13_q [E, 2*I_shard, H/2] / w13_s [E, 2*I_shard, H/32], and the matching K
+ * range of the down projection, w2_q [E, H, I_shard/2] / w2_s [E, H, I_shard/32]: exactly the
+ * weights of a layer with intermediate size I_shard (I_shard a multiple of 32).  Routing runs in
+ * full on every rank, so ids and weights are the same bits everywhere.  partial_out [M,H] fp32
+ * (16-byte aligned) receives sum_j w[t,j] * (W2_slice h_slice)[t,j] in slot order, NOT rounded.
+ * The ranks then exchange their partials (an all-gather into [G,M,H], rank order) and each calls
+ * moe_reduce_partials.  Workspace: moe_workspace_bytes(M, H, I_shard, E, k).  Other arguments,
+ * errors and status as moe_mxfp4_forward_ex.
+ */
+int moe_mxfp4_forward_partial(const void *x, const float *router_w, const float *router_bias,
+                              const uint8_t *w13_q, const uint8_t *w13_s, const uint8_t *w2_q, const uint8_t *w2_s,
+                              float *partial_out, int M, int H, int I_shard, int E, int k, int32_t *topk_ids_out,
+                              float *topk_w_out, int32_t *status_out, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/*
+ * out[t,c] = bf16( sum_{g = 0 .. G-1} partials[g][t][c] ) with g ascending: the fixed-order
+ * reduction of G ranks' moe_mxfp4_forward_partial outputs, stacked as partials [G,M,H] fp32
+ * (device, 16-byte aligned; out [M,H] bf16, 16-byte aligned, not overlapping it).  Every rank
+ * that reduces the same stack gets the same bits.  With G = 1 it returns what
+ * moe_mxfp4_forward_ex writes for the same layer.  H must be a multiple of 4.
+ * Asynchronous on `stream`; MOE_ERR_INVALID_ARG for G <= 0, M < 0, H <= 0 or a bad pointer.
+ */
+int moe_reduce_partials(const float *partials, int G, void *out_bf16, int M, int H, cudaStream_t stream);
+
 /* Entries of moe_mxfp4_forward_profile's output. */
 #define MOE_PROFILE_KERNELS 11
 
