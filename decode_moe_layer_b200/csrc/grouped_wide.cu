@@ -137,6 +137,40 @@ __device__ __forceinline__ float wide_clamp_swiglu(float g, float u)
     return a / (1.0f + expf(-a)) * c;
 }
 
+// One dequant thread's share of an A unit: packed row r of the stage (128-byte swizzled box
+// columns), sub-tiles j0 .. j0 + kSubsN - 1 (64 K each), E8M0 bytes eb (byte b of the unit's block
+// b, two blocks per sub-tile).  Each sub-tile's 64 weights become 32 TMEM columns of this thread's
+// lane, K 64c + 32h + 8u + i in the low half of column 32c + 16h + 4u + i and + 4 in its high half
+// (the P4 pairing).  kLarge: some byte of the warp exceeds 128, so the two-multiply decode.
+// The stores are left in flight; the caller waits for them.
+template <int kSubsN, bool kLarge>
+__device__ __forceinline__ void dequant_unit(const uint8_t *pk, int r, int j0, const uint32_t (&eb)[2], uint32_t a_unit)
+{
+    using namespace wide;
+#pragma unroll
+    for (int c = 0; c < kSubsN; ++c) {
+        const int j = j0 + c;
+        uint32_t f[32];
+        uint4 w[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int ch = (j & 3) * 2 + h;
+            w[h] = *reinterpret_cast<const uint4 *>(pk + (j >> 2) * kPackedCol + r * 128 + ((ch ^ (r & 7)) << 4));
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int b = 2 * c + h;
+            const uint32_t e = (eb[b >> 2] >> (8 * (b & 3))) & 0xFFu;
+            uint32_t(&fo)[16] = *reinterpret_cast<uint32_t(*)[16]>(&f[16 * h]);
+            mxfp4x8_to_bf16x2_p4(w[h].x, e, kLarge, *reinterpret_cast<uint32_t(*)[4]>(&fo[0]));
+            mxfp4x8_to_bf16x2_p4(w[h].y, e, kLarge, *reinterpret_cast<uint32_t(*)[4]>(&fo[4]));
+            mxfp4x8_to_bf16x2_p4(w[h].z, e, kLarge, *reinterpret_cast<uint32_t(*)[4]>(&fo[8]));
+            mxfp4x8_to_bf16x2_p4(w[h].w, e, kLarge, *reinterpret_cast<uint32_t(*)[4]>(&fo[12]));
+        }
+        tmem_st32(a_unit + static_cast<uint32_t>(32 * c), f);
+    }
+}
+
 template <bool kGateUp, bool kSmall>
 __global__ void __launch_bounds__(wide::kThreads, 1)
 grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap smap,
@@ -343,26 +377,24 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     mbar_wait(&a_empty[ab], ((unit_ctr / P::kABufs) & 1) ^ 1, aborted, status);
                     if (aborted) break;
                     tc_fence_after();   // the MMAs that read this A unit are complete
-                    for (int c = 0; c < P::kUnitSubs; ++c) {
-                        const int j = uu * P::kUnitSubs + c;   // 64-K sub-tile within the stage
-                        // 32 packed bytes of row r: box column j / 4, 16-byte chunks (j % 4) * 2 + h
-                        uint32_t f[32];
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int ch = (j & 3) * 2 + h;
-                            const uint4 w = *reinterpret_cast<const uint4 *>(pk + (j >> 2) * kPackedCol + r * 128 +
-                                                                             ((ch ^ (r & 7)) << 4));
-                            const uint32_t sbyte = sc[r * 16 + 2 * j + h];
-                            const bool large = __any_sync(0xffffffffu, sbyte > 128u);
-                            mxfp4x8_to_bf16x2_p4(w.x, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h]));
-                            mxfp4x8_to_bf16x2_p4(w.y, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h + 4]));
-                            mxfp4x8_to_bf16x2_p4(w.z, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h + 8]));
-                            mxfp4x8_to_bf16x2_p4(w.w, sbyte, large, *reinterpret_cast<uint32_t(*)[4]>(&f[16 * h + 12]));
-                        }
-                        // column 32c + 16h + 4u + i of the unit holds K 64c + 32h + 8u + i (low half) and
-                        // 64c + 32h + 8u + i + 4 (high half): MMA K positions 2 col, 2 col + 1 in P4 order
-                        tmem_st32(tmem + a_lane + static_cast<uint32_t>(P::kACol0 + ab * P::kACols + 32 * c), f);
+                    // the unit's E8M0 bytes of row r (2 per 64-K sub-tile), one load; the scale
+                    // folds into the decode's multiply unless some byte of the warp exceeds 128
+                    uint32_t eb[2];
+                    if (P::kUnitSubs == 4) {
+                        const uint2 v = *reinterpret_cast<const uint2 *>(sc + r * 16 + uu * 8);
+                        eb[0] = v.x;
+                        eb[1] = v.y;
+                    } else {
+                        eb[0] = *reinterpret_cast<const uint32_t *>(sc + r * 16 + uu * 4);
+                        eb[1] = 0;
                     }
+                    const bool large = __any_sync(0xffffffffu, __vcmpgtu4(eb[0], 0x80808080u) | __vcmpgtu4(eb[1], 0x80808080u));
+                    const uint32_t a_unit = tmem + a_lane + static_cast<uint32_t>(P::kACol0 + ab * P::kACols);
+                    if (!large)
+                        dequant_unit<P::kUnitSubs, false>(pk, r, uu * P::kUnitSubs, eb, a_unit);
+                    else
+                        dequant_unit<P::kUnitSubs, true>(pk, r, uu * P::kUnitSubs, eb, a_unit);
+                    tmem_wait_st();
                     if (quarter == 0 && lane == 0) a_item[ab] = item;
                     tc_fence_before();
                     __syncwarp();
@@ -401,37 +433,51 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int spb = subs_per_slot(nbox);
             const uint32_t idesc = umma_idesc_bf16(kRows, 16 * nbox);
             const uint32_t d_tmem = tmem + static_cast<uint32_t>(db * P::kAccCols);
+            // B descriptor units (16 bytes) between consecutive sub-tiles of a slot
+            const uint32_t b_step = static_cast<uint32_t>(nbox * kBBox) >> 4;
             for (int u = 0; u < n_units; ++u, ++unit_ctr) {
                 ab = unit_ctr % P::kABufs;
                 if (u > 0) mbar_wait(&a_full[ab], (unit_ctr / P::kABufs) & 1, aborted, status);
                 if (aborted) break;
                 tc_fence_after();
-                for (int c = 0; c < P::kUnitSubs; ++c) {
-                    const int j = u * P::kUnitSubs + c;
+                const uint32_t a_unit = tmem + static_cast<uint32_t>(P::kACol0 + ab * P::kACols);
+                // the unit's sub-tiles, one B slot at a time: a wait on the slot, then one elected
+                // lane issues all of the slot's MMAs of this unit back to back (the warp shares its
+                // scheduler with dequant warps, so every instruction it spends between MMAs delays
+                // the tensor pipe)
+                for (int c0 = 0; c0 < P::kUnitSubs;) {
+                    const int j = u * P::kUnitSubs + c0;
                     const int bb = bload % kBBufs, uo = j % spb;
                     if (uo == 0) {
                         mbar_wait(&b_full[bb], (bload / kBBufs) & 1, aborted, status);
                         if (aborted) break;
                         tc_fence_after();
                     }
-                    // operands computed by the whole warp; one elected lane issues
-                    const uint32_t a_tmem = tmem + static_cast<uint32_t>(P::kACol0 + ab * P::kACols + 32 * c);
-                    const uint64_t b_desc = umma_sdesc_sw128(smem_u32(smem + kOffB + bb * kBTile + uo * nbox * kBBox));
-                    const uint32_t first = (j == 0) ? 0u : 1u;
+                    const int nsub = min(spb - uo, P::kUnitSubs - c0);
+                    const bool slot_end = uo + nsub == spb;
+                    const bool unit_end = c0 + nsub == P::kUnitSubs;
+                    const uint64_t b0 = umma_sdesc_sw128(smem_u32(smem + kOffB + bb * kBTile + uo * nbox * kBBox));
                     if (elect_one()) {
-                        // K steps of 16 advance A by 8 columns and B by 32 bytes (2 in the descriptor)
-                        umma_f16_tmem_a(d_tmem, a_tmem, b_desc, idesc, first);
-                        umma_f16_tmem_a(d_tmem, a_tmem + 8, b_desc + 2, idesc, 1u);
-                        umma_f16_tmem_a(d_tmem, a_tmem + 16, b_desc + 4, idesc, 1u);
-                        umma_f16_tmem_a(d_tmem, a_tmem + 24, b_desc + 6, idesc, 1u);
-                        if (uo == spb - 1) umma_commit(smem_u32(&b_empty[bb]));   // the slot's last sub-tile
+#pragma unroll
+                        for (int c = 0; c < P::kUnitSubs; ++c) {
+                            if (c < nsub) {
+                                // K steps of 16 advance A by 8 columns and B by 32 bytes (2 in the descriptor)
+                                const uint32_t at = a_unit + static_cast<uint32_t>(32 * (c0 + c));
+                                const uint64_t bd = b0 + static_cast<uint64_t>(c) * b_step;
+                                umma_f16_tmem_a(d_tmem, at, bd, idesc, (j + c == 0) ? 0u : 1u);
+                                umma_f16_tmem_a(d_tmem, at + 8, bd + 2, idesc, 1u);
+                                umma_f16_tmem_a(d_tmem, at + 16, bd + 4, idesc, 1u);
+                                umma_f16_tmem_a(d_tmem, at + 24, bd + 6, idesc, 1u);
+                            }
+                        }
+                        if (slot_end) umma_commit(smem_u32(&b_empty[bb]));   // the slot's last sub-tile
+                        if (unit_end) umma_commit(smem_u32(&a_empty[ab]));
                     }
                     __syncwarp();
-                    if (uo == spb - 1) ++bload;
+                    if (slot_end) ++bload;
+                    c0 += nsub;
                 }
                 if (aborted) break;
-                if (elect_one()) umma_commit(smem_u32(&a_empty[ab]));
-                __syncwarp();
             }
             if (aborted) break;
             if (elect_one()) umma_commit(smem_u32(&d_full[db]));

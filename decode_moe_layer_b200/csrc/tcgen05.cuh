@@ -71,8 +71,9 @@ __device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
                  : "memory");
 }
 
-// 32 consecutive 32-bit columns of this thread's TMEM lane (lane as in tmem_ld16) from registers,
-// then wait until the stores are done.
+// 32 consecutive 32-bit columns of this thread's TMEM lane (lane as in tmem_ld16) from registers.
+// The store is asynchronous: tmem_wait_st() must follow before the columns are read by anything
+// else (the registers themselves are free again as soon as the instruction has issued).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32])
 {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -82,8 +83,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
                  "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]),
                  "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
                  : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+
+// Waits until every tcgen05.st this thread issued has completed.
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // The mbarrier receives one arrival when every tcgen05 operation this thread issued before
 // is complete.
