@@ -12,14 +12,19 @@
 //
 // Measured on this part (one CTA per SM issuing back to back): a kind::f16 MMA of 128 x N x 16
 // with A in tensor memory takes about 40-50 cycles for N <= 64 and N / 2 above; every
-// tcgen05.commit costs the issuing thread about 80 cycles and every mbarrier wait about 185, even
-// on a completed phase.  So the dequant warps hand the MMA warp large A units (a wait and a commit
-// cover 8 or 16 MMAs), and the tensor memory is split by tile size (two kernels):
+// tcgen05.commit costs the issuing thread about 80 cycles and a check of an mbarrier phase about
+// 100-130, even a completed one.  Inside this kernel the MMA warp shares its scheduler with
+// ALU-heavy dequant warps and gets a small share of the issue slots (a clock64 timeline of one
+// CTA: about 1500 cycles per 16-MMA unit, of which about 550 were its wait on the activation
+// slot), so everything that can leave the MMA warp does: the dequant warps hand it large A units
+// (one wait and one commit per 8 or 16 MMAs) only once their activations have landed, and its
+// loop keeps the arithmetic between MMAs minimal.  The tensor memory is split by tile size (two
+// kernels):
 //  * small tiles (kWideMinTokens .. kWideSmallMax assignments): two 64-column accumulators and
 //    three A units of 256 K (128 columns each);
 //  * large tiles (up to kWideTokens): two 192-column accumulators and two A units of 128 K.
 //
-// One persistent CTA per SM, 20 warps:
+// One persistent CTA per SM, 16 warps:
 //  * warp 0 (weights producer): per 512-K stage, TMA copies of the item's packed E2M1 rows
 //    (128 rows x 256 bytes, 128-byte swizzle) and their E8M0 scales into a 3-stage ring;
 //    items come from the call's work queue, the ids reach the other warps through shared
@@ -29,22 +34,24 @@
 //    into a 4-slot ring; a slot takes 1 to 8 consecutive 64-K sub-tiles, as many as fit, so
 //    that narrow tiles keep many sub-tiles in flight against the copies' latency.  Rows past
 //    the tile are read and ignored.
-//  * warps 4..15 (dequant, three groups of four): a group decodes a whole A unit, each thread
+//  * warp 3 (activations watcher): waits on every slot load in load order and publishes the
+//    count that has landed (a release store the dequant groups read with acquire loads).
+//  * warps 4..11 (dequant, two groups of four): a group decodes a whole A unit, each thread
 //    the weights of one row, to bf16 with the row's E8M0 block scales folded in
 //    (mxfp4x8_to_bf16x2_p4: exact for every scale byte whose scaled values are bf16 values),
 //    and stores them with tcgen05.st into the unit's A buffer in tensor memory (TMEM lane = A
 //    row; a warp reaches the 32 lanes of its warp index mod 4).  The groups take units in turn
-//    (group g always unit g), so one group's store latency overlaps the others' decoding.  The decode pairs K 8j+i with
-//    8j+i+4 in a TMEM column, so the activation rows are stored in the matching P4 K order
-//    (common.cuh): x by the router (gathered into x_perm by gather_wide_rows_kernel), h by the
-//    gate_up epilogues.  gate_up interleaves gate row i and up row i as A rows 2i, 2i+1, so one
-//    TMEM lane pair holds g and u.  A never passes through shared memory, which leaves
-//    shared-memory bandwidth to the TMA copies and the B operand.
+//    (group g always unit g), so one group's decoding overlaps the other's hand-over.  The
+//    decode pairs K 8j+i with 8j+i+4 in a TMEM column, so the activation rows are stored in the
+//    matching P4 K order (common.cuh): x by the router (gathered into x_perm by
+//    gather_wide_rows_kernel), h by the gate_up epilogues.  gate_up interleaves gate row i and
+//    up row i as A rows 2i, 2i+1, so one TMEM lane pair holds g and u.  A never passes through
+//    shared memory, which leaves shared-memory bandwidth to the TMA copies and the B operand.
 //  * warp 1 (MMA): one thread issues the unit's tcgen05.mma kind::f16 with bf16 operands (A
 //    from TMEM, B from shared memory; M 128, N = the tile's tokens rounded up to 16, K 16) into
 //    one of two TMEM accumulators, commits the consumed A unit and B slots and, per item, the
 //    accumulator.
-//  * warps 16..19 (epilogue): tcgen05.ld of the accumulator (warp w reads TMEM lanes
+//  * warps 12..15 (epilogue): tcgen05.ld of the accumulator (warp w reads TMEM lanes
 //    32 (w % 4) ..); gate_up pairs g and u with one shuffle, applies clamp-SwiGLU and the bf16
 //    rounding and stores h (bf16); down stores the assignment's fp32 row of y (the combine
 //    applies the routing weight).
@@ -65,12 +72,12 @@ constexpr int kSubK = 64;                                // K per B sub-tile (on
 constexpr int kSubs = kStageK / kSubK;                   // 8
 constexpr int kBBufs = 4, kDBufs = 2;
 constexpr int kItemQ = 8;
-// Warps: 0 weights producer, 1 MMA issuer, 2 activations producer, 3 idle, 4..15 dequant (three
-// groups of four: a group covers the 128 TMEM lanes and decodes whole A units, the groups taking
-// units in turn), 16..19 epilogue.
-constexpr int kWarps = 20;
+// Warps: 0 weights producer, 1 MMA issuer, 2 activations producer, 3 activations watcher, 4..11
+// dequant (two groups of four: a group covers the 128 TMEM lanes and decodes whole A units, the
+// groups taking units in turn), 12..15 epilogue.
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kWProd = 0, kMma = 1, kBProd = 2, kDeq0 = 4, kDeqGroups = 3, kDeqWarps = 4 * kDeqGroups;
+constexpr int kWProd = 0, kMma = 1, kBProd = 2, kBWatch = 3, kDeq0 = 4, kDeqGroups = 2, kDeqWarps = 4 * kDeqGroups;
 constexpr int kEpi0 = kDeq0 + kDeqWarps, kEpiWarps = 4;
 static_assert(kDeq0 % 4 == 0 && kEpi0 % 4 == 0, "a group of four warps reaches all 128 TMEM lanes");
 constexpr int kPackedStage = kRows * kStageK / 2;        // 32 KB: 2 box columns x 128 rows x 128 B
@@ -94,10 +101,13 @@ struct Part {
     static constexpr int kUnitSubs = kUnitK / kSubK;
     static constexpr int kACols = kUnitK / 2;                               // 2 bf16 per column
     static constexpr int kABufs = kSmall ? 3 : 2;
-    // Units rotate over as many dequant groups as there are A units, so that a group always
-    // refills the same unit and waits on its barrier phases in order (a parity wait cannot tell a
-    // phase from the one two before it); the large class leaves its third group idle.
-    static constexpr int kGroups = kABufs;
+    // Units rotate over the dequant groups and over the A buffers.  A group that waits for unit
+    // u's buffer (the release of unit u - kABufs) must know the phase before it (unit
+    // u - 2 kABufs) has completed, since a parity wait cannot tell a phase from the one two
+    // before it: its own previous unit u - kGroups waited for unit u - kGroups - kABufs, and
+    // units complete in order, so kGroups <= kABufs suffices.
+    static constexpr int kGroups = kDeqGroups;
+    static_assert(kGroups <= kABufs, "a group's waits see the phases in order");
     static constexpr int kACol0 = kDBufs * kAccCols;
     static_assert(kACol0 + kABufs * kACols <= 512, "TMEM budget");
     static_assert(kGroups <= kDeqGroups, "enough dequant groups");
@@ -143,6 +153,34 @@ __device__ __forceinline__ float wide_clamp_swiglu(float g, float u)
 // lane, K 64c + 32h + 8u + i in the low half of column 32c + 16h + 4u + i and + 4 in its high half
 // (the P4 pairing).  kLarge: some byte of the warp exceeds 128, so the two-multiply decode.
 // The stores are left in flight; the caller waits for them.
+__device__ __forceinline__ void st_release_shared(int *p, int v)
+{
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_shared(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+
+// Bounded poll (whole warp) until the count at p reaches `target` (acquire: what the publisher
+// observed before its release store is visible after).  Gives up like mbar_wait.
+__device__ __forceinline__ void poll_count(const int *p, int target, bool &aborted, const StatusPtrs &st)
+{
+    if (aborted) return;
+    if (__all_sync(0xffffffffu, ld_acquire_shared(p) >= target)) return;
+    const long long t0 = clock64();
+    while (!__all_sync(0xffffffffu, ld_acquire_shared(p) >= target)) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+            aborted = true;
+            record_timeout(st);
+            return;
+        }
+    }
+}
+
 template <int kSubsN, bool kLarge>
 __device__ __forceinline__ void dequant_unit(const uint8_t *pk, int r, int j0, const uint32_t (&eb)[2], uint32_t a_unit)
 {
@@ -192,6 +230,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
     volatile int *a_item = item_q + kItemQ;                                   // [kMaxABufs]
     volatile int *d_item = a_item + kMaxABufs;                                // [kDBufs]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(const_cast<int *>(d_item + kDBufs));
+    int *b_seq = reinterpret_cast<int *>(tmem_slot + 4);   // B slot loads known to have landed, in load order
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{a.status_ws, a.status_out};
@@ -221,6 +260,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
         }
         for (int i = 0; i < kItemQ; ++i) mbar_init(&pub[i], 1);
         mbar_init(mma_done, 1);
+        *b_seq = 0;
         fence_barrier_init();
     }
     if (warp == kMma) tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -332,11 +372,34 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             const int sc = issued - 1 - i;
             mbar_wait_drain(&b_full[sc % kBBufs], (sc / kBBufs) & 1, status);
         }
+    } else if (warp == kBWatch) {
+        // ------------------------------------------------------------ B landing watcher
+        // Waits on every activation slot load in load order (an in-order waiter always sees the
+        // load's own barrier phase) and publishes how many have landed.  The dequant group of a
+        // unit checks that count before it hands the unit to the MMA warp, so the MMA warp's only
+        // wait per unit is the unit's own.
+        int bload = 0;
+        for (int item_ctr = 0;; ++item_ctr) {
+            mbar_wait(&pub[item_ctr % kItemQ], (item_ctr / kItemQ) & 1, aborted, status);
+            aborted = __any_sync(0xffffffffu, aborted);
+            if (aborted) break;
+            const int item = item_q[item_ctr % kItemQ];
+            if (item < 0) break;
+            const WideTile *tp = a.tiles + item / row_blocks;
+            const int spb = subs_per_slot((__ldcg(&tp->count) + 15) / 16);
+            for (int j0 = 0; j0 < n_stages * kSubs; j0 += spb, ++bload) {
+                mbar_wait(&b_full[bload % kBBufs], (bload / kBBufs) & 1, aborted, status);
+                aborted = __any_sync(0xffffffffu, aborted);
+                if (aborted) break;
+                if (lane == 0) st_release_shared(b_seq, bload + 1);
+            }
+            if (aborted) break;
+        }
     } else if (warp >= kDeq0 && warp < kDeq0 + kDeqWarps) {
         // ------------------------------------------------------------ dequant warps
-        // group grp takes the units whose running index is grp mod P::kGroups (so always A unit
-        // grp); a warp stores TMEM lanes 32 (warp % 4) ..; its thread owns A row ar = that lane,
-        // all K of the unit.  Groups past P::kGroups take no unit but release every stage.
+        // group grp takes the units whose running index u is grp mod P::kGroups, into A buffer
+        // u mod P::kABufs; a warp stores TMEM lanes 32 (warp % 4) ..; its thread owns A row
+        // ar = that lane, all K of the unit.  Every group releases every stage.
         const int grp = (warp - kDeq0) >> 2;
         const int quarter = warp & 3;
         const int ar = 32 * quarter + lane;
@@ -345,6 +408,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
         const int r = kGateUp ? (ar >> 1) + (ar & 1) * 64 : ar;
         const uint32_t a_lane = static_cast<uint32_t>(32 * quarter) << 16;
         int stage_ctr = 0, unit_ctr = 0;   // every group counts every stage and unit
+        int bload_base = 0;                // activation slot loads of the items before this one
         for (int item_ctr = 0;; ++item_ctr) {
             // the item's first stage (or the end marker) names the item
             mbar_wait(&full_p[stage_ctr % kPStages], (stage_ctr / kPStages) & 1, aborted, status);
@@ -363,6 +427,9 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 }
                 break;
             }
+            // the item's activation slots (the loads the B producer issues for it, in order)
+            const WideTile *tp = a.tiles + item / row_blocks;
+            const int spb_shift = __ffs(subs_per_slot((__ldcg(&tp->count) + 15) / 16)) - 1;
             for (int st = 0; st < n_stages; ++st) {
                 const int s = stage_ctr % kPStages;
                 if (st > 0) {
@@ -395,7 +462,12 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     else
                         dequant_unit<P::kUnitSubs, true>(pk, r, uu * P::kUnitSubs, eb, a_unit);
                     tmem_wait_st();
-                    if (quarter == 0 && lane == 0) a_item[ab] = item;
+                    if (quarter == 0) {
+                        // the unit's activations have landed: the last slot load its sub-tiles use
+                        const int last_sub = (st * kUnitsPerStage + uu + 1) * P::kUnitSubs - 1;
+                        poll_count(b_seq, bload_base + (last_sub >> spb_shift) + 1, aborted, status);
+                        if (lane == 0) a_item[ab] = item;
+                    }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&a_full[ab]);
@@ -406,14 +478,19 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 ++stage_ctr;
             }
             if (aborted) break;
+            bload_base += (n_stages * kSubs) >> spb_shift;
         }
     } else if (warp == kMma) {
         // ------------------------------------------------------------ MMA issuer
+        // The warp shares its scheduler with ALU-heavy dequant warps and gets a small share of
+        // its issue slots, so its loop keeps the arithmetic between MMAs minimal: ring indices
+        // and phase bits advance incrementally, slot sizes are powers of two.
         int unit_ctr = 0, bload = 0;
+        int ab = 0;               // A buffer of unit unit_ctr (unit_ctr % kABufs)
+        uint32_t a_par = 0;       // phase parity of that buffer ((unit_ctr / kABufs) & 1)
         for (int item_ctr = 0;; ++item_ctr) {
             const int db = item_ctr % kDBufs;
-            int ab = unit_ctr % P::kABufs;
-            mbar_wait(&a_full[ab], (unit_ctr / P::kABufs) & 1, aborted, status);
+            mbar_wait(&a_full[ab], a_par, aborted, status);
             if (aborted) break;
             const int item = a_item[ab];
             // the accumulator's previous item must have left the epilogue (also before the end
@@ -430,29 +507,22 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
             if (lane == 0) d_item[db] = item;
             const WideTile *tp = a.tiles + item / row_blocks;
             const int nbox = (__ldcg(&tp->count) + 15) / 16;
-            const int spb = subs_per_slot(nbox);
+            const int spb = subs_per_slot(nbox);   // a power of two
             const uint32_t idesc = umma_idesc_bf16(kRows, 16 * nbox);
             const uint32_t d_tmem = tmem + static_cast<uint32_t>(db * P::kAccCols);
             // B descriptor units (16 bytes) between consecutive sub-tiles of a slot
             const uint32_t b_step = static_cast<uint32_t>(nbox * kBBox) >> 4;
             for (int u = 0; u < n_units; ++u, ++unit_ctr) {
-                ab = unit_ctr % P::kABufs;
-                if (u > 0) mbar_wait(&a_full[ab], (unit_ctr / P::kABufs) & 1, aborted, status);
+                if (u > 0) mbar_wait(&a_full[ab], a_par, aborted, status);
                 if (aborted) break;
                 tc_fence_after();
                 const uint32_t a_unit = tmem + static_cast<uint32_t>(P::kACol0 + ab * P::kACols);
-                // the unit's sub-tiles, one B slot at a time: a wait on the slot, then one elected
-                // lane issues all of the slot's MMAs of this unit back to back (the warp shares its
-                // scheduler with dequant warps, so every instruction it spends between MMAs delays
-                // the tensor pipe)
+                // the unit's sub-tiles, one B slot at a time (their activations have landed: the
+                // dequant group checked before handing the unit over); one elected lane issues all of
+                // the slot's MMAs of this unit back to back
                 for (int c0 = 0; c0 < P::kUnitSubs;) {
                     const int j = u * P::kUnitSubs + c0;
-                    const int bb = bload % kBBufs, uo = j % spb;
-                    if (uo == 0) {
-                        mbar_wait(&b_full[bb], (bload / kBBufs) & 1, aborted, status);
-                        if (aborted) break;
-                        tc_fence_after();
-                    }
+                    const int bb = bload & (kBBufs - 1), uo = j & (spb - 1);
                     const int nsub = min(spb - uo, P::kUnitSubs - c0);
                     const bool slot_end = uo + nsub == spb;
                     const bool unit_end = c0 + nsub == P::kUnitSubs;
@@ -478,6 +548,10 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                     c0 += nsub;
                 }
                 if (aborted) break;
+                if (++ab == P::kABufs) {
+                    ab = 0;
+                    a_par ^= 1u;
+                }
             }
             if (aborted) break;
             if (elect_one()) umma_commit(smem_u32(&d_full[db]));
