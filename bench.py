@@ -590,7 +590,9 @@ def run_case_sharded(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, 
         "warmup": args.warmup, "ms_per_step": mean_us / 1e3, "higher_is_better": False, "scaling": "strong",
         "vs_baseline": None, "dtype": "bf16 (MXFP4 weights decoded exactly to bf16), fp32 accumulate",
         "data": "synthetic",
-        "config": dict(workload_config(shape, M), parallelism="I-shard %d (I/%d = %d per GPU)" % (world, world, Is)),
+        "config": dict(workload_config(shape, M), parallelism="I-shard %d (I/%d = %d per GPU)" % (world, world, Is),
+                       timing="eager steps (this rank's share, NCCL all-gather, fixed-order reduction), CUDA "
+                              "events on the current stream, max over ranks"),
         "roofline_call": {"bound": call_bound, "roofline_us": roof_us, "frac": roof_us / mean_us,
                           "peaks": peak_kind, "algorithmic_bytes_per_gpu": work["bytes"],
                           "exchange_bytes_per_gpu": exchange, "touched_experts": work["touched"]},

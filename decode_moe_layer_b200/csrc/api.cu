@@ -74,6 +74,8 @@ Layout make_layout(int M, int H, int I, int E, int k)
     L.splits = route_plan(M, H, E).splits;
     L.partial = take(static_cast<size_t>(L.splits) * M * E * sizeof(float));
     L.x_p4 = take(static_cast<size_t>(M) * H * 2);
+    L.xmax = take(static_cast<size_t>(L.splits) * M * 4);
+    L.xshift = take(static_cast<size_t>(M) * 4);
     L.topk_ids = take(n * 4);
     L.topk_w = take(n * 4);
     L.offsets = take(static_cast<size_t>(E + 1) * 4);
@@ -354,7 +356,11 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     float *y = reinterpret_cast<float *>(ws + L.y);
     const WideLists wl = wide_lists(ws, L);
     __nv_bfloat16 *x_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_perm);
-    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width};
+    uint32_t *xmax = reinterpret_cast<uint32_t *>(ws + L.xmax);
+    int *xshift = reinterpret_cast<int *>(ws + L.xshift);
+    // the unfused path's remap reads the shifts route_topk writes; the fused one makes its own
+    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width,
+                     xshift, k};
     // The first kernel is ordered after everything before it on the stream; each later
     // kernel of the call is launched early (programmatic dependent launch) and waits on
     // device for its predecessor.  Event marks (profiling) break that overlap, so the
@@ -362,14 +368,14 @@ static int forward_impl(const void *x, const float *router_w, const float *route
     const bool pdl = (marks == nullptr);
 
     if (marks) MOE_TRY(marks->start(s));
-    MOE_TRY(launch_route_logits(x, router_w, partial, x_p4, status, status_out, M, H, E, s));
+    MOE_TRY(launch_route_logits(x, router_w, partial, x_p4, xmax, status, status_out, M, H, E, s));
     MOE_AFTER(marks, s, kProfLogits);
     if (fused_select(M, E, k)) {
-        MOE_TRY(launch_route_select_permute(partial, L.splits, router_bias, ids, tw, offsets, sorted_ids, inv_pos, to, M,
-                                            E, k, s, pdl));
+        MOE_TRY(launch_route_select_permute(partial, L.splits, router_bias, ids, tw, offsets, sorted_ids, inv_pos, to,
+                                            xmax, M, E, k, s, pdl));
         MOE_AFTER(marks, s, kProfSelect);
     } else {
-        MOE_TRY(launch_route_topk(partial, L.splits, router_bias, ids, tw, M, E, k, s, pdl));
+        MOE_TRY(launch_route_topk(partial, L.splits, router_bias, ids, tw, xmax, xshift, M, E, k, s, pdl));
         MOE_AFTER(marks, s, kProfSelect);
         MOE_TRY(launch_permute(ids, offsets, sorted_ids, inv_pos, to, M, E, k, s, pdl));
         MOE_AFTER(marks, s, kProfPermute);
@@ -480,9 +486,10 @@ int moe_route(const void *x_bf16, const float *router_w, const float *router_bia
     rc = library_workspace(stream, L.total, &ws);
     if (rc != MOE_OK) return rc;
     float *partial = reinterpret_cast<float *>(ws + L.partial);
-    MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, reinterpret_cast<int *>(ws + L.status), nullptr,
-                                M, H, E, stream));
-    MOE_TRY(launch_route_topk(partial, L.splits, router_bias, topk_ids, topk_w, M, E, k, stream, false));
+    MOE_TRY(launch_route_logits(x_bf16, router_w, partial, nullptr, nullptr, reinterpret_cast<int *>(ws + L.status),
+                                nullptr, M, H, E, stream));
+    MOE_TRY(launch_route_topk(partial, L.splits, router_bias, topk_ids, topk_w, nullptr, nullptr, M, E, k, stream,
+                              false));
     return MOE_OK;
 }
 
@@ -496,7 +503,7 @@ int moe_permute(const int32_t *topk_ids, int32_t *expert_offsets, int32_t *sorte
     if (!aligned(topk_ids, 4) || !aligned(expert_offsets, 4) || !aligned(sorted_ids, 4) || !aligned(inv_pos, 4))
         return MOE_ERR_INVALID_ARG;
     if (M == 0) return MOE_OK;
-    const TileOut none{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 8};
+    const TileOut none{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, 8, nullptr, k};
     MOE_TRY(launch_permute(topk_ids, expert_offsets, sorted_ids, inv_pos, none, M, E, k, stream, false));
     return MOE_OK;
 }
@@ -522,8 +529,12 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
     __nv_bfloat16 *x_perm = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_perm);
     __nv_bfloat16 *x_p4 = reinterpret_cast<__nv_bfloat16 *>(ws + L.x_p4);
     __nv_bfloat16 *h = static_cast<__nv_bfloat16 *>(h_bf16);
-    // the same tiles as a whole-layer call (mma.sync tiles, and tensor-core tiles)
-    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width};
+    int *xshift = reinterpret_cast<int *>(ws + L.xshift);
+    // the tokens' activation shifts (the whole layer's router computes them), then the same tiles
+    // as a whole-layer call (mma.sync tiles, and tensor-core tiles)
+    MOE_TRY(launch_row_shift(static_cast<const __nv_bfloat16 *>(x_bf16), xshift, M, H, stream));
+    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width,
+                     xshift, k};
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, to, status, E, stream));
     // x into the P4 K order the grouped GEMMs read (the whole layer's router writes it)
     MOE_TRY(launch_rows_to_p4(static_cast<const __nv_bfloat16 *>(x_bf16), x_p4, static_cast<size_t>(M), H, stream));
@@ -559,7 +570,9 @@ int moe_down_combine(const void *h_bf16, const uint8_t *w2_q, const uint8_t *w2_
     const WideLists wl = wide_lists(ws, L);
     __nv_bfloat16 *h_p4 = reinterpret_cast<__nv_bfloat16 *>(ws + L.h);
     float *y = reinterpret_cast<float *>(ws + L.y);
-    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width};
+    // (the down kernels scale h by a fixed power of two: no per-token shifts)
+    const TileOut to{tiles, n_tiles, L.wide ? wl.small : nullptr, wl.n_small, wl.large, wl.n_large, L.width, nullptr,
+                     k};
     MOE_TRY(launch_build_tiles(expert_offsets, sorted_ids, to, status, E, stream));
     // the caller's h rows (natural K order) into the P4 order the down kernels read
     MOE_TRY(launch_rows_to_p4(static_cast<const __nv_bfloat16 *>(h_bf16), h_p4, static_cast<size_t>(M) * k, I,

@@ -32,8 +32,15 @@
 //  * 16 compute warps = 2 m-tile pairs x 8 K slots.  Per stage a warp takes 4 of
 //    the 32 blocks of 32 K for its 2 m-tiles: a thread reads the 32-bit word q of
 //    its rows' 16-byte block (conflict-free thanks to the swizzle), decodes it
-//    exactly to bf16 (e2m1x8_to_bf16x2_p4) straight into MMA A-fragment registers,
-//    and runs two m16n8k16 bf16 MMAs per block.  Inside a block the K order is
+//    exactly to the codes' values times 2^-126 (e2m1x8_raw_p4: the E2M1 subnormal 0.5
+//    becomes a bf16 subnormal, which the MMA takes exactly) straight into MMA
+//    A-fragment registers, and runs two m16n8k16 bf16 MMAs per block.  The 2^126
+//    rides on the activations instead: each token's bf16 activations are multiplied by
+//    2^s (s: the token's activation shift, x_shift_from_max; a fixed kHShift for h)
+//    as the thread loads them, which keeps every product inside fp32's normal range,
+//    and the epilogue multiplies the sums by 2^(126 - s).  Both are powers of two, so
+//    the fp32 sums are the unshifted sums times 2^(s - 126), rounding for rounding;
+//    the shift costs one multiply per 8 activations against one per 2 weights.  Inside a block the K order is
 //    permuted identically for A and for the activation fragment: thread q's word
 //    covers K 8q..8q+7, its registers pair K 8q+i with 8q+i+4, and the activation
 //    rows are stored in that same P4 order (x by the router, h by gate_up).  So
@@ -50,8 +57,9 @@
 //    memory.  The weighted top-k combine that follows is its own small kernel
 //    (combine_kernel).
 // Both MMA operands are bf16: x as the caller gives it and h as gate_up rounds it (both
-// stored in the P4 K order of common.cuh), and the weights decoded exactly (every E2M1
-// value is a bf16 value); products accumulate in fp32.
+// stored in the P4 K order of common.cuh, both times an exact power of two), and the
+// weights decoded exactly (every E2M1 value times 2^-126 is a bf16 value); products
+// accumulate in fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -90,7 +98,7 @@ struct SmemPlan {
 };
 
 constexpr int kNumBars = 2 * kStages + 8 + kComputeWarps / 2;   // ring, scale buffers, partials, K-slot pairs
-constexpr int kMetaInts = 3 * (kItemQ + 2);                      // item ids, positions, counts
+constexpr int kMetaInts = (3 + kTileTokensMax) * (kItemQ + 2);   // item ids, positions, counts, token shifts
 
 template <int kN>
 __host__ __device__ inline SmemPlan smem_plan(int K)
@@ -106,6 +114,13 @@ __host__ __device__ inline SmemPlan smem_plan(int K)
     p.bars_off = p.red_off + T::kRedBufs * T::kRedFloats * 4;
     p.total = p.bars_off + kNumBars * 8 + kMetaInts * 4 + 1024;   // + alignment slack
     return p;
+}
+
+// v * 2^(126 - s) for an activation shift s in [-7, 127], in two exact power-of-two steps (the
+// factor alone can exceed fp32's range).
+__device__ __forceinline__ float unshift(float v, int s)
+{
+    return (v * 0x1p63f) * __int_as_float((190 - s) << 23);   // 2^63, then 2^(63 - s)
 }
 
 __device__ __forceinline__ float clamp_swiglu(float g, float u)
@@ -147,6 +162,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
     volatile int *red_item = item_cnt + kItemQ;                                       // [kRedBufs]
     volatile int *red_p0 = red_item + 2;                                              // [kRedBufs]
     volatile int *red_cnt = red_p0 + 2;                                               // [kRedBufs]
+    // the activation shift of each tile slot (item_sh: per item in flight; red_sh: per partial buffer)
+    volatile int *item_sh = red_cnt + 2;                                              // [kItemQ][16]
+    volatile int *red_sh = item_sh + kItemQ * kTileTokensMax;                         // [kRedBufs][16]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const StatusPtrs status{status_ws, status_out};
@@ -258,7 +276,7 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         for (;; ++item_ctr) {
             const int item = next_id;
             if (item >= n_items) break;
-            const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, flat = nx_flat;
+            const int e = nx_e, p0 = nx_p0, cnt = nx_cnt, flat = tile_flat_id(nx_flat);
             next_id = take();
             fetch(next_id);
             if (lane == 0) {   // published by the first stage's arrival
@@ -266,6 +284,9 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 item_p0[item_ctr % kItemQ] = p0;
                 item_cnt[item_ctr % kItemQ] = cnt;
             }
+            // the slots' activation shifts: x by its token's shift (packed with the flat id), h by
+            // the fixed one
+            if (lane < kTileTokensMax) item_sh[(item_ctr % kItemQ) * kTileTokensMax + lane] = kGateUp ? tile_shift(nx_flat) : kHShift;
             __syncwarp();   // orders these stores before the arrival of whichever lane issues it
             const int rb = item % row_blocks;
             // weight rows: gate_up = gate block a and up block b (32 rows each); down = one block of 64
@@ -420,8 +441,16 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 const int j = ep + T::kEpiWarps * m;
 #pragma unroll
                 for (int hf = 0; hf < T::kHalves; ++hf) {
-                    const float4 sum = sums[m][hf];
+                    float4 sum = sums[m][hf];
                     const int li0 = 8 * hf + 2 * q, li1 = li0 + 1;   // the fragment's two tile slots
+                    // back to the true scale: the sums carry 2^(shift - 126) (exact powers of two)
+                    if (kGateUp) {
+                        const int s0 = red_sh[b * kTileTokensMax + li0], s1 = red_sh[b * kTileTokensMax + li1];
+                        sum = make_float4(unshift(sum.x, s0), unshift(sum.y, s1), unshift(sum.z, s0), unshift(sum.w, s1));
+                    } else {
+                        constexpr float kBack = static_cast<float>(1u << (126 - kHShift));
+                        sum = make_float4(sum.x * kBack, sum.y * kBack, sum.z * kBack, sum.w * kBack);
+                    }
                     if (kGateUp) {
                         // h rounded to bf16 once, at column n (P4 storage order for the down kernels)
                         const int n = rb * 32 + 8 * j + g;
@@ -496,6 +525,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
         const bool two = kN == 16 && item_cnt[item_ctr % kItemQ] > 8;
         const uint8_t *sbi = sbuf + b * plan.sbuf_bytes;
         if (!stage_scales) mbar_wait(&sfull[b], (item_ctr >> 1) & 1, aborted, status);
+        // bf16x2 2^s of this thread's B-fragment tokens g and g + 8 (the activation shifts)
+        const uint32_t fac_g = static_cast<uint32_t>(item_sh[(item_ctr % kItemQ) * kTileTokensMax + g] + 127) * 0x00800080u;
+        const uint32_t fac_g8 =
+            static_cast<uint32_t>(item_sh[(item_ctr % kItemQ) * kTileTokensMax + g + 8] + 127) * 0x00800080u;
 
         float acc[kWarpMTiles][kVals];
 #pragma unroll
@@ -514,11 +547,17 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
 #pragma unroll
             for (int bi = 0; bi < kBlocksPerWarp; ++bi) {
                 if (c * kBlocksPerStage + blk_base + bi >= kblocks) continue;
-                // K 8q..8q+7 of token g (and g + 8), stored in P4 order like the decoded weights
-                const uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (blk_base + bi) + 8 * q) * 2);
+                // K 8q..8q+7 of token g (and g + 8), stored in P4 order like the decoded weights, times
+                // 2^(token's shift) (exact)
+                uint4 xb = *reinterpret_cast<const uint4 *>(xa + (32 * (blk_base + bi) + 8 * q) * 2);
+                xb = make_uint4(bf16x2_mul(xb.x, fac_g), bf16x2_mul(xb.y, fac_g), bf16x2_mul(xb.z, fac_g),
+                                bf16x2_mul(xb.w, fac_g));
                 uint4 xc = make_uint4(0u, 0u, 0u, 0u);   // token g + 8 (second n-tile)
-                if (kN == 16 && two)
+                if (kN == 16 && two) {
                     xc = *reinterpret_cast<const uint4 *>(xa + 8 * kActPitch + (32 * (blk_base + bi) + 8 * q) * 2);
+                    xc = make_uint4(bf16x2_mul(xc.x, fac_g8), bf16x2_mul(xc.y, fac_g8), bf16x2_mul(xc.z, fac_g8),
+                                    bf16x2_mul(xc.w, fac_g8));
+                }
                 const int sw = (((bb0 + bi) ^ g) << 4) + 4 * q;   // 128-byte swizzle: chunk ^ (row & 7)
 #pragma unroll
                 for (int m = 0; m < kWarpMTiles; ++m) {
@@ -526,9 +565,10 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                     const uint32_t wb = *reinterpret_cast<const uint32_t *>(st + bot_off[m] + sw);
                     const float st_scale = e8m0_scale(sc_base[top_sr[m] * s_pitch + sc_col0 + bi]);
                     const float sb_scale = e8m0_scale(sc_base[bot_sr[m] * s_pitch + sc_col0 + bi]);
+                    // the codes' values times 2^-126 (the shifted activations carry the 2^126)
                     uint32_t t[4], u[4];
-                    e2m1x8_to_bf16x2_p4(wt, t);
-                    e2m1x8_to_bf16x2_p4(wb, u);
+                    e2m1x8_raw_p4(wt, t);
+                    e2m1x8_raw_p4(wb, u);
                     // registers i = K (8q+i, 8q+i+4): the first MMA takes i = 0, 1, the second 2, 3.
                     // Each block's MMA pair starts from zero (no dependence on the previous block's
                     // MMAs) and its fp32 partial times the block scale (exact) joins the K slot's sums.
@@ -599,10 +639,13 @@ grouped_mxfp4_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_cons
                 }
                 *dst = o;
             }
-        if (warp == 0 && lane == 0) {
-            red_item[rb] = item_q[item_ctr % kItemQ];
-            red_p0[rb] = item_p0[item_ctr % kItemQ];
-            red_cnt[rb] = item_cnt[item_ctr % kItemQ];
+        if (warp == 0) {
+            if (lane == 0) {
+                red_item[rb] = item_q[item_ctr % kItemQ];
+                red_p0[rb] = item_p0[item_ctr % kItemQ];
+                red_cnt[rb] = item_cnt[item_ctr % kItemQ];
+            }
+            if (lane < kTileTokensMax) red_sh[rb * kTileTokensMax + lane] = item_sh[(item_ctr % kItemQ) * kTileTokensMax + lane];
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&rfull[rb]);

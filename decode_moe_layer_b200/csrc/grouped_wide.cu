@@ -485,7 +485,8 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
         // The warp shares its scheduler with ALU-heavy dequant warps and gets a small share of
         // its issue slots, so its loop keeps the arithmetic between MMAs minimal: ring indices
         // and phase bits advance incrementally, slot sizes are powers of two.
-        int unit_ctr = 0, bload = 0;
+        int unit_ctr = 0;
+        int bb = 0;               // slot of the current activation load (load count % kBBufs)
         int ab = 0;               // A buffer of unit unit_ctr (unit_ctr % kABufs)
         uint32_t a_par = 0;       // phase parity of that buffer ((unit_ctr / kABufs) & 1)
         for (int item_ctr = 0;; ++item_ctr) {
@@ -522,7 +523,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                 // the slot's MMAs of this unit back to back
                 for (int c0 = 0; c0 < P::kUnitSubs;) {
                     const int j = u * P::kUnitSubs + c0;
-                    const int bb = bload & (kBBufs - 1), uo = j & (spb - 1);
+                    const int uo = j & (spb - 1);
                     const int nsub = min(spb - uo, P::kUnitSubs - c0);
                     const bool slot_end = uo + nsub == spb;
                     const bool unit_end = c0 + nsub == P::kUnitSubs;
@@ -544,7 +545,7 @@ grouped_wide_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_const
                         if (unit_end) umma_commit(smem_u32(&a_empty[ab]));
                     }
                     __syncwarp();
-                    if (slot_end) ++bload;
+                    if (slot_end && ++bb == kBBufs) bb = 0;
                     c0 += nsub;
                 }
                 if (aborted) break;

@@ -82,12 +82,29 @@ constexpr int kMaxE = 1024;
 constexpr int kMaxK = 32;
 constexpr int kMaxAssignments = 16384;
 
+// Activation shift of the mma.sync kernels (grouped_gemm.cu): they multiply each token's bf16
+// activations by 2^s, s = clamp(120 - (exponent of the token's largest |x|), -7, 127), so that the
+// weights can enter the MMA undecoded-scale (E2M1 value x 2^-126) and every product stays inside
+// fp32's normal range; the epilogue multiplies the sums back by 2^(126 - s).  Both scalings are
+// powers of two, so the fp32 sums are the same numbers times 2^(s - 126).  m: the largest bf16
+// magnitude bits (|x| bits, 0 .. 0x7F7F) of the token's row.
+__host__ __device__ inline int x_shift_from_max(uint32_t m)
+{
+    const int s = 247 - static_cast<int>(m >> 7);   // 120 - (biased exponent - 127)
+    return s < -7 ? -7 : (s > 127 ? 127 : s);
+}
+constexpr int kHShift = 120;   // the same for h (|h| <= 49 < 2^6): a fixed shift
+
+__device__ __forceinline__ int tile_flat_id(int packed) { return packed & 0xFFFFFF; }
+__device__ __forceinline__ int tile_shift(int packed) { return packed >> 24; }   // arithmetic: signed
+
 struct ExpertTile {   // one expert's run of <= tile_width consecutive assignments
     int expert;
     int p0;           // first position in the expert-grouped order
     int count;
     int pad;
-    int flat[kTileTokensMax];   // flat assignment id t*k + j of each slot (sorted_ids[p0+i]); slots count..width-1
+    int flat[kTileTokensMax];   // flat assignment id t*k + j of each slot (sorted_ids[p0+i]) with its token's
+                                // activation shift in the top byte (pack_flat); slots count..width-1
                                 // repeat the last, slots past the width are not written
 };
 
@@ -139,7 +156,7 @@ __host__ __device__ inline bool wide_enabled(int M, int H, int I, int E, int k)
 
 // Byte offsets of every buffer inside one call's workspace (256-byte aligned).
 struct Layout {
-    size_t status, partial, x_p4, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y;
+    size_t status, partial, x_p4, xmax, xshift, topk_ids, topk_w, offsets, sorted_ids, inv_pos, tiles, n_tiles, h, y;
     size_t wide_small, n_wide_small, wide_large, n_wide_large, x_perm, total;
     int splits;   // router partial-logit slices (route_plan)
     int width;    // tile_width
@@ -194,10 +211,14 @@ __host__ __device__ inline int permute_smem_bytes(int E)
 
 // Kernel launchers (return cudaError_t of the launch).
 // x_p4 (nullable): x [M, H] rewritten in P4 K order for the grouped GEMMs.
-cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, void *x_p4, int *status,
-                                int32_t *status_out, int M, int H, int E, cudaStream_t s);
-cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
-                              int E, int k, cudaStream_t s, bool pdl);
+// xmax (when x_p4 is written): per H slice and token, the largest bf16 magnitude bits of x's row
+// in the slice, uint32 [splits][M]; the top-k kernels turn them into the per-token shifts.
+cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, void *x_p4, uint32_t *xmax,
+                                int *status, int32_t *status_out, int M, int H, int E, cudaStream_t s);
+cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
+                              const uint32_t *xmax, int *xshift, int M, int E, int k, cudaStream_t s, bool pdl);
+// Per-token shifts straight from x rows (the step-level gate_up entry point, which has no router).
+cudaError_t launch_row_shift(const __nv_bfloat16 *x, int *xshift, int M, int H, cudaStream_t s);
 // Tile outputs of the route remap: tiles of `width` (8 or 16) assignments for the mma.sync
 // kernels and, when wide_tiles is set, wide tiles (experts with at least kWideMinTokens
 // assignments) for the tensor-core kernels; such experts then get no mma.sync tiles.
@@ -209,10 +230,20 @@ struct TileOut {
     WideTile *wide_large;   // large tensor-core tiles (set whenever wide_tiles is)
     int *n_wide_large;
     int width;
+    const int *shift;       // per-token activation shifts packed into the tiles' flat ids (nullptr: 0)
+    int k;                  // top-k, to find a flat id's token
 };
+
+// A tile slot's flat id with its token's activation shift in the top byte (tile_flat_id and
+// tile_shift below take them apart; flat ids stay below 2^24).
+__device__ __forceinline__ int pack_flat(int f, const TileOut &to)
+{
+    const int sh = to.shift != nullptr ? to.shift[f / to.k] : 0;
+    return f | static_cast<int>(static_cast<uint32_t>(sh & 0xFF) << 24);
+}
 cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
-                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M,
-                                        int E, int k, cudaStream_t s, bool pdl);
+                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
+                                        const uint32_t *xmax, int M, int E, int k, cudaStream_t s, bool pdl);
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
                            int M, int E, int k, cudaStream_t s, bool pdl);
 // Tiles of both kinds from given expert offsets and sorted ids (the step-level entry points);

@@ -62,6 +62,31 @@ __global__ void __launch_bounds__(256) rows_to_p4_kernel(const uint4 *__restrict
     if (i < n_groups) dst[i] = p4_from_natural(src[i]);
 }
 
+// xshift[t] = the activation shift of row t of x (x_shift_from_max of its largest |x| bits), one
+// warp per row.
+__global__ void __launch_bounds__(256) row_shift_kernel(const uint4 *__restrict__ x, int *__restrict__ xshift, int M,
+                                                        int H)
+{
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (t >= M) return;
+    const uint4 *row = x + static_cast<size_t>(t) * (H / 8);
+    uint32_t m = 0;
+    for (int i = lane; i < H / 8; i += 32) {
+        const uint4 v = row[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) m = max(m, max(w[c] & 0x7FFFu, (w[c] >> 16) & 0x7FFFu));
+    }
+    m = __reduce_max_sync(0xffffffffu, m);
+    if (lane == 0) xshift[t] = x_shift_from_max(m);
+}
+
+cudaError_t launch_row_shift(const __nv_bfloat16 *x, int *xshift, int M, int H, cudaStream_t s)
+{
+    row_shift_kernel<<<(M + 7) / 8 > 0 ? (M + 7) / 8 : 1, 256, 0, s>>>(reinterpret_cast<const uint4 *>(x), xshift, M, H);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_permute(const int32_t *ids, int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
                            int M, int E, int k, cudaStream_t s, bool pdl)
 {

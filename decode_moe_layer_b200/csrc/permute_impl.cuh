@@ -186,7 +186,7 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
             } else if (tiles) {
                 const int slot = rank & (W - 1), tile_first = rank - slot;
                 ExpertTile *tp = tiles + sm.tb[e] + (rank >> wsh);
-                tp->flat[slot] = f;
+                tp->flat[slot] = pack_flat(f, to);
                 if (slot == 0) {
                     tp->expert = e;
                     tp->p0 = sm.off[e] + tile_first;
@@ -194,7 +194,7 @@ __device__ inline void rank_and_scatter(const int *s_e, int n, int E, int k, Ran
                     tp->pad = 0;
                 }
                 if (rank == cnt - 1)   // the last assignment repeats into the unused slots
-                    for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
+                    for (int j = slot + 1; j < W; ++j) tp->flat[j] = pack_flat(f, to);
             }
         }
     }
@@ -298,7 +298,7 @@ __device__ inline void scatter_assignment(int f, int e, int r, int c, const int 
     const int W = to.width, wsh = W == 16 ? 4 : 3;
     const int slot = r & (W - 1), tile_first = r - slot;
     ExpertTile *tp = to.tiles + tb[e] + (r >> wsh);
-    tp->flat[slot] = f;
+    tp->flat[slot] = pack_flat(f, to);
     if (slot == 0) {
         tp->expert = e;
         tp->p0 = off[e] + tile_first;
@@ -306,7 +306,7 @@ __device__ inline void scatter_assignment(int f, int e, int r, int c, const int 
         tp->pad = 0;
     }
     if (r == c - 1)   // the last assignment repeats into the unused slots
-        for (int j = slot + 1; j < W; ++j) tp->flat[j] = f;
+        for (int j = slot + 1; j < W; ++j) tp->flat[j] = pack_flat(f, to);
 }
 
 // Tiles from expert offsets (the step-level entry points, whose caller gives the permutation):
@@ -361,7 +361,7 @@ __device__ inline void emit_tiles(const int *off, int E, TileOut to, int *scan_b
             tl.p0 = off[e] + i * W;
             tl.count = min(W, cnt - i * W);
             tl.pad = 0;
-            for (int j = 0; j < W; ++j) tl.flat[j] = sorted_flat(tl.p0 + min(j, tl.count - 1));
+            for (int j = 0; j < W; ++j) tl.flat[j] = pack_flat(sorted_flat(tl.p0 + min(j, tl.count - 1)), to);
             to.tiles[base++] = tl;
         }
     }

@@ -62,13 +62,14 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 template <int kSteps, int kTiles>
 __global__ void __launch_bounds__(kRouteWarps * 32)
 route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr, float *__restrict__ partial,
-                    uint16_t *__restrict__ x_p4, int *status, int32_t *status_out, int M, int H, int E,
-                    int passes)
+                    uint16_t *__restrict__ x_p4, uint32_t *__restrict__ xmax, int *status, int32_t *status_out, int M,
+                    int H, int E, int passes)
 {
     constexpr int kPassK = 16 * kSteps;
     constexpr int kTokens = 8 * kTiles;
     constexpr int kPitch = kTokens + 8;                 // padded row of the warp partials
     __shared__ __align__(16) float red[kRouteWarps][kRouteExperts][kPitch];
+    __shared__ uint32_t xm[kRouteWarps][kTokens];   // per warp and token: largest |x| bits seen
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, q = lane & 3;
     const int e0 = blockIdx.x * kRouteExperts;
@@ -91,10 +92,13 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
     const int wg = split * kRouteWarps + warp;              // this warp's index along H
     const int ea = e0 + g, eb = e0 + g + 8;                 // its two W_r rows
     float acc[kTiles][4];
+    uint32_t amax[kTiles];   // largest |x| bits of token t0 + 8j + g among this lane's elements
 #pragma unroll
-    for (int j = 0; j < kTiles; ++j)
+    for (int j = 0; j < kTiles; ++j) {
+        amax[j] = 0;
 #pragma unroll
         for (int r = 0; r < 4; ++r) acc[j][r] = 0.f;
+    }
     for (int pass = 0; pass < passes; ++pass) {
         const int kw = (wg * passes + pass) * kPassK;       // first K of this pass
         // issue every load of the pass before any use: W_r rows and the token tiles' x words
@@ -139,6 +143,8 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
 #pragma unroll
                 for (int j = 0; j < kTiles; ++j) {
                     const uint2 mine = xv[j][s];
+                    amax[j] = max(amax[j], max(max(mine.x & 0x7FFFu, (mine.x >> 16) & 0x7FFFu),
+                                               max(mine.y & 0x7FFFu, (mine.y >> 16) & 0x7FFFu)));
                     const uint2 other = make_uint2(__shfl_xor_sync(0xffffffffu, mine.x, 1),
                                                    __shfl_xor_sync(0xffffffffu, mine.y, 1));
                     const bool odd = (q & 1) != 0;
@@ -156,8 +162,21 @@ route_logits_kernel(const uint16_t *__restrict__ x, const float *__restrict__ wr
     for (int j = 0; j < kTiles; ++j) {
         *reinterpret_cast<float2 *>(&red[warp][g][8 * j + 2 * q]) = make_float2(acc[j][0], acc[j][1]);
         *reinterpret_cast<float2 *>(&red[warp][g + 8][8 * j + 2 * q]) = make_float2(acc[j][2], acc[j][3]);
+        if (write_p4) {   // the four lanes of token g hold its 4-element groups of the warp's K
+            uint32_t m = amax[j];
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+            m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
+            if (q == 0) xm[warp][8 * j + g] = m;
+        }
     }
     __syncthreads();
+    if (write_p4 && xmax != nullptr && threadIdx.x < kTokens) {
+        const int t = t0 + threadIdx.x;
+        uint32_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kRouteWarps; ++w) m = max(m, xm[w][threadIdx.x]);
+        if (t < M) xmax[static_cast<size_t>(split) * M + t] = m;
+    }
     for (int i = threadIdx.x; i < kRouteExperts * kTokens; i += blockDim.x) {
         const int tl = i / kRouteExperts, el = i % kRouteExperts;   // consecutive threads: consecutive experts
         const int e = e0 + el, t = t0 + tl;
@@ -229,13 +248,20 @@ __device__ __forceinline__ void topk_from_values(const float (&v)[kPerLane], int
 template <int kPerLane>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float *__restrict__ partial, int splits,
                                                          const float *__restrict__ bias, int32_t *__restrict__ ids,
-                                                         float *__restrict__ wout, int M, int E, int k)
+                                                         float *__restrict__ wout, const uint32_t *__restrict__ xmax,
+                                                         int *__restrict__ xshift, int M, int E, int k)
 {
     pdl_wait();
     pdl_trigger();
     const int lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= M) return;
+    if (xmax != nullptr) {   // the token's activation shift, from its slices' largest |x|
+        uint32_t m = 0;
+        for (int sp = lane; sp < splits; sp += 32) m = max(m, xmax[static_cast<size_t>(sp) * M + t]);
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) xshift[t] = x_shift_from_max(m);
+    }
     float v[kPerLane];
 #pragma unroll
     for (int j = 0; j < kPerLane; ++j) v[j] = 0.f;
@@ -301,19 +327,28 @@ template <int kPerLane>
 __global__ void __launch_bounds__(kPermuteThreads, 1)
 route_select_permute_kernel(const float *__restrict__ partial, int splits, const float *__restrict__ bias,
                             int32_t *__restrict__ ids, float *__restrict__ wout, int32_t *__restrict__ offsets,
-                            int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos, TileOut to, int M,
-                            int E, int k)
+                            int32_t *__restrict__ sorted_ids, int32_t *__restrict__ inv_pos, TileOut to,
+                            const uint32_t *__restrict__ xmax, int M, int E, int k)
 {
     extern __shared__ __align__(16) uint8_t smem[];
     __shared__ int s_e[kPermuteThreads];                    // expert of assignment f
     __shared__ unsigned long long s_mask[kMaxE];            // bit t: token t chose the expert
     __shared__ int s_off[kMaxE], s_tb[kMaxE];                // first position, first mma.sync tile
     __shared__ int s_wb[kMaxE], s_wbl[kMaxE];                // first small / large tensor-core tile
+    __shared__ int s_shift[kFusedSelectMaxM];                // per token: activation shift of the mma.sync tiles
     float *s_log = reinterpret_cast<float *>(smem);         // [M][E]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     pdl_wait();
     pdl_trigger();
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_mask[e] = 0ull;
+    if (xmax != nullptr) {
+        for (int t = threadIdx.x; t < M; t += blockDim.x) {
+            uint32_t m = 0;
+            for (int sp = 0; sp < splits; ++sp) m = max(m, xmax[static_cast<size_t>(sp) * M + t]);
+            s_shift[t] = x_shift_from_max(m);
+        }
+        to.shift = s_shift;
+    }
     const int n_log = M * E;
     if (n_log <= kPermuteThreads)
         stage_logits<1, 32>(partial, splits, bias, n_log, E, s_log);
@@ -351,64 +386,65 @@ route_select_permute_kernel(const float *__restrict__ partial, int splits, const
 }
 
 template <int kSteps, int kTiles>
-static cudaError_t logits_launch(const void *x, const float *router_w, float *partial, void *x_p4, int *status,
-                                 int32_t *status_out, int M, int H, int E, const RoutePlan &plan, cudaStream_t s)
+static cudaError_t logits_launch(const void *x, const float *router_w, float *partial, void *x_p4, uint32_t *xmax,
+                                 int *status, int32_t *status_out, int M, int H, int E, const RoutePlan &plan,
+                                 cudaStream_t s)
 {
     const dim3 grid((E + kRouteExperts - 1) / kRouteExperts, plan.splits, plan.blocks_t);
     // first kernel of a call: fully ordered after whatever precedes it in the stream
     route_logits_kernel<kSteps, kTiles><<<grid, kRouteWarps * 32, 0, s>>>(
-        static_cast<const uint16_t *>(x), router_w, partial, static_cast<uint16_t *>(x_p4), status, status_out, M, H,
-        E, plan.passes);
+        static_cast<const uint16_t *>(x), router_w, partial, static_cast<uint16_t *>(x_p4), xmax, status, status_out,
+        M, H, E, plan.passes);
     return cudaGetLastError();
 }
 
-cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, void *x_p4, int *status,
-                                int32_t *status_out, int M, int H, int E, cudaStream_t s)
+cudaError_t launch_route_logits(const void *x, const float *router_w, float *partial, void *x_p4, uint32_t *xmax,
+                                int *status, int32_t *status_out, int M, int H, int E, cudaStream_t s)
 {
     const RoutePlan plan = route_plan(M, H, E);
     if (plan.tiles == 1 && plan.steps == 2)
-        return logits_launch<2, 1>(x, router_w, partial, x_p4, status, status_out, M, H, E, plan, s);
+        return logits_launch<2, 1>(x, router_w, partial, x_p4, xmax, status, status_out, M, H, E, plan, s);
     if (plan.tiles == 4 && plan.steps == 4)
-        return logits_launch<4, 4>(x, router_w, partial, x_p4, status, status_out, M, H, E, plan, s);
+        return logits_launch<4, 4>(x, router_w, partial, x_p4, xmax, status, status_out, M, H, E, plan, s);
     return cudaErrorInvalidConfiguration;   // route_plan yields only the two shapes above
 }
 
 template <int P>
-static cudaError_t topk_p(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M, int E,
-                          int k, cudaStream_t s, bool pdl)
+static cudaError_t topk_p(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
+                          const uint32_t *xmax, int *xshift, int M, int E, int k, cudaStream_t s, bool pdl)
 {
-    return launch_ex(route_topk_kernel<P>, dim3((M + 7) / 8), dim3(256), 0, s, pdl, partial, splits, bias, ids, w, M,
-                     E, k);
+    return launch_ex(route_topk_kernel<P>, dim3((M + 7) / 8), dim3(256), 0, s, pdl, partial, splits, bias, ids, w,
+                     xmax, xshift, M, E, k);
 }
 
-cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w, int M,
-                              int E, int k, cudaStream_t s, bool pdl)
+cudaError_t launch_route_topk(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
+                              const uint32_t *xmax, int *xshift, int M, int E, int k, cudaStream_t s, bool pdl)
 {
-    if (E <= 32) return topk_p<1>(partial, splits, bias, ids, w, M, E, k, s, pdl);
-    if (E <= 64) return topk_p<2>(partial, splits, bias, ids, w, M, E, k, s, pdl);
-    if (E <= 128) return topk_p<4>(partial, splits, bias, ids, w, M, E, k, s, pdl);
-    if (E <= 256) return topk_p<8>(partial, splits, bias, ids, w, M, E, k, s, pdl);
-    if (E <= 512) return topk_p<16>(partial, splits, bias, ids, w, M, E, k, s, pdl);
-    return topk_p<32>(partial, splits, bias, ids, w, M, E, k, s, pdl);
+    if (E <= 32) return topk_p<1>(partial, splits, bias, ids, w, xmax, xshift, M, E, k, s, pdl);
+    if (E <= 64) return topk_p<2>(partial, splits, bias, ids, w, xmax, xshift, M, E, k, s, pdl);
+    if (E <= 128) return topk_p<4>(partial, splits, bias, ids, w, xmax, xshift, M, E, k, s, pdl);
+    if (E <= 256) return topk_p<8>(partial, splits, bias, ids, w, xmax, xshift, M, E, k, s, pdl);
+    if (E <= 512) return topk_p<16>(partial, splits, bias, ids, w, xmax, xshift, M, E, k, s, pdl);
+    return topk_p<32>(partial, splits, bias, ids, w, xmax, xshift, M, E, k, s, pdl);
 }
 
 template <int P>
 static cudaError_t select_permute_p(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
-                                    int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M, int E,
-                                    int k, cudaStream_t s, bool pdl)
+                                    int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
+                                    const uint32_t *xmax, int M, int E, int k, cudaStream_t s, bool pdl)
 {
     const int smem = M * E * static_cast<int>(sizeof(float));
     cudaError_t e = ensure_max_smem(reinterpret_cast<const void *>(route_select_permute_kernel<P>), smem);
     if (e != cudaSuccess) return e;
     return launch_ex(route_select_permute_kernel<P>, dim3(1), dim3(kPermuteThreads), smem, s, pdl, partial, splits,
-                     bias, ids, w, offsets, sorted_ids, inv_pos, to, M, E, k);
+                     bias, ids, w, offsets, sorted_ids, inv_pos, to, xmax, M, E, k);
 }
 
 cudaError_t launch_route_select_permute(const float *partial, int splits, const float *bias, int32_t *ids, float *w,
-                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to, int M,
-                                        int E, int k, cudaStream_t s, bool pdl)
+                                        int32_t *offsets, int32_t *sorted_ids, int32_t *inv_pos, TileOut to,
+                                        const uint32_t *xmax, int M, int E, int k, cudaStream_t s, bool pdl)
 {
-#define MOE_SEL(P) select_permute_p<P>(partial, splits, bias, ids, w, offsets, sorted_ids, inv_pos, to, M, E, k, s, pdl)
+#define MOE_SEL(P) select_permute_p<P>(partial, splits, bias, ids, w, offsets, sorted_ids, inv_pos, to, xmax, M, E, k, s, pdl)
     if (E <= 32) return MOE_SEL(1);
     if (E <= 64) return MOE_SEL(2);
     if (E <= 128) return MOE_SEL(4);

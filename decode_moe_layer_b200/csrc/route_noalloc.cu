@@ -70,9 +70,9 @@ extern "C" int moe_route_noalloc(const void *x_bf16, const float *router_w, cons
     float *partial = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + kNoAllocStatusBytes);
     // every partial logit the top-k kernel reads is written first by the logits kernel, so
     // nothing in the array has to start at zero
-    cudaError_t e = launch_route_logits(x_bf16, router_w, partial, nullptr, status, nullptr, M, H, E, stream);
+    cudaError_t e = launch_route_logits(x_bf16, router_w, partial, nullptr, nullptr, status, nullptr, M, H, E, stream);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = launch_route_topk(partial, splits, router_bias, topk_ids, topk_w, M, E, k, stream, false);
+    e = launch_route_topk(partial, splits, router_bias, topk_ids, topk_w, nullptr, nullptr, M, E, k, stream, false);
     if (e != cudaSuccess) return cuda_fail(e);
     return MOE_OK;
 }
