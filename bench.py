@@ -98,9 +98,9 @@ def load_peaks():
 # --------------------------------------------------------------------------- algorithmic work
 
 # The library's split of an expert's assignments (moe_internal.h): tensor-core tiles when H and I are
-# multiples of 512, M >= 9 and the experts average >= 4.5 assignments, for the experts with 9 or
+# multiples of 512, M >= 5 and the experts average >= 2.5 assignments, for the experts with 5 or
 # more (small tiles up to 64, large tiles above); mma.sync tiles for the others.
-WIDE_MIN_TOKENS, WIDE_SMALL_MAX = 9, 64
+WIDE_MIN_TOKENS, WIDE_SMALL_MAX = 5, 64
 
 
 def expert_classes(shape, M, ids):

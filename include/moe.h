@@ -177,7 +177,7 @@ size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
 /*
  * Kernel launches one moe_mxfp4_forward / moe_mxfp4_forward_ex call enqueues for this shape
  * (router logits, top-k + permutation as one or two kernels, the grouped GEMMs, the gather and
- * tensor-core GEMMs when the call can give experts 9 or more assignments, the combine); 0 for M == 0 and a
+ * tensor-core GEMMs when the call can give experts 5 or more assignments, the combine); 0 for M == 0 and a
  * negative MOE_* status for an unsupported shape.  For sizing CUDA graphs and for accounting.
  */
 int moe_forward_launches(int M, int H, int I, int E, int k);

@@ -171,7 +171,7 @@ def check_h_bound(gpu_h, ref_bits, g, u, x_row_bits, w13_q_e, w13_s_e, what=""):
 # 16 once the experts average 6 or more assignments (else 8); when H and I are multiples of 512 and
 # the call is wide enough, tensor-core tiles for an expert with WIDE_MIN_TOKENS or more: one tile
 # up to WIDE_SMALL_MAX assignments, else tiles of up to WIDE_TOKENS.
-WIDE_MIN_TOKENS = 9
+WIDE_MIN_TOKENS = 5
 WIDE_SMALL_MAX = 64
 WIDE_TOKENS = 192
 
