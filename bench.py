@@ -83,6 +83,9 @@ def parse_args():
     p.add_argument("--headline-only", action="store_true", help="skip the other workloads' lines")
     p.add_argument("--other-steps", type=int, default=20, help="timed steps of the non-headline lines")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--shape", default=None, metavar="H,I,E,k",
+                   help="time one layer of this shape at --M instead of the workloads (same input recipe as "
+                        "the tiny workload; e.g. a reduced expert count for a profiler capture)")
     return p.parse_args()
 
 
@@ -333,8 +336,12 @@ def main():
     else:   # the other workloads first (fewer steps, no baselines), the headline last
         cases = [(c, False) for c in every if c != headline] + [(headline, True)]
 
+    if args.shape:
+        H, I, E, k = (int(v) for v in args.shape.split(","))
+        custom = gen.LayerShape("custom_h%d_i%d_e%d_k%d" % (H, I, E, k), H, I, E, k, (args.M,))
+        cases = [((0, args.M), True)]
     for (ci, M), is_headline in cases:
-        shape = gen.CONFIGS[ci]
+        shape = custom if args.shape else gen.CONFIGS[ci]
         steps = args.steps if (is_headline or args.sweep) else min(args.steps, args.other_steps)
         if world > 1:
             rec = run_case_sharded(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks,
@@ -360,7 +367,7 @@ def max_over_ranks(dist, values, device):
 
 def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, peaks, peak_kind, baselines, steps):
     H, I, E, k = shape.H, shape.I, shape.E, shape.k
-    inp = gen.make_inputs(ci, M, weights="torch", device=dev)
+    inp = gen.make_inputs(ci, M, shape=shape, weights="torch", device=dev)
     xb = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16)).to(dev).view(torch.bfloat16)
     wr = torch.from_numpy(inp.router_w).to(dev)
     bias = None if inp.router_bias is None else torch.from_numpy(inp.router_bias).to(dev)
@@ -493,7 +500,7 @@ def run_case(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, args, pe
         "clocks": clk,
     }
     if baselines and rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = gen.make_inputs(ci, M, weights="none")
+        host = gen.make_inputs(ci, M, shape=shape, weights="none")
         subsets, n_tok = oracle_token_sample(M, k)
         times, cores = time_oracle(host, subsets, 10.0, 30, 30.0)
         rec["cpu_baseline"] = {"value": statistics.mean(times) * 1e6 * M / n_tok, "unit": UNIT, "cores": cores,
@@ -506,7 +513,7 @@ def run_case_sharded(torch, moe, dist, barrier, world, rank, dev, shape, ci, M, 
     is this rank's share, the all-gather of the shares and the fixed-order reduction."""
     from decode_moe_layer_b200 import sharded
     H, I, E, k = shape.H, shape.I, shape.E, shape.k
-    inp = gen.make_inputs(ci, M, weights="torch", device=dev)
+    inp = gen.make_inputs(ci, M, shape=shape, weights="torch", device=dev)
     layer = sharded.IShardedLayer(inp.w13_q, inp.w13_s, inp.w2_q, inp.w2_s, k, device=dev)
     inp.w13_q = inp.w13_s = inp.w2_q = inp.w2_s = None
     torch.cuda.empty_cache()
