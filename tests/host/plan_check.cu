@@ -1,7 +1,9 @@
 // Host-side check of the launch-planning helpers in moe_internal.h over a grid of shapes: the
 // router plan covers every token and every K element and fills at most one wave of CTAs, the tile
-// width and fused-select switches follow their stated rules, and the per-shape shared-memory
-// needs fit a B200 CTA.  Built and run by tests/test_host_plan.py (no GPU needed).
+// width and fused-select switches follow their stated rules, the per-shape shared-memory needs fit
+// a B200 CTA, and the mma.sync kernels' activation shift keeps every finite bf16 row in range.
+// Built and run by tests/test_host_plan.py (no GPU needed).
+#include <cmath>
 #include <cstdio>
 
 #include "moe_internal.h"
@@ -75,7 +77,25 @@ int main()
     CHECK(permute_smem_bytes(kMaxE) <= 227 * 1024, 0, 0, kMaxE, 0);
     // the fused select's static arrays (token masks, offsets, tile bases, assignment experts)
     // plus its staged logits
-    CHECK(kMaxE * (8 + 4 * 4) + kPermuteThreads * 4 + kFusedSelectMaxLogits * 4 <= 227 * 1024, 0, 0, kMaxE, 0);
+    CHECK(kMaxE * (8 + 4 * 4) + kPermuteThreads * 4 + kFusedSelectMaxM * 4 + kFusedSelectMaxLogits * 4 <= 227 * 1024,
+          0, 0, kMaxE, 0);
+    // The mma.sync kernels' activation shift: for the largest |x| of a token (every finite bf16
+    // magnitude m), x * 2^s must stay below 2^121 (bf16 and the products stay finite: the weights
+    // enter as value * 2^-126 <= 6 * 2^-126), and reach 2^120 unless the shift is at its cap of 127
+    // (tiny rows), so that products keep fp32's normal range.
+    for (uint32_t m = 0; m <= 0x7F7Fu; ++m) {
+        const int s = x_shift_from_max(m);
+        const int e = static_cast<int>(m >> 7), mant = static_cast<int>(m & 0x7F);
+        const double v = e == 0 ? std::ldexp(static_cast<double>(mant), -133)
+                                : std::ldexp(1.0 + mant / 128.0, e - 127);
+        const double shifted = std::ldexp(v, s);
+        CHECK(s >= -7 && s <= 127, static_cast<int>(m), s, 0, 0);
+        CHECK(shifted < std::ldexp(1.0, 121), static_cast<int>(m), s, 0, 0);
+        CHECK(s == 127 || shifted >= std::ldexp(1.0, 120), static_cast<int>(m), s, 0, 0);
+        CHECK(s == 127 || e >= 1, static_cast<int>(m), s, 0, 0);
+    }
+    // h (|h| <= 49 from the clamps) with the fixed shift stays below 2^126
+    CHECK(std::ldexp(49.0, kHShift) < std::ldexp(1.0, 126), 0, kHShift, 0, 0);
     if (fails) {
         std::printf("%d failures\n", fails);
         return 1;

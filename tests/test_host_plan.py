@@ -1,5 +1,6 @@
 """Host-side launch planning (route plan, tile width, fused select, tensor-core switch, shared
-memory sizes) checked over a grid of shapes by a small host program built with nvcc."""
+memory sizes) checked over a grid of shapes, and the activation-shift rule over every finite bf16
+magnitude, by a small host program built with nvcc."""
 import os
 import shutil
 import subprocess
