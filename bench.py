@@ -106,17 +106,29 @@ def load_peaks():
 WIDE_MIN_TOKENS, WIDE_SMALL_MAX = 5, 64
 
 
+def wide_on(shape, M):
+    return (M >= WIDE_MIN_TOKENS and shape.H % 512 == 0 and shape.I % 512 == 0
+            and 2 * M * shape.k >= WIDE_MIN_TOKENS * shape.E)
+
+
+def down_fused(shape, M):
+    """The library runs down and the weighted combine as one launch at the smallest sizes: M <= 8,
+    I <= 1024, tiles of 8 assignments (M*k < 6E), no tensor-core tiles and at most 8 tiles."""
+    return (1 <= M <= 8 and shape.I <= 1024 and M * shape.k < 6 * shape.E and not wide_on(shape, M)
+            and min(M * shape.k, shape.E) <= 8)
+
+
 def expert_classes(shape, M, ids):
     """Per-expert assignment counts and class ('narrow', 'small', 'large') from the realised routing."""
     H, I, E, k = shape.H, shape.I, shape.E, shape.k
     counts = np.bincount(np.asarray(ids).reshape(-1), minlength=E)
-    wide_on = M >= WIDE_MIN_TOKENS and H % 512 == 0 and I % 512 == 0 and 2 * M * k >= WIDE_MIN_TOKENS * E
+    wide = wide_on(shape, M)
     cls = {}
     for e in range(E):
         c = int(counts[e])
         if c == 0:
             continue
-        if wide_on and c >= WIDE_MIN_TOKENS:
+        if wide and c >= WIDE_MIN_TOKENS:
             cls[e] = "small" if c <= WIDE_SMALL_MAX else "large"
         else:
             cls[e] = "narrow"
@@ -140,6 +152,9 @@ def algorithmic(shape, M, ids):
         if name.startswith("gate_up"):
             b = len(ex) * (2 * I * H * 17 // 32) + n_assign * H * 2 + n_assign * I * 2
             f = 4 * I * H * n_assign
+        elif name == "down" and down_fused(shape, M):   # with the combine: bf16 out, no fp32 rows
+            b = len(ex) * (I * H * 17 // 32) + n_assign * I * 2 + M * k * 4 + M * H * 2
+            f = 2 * I * H * n_assign
         else:
             b = len(ex) * (I * H * 17 // 32) + n_assign * I * 2 + n_assign * H * 4
             f = 2 * I * H * n_assign

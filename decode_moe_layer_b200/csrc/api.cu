@@ -9,6 +9,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "down_slab.h"
 #include "moe.h"
 #include "moe_internal.h"
 
@@ -300,6 +301,20 @@ static int run_down(const void *w2_q, const uint8_t *w2_s, const __nv_bfloat16 *
     return MOE_OK;
 }
 
+// The smallest calls (slab_enabled): the down projection and the weighted top-k combine in one
+// launch; weight boxes of 16 rows x 128 bytes (one slab).
+static int run_down_slab(const void *w2_q, const uint8_t *w2_s, const __nv_bfloat16 *h_p4, const ExpertTile *tiles,
+                         const int *n_tiles, const float *topk_w, void *out, bool f32_out, int *status,
+                         int32_t *status_out, int M, int H, int I, int E, int k, cudaStream_t s, bool pdl)
+{
+    CUtensorMap map;
+    int rc = make_weight_map(&map, w2_q, static_cast<uint64_t>(E) * H, static_cast<uint64_t>(I) / 2, kSlabRows);
+    if (rc != MOE_OK) return rc;
+    MOE_TRY(launch_down_slab(map, w2_s, h_p4, tiles, n_tiles, topk_w, out, f32_out, status, status_out, M, H, I, k, s,
+                             pdl));
+    return MOE_OK;
+}
+
 // The tensor-core path for the wide tiles of one projection (gate_up: x rows gathered into
 // expert-grouped P4 order -> h; down: h (P4) -> y).  Weight boxes of 64 rows x 128 bytes, scale
 // boxes of 64 rows x 16 bytes (one 512-element stage), activation boxes of 16 rows x 64 elements.
@@ -392,6 +407,13 @@ static int forward_impl(const void *x, const float *router_w, const float *route
                       pdl, marks);
         if (rc != MOE_OK) return rc;
     }
+    if (slab_enabled(M, I, E, k, L.width, L.wide)) {
+        // the smallest calls: down and the weighted top-k combine in one launch, no y round trip
+        rc = run_down_slab(w2_q, w2_s, h, tiles, n_tiles, tw, out, f32_out, status, status_out, M, H, I, E, k, s, pdl);
+        if (rc != MOE_OK) return rc;
+        MOE_AFTER(marks, s, kProfDown);
+        return MOE_OK;
+    }
     // down likewise, then the weighted top-k combine
     rc = run_down(w2_q, w2_s, h, sorted_ids, tiles, n_tiles, y, status, status_out, H, I, E, L.width, L.max_tiles, s,
                   pdl);
@@ -466,8 +488,10 @@ int moe_forward_launches(int M, int H, int I, int E, int k)
     const int rc = check_dims(M, H, I, E, k, true);
     if (rc != MOE_OK) return rc;
     if (M == 0) return 0;
-    // route_logits, select (+ permute), gate_up, down, combine; gather + four tensor-core GEMMs
-    return (fused_select(M, E, k) ? 5 : 6) + (wide_enabled(M, H, I, E, k) ? 5 : 0);
+    // route_logits, select (+ permute), gate_up, down, combine (down and combine one launch for the
+    // smallest calls); gather + four tensor-core GEMMs
+    const Layout L = make_layout(M, H, I, E, k);
+    return (fused_select(M, E, k) ? 5 : 6) + (L.wide ? 5 : 0) - (slab_enabled(M, I, E, k, L.width, L.wide) ? 1 : 0);
 }
 
 int moe_route(const void *x_bf16, const float *router_w, const float *router_bias, int32_t *topk_ids, float *topk_w,
@@ -577,6 +601,9 @@ int moe_down_combine(const void *h_bf16, const uint8_t *w2_q, const uint8_t *w2_
     // the caller's h rows (natural K order) into the P4 order the down kernels read
     MOE_TRY(launch_rows_to_p4(static_cast<const __nv_bfloat16 *>(h_bf16), h_p4, static_cast<size_t>(M) * k, I,
                               stream));
+    if (slab_enabled(M, I, E, k, L.width, L.wide))   // the same launch plan as a whole-layer call
+        return run_down_slab(w2_q, w2_s, h_p4, tiles, n_tiles, topk_w, out_bf16, false, status, nullptr, M, H, I, E, k,
+                             stream, false);
     rc = run_down(w2_q, w2_s, h_p4, sorted_ids, tiles, n_tiles, y, status, nullptr, H, I, E, L.width, L.max_tiles,
                   stream, false);
     if (rc != MOE_OK) return rc;

@@ -134,7 +134,11 @@ int moe_gate_up_swiglu(const void *x_bf16, const uint8_t *w13_q, const uint8_t *
  *   y[f] = W2_e h[inv position of f] (fp32 accumulation),
  *   out[t] = bf16_rne( sum_{j=0..k-1} topk_w[t,j] * y[t*k+j] ), summed in slot
  *   order j with no atomics.
- * Uses the library-owned workspace of `stream` for the fp32 per-assignment rows.
+ * For the smallest calls (I <= 1024 and at most 8 expert tiles: min(M*k, E) <= 8, with M <= 8,
+ * fewer than 6 assignments per expert on average and no expert tiles for the tensor cores) one
+ * kernel does both: each CTA owns 16 rows of H, keeps those rows of y for every assignment in
+ * shared memory and writes out.  Otherwise the fp32 rows of y go through the library-owned
+ * workspace of `stream` and a combine kernel.  Same bits either way.
  */
 int moe_down_combine(const void *h_bf16, const uint8_t *w2_q, const uint8_t *w2_s, const float *topk_w,
                      const int32_t *expert_offsets, const int32_t *sorted_ids, void *out_bf16,
@@ -177,7 +181,8 @@ size_t moe_workspace_bytes(int M, int H, int I, int E, int k);
 /*
  * Kernel launches one moe_mxfp4_forward / moe_mxfp4_forward_ex call enqueues for this shape
  * (router logits, top-k + permutation as one or two kernels, the grouped GEMMs, the gather and
- * tensor-core GEMMs when the call can give experts 5 or more assignments, the combine); 0 for M == 0 and a
+ * tensor-core GEMMs when the call can give experts 5 or more assignments, the combine -- one launch
+ * with the down GEMM for the smallest calls, see moe_down_combine); 0 for M == 0 and a
  * negative MOE_* status for an unsupported shape.  For sizing CUDA graphs and for accounting.
  */
 int moe_forward_launches(int M, int H, int I, int E, int k);
@@ -253,7 +258,8 @@ int moe_reduce_partials(const float *partials, int G, void *out_bf16, int M, int
  *   [2] route remap (0 when fused), [3] gate_up + clamp-SwiGLU on mma.sync tiles,
  *   [4] gather of the tensor-core tiles' x rows, [5] / [6] gate_up + clamp-SwiGLU on small /
  *   large tensor-core tiles, [7] down on mma.sync tiles, [8] / [9] down on small / large
- *   tensor-core tiles, [10] the weighted top-k combine.
+ *   tensor-core tiles, [10] the weighted top-k combine (for the smallest calls [7] is down and
+ *   the combine in one launch and [10] is 0; see moe_down_combine).
  * Kernels run back to back here instead of overlapping their launches as in
  * moe_mxfp4_forward_ex, so the sum exceeds a normal call's time.
  */

@@ -105,9 +105,11 @@ def test_forward_launch_counts():
     # 5 launches at decode sizes (fused select), 6 with the separate top-k + permutation, and 5
     # more (the gather and the small- and large-tile tensor-core GEMMs of both projections) once the
     # tensor-core path is on: H and I multiples of 512, M >= 5 and experts averaging >= 2.5
-    # assignments
+    # assignments; one fewer when down and the combine are one launch (I <= 1024, at most 8 tiles)
     lib = moe.load()
     assert lib.moe_forward_launches(0, 2048, 768, 128, 8) == 0
+    assert lib.moe_forward_launches(1, 2048, 768, 128, 8) == 4
+    assert lib.moe_forward_launches(2, 1024, 512, 16, 4) == 4
     assert lib.moe_forward_launches(8, 2048, 768, 128, 8) == 5
     assert lib.moe_forward_launches(1, 7168, 2048, 256, 8) == 5
     assert lib.moe_forward_launches(32, 7168, 2048, 256, 8) == 5
